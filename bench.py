@@ -1,0 +1,397 @@
+#!/usr/bin/env python
+"""Benchmark of the H-BitLinear forward pass (BitNet v2) on B200.
+
+Workload (one step = one pass of the whole layer over one batch):
+  ffn_wdown: X bf16 [8192 x 16384] (silu(a)*b, 1% outlier channels x40) ->
+  RMSNorm -> online Hadamard transform -> INT4 absmean codes -> ternary matmul
+  with W [4096 x 16384] (2-bit packed, absmean) -> bf16 Y [8192 x 4096].
+The packed weights are made once (offline step, not timed).
+
+Prints one JSON line (rank 0).  `value` is device-timed tokens/s with inputs
+resident in HBM (inputs larger than L2); `e2e` is the same metric through the
+host-buffer C-ABI call with the host<->device copies inside the timed region.
+`roofline` covers the dominant kernel, timed live with CUDA events on its
+stream; `quant` reports the fused norm+transform+quantisation kernel on the
+8192 x 4096 workload in GB/s against the measured HBM copy bandwidth.
+Multi-GPU (torchrun): every rank runs its own 8192-token batch with a replica
+of the packed weights (rows shard with no collective), weak scaling; times
+are the max over ranks.
+
+--impl reference times the CPU oracle (the plain scalar C statement of the
+layer, test infrastructure) on a bounded sample of the same workload.
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "H-BitLinear tokens/s (7B W_down, a4) & FWHT+quant GB/s, % roofline"
+UNIT = "tokens/s"
+M_TOK, K_IN, N_OUT, BITS = 8192, 16384, 4096, 4
+QM, QK = 8192, 4096  # quant workload
+WORKLOAD = "ffn_wdown: X bf16 [8192 x 16384] -> Y bf16 [8192 x 4096], INT4 absmean act, " \
+           "ternary W [4096 x 16384] 2-bit packed"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="hbl", choices=["hbl", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--kernel-iters", type=int, default=200,
+                    help="iterations of the per-kernel timing loops")
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d["bf16_tflops_sustained"], "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(prefix="hbl_clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", str(self.gpu)], stdout=self.out,
+                stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        res = {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        if self.proc is None:
+            return res
+        time.sleep(0.2)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.out.close()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for nm, v in zip(names, parts[5:9]):
+                    if v.lower().startswith("active"):
+                        reasons.add(nm)
+        os.unlink(self.path)
+        if sm:
+            res = {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
+                   "reasons": sorted(reasons), "samples": len(sm)}
+        return res
+
+
+def source_hash(*names):
+    h = hashlib.sha256()
+    for n in names:
+        with open(os.path.join(ROOT, "hadamard_rotated_int4_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel_key, src_hash):
+    """DRAM bytes per launch from a committed ncu capture, if the kernel is unchanged."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(kernel_key)
+    if not e or e.get("source_hash") != src_hash:
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+def cpu_baseline(X_bits, packed, alpha, target_s=15.0):
+    """The oracle, as it stands, on a bounded sample of the workload's rows."""
+    import numpy as np
+
+    import oracle
+
+    threads = os.cpu_count() or 1
+    rows = min(threads, 64)
+    t0 = time.perf_counter()
+    oracle.hbitlinear_forward(X_bits[:rows], packed, alpha, BITS, threads=threads)
+    dt = time.perf_counter() - t0
+    if dt < target_s / 3:
+        scale = max(1, int(target_s / max(dt, 1e-3)))
+        rows = min(M_TOK, rows * scale)
+        t0 = time.perf_counter()
+        oracle.hbitlinear_forward(X_bits[:rows], packed, alpha, BITS, threads=threads)
+        dt = time.perf_counter() - t0
+    used = min(threads, rows)
+    return {"value": rows / dt, "unit": UNIT, "cores": used, "kind": "oracle",
+            "sample": "%d of the 8192 token rows of the ffn_wdown workload (full K, full N), "
+                      "scalar C oracle, rows split over %d threads, %.1f s" % (rows, used, dt)}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import numpy as np
+
+    import oracle
+    from hadamard_rotated_int4_b200 import inputs
+
+    X = inputs.activations("ffn_wdown")
+    W = inputs.weights("ffn_wdown")
+    packed, alpha = oracle.pack_ternary(W)
+    threads = os.cpu_count() or 1
+    rows_per_step = min(8192, max(1, threads))
+    for i in range(args.warmup):
+        oracle.hbitlinear_forward(X[i * rows_per_step:(i + 1) * rows_per_step], packed, alpha,
+                                  BITS, threads=threads)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        lo = (i * rows_per_step) % (M_TOK - rows_per_step + 1)
+        oracle.hbitlinear_forward(X[lo:lo + rows_per_step], packed, alpha, BITS, threads=threads)
+    dt = time.perf_counter() - t0
+    value = args.steps * rows_per_step / dt
+    used = min(threads, rows_per_step)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * dt / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "s8", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "M": M_TOK, "K": K_IN, "N": N_OUT, "act_bits": BITS,
+                   "parallelism": "replicas by token rows (no collective)"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": used, "kind": "oracle",
+                         "sample": "each step: %d token rows of the ffn_wdown workload (full K "
+                                   "and N), scalar C oracle over %d threads" % (rows_per_step,
+                                                                                used)},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+    return 0
+
+
+def run_hbl(args):
+    import numpy as np
+    import torch
+
+    import hadamard_rotated_int4_b200 as hbl
+    from hadamard_rotated_int4_b200 import dist as hdist
+    from hadamard_rotated_int4_b200 import inputs
+
+    rank, local_rank, world = hdist.env_rank()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    pg = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+        pg = dist
+
+    def barrier():
+        if pg is not None:
+            pg.barrier()
+        torch.cuda.synchronize()
+
+    pk = peaks()
+    # ---- inputs: each rank its own 8192-token batch; the same weights everywhere
+    X_bits = inputs.activations("ffn_wdown", seed=rank)
+    W = inputs.weights("ffn_wdown")
+    Xd = torch.from_numpy(X_bits.view(np.int16)).view(torch.bfloat16).to(dev)
+    packed, alpha = hbl.pack_ternary(torch.from_numpy(W).to(dev))
+    ws = torch.empty(hbl.workspace_size(hbl.OP_HBITLINEAR_FORWARD, M_TOK, K_IN, N_OUT, BITS),
+                     dtype=torch.uint8, device=dev)
+    Y = torch.empty((M_TOK, N_OUT), dtype=torch.bfloat16, device=dev)
+    status = hbl.new_status(dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        hbl.hbitlinear_forward(Xd, packed, alpha, BITS, ws=ws, out=Y, status=status)
+
+    sampler = ClockSampler(local_rank)
+    for _ in range(max(3, args.warmup)):
+        step()
+    barrier()
+    sampler.start()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    barrier()
+    t_dev_ms = e0.elapsed_time(e1)
+    t_max_ms = hdist.max_over_ranks(t_dev_ms, dev)
+    value = world * M_TOK * args.steps / (t_max_ms / 1e3)
+
+    # ---- per-kernel timing (same kernels, through the two-call C-ABI path)
+    codes = torch.empty((M_TOK, K_IN // 2), dtype=torch.uint8, device=dev)
+    scales = torch.empty(M_TOK, dtype=torch.float32, device=dev)
+    rowsum = torch.empty(M_TOK, dtype=torch.int32, device=dev)
+    gws = torch.empty(max(16, hbl.workspace_size(hbl.OP_TERNARY_GEMM, M_TOK, K_IN, N_OUT, BITS)),
+                      dtype=torch.uint8, device=dev)
+    iters = max(args.kernel_iters, args.steps)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(iters)]
+    for i in range(3):
+        hbl.norm_fwht_quant(Xd, BITS, out=(codes, scales, rowsum))
+        hbl.ternary_gemm(codes, scales, rowsum, BITS, K_IN, packed, alpha, ws=gws, out=Y)
+    torch.cuda.synchronize()
+    for i in range(iters):
+        evs[i][0].record(stream)
+        hbl.norm_fwht_quant(Xd, BITS, out=(codes, scales, rowsum))
+        evs[i][1].record(stream)
+        hbl.ternary_gemm(codes, scales, rowsum, BITS, K_IN, packed, alpha, ws=gws, out=Y,
+                         status=status)
+        evs[i][2].record(stream)
+    torch.cuda.synchronize()
+    t_k1 = statistics.mean(e[0].elapsed_time(e[1]) for e in evs) * 1e-3
+    t_k2 = statistics.mean(e[1].elapsed_time(e[2]) for e in evs) * 1e-3
+
+    # ---- quant workload: 8192 x 4096, a4 and a8, 4 rotating inputs (256 MB > L2)
+    qX = [torch.from_numpy(inputs.activations("quant", seed=s).view(np.int16)).view(
+        torch.bfloat16).to(dev) for s in range(4)]
+    quant = {}
+    for bits in (4, 8):
+        qc = torch.empty((QM, QK if bits == 8 else QK // 2), dtype=torch.uint8, device=dev)
+        qs = torch.empty(QM, dtype=torch.float32, device=dev)
+        qr = torch.empty(QM, dtype=torch.int32, device=dev)
+        for i in range(4):
+            hbl.norm_fwht_quant(qX[i], bits, out=(qc, qs, qr))
+        torch.cuda.synchronize()
+        qi = max(args.kernel_iters, 40)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for i in range(qi):
+            hbl.norm_fwht_quant(qX[i % 4], bits, out=(qc, qs, qr))
+        b.record(stream)
+        torch.cuda.synchronize()
+        t = a.elapsed_time(b) * 1e-3 / qi
+        nbytes = QM * QK * 2 + QM * QK * bits // 8 + QM * 4 + QM * 4
+        gbs = nbytes / t / 1e9
+        quant["a%d" % bits] = {"workload": "quant 8192 x 4096 Student-t nu=3, 1% channels x20",
+                               "us": t * 1e6, "bytes": nbytes, "achieved_gbs": gbs,
+                               "frac": gbs / pk["hbm_gbs"]}
+    del qX
+    clocks = sampler.stop()
+
+    # ---- end to end through the host-buffer call: H2D X, forward, D2H Y
+    Xh = torch.from_numpy(X_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
+    Yh = torch.empty((M_TOK, N_OUT), dtype=torch.bfloat16).pin_memory()
+    hws = torch.empty(hbl.workspace_size(hbl.OP_HBITLINEAR_FORWARD_HOSTIO, M_TOK, K_IN, N_OUT,
+                                         BITS), dtype=torch.uint8, device=dev)
+    del Xd
+    for _ in range(2):
+        hbl.hbitlinear_forward_hostio(Xh, packed, alpha, BITS, Yh, hws, status=status)
+    barrier()
+    e2e_steps = max(3, min(args.steps, 20))
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(e2e_steps):
+        hbl.hbitlinear_forward_hostio(Xh, packed, alpha, BITS, Yh, hws, status=status)
+    b.record(stream)
+    barrier()
+    t_e2e = hdist.max_over_ranks(a.elapsed_time(b), dev) * 1e-3
+    e2e_value = world * M_TOK * e2e_steps / t_e2e
+    st = int(status[0].item())
+
+    # ---- roofline of the dominant kernel
+    ops = 2.0 * M_TOK * N_OUT * K_IN
+    if t_k2 >= t_k1:
+        achieved = ops / t_k2 / 1e12
+        peak = 2.0 * pk["bf16_tflops_sustained"]
+        roof = {"bound": "tensor", "kernel": "ternary_gemm_tc (tcgen05 kind::i8)",
+                "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                "peak_note": "int8 dense = %s sustained bf16 %.1f TFLOP/s x 2 (nominal "
+                             "int8:bf16 ratio)" % (pk["source"], pk["bf16_tflops_sustained"]),
+                "traffic": recorded_traffic("gemm_tc_a4_ffn_wdown",
+                                            source_hash("k2_ternary_gemm_tc.cu")),
+                "us_per_launch": t_k2 * 1e6}
+    else:
+        nbytes = M_TOK * K_IN * 2 + M_TOK * K_IN // 2 + 8 * M_TOK
+        achieved = nbytes / t_k1 / 1e9
+        roof = {"bound": "hbm", "kernel": "norm_fwht_quant", "achieved": achieved,
+                "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": achieved / pk["hbm_gbs"],
+                "traffic": recorded_traffic("norm_fwht_quant_a4_ffn_wdown",
+                                            source_hash("k1_impl.cuh")),
+                "us_per_launch": t_k1 * 1e6}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": t_max_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "s8", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "M": M_TOK, "K": K_IN, "N": N_OUT, "act_bits": BITS,
+                   "global_batch": world * M_TOK,
+                   "parallelism": "replicas by token rows (no collective)" if world > 1
+                   else "single GPU",
+                   "l2": "inputs larger than L2 (X 268 MB per step)"},
+        "roofline": roof,
+        "kernels_us": {"norm_fwht_quant": t_k1 * 1e6, "ternary_gemm_tc": t_k2 * 1e6},
+        "quant": quant,
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": M_TOK * K_IN * 2,
+                "d2h_bytes_per_step": M_TOK * N_OUT * 2, "steps": e2e_steps,
+                "api": "hbl_hbitlinear_forward_hostio (pinned host buffers)"},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clocks,
+        "device_status": st,
+        "peaks": pk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+
+        wp, wa = oracle.pack_ternary(W)
+        line["cpu_baseline"] = cpu_baseline(X_bits, wp, wa)
+    if rank == 0:
+        print(json.dumps(line))
+    if pg is not None:
+        pg.barrier()
+        pg.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_hbl(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,218 @@
+"""Python binding of libhbl.so, the sm_100a H-BitLinear library (BitNet v2).
+
+Argument marshalling only: every step of the layer runs in the library's CUDA
+kernels.  torch supplies device memory and the current CUDA stream.  There is
+no CPU fallback: calls raise if the library is not built or the device is not
+an sm_100 GPU.
+
+Names follow include/hbl.h:
+  pack_ternary(W)                         -> (W_packed int32 view [N, K/16], alpha [1])
+  norm_fwht(X)                            -> V fp32 [M, K]
+  norm_fwht_quant(X, act_bits)            -> (codes uint8, scales fp32 [M], rowsum int32 [M])
+  ternary_gemm(codes, scales, rowsum, act_bits, K, W_packed, alpha)  -> Y bf16 [M, N] (, acc)
+  hbitlinear_forward(X, W_packed, alpha, act_bits)                   -> Y bf16 [M, N]
+  hbitlinear_forward_hostio(X_host, W_packed, alpha, act_bits, Y_host, ws)
+"""
+import ctypes
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libhbl.so")
+
+HBL_OK = 0
+STATUS_NAMES = {0: "HBL_OK", 1: "HBL_ERR_INVALID_ARG", 2: "HBL_ERR_SHAPE", 3: "HBL_ERR_ALIGNMENT",
+                4: "HBL_ERR_UNSUPPORTED_ARCH", 5: "HBL_ERR_WORKSPACE", 6: "HBL_ERR_CUDA",
+                7: "HBL_ERR_TIMEOUT"}
+OP_PACK_TERNARY, OP_TERNARY_GEMM, OP_HBITLINEAR_FORWARD, OP_HBITLINEAR_FORWARD_HOSTIO = 0, 1, 2, 3
+EXPORTS = ("hbl_status_string", "hbl_version", "hbl_set_gemm_path", "hbl_workspace_size",
+           "hbl_pack_ternary", "hbl_norm_fwht", "hbl_norm_fwht_quant", "hbl_ternary_gemm",
+           "hbl_hbitlinear_forward", "hbl_hbitlinear_forward_hostio")
+
+_lib = None
+
+
+class HblError(RuntimeError):
+    def __init__(self, status, what):
+        self.status = status
+        super().__init__("%s failed: %s (%s)" % (what, STATUS_NAMES.get(status, status),
+                                                  lib().hbl_status_string(status).decode()))
+
+
+def lib():
+    """Load libhbl.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError("libhbl.so is not built (run __graft_entry__.build() or "
+                               "python hadamard_rotated_int4_b200/build.py)")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I, F, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+        L.hbl_status_string.restype = ctypes.c_char_p
+        L.hbl_status_string.argtypes = [I]
+        L.hbl_version.restype = I
+        L.hbl_version.argtypes = []
+        L.hbl_set_gemm_path.restype = I
+        L.hbl_set_gemm_path.argtypes = [I]
+        L.hbl_workspace_size.restype = I
+        L.hbl_workspace_size.argtypes = [I, I, I, I, I, ctypes.POINTER(SZ)]
+        L.hbl_pack_ternary.restype = I
+        L.hbl_pack_ternary.argtypes = [P, I, I, F, P, P, P, SZ, P]
+        L.hbl_norm_fwht.restype = I
+        L.hbl_norm_fwht.argtypes = [P, P, I, I, F, P, P, P]
+        L.hbl_norm_fwht_quant.restype = I
+        L.hbl_norm_fwht_quant.argtypes = [P, P, I, I, F, F, I, P, P, P, P, P]
+        L.hbl_ternary_gemm.restype = I
+        L.hbl_ternary_gemm.argtypes = [P, P, P, I, I, I, P, P, I, P, P, P, SZ, P, P]
+        L.hbl_hbitlinear_forward.restype = I
+        L.hbl_hbitlinear_forward.argtypes = [P, P, I, I, I, P, P, I, F, F, P, P, SZ, P, P]
+        L.hbl_hbitlinear_forward_hostio.restype = I
+        L.hbl_hbitlinear_forward_hostio.argtypes = [P, P, I, I, I, P, P, I, F, F, P, P, SZ, P, P]
+        _lib = L
+    return _lib
+
+
+def _check(status, what):
+    if status != HBL_OK:
+        raise HblError(status, what)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream():
+    import torch
+
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _dev(t, dtype, name):
+    import torch
+
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError("%s must be a CUDA tensor" % name)
+    if t.dtype != dtype:
+        raise TypeError("%s must be %s, got %s" % (name, dtype, t.dtype))
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+    return t
+
+
+def workspace_size(op, M, K, N, act_bits):
+    out = ctypes.c_size_t(0)
+    _check(lib().hbl_workspace_size(op, M, K, N, act_bits, ctypes.byref(out)), "workspace_size")
+    return out.value
+
+
+def set_gemm_path(path):
+    """0 = automatic, 1 = tensor cores, 2 = CUDA-core GEMV (process-wide)."""
+    _check(lib().hbl_set_gemm_path(int(path)), "set_gemm_path")
+
+
+def _workspace(nbytes, device):
+    import torch
+
+    return torch.empty(max(int(nbytes), 16), dtype=torch.uint8, device=device)
+
+
+def new_status(device):
+    import torch
+
+    return torch.zeros(4, dtype=torch.int32, device=device)
+
+
+def pack_ternary(W, eps=1e-5, ws=None):
+    import torch
+
+    _dev(W, torch.float32, "W")
+    N, K = W.shape
+    packed = torch.empty((N, K // 16), dtype=torch.int32, device=W.device)
+    alpha = torch.empty(4, dtype=torch.float32, device=W.device)
+    need = workspace_size(OP_PACK_TERNARY, 0, K, N, 0)
+    if ws is None:
+        ws = _workspace(need, W.device)
+    _check(lib().hbl_pack_ternary(_ptr(W), N, K, float(eps), _ptr(packed), _ptr(alpha), _ptr(ws),
+                                  ws.numel(), _stream()), "hbl_pack_ternary")
+    return packed, alpha[:1]
+
+
+def norm_fwht(X, gain=None, norm_eps=1e-6, status=None):
+    import torch
+
+    _dev(X, torch.bfloat16, "X")
+    M, K = X.shape
+    V = torch.empty((M, K), dtype=torch.float32, device=X.device)
+    _check(lib().hbl_norm_fwht(_ptr(X), _ptr(gain), M, K, float(norm_eps), _ptr(V), _ptr(status),
+                               _stream()), "hbl_norm_fwht")
+    return V
+
+
+def codes_shape(M, K, act_bits):
+    return (M, K if act_bits == 8 else K // 2)
+
+
+def norm_fwht_quant(X, act_bits, gain=None, norm_eps=1e-6, quant_eps=1e-5, out=None,
+                    status=None):
+    import torch
+
+    _dev(X, torch.bfloat16, "X")
+    M, K = X.shape
+    if out is None:
+        codes = torch.empty(codes_shape(M, K, act_bits), dtype=torch.uint8, device=X.device)
+        scales = torch.empty(max(M, 4), dtype=torch.float32, device=X.device)
+        rowsum = torch.empty(max(M, 4), dtype=torch.int32, device=X.device)
+    else:
+        codes, scales, rowsum = out
+    _check(lib().hbl_norm_fwht_quant(_ptr(X), _ptr(gain), M, K, float(norm_eps),
+                                     float(quant_eps), int(act_bits), _ptr(codes), _ptr(scales),
+                                     _ptr(rowsum), _ptr(status), _stream()),
+           "hbl_norm_fwht_quant")
+    return codes, scales[:M], rowsum[:M]
+
+
+def ternary_gemm(codes, scales, rowsum, act_bits, K, W_packed, alpha, want_acc=False, ws=None,
+                 out=None, status=None):
+    import torch
+
+    M = codes.shape[0]
+    N = W_packed.shape[0]
+    Y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16,
+                                                device=codes.device)
+    acc = torch.empty((M, N), dtype=torch.int32, device=codes.device) if want_acc else None
+    need = workspace_size(OP_TERNARY_GEMM, M, K, N, act_bits)
+    if ws is None:
+        ws = _workspace(need, codes.device)
+    _check(lib().hbl_ternary_gemm(_ptr(codes), _ptr(scales), _ptr(rowsum), int(act_bits), M, K,
+                                  _ptr(W_packed), _ptr(alpha), N, _ptr(Y), _ptr(acc), _ptr(ws),
+                                  ws.numel(), _ptr(status), _stream()), "hbl_ternary_gemm")
+    return (Y, acc) if want_acc else Y
+
+
+def hbitlinear_forward(X, W_packed, alpha, act_bits, gain=None, norm_eps=1e-6, quant_eps=1e-5,
+                       ws=None, out=None, status=None):
+    import torch
+
+    _dev(X, torch.bfloat16, "X")
+    M, K = X.shape
+    N = W_packed.shape[0]
+    Y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=X.device)
+    if ws is None:
+        ws = _workspace(workspace_size(OP_HBITLINEAR_FORWARD, M, K, N, act_bits), X.device)
+    _check(lib().hbl_hbitlinear_forward(_ptr(X), _ptr(gain), M, K, N, _ptr(W_packed),
+                                        _ptr(alpha), int(act_bits), float(norm_eps),
+                                        float(quant_eps), _ptr(Y), _ptr(ws), ws.numel(),
+                                        _ptr(status), _stream()), "hbl_hbitlinear_forward")
+    return Y
+
+
+def hbitlinear_forward_hostio(X_host, W_packed, alpha, act_bits, Y_host, ws, gain=None,
+                              norm_eps=1e-6, quant_eps=1e-5, status=None):
+    """Host bf16 X in, host bf16 Y out (pinned memory makes the copies asynchronous)."""
+    M, K = X_host.shape
+    N = W_packed.shape[0]
+    _check(lib().hbl_hbitlinear_forward_hostio(_ptr(X_host), _ptr(gain), M, K, N, _ptr(W_packed),
+                                               _ptr(alpha), int(act_bits), float(norm_eps),
+                                               float(quant_eps), _ptr(Y_host), _ptr(ws),
+                                               ws.numel(), _ptr(status), _stream()),
+           "hbl_hbitlinear_forward_hostio")
+    return Y_host

@@ -1,0 +1,333 @@
+// api.cu -- the C ABI of libhbl: argument validation (before any CUDA call),
+// device checks, workspace carving and dispatch to the sm_100a kernels.
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include <atomic>
+#include <mutex>
+#include <unordered_map>
+
+#include "hbl.h"
+#include "hbl_launch.h"
+
+namespace hbl {
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+struct DevInfo {
+    std::atomic<int> state{0};  // 0 unknown, 1 ok, 2 unsupported
+    int sms = 0;
+};
+DevInfo g_dev[kMaxDevices];
+std::atomic<int> g_path{0};  // 0 auto, 1 tensor core, 2 CUDA-core GEMV
+
+bool is_pow2(int64_t v) { return v > 0 && (v & (v - 1)) == 0; }
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool finite_nonneg(float e) { return isfinite(e) && e >= 0.0f; }
+size_t up256(size_t v) { return (v + 255) & ~(size_t)255; }
+
+hbl_status check_k(int K) {
+    return (K >= 16 && K <= 32768 && is_pow2(K)) ? HBL_OK : HBL_ERR_SHAPE;
+}
+hbl_status check_n(int N) { return (N >= 16 && N % 16 == 0) ? HBL_OK : HBL_ERR_SHAPE; }
+
+// Current device must be sm_100; caches the SM count.
+hbl_status device(int* sms) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return HBL_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return HBL_ERR_CUDA;
+    DevInfo& d = g_dev[dev];
+    int st = d.state.load(std::memory_order_acquire);
+    if (st == 0) {
+        int major = 0, minor = 0, n = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return HBL_ERR_CUDA;
+        d.sms = n;
+        st = (major == 10 && minor == 0) ? 1 : 2;
+        d.state.store(st, std::memory_order_release);
+    }
+    if (st != 1) return HBL_ERR_UNSUPPORTED_ARCH;
+    *sms = d.sms;
+    return HBL_OK;
+}
+
+int codes_row_bytes(int K, int act_bits) { return act_bits == 8 ? K : K / 2; }
+
+bool use_gemv(int64_t M) {
+    const int path = g_path.load();
+    if (path == 1) return false;
+    if (path == 2) return true;
+    return M <= gemv_max_m();
+}
+
+size_t gemm_ws(int64_t M, int K, int N, int sms_guess) {
+    if (!use_gemv(M)) return 0;
+    const int64_t mchunk = M < gemv_max_m() ? M : gemv_max_m();
+    return gemv_workspace(mchunk, K, N, sms_guess);
+}
+
+// SM count for sizing when no device is queried yet (workspace queries must
+// not need a GPU): the split factor only grows with SM count, so size for 148.
+constexpr int kSizingSms = 148;
+
+hbl_status run_gemm(const GemmArgs& a, void* ws, size_t ws_bytes, cudaStream_t s, int sms) {
+    if (!use_gemv(a.M)) return launch_gemm_tc(a, s, sms);
+    // CUDA-core path in chunks of up to gemv_max_m() tokens (workspace reused in order)
+    const int64_t step = gemv_max_m();
+    for (int64_t r0 = 0; r0 < a.M; r0 += step) {
+        GemmArgs c = a;
+        c.M = (a.M - r0) < step ? (a.M - r0) : step;
+        c.codes = static_cast<const uint8_t*>(a.codes) + r0 * codes_row_bytes(a.K, a.act_bits);
+        c.scales = a.scales + r0;
+        c.rowsum = a.rowsum + r0;
+        c.Y = a.Y + r0 * a.N;
+        c.acc_out = a.acc_out ? a.acc_out + r0 * a.N : nullptr;
+        hbl_status st = launch_gemv(c, ws, ws_bytes, s, sms);
+        if (st != HBL_OK) return st;
+    }
+    return HBL_OK;
+}
+
+}  // namespace
+
+bool smem_attr_once(const void* func, int bytes) {
+    static std::mutex mu;
+    static std::unordered_map<uint64_t, int> done;  // (device, func) -> bytes set
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return false;
+    const uint64_t key = (reinterpret_cast<uintptr_t>(func) << 6) ^ (uint64_t)dev;
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = done.find(key);
+    if (it != done.end() && it->second >= bytes) return true;
+    if (cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
+        cudaSuccess)
+        return false;
+    done[key] = bytes;
+    return true;
+}
+
+}  // namespace hbl
+
+using namespace hbl;
+
+extern "C" {
+
+const char* hbl_status_string(int status) {
+    switch (status) {
+        case HBL_OK: return "ok";
+        case HBL_ERR_INVALID_ARG: return "invalid argument";
+        case HBL_ERR_SHAPE: return "unsupported shape";
+        case HBL_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
+        case HBL_ERR_UNSUPPORTED_ARCH: return "device is not sm_100";
+        case HBL_ERR_WORKSPACE: return "workspace missing or too small";
+        case HBL_ERR_CUDA: return "CUDA runtime error";
+        case HBL_ERR_TIMEOUT: return "device-side wait timed out";
+        default: return "unknown status";
+    }
+}
+
+int hbl_version(void) { return 100; }
+
+int hbl_set_gemm_path(int path) {
+    if (path < 0 || path > 2) return HBL_ERR_INVALID_ARG;
+    g_path.store(path);
+    return HBL_OK;
+}
+
+hbl_status hbl_workspace_size(int op, int M, int K, int N, int act_bits, size_t* bytes) {
+    if (bytes == nullptr) return HBL_ERR_INVALID_ARG;
+    *bytes = 0;
+    switch (op) {
+        case HBL_OP_PACK_TERNARY:
+            if (N < 1) return HBL_ERR_SHAPE;
+            if (check_k(K) != HBL_OK) return HBL_ERR_SHAPE;
+            *bytes = pack_ternary_workspace(N, K);
+            return HBL_OK;
+        case HBL_OP_TERNARY_GEMM:
+        case HBL_OP_HBITLINEAR_FORWARD:
+        case HBL_OP_HBITLINEAR_FORWARD_HOSTIO: {
+            if (M < 0 || check_k(K) != HBL_OK || check_n(N) != HBL_OK) return HBL_ERR_SHAPE;
+            if (act_bits != 4 && act_bits != 8) return HBL_ERR_INVALID_ARG;
+            size_t b = up256(gemm_ws(M, K, N, kSizingSms));
+            if (op != HBL_OP_TERNARY_GEMM) {
+                b += up256((size_t)M * codes_row_bytes(K, act_bits));  // codes
+                b += up256((size_t)M * 4) * 2;                         // scales, rowsum
+            }
+            if (op == HBL_OP_HBITLINEAR_FORWARD_HOSTIO) {
+                b += up256((size_t)M * K * 2);  // device copy of X
+                b += up256((size_t)M * N * 2);  // device copy of Y
+            }
+            *bytes = b;
+            return HBL_OK;
+        }
+        default: return HBL_ERR_INVALID_ARG;
+    }
+}
+
+hbl_status hbl_pack_ternary(const float* W, int N, int K, float eps, uint32_t* W_packed,
+                            float* alpha, void* ws, size_t ws_bytes, void* stream) {
+    if (!W || !W_packed || !alpha) return HBL_ERR_INVALID_ARG;
+    if (!finite_nonneg(eps)) return HBL_ERR_INVALID_ARG;
+    if (N < 1 || check_k(K) != HBL_OK) return HBL_ERR_SHAPE;
+    if (!aligned16(W) || !aligned16(W_packed) || !aligned16(alpha)) return HBL_ERR_ALIGNMENT;
+    if (ws == nullptr || ws_bytes < pack_ternary_workspace(N, K)) return HBL_ERR_WORKSPACE;
+    if (!aligned16(ws)) return HBL_ERR_ALIGNMENT;
+    int sms = 0;
+    hbl_status st = device(&sms);
+    if (st != HBL_OK) return st;
+    return launch_pack_ternary(W, N, K, eps, W_packed, alpha, ws,
+                               static_cast<cudaStream_t>(stream), sms);
+}
+
+static hbl_status check_act_args(const uint16_t* X, const float* gain, int M, int K,
+                                 float norm_eps) {
+    if (!X) return HBL_ERR_INVALID_ARG;
+    if (!finite_nonneg(norm_eps)) return HBL_ERR_INVALID_ARG;
+    if (M < 0 || check_k(K) != HBL_OK) return HBL_ERR_SHAPE;
+    if (!aligned16(X) || (gain && !aligned16(gain))) return HBL_ERR_ALIGNMENT;
+    return HBL_OK;
+}
+
+hbl_status hbl_norm_fwht(const uint16_t* X, const float* gain, int M, int K, float norm_eps,
+                         float* V, int32_t* dev_status, void* stream) {
+    (void)dev_status;
+    hbl_status st = check_act_args(X, gain, M, K, norm_eps);
+    if (st != HBL_OK) return st;
+    if (!V) return HBL_ERR_INVALID_ARG;
+    if (!aligned16(V)) return HBL_ERR_ALIGNMENT;
+    if (M == 0) return HBL_OK;
+    int sms = 0;
+    if ((st = device(&sms)) != HBL_OK) return st;
+    return launch_norm_fwht_quant(X, gain, M, K, norm_eps, 0.f, 0, nullptr, nullptr, nullptr, V,
+                                  static_cast<cudaStream_t>(stream), sms);
+}
+
+hbl_status hbl_norm_fwht_quant(const uint16_t* X, const float* gain, int M, int K,
+                               float norm_eps, float quant_eps, int act_bits, void* codes,
+                               float* scales, int32_t* rowsum, int32_t* dev_status,
+                               void* stream) {
+    (void)dev_status;
+    hbl_status st = check_act_args(X, gain, M, K, norm_eps);
+    if (st != HBL_OK) return st;
+    if (act_bits != 4 && act_bits != 8) return HBL_ERR_INVALID_ARG;
+    if (!finite_nonneg(quant_eps)) return HBL_ERR_INVALID_ARG;
+    if (!codes || !scales) return HBL_ERR_INVALID_ARG;
+    if (!aligned16(codes) || !aligned16(scales) || (rowsum && !aligned16(rowsum)))
+        return HBL_ERR_ALIGNMENT;
+    if (M == 0) return HBL_OK;
+    int sms = 0;
+    if ((st = device(&sms)) != HBL_OK) return st;
+    return launch_norm_fwht_quant(X, gain, M, K, norm_eps, quant_eps, act_bits, codes, scales,
+                                  rowsum, nullptr, static_cast<cudaStream_t>(stream), sms);
+}
+
+hbl_status hbl_ternary_gemm(const void* codes, const float* scales, const int32_t* rowsum,
+                            int act_bits, int M, int K, const uint32_t* W_packed,
+                            const float* alpha, int N, uint16_t* Y, int32_t* acc_out,
+                            void* ws, size_t ws_bytes, int32_t* dev_status, void* stream) {
+    if (!codes || !scales || !rowsum || !W_packed || !alpha || !Y) return HBL_ERR_INVALID_ARG;
+    if (act_bits != 4 && act_bits != 8) return HBL_ERR_INVALID_ARG;
+    if (M < 0 || check_k(K) != HBL_OK || check_n(N) != HBL_OK) return HBL_ERR_SHAPE;
+    if (!aligned16(codes) || !aligned16(scales) || !aligned16(rowsum) || !aligned16(W_packed) ||
+        !aligned16(alpha) || !aligned16(Y) || (acc_out && !aligned16(acc_out)) ||
+        (dev_status && !aligned16(dev_status)))
+        return HBL_ERR_ALIGNMENT;
+    const size_t need = gemm_ws(M, K, N, kSizingSms);
+    if (need > 0 && (ws == nullptr || ws_bytes < need)) return HBL_ERR_WORKSPACE;
+    if (ws && !aligned16(ws)) return HBL_ERR_ALIGNMENT;
+    if (M == 0) return HBL_OK;
+    int sms = 0;
+    hbl_status st = device(&sms);
+    if (st != HBL_OK) return st;
+    GemmArgs a{codes, scales, rowsum, act_bits, M, K, W_packed, alpha, N, Y, acc_out, dev_status};
+    return run_gemm(a, ws, ws_bytes, static_cast<cudaStream_t>(stream), sms);
+}
+
+static hbl_status forward_impl(const uint16_t* X, const float* gain, int M, int K, int N,
+                               const uint32_t* W_packed, const float* alpha, int act_bits,
+                               float norm_eps, float quant_eps, uint16_t* Y, uint8_t* ws,
+                               size_t ws_bytes, int32_t* dev_status, cudaStream_t s, int sms) {
+    const size_t cb = up256((size_t)M * codes_row_bytes(K, act_bits));
+    const size_t sb = up256((size_t)M * 4);
+    uint8_t* codes = ws;
+    float* scales = reinterpret_cast<float*>(ws + cb);
+    int32_t* rowsum = reinterpret_cast<int32_t*>(ws + cb + sb);
+    uint8_t* gws = ws + cb + 2 * sb;
+    const size_t gws_bytes = ws_bytes - (cb + 2 * sb);
+    hbl_status st = launch_norm_fwht_quant(X, gain, M, K, norm_eps, quant_eps, act_bits, codes,
+                                           scales, rowsum, nullptr, s, sms);
+    if (st != HBL_OK) return st;
+    GemmArgs a{codes, scales, rowsum, act_bits, M, K, W_packed, alpha, N, Y, nullptr, dev_status};
+    return run_gemm(a, gws, gws_bytes, s, sms);
+}
+
+static hbl_status check_forward(const uint16_t* X, const float* gain, int M, int K, int N,
+                                const uint32_t* W_packed, const float* alpha, int act_bits,
+                                float norm_eps, float quant_eps, const uint16_t* Y, void* ws,
+                                size_t ws_bytes, int32_t* dev_status, int op, bool host_xy) {
+    if (!X || !W_packed || !alpha || !Y) return HBL_ERR_INVALID_ARG;
+    if (act_bits != 4 && act_bits != 8) return HBL_ERR_INVALID_ARG;
+    if (!finite_nonneg(norm_eps) || !finite_nonneg(quant_eps)) return HBL_ERR_INVALID_ARG;
+    if (M < 0 || check_k(K) != HBL_OK || check_n(N) != HBL_OK) return HBL_ERR_SHAPE;
+    if ((!host_xy && (!aligned16(X) || !aligned16(Y))) || (gain && !aligned16(gain)) ||
+        !aligned16(W_packed) || !aligned16(alpha) || (dev_status && !aligned16(dev_status)))
+        return HBL_ERR_ALIGNMENT;
+    size_t need = 0;
+    hbl_workspace_size(op, M, K, N, act_bits, &need);
+    if (ws == nullptr || ws_bytes < need) return HBL_ERR_WORKSPACE;
+    if (!aligned16(ws)) return HBL_ERR_ALIGNMENT;
+    return HBL_OK;
+}
+
+hbl_status hbl_hbitlinear_forward(const uint16_t* X, const float* gain, int M, int K, int N,
+                                  const uint32_t* W_packed, const float* alpha, int act_bits,
+                                  float norm_eps, float quant_eps, uint16_t* Y, void* ws,
+                                  size_t ws_bytes, int32_t* dev_status, void* stream) {
+    hbl_status st = check_forward(X, gain, M, K, N, W_packed, alpha, act_bits, norm_eps,
+                                  quant_eps, Y, ws, ws_bytes, dev_status,
+                                  HBL_OP_HBITLINEAR_FORWARD, false);
+    if (st != HBL_OK) return st;
+    if (M == 0) return HBL_OK;
+    int sms = 0;
+    if ((st = device(&sms)) != HBL_OK) return st;
+    return forward_impl(X, gain, M, K, N, W_packed, alpha, act_bits, norm_eps, quant_eps, Y,
+                        static_cast<uint8_t*>(ws), ws_bytes, dev_status,
+                        static_cast<cudaStream_t>(stream), sms);
+}
+
+hbl_status hbl_hbitlinear_forward_hostio(const uint16_t* X_host, const float* gain, int M,
+                                         int K, int N, const uint32_t* W_packed,
+                                         const float* alpha, int act_bits, float norm_eps,
+                                         float quant_eps, uint16_t* Y_host, void* ws,
+                                         size_t ws_bytes, int32_t* dev_status, void* stream) {
+    hbl_status st = check_forward(X_host, gain, M, K, N, W_packed, alpha, act_bits, norm_eps,
+                                  quant_eps, Y_host, ws, ws_bytes, dev_status,
+                                  HBL_OP_HBITLINEAR_FORWARD_HOSTIO, true);
+    if (st != HBL_OK) return st;
+    if (M == 0) return HBL_OK;
+    int sms = 0;
+    if ((st = device(&sms)) != HBL_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t xb = up256((size_t)M * K * 2), yb = up256((size_t)M * N * 2);
+    uint8_t* w8 = static_cast<uint8_t*>(ws);
+    uint16_t* Xd = reinterpret_cast<uint16_t*>(w8);
+    uint16_t* Yd = reinterpret_cast<uint16_t*>(w8 + xb);
+    uint8_t* fws = w8 + xb + yb;
+    const size_t fws_bytes = ws_bytes - xb - yb;
+    if (cudaMemcpyAsync(Xd, X_host, (size_t)M * K * 2, cudaMemcpyHostToDevice, s) != cudaSuccess)
+        return HBL_ERR_CUDA;
+    st = forward_impl(Xd, gain, M, K, N, W_packed, alpha, act_bits, norm_eps, quant_eps, Yd, fws,
+                      fws_bytes, dev_status, s, sms);
+    if (st != HBL_OK) return st;
+    if (cudaMemcpyAsync(Y_host, Yd, (size_t)M * N * 2, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return HBL_ERR_CUDA;
+    return HBL_OK;
+}
+
+}  // extern "C"

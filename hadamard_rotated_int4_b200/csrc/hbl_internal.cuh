@@ -1,0 +1,108 @@
+// hbl_internal.cuh -- device helpers shared by the sm_100a kernels of libhbl.
+// Inline PTX wrappers (cp.async, bulk prefetch, named barriers, packed fp32x2
+// arithmetic, mbarriers, TMA, tcgen05) and a compile-time loop helper.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <type_traits>
+#include <utility>
+
+#include "hbl.h"
+
+namespace hbl {
+
+// ------------------------------------------------------------ compile time
+
+template <int I>
+using ic = std::integral_constant<int, I>;
+
+template <int Begin, int End, class F>
+__device__ __forceinline__ void static_for(F&& f) {
+    if constexpr (Begin < End) {
+        f(ic<Begin>{});
+        static_for<Begin + 1, End>(f);
+    }
+}
+
+__host__ __device__ constexpr int ilog2(unsigned v) {
+    int r = 0;
+    while ((1u << r) < v) ++r;
+    return r;
+}
+
+// ------------------------------------------------------------ status
+
+// First non-zero status wins; the host reads it after synchronising.
+__device__ __forceinline__ void report_status(int32_t* st, int code) {
+    if (st != nullptr) atomicCAS(reinterpret_cast<int*>(st), 0, code);
+}
+
+// Upper bound on spins of any device-side wait (each spin also sleeps), so a
+// wait that can never be satisfied returns an error instead of hanging.
+constexpr uint32_t kSpinLimit = 1u << 22;
+
+// ------------------------------------------------------------ memory
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// 16-byte async copy global -> shared; src_bytes 0 zero-fills without reading.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, int src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src),
+                 "r"(src_bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+    asm volatile("cp.async.commit_group;\n" ::: "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+    asm volatile("cp.async.wait_group 0;\n" ::: "memory");
+}
+
+// Hint: bring [src, src + bytes) into L2 (bytes a multiple of 16, src 16B aligned).
+__device__ __forceinline__ void prefetch_l2_bulk(const void* src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;\n" ::"l"(src), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void named_barrier(int id, int nthreads) {
+    asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];\n"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(addr)
+                 : "memory");
+    return v;
+}
+__device__ __forceinline__ void sts128(uint32_t addr, uint4 v) {
+    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};\n" ::"r"(addr), "r"(v.x), "r"(v.y),
+                 "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+
+// ------------------------------------------------------------ fp32x2 (sm_100)
+
+__device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+__device__ __forceinline__ float2 sub2(float2 a, float2 b) {
+    unsigned long long ra, rb, rd;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(ra) : "f"(a.x), "f"(a.y));
+    asm("mov.b64 %0, {%1, %2};" : "=l"(rb) : "f"(b.x), "f"(b.y));
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(rd) : "l"(ra), "l"(rb));
+    float2 d;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(d.x), "=f"(d.y) : "l"(rd));
+    return d;
+}
+
+// bf16 pair (low half = first element) -> two fp32 (exact widening).
+__device__ __forceinline__ float2 bf16x2_to_f2(uint32_t w) {
+    return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+
+}  // namespace hbl

@@ -1,0 +1,51 @@
+// hbl_launch.h -- host-side launchers of the sm_100a kernels (internal to libhbl).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "hbl.h"
+
+namespace hbl {
+
+// Sets the dynamic shared-memory limit of `func` once per device (idempotent).
+bool smem_attr_once(const void* func, int bytes);
+
+// K1: mode 0 writes fp32 V, mode 4/8 writes INT4/INT8 codes + scales (+ rowsum).
+hbl_status launch_norm_fwht_quant(const uint16_t* X, const float* gain, int64_t M, int K,
+                                  float norm_eps, float quant_eps, int mode, void* codes,
+                                  float* scales, int32_t* rowsum, float* V, cudaStream_t stream,
+                                  int num_sms);
+
+// K0: absmean ternarisation + 2-bit packing (K a power of two).
+size_t pack_ternary_workspace(int N, int K);
+hbl_status launch_pack_ternary(const float* W, int N, int K, float eps, uint32_t* W_packed,
+                               float* alpha, void* ws, cudaStream_t stream, int num_sms);
+
+// Ternary GEMM back ends.  All compute acc = sum_k q*t exactly, Y = bf16(acc*alpha*s).
+struct GemmArgs {
+    const void* codes;
+    const float* scales;
+    const int32_t* rowsum;
+    int act_bits;
+    int64_t M;
+    int K;
+    const uint32_t* W_packed;
+    const float* alpha;
+    int N;
+    uint16_t* Y;
+    int32_t* acc_out;
+    int32_t* dev_status;
+};
+
+// K2: tcgen05 tensor-core GEMM (TMEM accumulators), any M.
+hbl_status launch_gemm_tc(const GemmArgs& a, cudaStream_t stream, int num_sms);
+
+// K3: CUDA-core split-K GEMV for small M (M <= gemv_max_m()).
+int gemv_max_m();
+size_t gemv_workspace(int64_t M, int K, int N, int num_sms);
+hbl_status launch_gemv(const GemmArgs& a, void* ws, size_t ws_bytes, cudaStream_t stream,
+                       int num_sms);
+
+}  // namespace hbl

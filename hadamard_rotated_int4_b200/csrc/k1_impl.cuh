@@ -1,0 +1,605 @@
+// k1_impl.cuh -- fused RMSNorm + online Walsh-Hadamard transform +
+// per-token INT8 (absmax) / INT4 (absmean) quantisation, one token row per
+// group of T threads, for sm_100a.
+//
+// What it computes (BitNet v2 write-up, 0755model.com, sections
+// "BitNet v2：原生4位激活" and "H-BitLinear"; shengxinai.com section 2.2):
+//   r = 1/sqrt(tree_sum(x*x) * (1/K) + norm_eps),  u = (x * r) * gain
+//   v = (u . H_K) * c_K                        (butterflies h = 1, 2, ..., K/2)
+//   INT8: q = clip(rhe(v * (127/(max|v| + eps))), -128, 127), scale = max|v|/127
+//   INT4: beta = tree_sum(|v|) * (1/K), q = clip(rhe(v * (sqrt7/(beta+eps))), -8, 7),
+//         scale = beta/sqrt7
+// Every fp32 operation is a single IEEE round-to-nearest operation (no FMA
+// contraction, explicit _rn intrinsics), the butterfly stages run in ascending
+// order and every sum is the perfect pairwise tree over index order, so the
+// codes are bit-identical to a scalar evaluation in that order.
+//
+// Thread mapping.  Each thread holds R = 128 fp32 values of its row (R = K for
+// K < 128).  Index bits of the row are assigned to register bits and thread
+// bits by a sequence of layouts:
+//   N  (natural): register bits <-> index bits 0..6, thread bits <-> 7..L-1.
+//      Stages 0..6 run in registers.
+//   P_b (pass b): register bits <-> {0, 1} + stage bits [b, b+5) (+ the lowest
+//      free bits when fewer than 5 stages remain), thread bits <-> the rest.
+//      Index bits 0 and 1 stay in registers so every shared-memory access is a
+//      16-byte vector.  Stages [b, b+5) run in registers.
+// Between layouts the row is written to shared memory and read back; an XOR
+// swizzle of the 16-byte chunk index keeps every access of every layout free
+// of bank conflicts.  K = 4096 needs one exchange, K = 16384 two.
+// The row is staged bf16 -> shared memory with coalesced 16-byte cp.async
+// (swizzled so the per-thread reads are conflict-free too), and the next
+// group's rows are prefetched into L2 with one bulk prefetch.
+#pragma once
+#include <cuda_runtime.h>
+#include <math.h>
+
+#include "hbl_internal.cuh"
+#include "hbl_launch.h"
+
+namespace hbl {
+namespace k1 {
+
+constexpr int kRegLog = 7;
+constexpr int kRedFloats = 128;  // per-group cross-warp reduction scratch
+
+template <int L>
+struct Cfg {
+    static constexpr int K = 1 << L;
+    static constexpr int r = L < kRegLog ? L : kRegLog;
+    static constexpr int R = 1 << r;           // values per thread
+    static constexpr int t = L - r;            // thread bits of a row
+    static constexpr int T = 1 << t;           // threads per row
+    static constexpr int W = T > 32 ? T : 32;  // threads sharing one staging buffer
+    static constexpr int kRowsPerGroup = W / T;
+    static constexpr int kGroupsPerCta = T >= 128 ? 1 : 128 / W;
+    static constexpr int kCtaThreads = kGroupsPerCta * W;
+    static constexpr int kLaneBits = t < 5 ? t : 5;
+    static constexpr int kWarpBits = t > 5 ? t - 5 : 0;
+    static constexpr int kPasses = L <= kRegLog ? 0 : (L - kRegLog + 4) / 5;
+    static constexpr int kBufBytes = kRowsPerGroup * K * 4;  // fp32 row(s) of the group
+    static constexpr int kStageShift = ilog2(R / 8);         // chunks per thread = R/8
+    static constexpr int kSmemBytes = kGroupsPerCta * (kBufBytes + kRedFloats * 4);
+    // 3 CTAs (12 warps) per SM where the register budget (170) suffices
+    static constexpr int kMinBlocks = kCtaThreads >= 256 ? 1 : ((L >= 8 && L != 12) ? 2 : 3);
+};
+
+// Layout p: 0 = natural, p >= 1 = pass p (stage base 7 + 5 (p - 1)).
+template <int L>
+struct Lay {
+    using C = Cfg<L>;
+    __host__ __device__ static constexpr uint32_t reg_mask(int p) {
+        if (p == 0) return (1u << C::r) - 1u;
+        int b = kRegLog + 5 * (p - 1);
+        int n = (L - b) < 5 ? (L - b) : 5;
+        uint32_t m = 3u;
+        for (int s = b; s < b + n; ++s) m |= 1u << s;
+        int cnt = 2 + n;
+        for (int f = 2; cnt < kRegLog; ++f)
+            if (!((m >> f) & 1u)) {
+                m |= 1u << f;
+                ++cnt;
+            }
+        return m;
+    }
+    __host__ __device__ static constexpr int reg_idx(int p, int rb) {
+        uint32_t m = reg_mask(p);
+        int c = 0;
+        for (int i = 0; i < 32; ++i)
+            if ((m >> i) & 1u) {
+                if (c == rb) return i;
+                ++c;
+            }
+        return -1;
+    }
+    __host__ __device__ static constexpr int thr_idx(int p, int tb) {
+        uint32_t m = reg_mask(p);
+        int c = 0;
+        for (int i = 0; i < L; ++i)
+            if (!((m >> i) & 1u)) {
+                if (c == tb) return i;
+                ++c;
+            }
+        return -1;
+    }
+    __host__ __device__ static constexpr int reg_off(int p, int i) {
+        int e = 0;
+        for (int rb = 0; rb < C::r; ++rb)
+            if ((i >> rb) & 1) e |= 1 << reg_idx(p, rb);
+        return e;
+    }
+    __host__ __device__ static constexpr int reg_bit_of(int p, int idx) {
+        for (int rb = 0; rb < C::r; ++rb)
+            if (reg_idx(p, rb) == idx) return rb;
+        return -1;
+    }
+    // number of lowest index bits held in registers (the contiguous run)
+    __host__ __device__ static constexpr int run_bits(int p) {
+        uint32_t m = reg_mask(p);
+        int c = 0;
+        while (c < L && ((m >> c) & 1u)) ++c;
+        return c;
+    }
+};
+
+// XOR swizzle of a 16-byte chunk index for the fp32 row exchanges; linear over
+// GF(2), so swz(a ^ b) = swz(a) ^ swz(b).
+__host__ __device__ constexpr uint32_t swz(uint32_t ch) {
+    uint32_t b3 = (ch >> 3) & 1u, b4 = (ch >> 4) & 1u, b5 = (ch >> 5) & 1u;
+    uint32_t b6 = (ch >> 6) & 1u, b7 = (ch >> 7) & 1u;
+    return ch ^ ((b3 ^ b4 ^ b5) | ((b3 ^ b6) << 1) | ((b4 ^ b7) << 2));
+}
+// Swizzle of the bf16 staging chunks (8 elements each); linear too.
+template <int S>
+__host__ __device__ constexpr uint32_t stage_swz(uint32_t g) {
+    return g ^ ((g >> S) & 7u);
+}
+
+struct Params {
+    const uint16_t* X;
+    const float* gain;
+    int64_t M;
+    float norm_eps, quant_eps, cK, s7;
+    uint8_t* codes;
+    float* scales;
+    int32_t* rowsum;
+    float* V;
+};
+
+template <int T>
+__device__ __forceinline__ void group_sync(int grp) {
+    if constexpr (T <= 32)
+        __syncwarp();
+    else
+        named_barrier(1 + grp, T);
+}
+
+// ---- register-level pieces ------------------------------------------------
+
+// Butterfly stage on register bit RB of the float2 array (R/2 entries).
+template <int R, int RB>
+__device__ __forceinline__ void stage_regs(float2 (&d)[R / 2]) {
+    if constexpr (RB == 0) {
+        static_for<0, R / 2>([&](auto kk) {
+            constexpr int k = decltype(kk)::value;
+            float a = d[k].x, b = d[k].y;
+            d[k].x = __fadd_rn(a, b);
+            d[k].y = __fsub_rn(a, b);
+        });
+    } else {
+        constexpr int h = 1 << (RB - 1);
+        static_for<0, R / 2>([&](auto kk) {
+            constexpr int k = decltype(kk)::value;
+            if constexpr ((k & h) == 0) {
+                float2 a = d[k], b = d[k | h];
+                d[k] = add2(a, b);
+                d[k | h] = sub2(a, b);
+            }
+        });
+    }
+}
+
+// Perfect pairwise tree (index order) of f(k) for k in [0, N), streaming with a
+// stack of partial sums so only log2(N) partials stay live.
+template <int N, class F>
+__device__ __forceinline__ float stream_tree(F&& f) {
+    constexpr int D = ilog2(N) + 1;
+    float stk[D] = {};
+    float out = 0.f;
+    static_for<0, N>([&](auto kk) {
+        constexpr int k = decltype(kk)::value;
+        float x = f(kk);
+        constexpr int ones = [] {
+            int c = 0;
+            while ((k >> c) & 1) ++c;
+            return c;
+        }();
+        static_for<0, ones>([&](auto ll) {
+            constexpr int l = decltype(ll)::value;
+            x = __fadd_rn(stk[l], x);
+        });
+        if constexpr (k == N - 1)
+            out = x;
+        else
+            stk[ones] = x;
+    });
+    return out;
+}
+
+// ---- the kernel -------------------------------------------------------------
+
+// MODE: 0 = write fp32 V (norm + transform only), 4 = INT4 codes, 8 = INT8 codes.
+// GAIN: multiply by the per-channel RMSNorm gain (false: gain of one, exact skip).
+template <int L, int MODE, bool GAIN>
+__global__ void __launch_bounds__(Cfg<L>::kCtaThreads, Cfg<L>::kMinBlocks)
+    norm_fwht_quant_kernel(Params p) {
+    using C = Cfg<L>;
+    using Y = Lay<L>;
+    constexpr int R = C::R, T = C::T, W = C::W, K = C::K;
+    constexpr int P_LAST = C::kPasses;
+    extern __shared__ __align__(128) uint8_t smem[];
+
+    const int tid = threadIdx.x;
+    const int grp = tid / W;
+    const int w = tid % W;
+    const int lane = tid & 31;
+    const int j = (T >= 32) ? w : (lane % T);    // thread index within its row
+    const int rig = (T >= 32) ? 0 : (lane / T);  // row within the group
+    const int wig = w >> 5;                      // warp within the row (T > 32)
+    uint8_t* buf = smem + grp * C::kBufBytes;
+    const uint32_t buf_s = smem_addr(buf);
+    float* red = reinterpret_cast<float*>(smem + C::kGroupsPerCta * C::kBufBytes) +
+                 grp * kRedFloats;
+
+    // thread part of the element index in layout P (plus the row offset)
+    auto thr_off = [&](auto pp) -> uint32_t {
+        constexpr int P = decltype(pp)::value;
+        uint32_t e = 0;
+        static_for<0, C::t>([&](auto tt) {
+            constexpr int tb = decltype(tt)::value;
+            constexpr int sh = Y::thr_idx(P, tb);
+            e |= ((uint32_t)(j >> tb) & 1u) << sh;
+        });
+        return e + (uint32_t)rig * K;
+    };
+
+    // sum over the threads of a row, ascending thread bits (lanes by xor
+    // shuffle, warps through shared memory in warp order)
+    auto row_sum = [&](float x) -> float {
+        static_for<0, C::kLaneBits>([&](auto tt) {
+            constexpr int tb = decltype(tt)::value;
+            x = __fadd_rn(x, __shfl_xor_sync(0xffffffffu, x, 1 << tb));
+        });
+        if constexpr (C::kWarpBits > 0) {
+            constexpr int NW = 1 << C::kWarpBits;
+            if (lane == 0) red[wig] = x;
+            group_sync<T>(grp);
+            x = stream_tree<NW>([&](auto kk) { return red[decltype(kk)::value]; });
+            group_sync<T>(grp);
+        }
+        return x;
+    };
+    auto row_max = [&](float x) -> float {
+        static_for<0, C::kLaneBits>([&](auto tt) {
+            constexpr int tb = decltype(tt)::value;
+            x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 1 << tb));
+        });
+        if constexpr (C::kWarpBits > 0) {
+            constexpr int NW = 1 << C::kWarpBits;
+            if (lane == 0) red[wig] = x;
+            group_sync<T>(grp);
+            x = red[0];
+            static_for<1, NW>([&](auto kk) { x = fmaxf(x, red[decltype(kk)::value]); });
+            group_sync<T>(grp);
+        }
+        return x;
+    };
+    auto row_isum = [&](int x) -> int {
+        static_for<0, C::kLaneBits>([&](auto tt) {
+            constexpr int tb = decltype(tt)::value;
+            x += __shfl_xor_sync(0xffffffffu, x, 1 << tb);
+        });
+        if constexpr (C::kWarpBits > 0) {
+            constexpr int NW = 1 << C::kWarpBits;
+            int* ired = reinterpret_cast<int*>(red);
+            if (lane == 0) ired[wig] = x;
+            group_sync<T>(grp);
+            x = 0;
+            static_for<0, NW>([&](auto kk) { x += ired[decltype(kk)::value]; });
+            group_sync<T>(grp);
+        }
+        return x;
+    };
+
+    const int64_t stride_groups = (int64_t)gridDim.x * C::kGroupsPerCta;
+    for (int64_t rg = (int64_t)blockIdx.x * C::kGroupsPerCta + grp;; rg += stride_groups) {
+        const int64_t row0 = rg * C::kRowsPerGroup;
+        if (row0 >= p.M) break;
+        const int64_t row = row0 + rig;
+
+        // ---- stage the group's bf16 rows in shared memory (coalesced)
+        {
+            const uint16_t* src0 = p.X + row0 * K;
+            const uint32_t wsw = stage_swz<C::kStageShift>((uint32_t)w);
+            static_for<0, R / 8>([&](auto ii) {
+                constexpr int i = decltype(ii)::value;
+                const int g = i * W + w;
+                const bool ok = row0 + ((g * 8) >> L) < p.M;
+                const uint32_t phys = stage_swz<C::kStageShift>((uint32_t)(i * W)) ^ wsw;
+                cp_async16(buf_s + phys * 16u, ok ? (const void*)(src0 + g * 8) : (const void*)p.X,
+                           ok ? 16 : 0);
+            });
+            cp_async_commit();
+            if (w == 0) {
+                const int64_t nrow0 = row0 + stride_groups * C::kRowsPerGroup;
+                if (nrow0 < p.M) {
+                    int64_t nrows = p.M - nrow0;
+                    if (nrows > C::kRowsPerGroup) nrows = C::kRowsPerGroup;
+                    prefetch_l2_bulk(p.X + nrow0 * K, (uint32_t)(nrows * K * 2));
+                }
+            }
+            cp_async_wait_all();
+            group_sync<T>(grp);
+        }
+
+        float2 d[R / 2];
+        {
+            const uint32_t base = stage_swz<C::kStageShift>((uint32_t)w << C::kStageShift);
+            static_for<0, R / 8>([&](auto ii) {
+                constexpr int i = decltype(ii)::value;
+                uint4 q = lds128(buf_s + (base ^ (uint32_t)i) * 16u);
+                d[4 * i + 0] = bf16x2_to_f2(q.x);
+                d[4 * i + 1] = bf16x2_to_f2(q.y);
+                d[4 * i + 2] = bf16x2_to_f2(q.z);
+                d[4 * i + 3] = bf16x2_to_f2(q.w);
+            });
+        }
+        group_sync<T>(grp);  // staging buffer free again
+
+        // ---- RMSNorm: tree(x*x) over the row, ascending index order
+        float ss = stream_tree<R / 2>([&](auto kk) {
+            constexpr int k = decltype(kk)::value;
+            float2 q = mul2(d[k], d[k]);
+            return __fadd_rn(q.x, q.y);
+        });
+        ss = row_sum(ss);
+        const float ms = __fmul_rn(ss, 1.0f / (float)K);
+        const float rn = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, p.norm_eps)));
+        {
+            const float2 r2 = make_float2(rn, rn);
+            static_for<0, R / 2>([&](auto kk) {
+                constexpr int k = decltype(kk)::value;
+                d[k] = mul2(d[k], r2);
+            });
+            if constexpr (GAIN) {
+                const float* g = p.gain + (thr_off(ic<0>{}) - (uint32_t)rig * K);
+                static_for<0, R / 4>([&](auto cc) {
+                    constexpr int c = decltype(cc)::value;
+                    float4 gv = *reinterpret_cast<const float4*>(g + 4 * c);
+                    d[2 * c] = mul2(d[2 * c], make_float2(gv.x, gv.y));
+                    d[2 * c + 1] = mul2(d[2 * c + 1], make_float2(gv.z, gv.w));
+                });
+            }
+        }
+
+        // ---- Walsh-Hadamard butterflies: natural layout, stages 0..r-1
+        static_for<0, C::r>([&](auto rr) { stage_regs<R, decltype(rr)::value>(d); });
+
+        // ---- exchanges through shared memory, one per pass
+        static_for<1, P_LAST + 1>([&](auto pp) {
+            constexpr int P = decltype(pp)::value;
+            {  // write in layout P-1
+                const uint32_t tb = swz(thr_off(ic<P - 1>{}) >> 2);
+                static_for<0, R / 4>([&](auto cc) {
+                    constexpr int c = decltype(cc)::value;
+                    constexpr uint32_t rc = swz((uint32_t)Y::reg_off(P - 1, 4 * c) >> 2);
+                    uint4 v;
+                    v.x = __float_as_uint(d[2 * c].x);
+                    v.y = __float_as_uint(d[2 * c].y);
+                    v.z = __float_as_uint(d[2 * c + 1].x);
+                    v.w = __float_as_uint(d[2 * c + 1].y);
+                    sts128(buf_s + ((tb ^ rc) << 4), v);
+                });
+            }
+            group_sync<T>(grp);
+            {  // read in layout P
+                const uint32_t tb = swz(thr_off(ic<P>{}) >> 2);
+                static_for<0, R / 4>([&](auto cc) {
+                    constexpr int c = decltype(cc)::value;
+                    constexpr uint32_t rc = swz((uint32_t)Y::reg_off(P, 4 * c) >> 2);
+                    uint4 v = lds128(buf_s + ((tb ^ rc) << 4));
+                    d[2 * c] = make_float2(__uint_as_float(v.x), __uint_as_float(v.y));
+                    d[2 * c + 1] = make_float2(__uint_as_float(v.z), __uint_as_float(v.w));
+                });
+            }
+            group_sync<T>(grp);
+            constexpr int b = kRegLog + 5 * (P - 1);
+            constexpr int n = (L - b) < 5 ? (L - b) : 5;
+            static_for<0, n>([&](auto ss_) {
+                constexpr int s = b + decltype(ss_)::value;
+                stage_regs<R, Y::reg_bit_of(P, s)>(d);
+            });
+        });
+
+        // ---- normalise by 1/sqrt(K)
+        {
+            const float2 c2 = make_float2(p.cK, p.cK);
+            static_for<0, R / 2>([&](auto kk) {
+                constexpr int k = decltype(kk)::value;
+                d[k] = mul2(d[k], c2);
+            });
+        }
+
+        const uint32_t toff = thr_off(ic<P_LAST>{});  // includes rig * K
+        constexpr int RUN = Y::run_bits(P_LAST);       // contiguous run length 2^RUN
+
+        if constexpr (MODE == 0) {
+            if (row < p.M) {
+                float* vrow = p.V + row0 * K;
+                static_for<0, R / 4>([&](auto cc) {
+                    constexpr int c = decltype(cc)::value;
+                    constexpr uint32_t e = (uint32_t)Y::reg_off(P_LAST, 4 * c);
+                    *reinterpret_cast<float4*>(vrow + (toff | e)) =
+                        make_float4(d[2 * c].x, d[2 * c].y, d[2 * c + 1].x, d[2 * c + 1].y);
+                });
+            }
+        } else {
+            // ---- per-token statistic
+            float stat;
+            if constexpr (MODE == 8) {
+                float m = 0.f;
+                static_for<0, R / 2>([&](auto kk) {
+                    constexpr int k = decltype(kk)::value;
+                    m = fmaxf(m, fmaxf(fabsf(d[k].x), fabsf(d[k].y)));
+                });
+                stat = row_max(m);
+            } else {
+                // tree_sum(|v|): runs in registers, then lanes: the first NSC
+                // lane levels scatter the remaining register partials (each
+                // lane keeps the half its lane bit selects), the rest add.
+                constexpr int NRUN = R >> RUN;  // partials per thread after the runs
+                constexpr int NSC = ilog2(NRUN);
+                static_assert(NSC <= C::kLaneBits, "partials exceed lane bits");
+                const float total_thread = [&] {
+                    float stk[NSC + 1] = {};
+                    float fin = 0.f;
+                    static_for<0, NRUN>([&](auto mm) {
+                        constexpr int m = decltype(mm)::value;
+                        constexpr int RL = 1 << RUN;  // elements per run
+                        float x = stream_tree<RL / 2>([&](auto kk) {
+                            constexpr int k = (m * RL) / 2 + decltype(kk)::value;
+                            return __fadd_rn(fabsf(d[k].x), fabsf(d[k].y));
+                        });
+                        constexpr int ones = [] {
+                            int c = 0;
+                            while (c < NSC && ((m >> c) & 1)) ++c;
+                            return c;
+                        }();
+                        static_for<0, ones>([&](auto ll) {
+                            constexpr int l = decltype(ll)::value;
+                            const bool hi = (j >> l) & 1;
+                            const float a = stk[l];  // partial bit = 0
+                            const float keep = hi ? x : a;
+                            const float send = hi ? a : x;
+                            x = __fadd_rn(keep, __shfl_xor_sync(0xffffffffu, send, 1 << l));
+                        });
+                        if constexpr (m == NRUN - 1)
+                            fin = x;
+                        else
+                            stk[ones] = x;
+                    });
+                    return fin;
+                }();
+                float x = total_thread;
+                static_for<NSC, C::kLaneBits>([&](auto tt) {
+                    constexpr int tb = decltype(tt)::value;
+                    x = __fadd_rn(x, __shfl_xor_sync(0xffffffffu, x, 1 << tb));
+                });
+                if constexpr (C::kWarpBits == 0) {
+                    static_for<0, NSC>([&](auto ll) {
+                        constexpr int l = decltype(ll)::value;
+                        x = __fadd_rn(x, __shfl_xor_sync(0xffffffffu, x, 1 << l));
+                    });
+                } else {
+                    constexpr int WB = C::kWarpBits;
+                    constexpr int NV = 1 << (WB + NSC);
+                    static_assert(NV <= kRedFloats, "reduction scratch too small");
+                    if ((lane >> NSC) == 0) red[wig | (lane << WB)] = x;
+                    group_sync<T>(grp);
+                    x = stream_tree<NV>([&](auto kk) { return red[decltype(kk)::value]; });
+                    group_sync<T>(grp);
+                }
+                stat = __fmul_rn(x, 1.0f / (float)K);
+            }
+
+            const float cq = (MODE == 8) ? 127.0f : p.s7;
+            const float inv = __fdiv_rn(cq, __fadd_rn(stat, p.quant_eps));
+            const float lo = (MODE == 8) ? -128.0f : -8.0f;
+            const float hi = (MODE == 8) ? 127.0f : 7.0f;
+            const float2 inv2 = make_float2(inv, inv);
+            const float2 magic2 = make_float2(12582912.0f, 12582912.0f);  // 1.5 * 2^23
+
+            // codes: round-half-even via the 1.5*2^23 addition; the code is the
+            // low bits of the sum's bit pattern.  Packed word by word, run by run.
+            constexpr int RL = 1 << RUN;                       // elements per run
+            constexpr int BYTES = (MODE == 8) ? RL : RL / 2;   // code bytes per run
+            constexpr int EPW = (MODE == 8) ? 4 : (RL >= 8 ? 8 : 4);  // elements per word
+            constexpr int NWORD = RL / EPW;
+            const bool row_ok = row < p.M;
+            uint8_t* crow = p.codes + row0 * (int64_t)((K * MODE) / 8);
+            uint32_t qsum = 0;
+            static_for<0, R / RL>([&](auto mm) {
+                constexpr int m = decltype(mm)::value;
+                uint32_t wv[NWORD];
+                static_for<0, NWORD>([&](auto ww) {
+                    constexpr int wi = decltype(ww)::value;
+                    uint32_t qv[EPW];
+                    static_for<0, EPW / 2>([&](auto kk) {
+                        constexpr int k = (m * RL + wi * EPW) / 2 + decltype(kk)::value;
+                        float2 y = mul2(d[k], inv2);
+                        y.x = fminf(fmaxf(y.x, lo), hi);
+                        y.y = fminf(fmaxf(y.y, lo), hi);
+                        y = add2(y, magic2);
+                        qv[2 * decltype(kk)::value] = __float_as_uint(y.x);
+                        qv[2 * decltype(kk)::value + 1] = __float_as_uint(y.y);
+                    });
+                    static_for<0, EPW>([&](auto ee) { qsum += qv[decltype(ee)::value]; });
+                    if constexpr (MODE == 8) {
+                        const uint32_t lo2 = __byte_perm(qv[0], qv[1], 0x0040);
+                        const uint32_t hi2 = __byte_perm(qv[2], qv[3], 0x0040);
+                        wv[wi] = __byte_perm(lo2, hi2, 0x5410);
+                    } else {
+                        uint32_t acc = 0;
+                        static_for<0, EPW>([&](auto ee) {
+                            constexpr int e = decltype(ee)::value;
+                            acc |= (qv[e] & 0xFu) << (4 * e);
+                        });
+                        wv[wi] = acc;
+                    }
+                });
+                if (row_ok) {
+                    constexpr uint32_t e0 = (uint32_t)Y::reg_off(P_LAST, m * RL);
+                    uint8_t* dst = crow + (((toff | e0) * MODE) >> 3);
+                    if constexpr (BYTES == 2) {
+                        *reinterpret_cast<uint16_t*>(dst) = (uint16_t)wv[0];
+                    } else if constexpr (BYTES == 4) {
+                        *reinterpret_cast<uint32_t*>(dst) = wv[0];
+                    } else if constexpr (BYTES == 8) {
+                        *reinterpret_cast<uint2*>(dst) = make_uint2(wv[0], wv[1]);
+                    } else {
+                        static_for<0, BYTES / 16>([&](auto vv) {
+                            constexpr int v = decltype(vv)::value;
+                            *reinterpret_cast<uint4*>(dst + 16 * v) =
+                                make_uint4(wv[4 * v], wv[4 * v + 1], wv[4 * v + 2], wv[4 * v + 3]);
+                        });
+                    }
+                }
+            });
+            // sum of codes: each term is 0x4B400000 + q (mod 2^32)
+            int qs = (int)(qsum - (uint32_t)R * 0x4B400000u);
+            qs = row_isum(qs);
+
+            if (row_ok) {
+                if (j == 0) {
+                    p.scales[row] = __fdiv_rn(stat, cq);
+                    if (p.rowsum != nullptr) p.rowsum[row] = qs;
+                }
+            }
+        }
+    }
+}
+
+template <int L, int MODE, bool GAIN>
+static hbl_status launch_one(const Params& prm, cudaStream_t stream, int num_sms) {
+    using C = Cfg<L>;
+    auto kern = norm_fwht_quant_kernel<L, MODE, GAIN>;
+    if (!smem_attr_once(reinterpret_cast<const void*>(kern), C::kSmemBytes)) return HBL_ERR_CUDA;
+    const int64_t groups = (prm.M + C::kRowsPerGroup - 1) / C::kRowsPerGroup;
+    const int64_t ctas_needed = (groups + C::kGroupsPerCta - 1) / C::kGroupsPerCta;
+    int64_t grid = (int64_t)num_sms * C::kMinBlocks;
+    if (ctas_needed < grid) grid = ctas_needed;
+    if (grid < 1) grid = 1;
+    kern<<<(unsigned)grid, C::kCtaThreads, C::kSmemBytes, stream>>>(prm);
+    return cudaGetLastError() == cudaSuccess ? HBL_OK : HBL_ERR_CUDA;
+}
+
+template <int MODE, bool GAIN>
+hbl_status dispatch(int L, const Params& prm, cudaStream_t s, int sms) {
+    switch (L) {
+        case 4: return launch_one<4, MODE, GAIN>(prm, s, sms);
+        case 5: return launch_one<5, MODE, GAIN>(prm, s, sms);
+        case 6: return launch_one<6, MODE, GAIN>(prm, s, sms);
+        case 7: return launch_one<7, MODE, GAIN>(prm, s, sms);
+        case 8: return launch_one<8, MODE, GAIN>(prm, s, sms);
+        case 9: return launch_one<9, MODE, GAIN>(prm, s, sms);
+        case 10: return launch_one<10, MODE, GAIN>(prm, s, sms);
+        case 11: return launch_one<11, MODE, GAIN>(prm, s, sms);
+        case 12: return launch_one<12, MODE, GAIN>(prm, s, sms);
+        case 13: return launch_one<13, MODE, GAIN>(prm, s, sms);
+        case 14: return launch_one<14, MODE, GAIN>(prm, s, sms);
+        case 15: return launch_one<15, MODE, GAIN>(prm, s, sms);
+        default: return HBL_ERR_SHAPE;
+    }
+}
+
+}  // namespace k1
+}  // namespace hbl

@@ -1,0 +1,175 @@
+/*
+ * hbl.h -- C ABI of the B200 (sm_100a) H-BitLinear library (libhbl.so).
+ *
+ * H-BitLinear is the linear layer of BitNet v2 that replaces the attention
+ * output projection (Wo) and the FFN down projection (W_down).  Per token row
+ * x it computes
+ *
+ *     y = (alpha * s_x) * ( Quant_act( H_K/sqrt(K) . RMSNorm(x) ) . W_t^T )
+ *
+ * Sources: the BitNet v2 write-up on 0755model.com, sections
+ * "BitNet v2：原生4位激活" (RMS normalisation, no bias; H-BitLinear at Wo and
+ * W_down) and "H-BitLinear" (per-tensor absmean ternary weights; online
+ * Hadamard transform before activation quantisation, computed with the fast
+ * Hadamard transform in O(n log n); INT8 / INT4 activation quantisers; the
+ * layer's overall expression LN -> Hadamard -> quantise -> matmul); the
+ * shengxinai.com explainer, section 2.2 (4-bit activations take 16 values);
+ * the "[论文品鉴] 1-bit LLM" post, section "掩码存储" (ternary weights packed
+ * several to an integer).  The pages show their formulas as images only; the
+ * formulas used are written out at each call below.
+ *
+ * Conventions for every call:
+ *   - Pointers are device pointers owned by the caller, unless a call says
+ *     "host".  The library allocates no memory; scratch space comes from the
+ *     caller's workspace `ws` of at least hbl_workspace_size() bytes.
+ *   - Every device pointer must be 16-byte aligned (HBL_ERR_ALIGNMENT).
+ *   - bf16 tensors are passed as uint16_t bit patterns.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls are
+ *     asynchronous: HBL_OK means the arguments were valid and the kernels were
+ *     launched.  Errors are returned before any launch; nothing is written then.
+ *   - `dev_status` (nullable) is a device int32 the kernels set to a non-zero
+ *     hbl_status if a bounded device-side wait gives up (HBL_ERR_TIMEOUT); the
+ *     caller reads it after synchronising.  Kernels never trap.
+ *   - Shapes: K is a power of two with 16 <= K <= 32768 (the fast transform
+ *     needs a power of two); M >= 0 (M == 0 launches nothing); N >= 16 and
+ *     N % 16 == 0.  Violations return HBL_ERR_SHAPE.
+ *   - act_bits is 4 or 8.  Codes layout: act_bits 8 -> int8 [M x K] row-major;
+ *     act_bits 4 -> two's-complement nibbles [M x K/2], element 2j in the low
+ *     nibble of byte j.
+ *   - Packed ternary weights: uint32 [N x K/16] row-major; word (n, k/16) holds
+ *     16 weights; local weight j = k % 16 sits at bits [8*(j%4) + 2*(j/4), +2)
+ *     as the code t + 1 (0 -> -1, 1 -> 0, 2 -> +1; 3 is never written).
+ *   - Only sm_100 devices are supported (HBL_ERR_UNSUPPORTED_ARCH otherwise).
+ *   - Non-finite inputs give unspecified (but memory-safe) results.
+ */
+#ifndef HBL_H
+#define HBL_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__) || defined(__clang__)
+#define HBL_API __attribute__((visibility("default")))
+#else
+#define HBL_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    HBL_OK = 0,
+    HBL_ERR_INVALID_ARG = 1,      /* null pointer, bad act_bits, negative/non-finite eps, bad op */
+    HBL_ERR_SHAPE = 2,            /* K not a power of two in [16, 32768], N % 16, M < 0 */
+    HBL_ERR_ALIGNMENT = 3,        /* a pointer is not 16-byte aligned */
+    HBL_ERR_UNSUPPORTED_ARCH = 4, /* current device is not sm_100 */
+    HBL_ERR_WORKSPACE = 5,        /* ws is NULL or smaller than hbl_workspace_size() */
+    HBL_ERR_CUDA = 6,             /* a CUDA runtime call failed (launch, copy, query) */
+    HBL_ERR_TIMEOUT = 7           /* a bounded device-side wait gave up (dev_status only) */
+} hbl_status;
+
+/* Static string for a status code ("unknown status" for other values). */
+HBL_API const char* hbl_status_string(int status);
+
+/* Library ABI version (major * 10000 + minor * 100 + patch). */
+HBL_API int hbl_version(void);
+
+/* Choice of ternary-GEMM back end (test and tuning aid; process-wide, not
+ * synchronised with calls in flight on other threads):
+ *   0 = automatic (CUDA-core split-K GEMV for M <= 8 tokens, tcgen05 tensor
+ *       cores otherwise), 1 = always tensor cores, 2 = always the GEMV path
+ *       (large M runs in chunks of 8 tokens).
+ * hbl_workspace_size() answers for the path in force.  Returns HBL_OK or
+ * HBL_ERR_INVALID_ARG.  This call has no counterpart on the BitNet v2 pages. */
+HBL_API int hbl_set_gemm_path(int path);
+
+/* Operation identifiers for hbl_workspace_size(). */
+enum {
+    HBL_OP_PACK_TERNARY = 0,
+    HBL_OP_TERNARY_GEMM = 1,
+    HBL_OP_HBITLINEAR_FORWARD = 2,
+    HBL_OP_HBITLINEAR_FORWARD_HOSTIO = 3
+};
+
+/* Bytes of device workspace that `op` needs for the given shape (0 is a valid
+ * answer).  Unused shape arguments may be 0.  Writes *bytes; HBL_ERR_SHAPE or
+ * HBL_ERR_INVALID_ARG on bad input. */
+HBL_API hbl_status hbl_workspace_size(int op, int M, int K, int N, int act_bits, size_t* bytes);
+
+/* Ternary weight quantisation and packing (offline, once per weight).
+ * Formula (per-tensor absmean; the page's formula is an image):
+ *   alpha = S / (float)(N*K),  S = fp32 left-complete pairwise tree sum of |W|
+ *           over the row-major flat index (row sums, then a tree over rows);
+ *   t     = clip(round_half_even(W / (alpha + eps)), -1, 1)   (IEEE division);
+ * W:        fp32 [N x K] row-major, device.
+ * W_packed: uint32 [N x K/16] out, layout above.   alpha: device float, out.
+ * ws:       >= hbl_workspace_size(HBL_OP_PACK_TERNARY, 0, K, N, 0) bytes.
+ * K follows the layer's rule (a power of two in [16, 32768]); N >= 1. */
+HBL_API hbl_status hbl_pack_ternary(const float* W, int N, int K, float eps, uint32_t* W_packed,
+                            float* alpha, void* ws, size_t ws_bytes, void* stream);
+
+/* RMSNorm followed by the normalised online Hadamard transform, fp32 out:
+ *   r = 1 / sqrt(tree_sum(x*x) * (1/K) + norm_eps),   u = (x * r) * gain
+ *   V = (u . H_K) * c_K,   c_K = fp32(1/sqrt(K)),
+ * H_K the Sylvester Hadamard matrix in natural order, evaluated as butterfly
+ * stages h = 1, 2, ..., K/2 in that order, (a, b) -> (a + b, a - b).
+ * X: bf16 [M x K]; gain: fp32 [K] or NULL (all ones); V: fp32 [M x K] out.
+ * This exposes the first two steps of the layer on their own. */
+HBL_API hbl_status hbl_norm_fwht(const uint16_t* X, const float* gain, int M, int K, float norm_eps,
+                         float* V, int32_t* dev_status, void* stream);
+
+/* Fused RMSNorm + online Hadamard transform + per-token activation quantisation
+ * (one kernel; V above is never written to memory).
+ *   act_bits 8 (absmax):  gamma = max|v|;  q = clip(rhe(v * (127/(gamma+eps))), -128, 127);
+ *                         scale = gamma / 127
+ *   act_bits 4 (absmean): beta = tree_sum(|v|) * (1/K);
+ *                         q = clip(rhe(v * (sqrt7/(beta+eps))), -8, 7);  scale = beta / sqrt7
+ * rhe = round half to even; 127/(gamma+eps) and sqrt7/(beta+eps) are one IEEE
+ * division per row; sqrt7 = fp32(sqrt(7)).
+ * codes: out, layout above.  scales: fp32 [M] out.  rowsum: int32 [M] out = sum
+ * of the row's codes, or NULL. */
+HBL_API hbl_status hbl_norm_fwht_quant(const uint16_t* X, const float* gain, int M, int K,
+                               float norm_eps, float quant_eps, int act_bits, void* codes,
+                               float* scales, int32_t* rowsum, int32_t* dev_status,
+                               void* stream);
+
+/* Ternary x integer matmul with int32 accumulation and bf16 dequantisation:
+ *   acc[m][n] = sum_k q[m][k] * t[n][k]            (exact)
+ *   Y[m][n]   = bf16_rne( (float)acc * (alpha * scales[m]) )
+ * codes/scales/rowsum as written by hbl_norm_fwht_quant (rowsum is REQUIRED:
+ * the kernels multiply by the stored code t+1 and subtract rowsum[m]).
+ * W_packed/alpha as written by hbl_pack_ternary.  Y: bf16 [M x N] out.
+ * acc_out: int32 [M x N] out, or NULL (debug/parity aid).
+ * ws: >= hbl_workspace_size(HBL_OP_TERNARY_GEMM, M, K, N, act_bits) bytes
+ * (may be NULL when that size is 0). */
+HBL_API hbl_status hbl_ternary_gemm(const void* codes, const float* scales, const int32_t* rowsum,
+                            int act_bits, int M, int K, const uint32_t* W_packed,
+                            const float* alpha, int N, uint16_t* Y, int32_t* acc_out,
+                            void* ws, size_t ws_bytes, int32_t* dev_status, void* stream);
+
+/* The whole layer: hbl_norm_fwht_quant into workspace, then hbl_ternary_gemm.
+ * X: bf16 [M x K]; Y: bf16 [M x N] out; other arguments as above.
+ * ws: >= hbl_workspace_size(HBL_OP_HBITLINEAR_FORWARD, M, K, N, act_bits). */
+HBL_API hbl_status hbl_hbitlinear_forward(const uint16_t* X, const float* gain, int M, int K, int N,
+                                  const uint32_t* W_packed, const float* alpha, int act_bits,
+                                  float norm_eps, float quant_eps, uint16_t* Y, void* ws,
+                                  size_t ws_bytes, int32_t* dev_status, void* stream);
+
+/* The whole layer with HOST activations in and HOST outputs out: copies X_host
+ * to the device, runs hbl_hbitlinear_forward, copies Y back to Y_host, all on
+ * `stream` (asynchronous; pinned host memory makes the copies asynchronous).
+ * X_host: bf16 [M x K] host; Y_host: bf16 [M x N] host, out.
+ * ws: >= hbl_workspace_size(HBL_OP_HBITLINEAR_FORWARD_HOSTIO, M, K, N, act_bits)
+ * bytes of device memory (it holds the device copies of X and Y as well). */
+HBL_API hbl_status hbl_hbitlinear_forward_hostio(const uint16_t* X_host, const float* gain, int M,
+                                         int K, int N, const uint32_t* W_packed,
+                                         const float* alpha, int act_bits, float norm_eps,
+                                         float quant_eps, uint16_t* Y_host, void* ws,
+                                         size_t ws_bytes, int32_t* dev_status, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HBL_H */

@@ -1,0 +1,120 @@
+"""The C ABI: the library loads, exports every call include/hbl.h declares, and
+rejects bad arguments on the host before touching the GPU.  CPU only: every
+call here fails validation before any CUDA call, so no device is needed."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import hadamard_rotated_int4_b200 as hbl
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "hbl.h")
+
+# fake but 16-byte-aligned device addresses: validation never dereferences them
+A = ctypes.c_void_p(0x10000)
+B = ctypes.c_void_p(0x20000)
+C = ctypes.c_void_p(0x30000)
+D = ctypes.c_void_p(0x40000)
+E = ctypes.c_void_p(0x50000)
+MIS = ctypes.c_void_p(0x10004)  # misaligned
+NUL = None
+
+
+def declared():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"HBL_API\s+[\w\s\*]*?\b(hbl_\w+)\s*\(", src)))
+
+
+def test_header_declares_the_expected_calls():
+    names = declared()
+    for n in ("hbl_pack_ternary", "hbl_norm_fwht_quant", "hbl_ternary_gemm",
+              "hbl_hbitlinear_forward", "hbl_workspace_size", "hbl_status_string"):
+        assert n in names
+    assert set(names) == set(hbl.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol():
+    lib = hbl.lib()
+    for n in declared():
+        assert hasattr(lib, n), n
+    out = os.popen("nm -D --defined-only %s" % hbl.LIB_PATH).read()
+    exported = set(re.findall(r"\bT (hbl_\w+)", out))
+    assert set(declared()) <= exported
+
+
+def test_status_strings_and_version():
+    lib = hbl.lib()
+    for code in range(8):
+        assert lib.hbl_status_string(code).decode() not in ("", "unknown status")
+    assert lib.hbl_status_string(99).decode() == "unknown status"
+    assert lib.hbl_version() >= 100
+
+
+def test_workspace_sizes():
+    # pack: one float per weight row (rounded to 256 B)
+    assert hbl.workspace_size(hbl.OP_PACK_TERNARY, 0, 4096, 100, 0) == 512
+    # forward: codes + scales + rowsum, each 256-aligned (tensor-core path: no GEMM scratch)
+    hbl.set_gemm_path(1)
+    try:
+        M, K, N = 8192, 16384, 4096
+        got = hbl.workspace_size(hbl.OP_HBITLINEAR_FORWARD, M, K, N, 4)
+        assert got == M * K // 2 + 2 * M * 4
+        got8 = hbl.workspace_size(hbl.OP_HBITLINEAR_FORWARD, M, K, N, 8)
+        assert got8 == M * K + 2 * M * 4
+        hio = hbl.workspace_size(hbl.OP_HBITLINEAR_FORWARD_HOSTIO, M, K, N, 4)
+        assert hio == got + M * K * 2 + M * N * 2
+        assert hbl.workspace_size(hbl.OP_TERNARY_GEMM, M, K, N, 4) == 0
+    finally:
+        hbl.set_gemm_path(0)
+    # small M uses the split-K GEMV, which needs integer partials
+    assert hbl.workspace_size(hbl.OP_TERNARY_GEMM, 1, 16384, 4096, 4) > 0
+
+
+@pytest.mark.parametrize("K", [0, 8, 24, 100, 65536])
+def test_bad_K_is_a_shape_error(K):
+    lib = hbl.lib()
+    s = lib.hbl_norm_fwht_quant(A, NUL, 4, K, 1e-6, 1e-5, 4, B, C, D, NUL, NUL)
+    assert s == 2
+    sz = ctypes.c_size_t()
+    assert lib.hbl_workspace_size(hbl.OP_HBITLINEAR_FORWARD, 4, K, 64, 4, ctypes.byref(sz)) == 2
+
+
+def test_validation_errors():
+    lib = hbl.lib()
+    # null pointer, bad act_bits, bad eps
+    assert lib.hbl_norm_fwht_quant(NUL, NUL, 4, 256, 1e-6, 1e-5, 4, B, C, D, NUL, NUL) == 1
+    assert lib.hbl_norm_fwht_quant(A, NUL, 4, 256, 1e-6, 1e-5, 3, B, C, D, NUL, NUL) == 1
+    assert lib.hbl_norm_fwht_quant(A, NUL, 4, 256, -1.0, 1e-5, 4, B, C, D, NUL, NUL) == 1
+    assert lib.hbl_norm_fwht_quant(A, NUL, 4, 256, float("nan"), 1e-5, 4, B, C, D, NUL, NUL) == 1
+    # negative M
+    assert lib.hbl_norm_fwht_quant(A, NUL, -1, 256, 1e-6, 1e-5, 4, B, C, D, NUL, NUL) == 2
+    # misaligned pointers
+    assert lib.hbl_norm_fwht_quant(MIS, NUL, 4, 256, 1e-6, 1e-5, 4, B, C, D, NUL, NUL) == 3
+    assert lib.hbl_norm_fwht_quant(A, MIS, 4, 256, 1e-6, 1e-5, 4, B, C, D, NUL, NUL) == 3
+    assert lib.hbl_norm_fwht(A, NUL, 4, 256, 1e-6, MIS, NUL, NUL) == 3
+    # M == 0 is a no-op that succeeds without a device
+    assert lib.hbl_norm_fwht_quant(A, NUL, 0, 256, 1e-6, 1e-5, 4, B, C, D, NUL, NUL) == 0
+    # GEMM: N not a multiple of 16, rowsum required, workspace required for small M
+    gemm = lib.hbl_ternary_gemm
+    assert gemm(A, B, C, 4, 64, 256, D, E, 40, A, NUL, NUL, 0, NUL, NUL) == 2
+    assert gemm(A, B, NUL, 4, 64, 256, D, E, 64, A, NUL, NUL, 0, NUL, NUL) == 1
+    assert gemm(A, B, C, 4, 1, 256, D, E, 64, A, NUL, NUL, 0, NUL, NUL) == 5
+    # forward: workspace too small
+    fwd = lib.hbl_hbitlinear_forward
+    assert fwd(A, NUL, 64, 256, 64, B, C, 4, 1e-6, 1e-5, D, E, 16, NUL, NUL) == 5
+    assert fwd(A, NUL, 64, 256, 64, B, C, 5, 1e-6, 1e-5, D, E, 1 << 20, NUL, NUL) == 1
+    # pack
+    pack = lib.hbl_pack_ternary
+    assert pack(A, 16, 100, 1e-5, B, C, D, 1024, NUL) == 2
+    assert pack(A, 16, 256, 1e-5, B, C, NUL, 0, NUL) == 5
+    assert pack(A, 0, 256, 1e-5, B, C, D, 1024, NUL) == 2
+    assert lib.hbl_set_gemm_path(7) == 1
+
+
+def test_binding_rejects_non_cuda_tensors():
+    import torch
+
+    with pytest.raises(TypeError):
+        hbl.norm_fwht_quant(torch.zeros(4, 256, dtype=torch.bfloat16), 4)

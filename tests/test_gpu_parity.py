@@ -1,0 +1,292 @@
+"""GPU parity: the CUDA path through the C ABI against the CPU oracle on the
+same seeded inputs.  Integer outputs (codes, rowsum, packed weights, int32
+accumulators) and the fp32 per-token scales and alpha must be bit-identical;
+fp32 transform values are bit-identical to the oracle's fp32 evaluation and
+within 1e-6 (relative to the row's largest |v|) of the fp64 evaluation; bf16
+outputs must be within 1 bf16 ulp (they are expected bit-identical, since both
+sides evaluate the same IEEE operations in the same order).
+"""
+import numpy as np
+import pytest
+import torch
+
+import hadamard_rotated_int4_b200 as hbl
+import oracle
+from hadamard_rotated_int4_b200 import inputs
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+
+
+def to_dev_bf16(bits):
+    return torch.from_numpy(bits.view(np.int16).copy()).view(torch.bfloat16).to(DEV)
+
+
+def bf16_bits(t):
+    return t.view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def bf16_ulp_diff(a_bits, b_bits):
+    a = a_bits.astype(np.int32)
+    b = b_bits.astype(np.int32)
+    # order-preserving map of bf16 bit patterns to integers
+    a = np.where(a & 0x8000, 0x8000 - a, a)
+    b = np.where(b & 0x8000, 0x8000 - b, b)
+    return np.abs(a - b)
+
+
+def acts(M, K, seed=0, kind="gauss"):
+    if kind == "gauss":
+        return inputs.gaussian_acts(M, K, seed=seed, frac=0.01, mult=30.0)
+    if kind == "t":
+        return inputs.student_t_acts(M, K, seed=seed)
+    if kind == "swiglu":
+        return inputs.swiglu_acts(M, K, seed=seed)
+    raise KeyError(kind)
+
+
+# ------------------------------------------------------------ norm + FWHT
+
+@pytest.mark.parametrize("K", [16, 32, 64, 128, 256, 512, 1024, 2048, 4096, 8192, 16384, 32768])
+@pytest.mark.parametrize("M", [1, 37])
+def test_norm_fwht_values(K, M):
+    X = acts(M, K, seed=K + M)
+    V = hbl.norm_fwht(to_dev_bf16(X)).cpu().numpy()
+    want32 = oracle.norm_fwht(X)
+    assert np.array_equal(V.view(np.uint32), want32.view(np.uint32))
+    want64 = oracle.norm_fwht_f64(X)
+    rel = np.abs(V - want64).max(axis=1) / np.abs(want64).max(axis=1)
+    assert rel.max() < 1e-6
+
+
+@pytest.mark.parametrize("K", [256, 4096])
+def test_norm_fwht_with_gain(K):
+    X = acts(5, K, seed=3)
+    g = np.random.default_rng(1).uniform(0.5, 1.5, K).astype(np.float32)
+    V = hbl.norm_fwht(to_dev_bf16(X), gain=torch.from_numpy(g).to(DEV)).cpu().numpy()
+    assert np.array_equal(V.view(np.uint32), oracle.norm_fwht(X, gain=g).view(np.uint32))
+
+
+# ------------------------------------------------- fused norm+FWHT+quant
+
+def check_quant(X, bits, gain=None):
+    g_dev = None if gain is None else torch.from_numpy(gain).to(DEV)
+    codes, scales, rowsum = hbl.norm_fwht_quant(to_dev_bf16(X), bits, gain=g_dev)
+    torch.cuda.synchronize()
+    wc, ws, wr = oracle.norm_fwht_quant(X, bits, gain=gain)
+    c = codes.cpu().numpy()
+    if not np.array_equal(c, wc):
+        bad = np.argwhere(c != wc)
+        raise AssertionError("codes differ at %d bytes, first %s" % (len(bad), bad[:5].tolist()))
+    assert np.array_equal(scales.cpu().numpy().view(np.uint32), ws.view(np.uint32))
+    assert np.array_equal(rowsum.cpu().numpy(), wr)
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("K", [16, 32, 64, 128, 256, 512, 1024, 2048, 4096, 8192, 16384, 32768])
+def test_quant_all_K(bits, K):
+    M = 45  # ragged against every rows-per-group size
+    check_quant(acts(M, K, seed=K, kind="t"), bits)
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("K", [256, 2048, 16384])
+def test_quant_with_gain(bits, K):
+    g = np.random.default_rng(K).uniform(0.25, 2.0, K).astype(np.float32)
+    check_quant(acts(9, K, seed=5), bits, gain=g)
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+def test_quant_edge_rows(bits):
+    K = 4096
+    X = acts(6, K, seed=2)
+    X[0] = 0                                      # zero row
+    X[1] = np.uint16(0x3F80)                      # constant 1.0
+    X[2, :] = 0
+    X[2, 17] = np.uint16(0x4120)                  # single spike (10.0)
+    X[3] = np.uint16(0x0001)                      # smallest bf16 subnormal
+    X[4, ::2] = np.uint16(0x7F00)                 # large values (~1.7e38)
+    check_quant(X, bits)
+
+
+def test_quant_workloads_full_size():
+    # quant workload (8192 x 4096, Student-t, 1% channels x 20), both widths
+    X = inputs.activations("quant")
+    for bits in (4, 8):
+        check_quant(X, bits)
+
+
+def test_quant_empty_M():
+    codes, scales, rowsum = hbl.norm_fwht_quant(
+        torch.zeros((0, 256), dtype=torch.bfloat16, device=DEV), 4)
+    assert codes.numel() == 0
+
+
+def test_quant_deterministic():
+    X = to_dev_bf16(acts(300, 4096, seed=9))
+    c0, s0, r0 = hbl.norm_fwht_quant(X, 4)
+    for _ in range(5):
+        c, s, r = hbl.norm_fwht_quant(X, 4)
+        assert torch.equal(c, c0) and torch.equal(s, s0) and torch.equal(r, r0)
+
+
+# ------------------------------------------------------------ ternary pack
+
+@pytest.mark.parametrize("N,K", [(16, 16), (48, 256), (128, 256), (100, 2048), (4096, 4096),
+                                 (4096, 16384)])
+def test_pack_ternary(N, K):
+    W = inputs.latent_weights(N, K, seed=N + K)
+    packed, alpha = hbl.pack_ternary(torch.from_numpy(W).to(DEV))
+    wp, wa = oracle.pack_ternary(W)
+    assert alpha.cpu().numpy()[0].view(np.uint32) == np.float32(wa).view(np.uint32)
+    assert np.array_equal(packed.cpu().numpy().view(np.uint32), wp)
+
+
+# ------------------------------------------------------------ GEMM
+
+def make_gemm_case(M, K, N, bits, seed=0):
+    X = acts(M, K, seed=seed, kind="swiglu")
+    codes, scales, rowsum = oracle.norm_fwht_quant(X, bits)
+    W = inputs.latent_weights(N, K, seed=seed)
+    packed, alpha = oracle.pack_ternary(W)
+    return codes, scales, rowsum, packed, alpha
+
+
+def run_gemm(codes, scales, rowsum, bits, K, packed, alpha, path):
+    hbl.set_gemm_path(path)
+    try:
+        Y, acc = hbl.ternary_gemm(
+            torch.from_numpy(codes).to(DEV), torch.from_numpy(scales).to(DEV),
+            torch.from_numpy(rowsum).to(DEV), bits, K,
+            torch.from_numpy(packed.view(np.int32)).to(DEV),
+            torch.from_numpy(np.array([alpha, 0, 0, 0], dtype=np.float32)).to(DEV),
+            want_acc=True)
+        torch.cuda.synchronize()
+    finally:
+        hbl.set_gemm_path(0)
+    return bf16_bits(Y), acc.cpu().numpy()
+
+
+@pytest.mark.parametrize("path", [1, 2])
+@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("M,K,N", [(1, 256, 128), (3, 16, 16), (8, 64, 48), (9, 128, 272),
+                                   (127, 256, 256), (128, 512, 256), (129, 2048, 512),
+                                   (300, 4096, 272)])
+def test_gemm_paths(path, bits, M, K, N):
+    if path == 2 and M > 129:
+        M = 40  # the CUDA-core path is exercised in 8-token chunks; keep it quick
+    codes, scales, rowsum, packed, alpha = make_gemm_case(M, K, N, bits, seed=M + N)
+    Y, acc = run_gemm(codes, scales, rowsum, bits, K, packed, alpha, path)
+    wY, wacc = oracle.ternary_gemm(codes, scales, bits, K, packed, alpha)
+    assert np.array_equal(acc, wacc)
+    assert bf16_ulp_diff(Y, wY).max() <= 1
+    assert np.array_equal(Y, wY)
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+def test_gemm_identity_weights(bits):
+    K = 256
+    codes, scales, rowsum, _, _ = make_gemm_case(130, K, 16, bits)
+    pI = oracle.pack_codes(np.eye(K, dtype=np.int8))
+    Y, acc = run_gemm(codes, scales, rowsum, bits, K, pI, np.float32(1.0), 1)
+    assert np.array_equal(acc, oracle.decode_codes(codes, K, bits).astype(np.int32))
+
+
+# ------------------------------------------------------------ whole layer
+
+def forward(X, packed, alpha, bits, path=0):
+    hbl.set_gemm_path(path)
+    try:
+        Y = hbl.hbitlinear_forward(
+            to_dev_bf16(X), torch.from_numpy(packed.view(np.int32)).to(DEV),
+            torch.from_numpy(np.array([alpha, 0, 0, 0], dtype=np.float32)).to(DEV), bits)
+        torch.cuda.synchronize()
+    finally:
+        hbl.set_gemm_path(0)
+    return bf16_bits(Y)
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+def test_forward_tiny_workload(bits):
+    X = inputs.activations("tiny")
+    packed, alpha = oracle.pack_ternary(inputs.weights("tiny"))
+    for path in (0, 1, 2):
+        Y = forward(X, packed, alpha, bits, path)
+        assert np.array_equal(Y, oracle.hbitlinear_forward(X, packed, alpha, bits))
+
+
+def test_forward_attn_wo_workload_sampled_rows():
+    X = inputs.activations("attn_wo")
+    W = inputs.weights("attn_wo")
+    Wd = torch.from_numpy(W).to(DEV)
+    p_dev, a_dev = hbl.pack_ternary(Wd)
+    packed, alpha = oracle.pack_ternary(W)
+    assert np.array_equal(p_dev.cpu().numpy().view(np.uint32), packed)
+    Y = forward(X, packed, alpha, 4)
+    rows = np.random.default_rng(0).choice(X.shape[0], 48, replace=False)
+    rows = np.concatenate([rows, [0, X.shape[0] - 1]])
+    want = oracle.hbitlinear_forward(X, packed, alpha, 4, rows=rows)
+    assert np.array_equal(Y[rows], want)
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("bits", [4, 8])
+def test_ffn_wdown_workload_full_quant_sampled_gemm(bits):
+    # 8192 x 16384 -> 4096: codes/scales/rowsum checked on every row, outputs on
+    # sampled rows (the launch configuration the benchmark times)
+    X = inputs.activations("ffn_wdown")
+    W = inputs.weights("ffn_wdown")
+    packed, alpha = oracle.pack_ternary(W)
+    Xd = to_dev_bf16(X)
+    codes, scales, rowsum = hbl.norm_fwht_quant(Xd, bits)
+    wc, ws, wr = oracle.norm_fwht_quant(X, bits)
+    assert np.array_equal(codes.cpu().numpy(), wc)
+    assert np.array_equal(scales.cpu().numpy().view(np.uint32), ws.view(np.uint32))
+    assert np.array_equal(rowsum.cpu().numpy(), wr)
+    Y = bf16_bits(hbl.hbitlinear_forward(
+        Xd, torch.from_numpy(packed.view(np.int32)).to(DEV),
+        torch.from_numpy(np.array([alpha, 0, 0, 0], dtype=np.float32)).to(DEV), bits))
+    rows = np.concatenate([np.random.default_rng(1).choice(8192, 14, replace=False), [0, 8191]])
+    wY, wacc = oracle.ternary_gemm(wc, ws, bits, 16384, packed, alpha, rows=rows)
+    assert np.array_equal(Y[rows], wY)
+
+
+@pytest.mark.parametrize("T", list(inputs.DECODE_TOKENS))
+@pytest.mark.parametrize("shape", ["wo", "wdown"])
+def test_decode_sweep(T, shape):
+    K = 4096 if shape == "wo" else 16384
+    N = 4096
+    X = inputs.activations("decode_" + shape, M=T, K=K, seed=T)
+    W = inputs.latent_weights(N, K, seed=7)
+    packed, alpha = oracle.pack_ternary(W)
+    Y = forward(X, packed, alpha, 4)
+    rows = np.arange(T) if T <= 8 else np.concatenate([np.arange(4), [T - 1]])
+    want = oracle.hbitlinear_forward(X, packed, alpha, 4, rows=rows)
+    assert np.array_equal(Y[rows], want)
+
+
+def test_hostio_matches_device_forward():
+    X = inputs.activations("tiny")
+    packed, alpha = oracle.pack_ternary(inputs.weights("tiny"))
+    M, K = X.shape
+    N = packed.shape[0]
+    ws = torch.empty(hbl.workspace_size(hbl.OP_HBITLINEAR_FORWARD_HOSTIO, M, K, N, 4),
+                     dtype=torch.uint8, device=DEV)
+    Xh = torch.from_numpy(X.view(np.int16).copy()).view(torch.bfloat16).pin_memory()
+    Yh = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
+    hbl.hbitlinear_forward_hostio(
+        Xh, torch.from_numpy(packed.view(np.int32)).to(DEV),
+        torch.from_numpy(np.array([alpha, 0, 0, 0], dtype=np.float32)).to(DEV), 4, Yh, ws)
+    torch.cuda.synchronize()
+    assert np.array_equal(Yh.view(torch.int16).numpy().view(np.uint16),
+                          oracle.hbitlinear_forward(X, packed, alpha, 4))
+
+
+def test_status_word_stays_clear():
+    st = hbl.new_status(DEV)
+    X = to_dev_bf16(acts(200, 2048, seed=1))
+    packed, alpha = hbl.pack_ternary(torch.from_numpy(inputs.latent_weights(256, 2048)).to(DEV))
+    hbl.hbitlinear_forward(X, packed, alpha, 4, status=st)
+    torch.cuda.synchronize()
+    assert int(st[0].item()) == 0
