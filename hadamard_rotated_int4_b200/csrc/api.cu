@@ -185,11 +185,13 @@ hbl_status hbl_pack_ternary(const float* W, int N, int K, float eps, uint32_t* W
                                static_cast<cudaStream_t>(stream), sms);
 }
 
+// Scalars and shapes first; pointers only matter when there is work (M > 0).
 static hbl_status check_act_args(const uint16_t* X, const float* gain, int M, int K,
                                  float norm_eps) {
-    if (!X) return HBL_ERR_INVALID_ARG;
     if (!finite_nonneg(norm_eps)) return HBL_ERR_INVALID_ARG;
     if (M < 0 || check_k(K) != HBL_OK) return HBL_ERR_SHAPE;
+    if (M == 0) return HBL_OK;
+    if (!X) return HBL_ERR_INVALID_ARG;
     if (!aligned16(X) || (gain && !aligned16(gain))) return HBL_ERR_ALIGNMENT;
     return HBL_OK;
 }
@@ -199,9 +201,9 @@ hbl_status hbl_norm_fwht(const uint16_t* X, const float* gain, int M, int K, flo
     (void)dev_status;
     hbl_status st = check_act_args(X, gain, M, K, norm_eps);
     if (st != HBL_OK) return st;
+    if (M == 0) return HBL_OK;
     if (!V) return HBL_ERR_INVALID_ARG;
     if (!aligned16(V)) return HBL_ERR_ALIGNMENT;
-    if (M == 0) return HBL_OK;
     int sms = 0;
     if ((st = device(&sms)) != HBL_OK) return st;
     return launch_norm_fwht_quant(X, gain, M, K, norm_eps, 0.f, 0, nullptr, nullptr, nullptr, V,
@@ -217,10 +219,10 @@ hbl_status hbl_norm_fwht_quant(const uint16_t* X, const float* gain, int M, int 
     if (st != HBL_OK) return st;
     if (act_bits != 4 && act_bits != 8) return HBL_ERR_INVALID_ARG;
     if (!finite_nonneg(quant_eps)) return HBL_ERR_INVALID_ARG;
+    if (M == 0) return HBL_OK;
     if (!codes || !scales) return HBL_ERR_INVALID_ARG;
     if (!aligned16(codes) || !aligned16(scales) || (rowsum && !aligned16(rowsum)))
         return HBL_ERR_ALIGNMENT;
-    if (M == 0) return HBL_OK;
     int sms = 0;
     if ((st = device(&sms)) != HBL_OK) return st;
     return launch_norm_fwht_quant(X, gain, M, K, norm_eps, quant_eps, act_bits, codes, scales,
@@ -231,9 +233,10 @@ hbl_status hbl_ternary_gemm(const void* codes, const float* scales, const int32_
                             int act_bits, int M, int K, const uint32_t* W_packed,
                             const float* alpha, int N, uint16_t* Y, int32_t* acc_out,
                             void* ws, size_t ws_bytes, int32_t* dev_status, void* stream) {
-    if (!codes || !scales || !rowsum || !W_packed || !alpha || !Y) return HBL_ERR_INVALID_ARG;
     if (act_bits != 4 && act_bits != 8) return HBL_ERR_INVALID_ARG;
     if (M < 0 || check_k(K) != HBL_OK || check_n(N) != HBL_OK) return HBL_ERR_SHAPE;
+    if (M == 0) return HBL_OK;
+    if (!codes || !scales || !rowsum || !W_packed || !alpha || !Y) return HBL_ERR_INVALID_ARG;
     if (!aligned16(codes) || !aligned16(scales) || !aligned16(rowsum) || !aligned16(W_packed) ||
         !aligned16(alpha) || !aligned16(Y) || (acc_out && !aligned16(acc_out)) ||
         (dev_status && !aligned16(dev_status)))
@@ -241,7 +244,6 @@ hbl_status hbl_ternary_gemm(const void* codes, const float* scales, const int32_
     const size_t need = gemm_ws(M, K, N, kSizingSms);
     if (need > 0 && (ws == nullptr || ws_bytes < need)) return HBL_ERR_WORKSPACE;
     if (ws && !aligned16(ws)) return HBL_ERR_ALIGNMENT;
-    if (M == 0) return HBL_OK;
     int sms = 0;
     hbl_status st = device(&sms);
     if (st != HBL_OK) return st;
@@ -271,10 +273,11 @@ static hbl_status check_forward(const uint16_t* X, const float* gain, int M, int
                                 const uint32_t* W_packed, const float* alpha, int act_bits,
                                 float norm_eps, float quant_eps, const uint16_t* Y, void* ws,
                                 size_t ws_bytes, int32_t* dev_status, int op, bool host_xy) {
-    if (!X || !W_packed || !alpha || !Y) return HBL_ERR_INVALID_ARG;
     if (act_bits != 4 && act_bits != 8) return HBL_ERR_INVALID_ARG;
     if (!finite_nonneg(norm_eps) || !finite_nonneg(quant_eps)) return HBL_ERR_INVALID_ARG;
     if (M < 0 || check_k(K) != HBL_OK || check_n(N) != HBL_OK) return HBL_ERR_SHAPE;
+    if (M == 0) return HBL_OK;
+    if (!X || !W_packed || !alpha || !Y) return HBL_ERR_INVALID_ARG;
     if ((!host_xy && (!aligned16(X) || !aligned16(Y))) || (gain && !aligned16(gain)) ||
         !aligned16(W_packed) || !aligned16(alpha) || (dev_status && !aligned16(dev_status)))
         return HBL_ERR_ALIGNMENT;
