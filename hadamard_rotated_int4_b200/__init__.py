@@ -12,6 +12,7 @@ Names follow include/hbl.h:
   ternary_gemm(codes, scales, rowsum, act_bits, K, W_packed, alpha)  -> Y bf16 [M, N] (, acc)
   hbitlinear_forward(X, W_packed, alpha, act_bits)                   -> Y bf16 [M, N]
   hbitlinear_forward_hostio(X_host, W_packed, alpha, act_bits, Y_host, ws)
+  ternary_gemv_noalloc(codes, scales, rowsum, act_bits, K, W_packed, alpha)  -> Y (, acc)
 """
 import ctypes
 import os
@@ -26,7 +27,8 @@ STATUS_NAMES = {0: "HBL_OK", 1: "HBL_ERR_INVALID_ARG", 2: "HBL_ERR_SHAPE", 3: "H
 OP_PACK_TERNARY, OP_TERNARY_GEMM, OP_HBITLINEAR_FORWARD, OP_HBITLINEAR_FORWARD_HOSTIO = 0, 1, 2, 3
 EXPORTS = ("hbl_status_string", "hbl_version", "hbl_set_gemm_path", "hbl_workspace_size",
            "hbl_pack_ternary", "hbl_norm_fwht", "hbl_norm_fwht_quant", "hbl_ternary_gemm",
-           "hbl_hbitlinear_forward", "hbl_hbitlinear_forward_hostio")
+           "hbl_hbitlinear_forward", "hbl_hbitlinear_forward_hostio",
+           "hbl_ternary_gemv_noalloc")
 
 _lib = None
 
@@ -67,6 +69,8 @@ def lib():
         L.hbl_hbitlinear_forward.argtypes = [P, P, I, I, I, P, P, I, F, F, P, P, SZ, P, P]
         L.hbl_hbitlinear_forward_hostio.restype = I
         L.hbl_hbitlinear_forward_hostio.argtypes = [P, P, I, I, I, P, P, I, F, F, P, P, SZ, P, P]
+        L.hbl_ternary_gemv_noalloc.restype = I
+        L.hbl_ternary_gemv_noalloc.argtypes = [P, P, P, I, I, I, P, P, I, P, P, P, P]
         _lib = L
     return _lib
 
@@ -185,6 +189,24 @@ def ternary_gemm(codes, scales, rowsum, act_bits, K, W_packed, alpha, want_acc=F
     _check(lib().hbl_ternary_gemm(_ptr(codes), _ptr(scales), _ptr(rowsum), int(act_bits), M, K,
                                   _ptr(W_packed), _ptr(alpha), N, _ptr(Y), _ptr(acc), _ptr(ws),
                                   ws.numel(), _ptr(status), _stream()), "hbl_ternary_gemm")
+    return (Y, acc) if want_acc else Y
+
+
+def ternary_gemv_noalloc(codes, scales, rowsum, act_bits, K, W_packed, alpha, want_acc=False,
+                         out=None, status=None):
+    """hbl_ternary_gemv_noalloc: the split-K GEMV with the library's fixed scratch
+    array (no workspace argument; the library allocates nothing)."""
+    import torch
+
+    M = codes.shape[0]
+    N = W_packed.shape[0]
+    Y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16,
+                                                device=codes.device)
+    acc = torch.empty((M, N), dtype=torch.int32, device=codes.device) if want_acc else None
+    _check(lib().hbl_ternary_gemv_noalloc(_ptr(codes), _ptr(scales), _ptr(rowsum),
+                                          int(act_bits), M, K, _ptr(W_packed), _ptr(alpha), N,
+                                          _ptr(Y), _ptr(acc), _ptr(status), _stream()),
+           "hbl_ternary_gemv_noalloc")
     return (Y, acc) if want_acc else Y
 
 

@@ -333,4 +333,47 @@ hbl_status hbl_hbitlinear_forward_hostio(const uint16_t* X_host, const float* ga
     return HBL_OK;
 }
 
+
+// Allocation-free ternary GEMV: the CUDA-core split-K path with its partial
+// sums in the library's fixed 2 MiB device array instead of caller workspace.
+hbl_status hbl_ternary_gemv_noalloc(const void* codes, const float* scales,
+                                    const int32_t* rowsum, int act_bits, int M, int K,
+                                    const uint32_t* W_packed, const float* alpha, int N,
+                                    uint16_t* Y, int32_t* acc_out, int32_t* dev_status,
+                                    void* stream) {
+    if (act_bits != 4 && act_bits != 8) return HBL_ERR_INVALID_ARG;
+    if (M < 0 || check_k(K) != HBL_OK || check_n(N) != HBL_OK) return HBL_ERR_SHAPE;
+    const int64_t mchunk = M < gemv_max_m() ? M : gemv_max_m();
+    if (gemv_workspace(mchunk, K, N, kSizingSms) > gemv_noalloc_scratch_bytes())
+        return HBL_ERR_WORKSPACE;  // shape needs more than the fixed scratch holds
+    if (M == 0) return HBL_OK;
+    if (!codes || !scales || !rowsum || !W_packed || !alpha || !Y) return HBL_ERR_INVALID_ARG;
+    if (!aligned16(codes) || !aligned16(scales) || !aligned16(rowsum) || !aligned16(W_packed) ||
+        !aligned16(alpha) || !aligned16(Y) || (acc_out && !aligned16(acc_out)) ||
+        (dev_status && !aligned16(dev_status)))
+        return HBL_ERR_ALIGNMENT;
+    int sms = 0;
+    hbl_status st = device(&sms);
+    if (st != HBL_OK) return st;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return HBL_ERR_CUDA;
+    void* scratch = gemv_noalloc_scratch(dev);
+    if (scratch == nullptr) return HBL_ERR_CUDA;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int64_t step = gemv_max_m();
+    for (int64_t r0 = 0; r0 < M; r0 += step) {
+        GemmArgs c{codes, scales, rowsum, act_bits, M, K, W_packed, alpha, N, Y, acc_out,
+                   dev_status};
+        c.M = (M - r0) < step ? (M - r0) : step;
+        c.codes = static_cast<const uint8_t*>(codes) + r0 * codes_row_bytes(K, act_bits);
+        c.scales = scales + r0;
+        c.rowsum = rowsum + r0;
+        c.Y = Y + r0 * N;
+        c.acc_out = acc_out ? acc_out + r0 * N : nullptr;
+        st = launch_gemv(c, scratch, gemv_noalloc_scratch_bytes(), s, sms);
+        if (st != HBL_OK) return st;
+    }
+    return HBL_OK;
+}
+
 }  // extern "C"

@@ -48,4 +48,8 @@ size_t gemv_workspace(int64_t M, int K, int N, int num_sms);
 hbl_status launch_gemv(const GemmArgs& a, void* ws, size_t ws_bytes, cudaStream_t stream,
                        int num_sms);
 
+// Fixed scratch of the allocation-free GEMV entry point (file-scope device array).
+size_t gemv_noalloc_scratch_bytes();
+void* gemv_noalloc_scratch(int dev);
+
 }  // namespace hbl

@@ -16,6 +16,8 @@
 #include "hbl_internal.cuh"
 #include "hbl_launch.h"
 
+#include <atomic>
+
 namespace hbl {
 namespace k3 {
 
@@ -200,6 +202,40 @@ hbl_status launch_gemv(const GemmArgs& a, void* ws, size_t ws_bytes, cudaStream_
     k3::gemv_epilogue_kernel<<<(unsigned)eb, 256, 0, stream>>>(part, ks, M, a.N, a.rowsum,
                                                                a.scales, a.alpha, a.Y, a.acc_out);
     return cudaGetLastError() == cudaSuccess ? HBL_OK : HBL_ERR_CUDA;
+}
+
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant: the split-K partials live in a fixed device array
+// owned by this file instead of caller-provided workspace.  Some callers cannot
+// hand the library scratch memory or let it allocate: an engine's custom-op or
+// plugin hook that receives only its inputs and outputs, or a per-token decode
+// loop that must not take the allocator's lock, stall on an implicit device
+// synchronisation, or fail with out-of-memory halfway through a step.
+// The array below is reserved on every GPU that loads the library and stays
+// reserved until the process exits.  Its host-side name is only a stand-in,
+// never a device address, so the address is looked up once per device with
+// cudaGetSymbolAddress while that device is current.
+constexpr size_t kNoAllocScratchBytes = (size_t)2 << 20;  // 2 MiB
+static __device__ __align__(256) int32_t g_noalloc_scratch[kNoAllocScratchBytes / 4];
+
+namespace {
+constexpr int kNoAllocMaxDevices = 64;
+std::atomic<void*> g_noalloc_ptr[kNoAllocMaxDevices];
+}  // namespace
+
+size_t gemv_noalloc_scratch_bytes() { return kNoAllocScratchBytes; }
+
+// Device address of the fixed scratch array on the current device, or null.
+void* gemv_noalloc_scratch(int dev) {
+    if (dev < 0 || dev >= kNoAllocMaxDevices) return nullptr;
+    void* p = g_noalloc_ptr[dev].load(std::memory_order_acquire);
+    if (p != nullptr) return p;
+    void* q = nullptr;
+    if (cudaGetSymbolAddress(&q, g_noalloc_scratch) != cudaSuccess || q == nullptr)
+        return nullptr;
+    g_noalloc_ptr[dev].store(q, std::memory_order_release);
+    return q;
 }
 
 }  // namespace hbl

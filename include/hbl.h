@@ -168,6 +168,33 @@ HBL_API hbl_status hbl_hbitlinear_forward_hostio(const uint16_t* X_host, const f
                                          float quant_eps, uint16_t* Y_host, void* ws,
                                          size_t ws_bytes, int32_t* dev_status, void* stream);
 
+/* Allocation-free ternary GEMV (no counterpart on the BitNet v2 pages; it is a
+ * deployment aid).  Same arguments, layouts and results as hbl_ternary_gemm
+ * run on its CUDA-core split-K path, but without a workspace argument: the
+ * split-K partial sums live in one fixed 2 MiB array that the library reserves
+ * on every GPU that loads it, until the process exits.
+ * For callers that cannot supply scratch memory or let a library allocate:
+ * e.g. an engine's custom-op hook that is handed only inputs and outputs, or a
+ * token-by-token decode loop that must not block on the allocator, trigger an
+ * implicit device synchronisation, or risk an out-of-memory failure mid-step.
+ * This call never allocates device or host memory.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ *   - All calls on a device share the array and leave their partial sums in
+ *     it; nothing in it needs to start at zero (every partial read is written
+ *     first by the same call).  Calls that overlap on the GPU (two streams or
+ *     two host threads at once) race on the array: serialise them.
+ *   - Shapes whose partials exceed the array (ksplit * min(M, 8) * N * 4 bytes,
+ *     ksplit chosen as for hbl_ternary_gemm) return HBL_ERR_WORKSPACE before
+ *     any launch; e.g. N = 4096 with K = 16384 needs 1 MiB at M >= 8.
+ *   - M > 8 runs in consecutive 8-token chunks on `stream`. */
+HBL_API hbl_status hbl_ternary_gemv_noalloc(const void* codes, const float* scales,
+                                            const int32_t* rowsum, int act_bits, int M, int K,
+                                            const uint32_t* W_packed, const float* alpha, int N,
+                                            uint16_t* Y, int32_t* acc_out, int32_t* dev_status,
+                                            void* stream);
+
 #ifdef __cplusplus
 }
 #endif
