@@ -143,11 +143,19 @@ ORACLE_API float oracle_sqrt7(void) { return (float)sqrt(7.0); }
  * description uses RMS normalisation without bias; the RMS reading is taken. */
 static void rmsnorm_row_f32(const uint16_t* xb, const float* gain, int K, float norm_eps,
                             float* u, float* scratch) {
-    for (int k = 0; k < K; ++k) {
-        float x = oracle_bf16_to_f32(xb[k]);
-        scratch[k] = x * x;
+    /* Leaves of the tree are pairs: x0*x0 + x1*x1 with one rounding.  For bf16
+     * inputs each square is exact in binary32 (8-bit significands), so this
+     * equals rounding the two squares first whenever they do not underflow. */
+    if (K == 1) {
+        float x = oracle_bf16_to_f32(xb[0]);
+        scratch[0] = x * x;
     }
-    float ss = tree_sum_f32(scratch, K);
+    for (int k = 0; k + 1 < K; k += 2) {
+        float x0 = oracle_bf16_to_f32(xb[k]);
+        float x1 = oracle_bf16_to_f32(xb[k + 1]);
+        scratch[k / 2] = fmaf(x0, x0, x1 * x1);
+    }
+    float ss = tree_sum_f32(scratch, K == 1 ? 1 : K / 2);
     float ms = ss * (1.0f / (float)K);
     float r = 1.0f / sqrtf(ms + norm_eps);
     for (int k = 0; k < K; ++k) {
@@ -221,16 +229,17 @@ ORACLE_API int oracle_norm_fwht_f64(const uint16_t* X, const float* gain, int M,
  *                           scale = gamma / 127.
  *   act_bits = 4 (absmean): beta = tree_sum(|v|) * (1/K);
  *                           q = clip(round(v * (sqrt7/(beta+eps))), -8, 7);  scale = beta / sqrt7.
- * round = nearest, ties to even.  The reciprocal constant C/(x+eps) is one IEEE
- * division per row, then one multiply per element.
+ * round = nearest, ties to even.  The reciprocal constant inv = C/(x+eps) is one
+ * IEEE division per row; each code rounds the exact product v * inv (the
+ * product of two binary32 numbers is exact in binary64) once to an integer.
  * Codes: act_bits 8 -> one int8 per element, row-major [M x K];
  *        act_bits 4 -> two's-complement nibbles, element 2j in the low nibble of
  *        byte j of the row, [M x K/2].
  * rowsum (nullable) = sum of the row's integer codes. */
-static int8_t clip_round(float y, int lo, int hi) {
-    float r = rintf(y);
-    if (r < (float)lo) r = (float)lo;
-    if (r > (float)hi) r = (float)hi;
+static int8_t clip_round(double y, int lo, int hi) {
+    double r = rint(y);
+    if (r < (double)lo) r = (double)lo;
+    if (r > (double)hi) r = (double)hi;
     return (int8_t)r;
 }
 
@@ -261,7 +270,7 @@ ORACLE_API int oracle_quantize_rows(const float* V, int M, int K, float quant_ep
         }
         int32_t sum = 0;
         for (int k = 0; k < K; ++k) {
-            float y = v[k] * inv;
+            double y = (double)v[k] * (double)inv; /* exact */
             q[k] = clip_round(y, lo, hi);
             sum += q[k];
         }
@@ -333,7 +342,7 @@ ORACLE_API int oracle_ternarize(const float* W, int N, int K, float eps, int8_t*
     free(a);
     float d = alpha + eps;
     if (t_out)
-        for (int64_t i = 0; i < nk; ++i) t_out[i] = clip_round(W[i] / d, -1, 1);
+        for (int64_t i = 0; i < nk; ++i) t_out[i] = clip_round((double)(W[i] / d), -1, 1);
     *alpha_out = alpha;
     return 0;
 }

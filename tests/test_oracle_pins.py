@@ -223,6 +223,37 @@ def test_int4_ties_hand_case():
     assert rowsum[0] == g["expected_rowsum"]
 
 
+def _tie_case():
+    """Find binary32 gamma, v with inv = fl(127/gamma) such that fl(v*inv) is a
+    .5 tie while the exact product is not: one rounding of the exact product
+    and rounding the binary32 product then the tie give different integers."""
+    rng = np.random.default_rng(123)
+    for _ in range(200000):
+        gamma = np.float32(rng.uniform(100.0, 127.0))
+        inv = np.float32(127.0) / gamma
+        k = int(rng.integers(1, 60))
+        v = np.float32((k + 0.5) / float(inv))
+        for cand in (v, np.nextafter(v, np.float32(0)), np.nextafter(v, np.float32(1e9))):
+            if abs(float(cand)) > float(gamma):
+                continue
+            p32 = np.float32(cand * inv)
+            ex = Fraction(float(cand)) * Fraction(float(inv))
+            if float(p32) == k + 0.5 and ex != Fraction(2 * k + 1, 2):
+                if round(ex) != round(Fraction(float(p32))):
+                    return gamma, cand, inv, ex, p32
+    raise AssertionError("no tie case found")
+
+
+def test_quantiser_rounds_the_exact_product_once():
+    # Reading: each code rounds the exact product v * (127/(gamma+eps)) once.
+    gamma, v, inv, exact, p32 = _tie_case()
+    row = np.array([[v, gamma]], dtype=np.float32)
+    codes, _, _ = oracle.quantize_rows(row, 8, quant_eps=0.0)
+    got = int(codes.view(np.int8)[0, 0])
+    assert got == round(exact)
+    assert got != round(Fraction(float(p32)))
+
+
 def test_int4_clip_hand_case():
     g = _golden()["int4_clip"]
     v = np.array([g["input"]], dtype=np.float32)
@@ -261,7 +292,8 @@ def test_quantiser_brute_force_rounding(bits):
             inv = oracle.sqrt7() / (beta + np.float32(1e-5))
             scale = beta / oracle.sqrt7()
         for k in range(K):
-            y = float(np.float32(row[k]) * np.float32(inv))
+            # the exact product of the two binary32 values, rounded once
+            y = Fraction(float(row[k])) * Fraction(float(inv))
             assert q[m, k] == min(hi, max(lo, round(y)))
         assert scales[m] == np.float32(scale)
         assert rowsum[m] == q[m].sum()
