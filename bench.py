@@ -50,6 +50,9 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--kernel-iters", type=int, default=200,
                     help="iterations of the per-kernel timing loops")
+    ap.add_argument("--only", default=None, choices=["forward", "gemm", "quant4", "quant8"],
+                    help="run only this case (a few launches, for profiler captures); prints a "
+                         "short JSON line, not the benchmark line")
     return ap.parse_args()
 
 
@@ -262,23 +265,25 @@ def run_hbl(args):
     t_max_ms = hdist.max_over_ranks(t_dev_ms, dev)
     value = world * M_TOK * args.steps / (t_max_ms / 1e3)
 
-    # ---- per-kernel timing (same kernels, through the two-call C-ABI path)
-    codes = torch.empty((M_TOK, K_IN // 2), dtype=torch.uint8, device=dev)
+    # ---- per-kernel timing: the forward's two kernels through the two-call
+    # C-ABI path with the same (32-row interleaved, one byte per code) layout
+    IL = hbl.ACT_INT4_I32
+    codes = torch.empty(hbl.codes_shape(M_TOK, K_IN, IL), dtype=torch.uint8, device=dev)
     scales = torch.empty(M_TOK, dtype=torch.float32, device=dev)
     rowsum = torch.empty(M_TOK, dtype=torch.int32, device=dev)
-    gws = torch.empty(max(16, hbl.workspace_size(hbl.OP_TERNARY_GEMM, M_TOK, K_IN, N_OUT, BITS)),
+    gws = torch.empty(max(16, hbl.workspace_size(hbl.OP_TERNARY_GEMM, M_TOK, K_IN, N_OUT, IL)),
                       dtype=torch.uint8, device=dev)
     iters = max(args.kernel_iters, args.steps)
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(iters)]
     for i in range(3):
-        hbl.norm_fwht_quant(Xd, BITS, out=(codes, scales, rowsum))
-        hbl.ternary_gemm(codes, scales, rowsum, BITS, K_IN, packed, alpha, ws=gws, out=Y)
+        hbl.norm_fwht_quant(Xd, IL, out=(codes, scales, rowsum))
+        hbl.ternary_gemm(codes, scales, rowsum, IL, K_IN, packed, alpha, ws=gws, out=Y)
     torch.cuda.synchronize()
     for i in range(iters):
         evs[i][0].record(stream)
-        hbl.norm_fwht_quant(Xd, BITS, out=(codes, scales, rowsum))
+        hbl.norm_fwht_quant(Xd, IL, out=(codes, scales, rowsum))
         evs[i][1].record(stream)
-        hbl.ternary_gemm(codes, scales, rowsum, BITS, K_IN, packed, alpha, ws=gws, out=Y,
+        hbl.ternary_gemm(codes, scales, rowsum, IL, K_IN, packed, alpha, ws=gws, out=Y,
                          status=status)
         evs[i][2].record(stream)
     torch.cuda.synchronize()
@@ -337,15 +342,15 @@ def run_hbl(args):
     if t_k2 >= t_k1:
         achieved = ops / t_k2 / 1e12
         peak = 2.0 * pk["bf16_tflops_sustained"]
-        roof = {"bound": "tensor", "kernel": "ternary_gemm_tc (tcgen05 kind::i8)",
+        roof = {"bound": "tensor", "kernel": "gemm_ts (tcgen05 kind::i8, activations in TMEM)",
                 "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                 "peak_note": "int8 dense = %s sustained bf16 %.1f TFLOP/s x 2 (nominal "
                              "int8:bf16 ratio)" % (pk["source"], pk["bf16_tflops_sustained"]),
-                "traffic": recorded_traffic("gemm_tc_a4_ffn_wdown",
-                                            source_hash("k2_ternary_gemm_tc.cu")),
+                "traffic": recorded_traffic("gemm_ts_a4_ffn_wdown",
+                                            source_hash("k2b_ternary_gemm_ts.cu")),
                 "us_per_launch": t_k2 * 1e6}
     else:
-        nbytes = M_TOK * K_IN * 2 + M_TOK * K_IN // 2 + 8 * M_TOK
+        nbytes = M_TOK * K_IN * 2 + M_TOK * K_IN + 8 * M_TOK  # one-byte codes in the forward
         achieved = nbytes / t_k1 / 1e9
         roof = {"bound": "hbm", "kernel": "norm_fwht_quant", "achieved": achieved,
                 "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": achieved / pk["hbm_gbs"],
@@ -363,7 +368,7 @@ def run_hbl(args):
                    else "single GPU",
                    "l2": "inputs larger than L2 (X 268 MB per step)"},
         "roofline": roof,
-        "kernels_us": {"norm_fwht_quant": t_k1 * 1e6, "ternary_gemm_tc": t_k2 * 1e6},
+        "kernels_us": {"norm_fwht_quant": t_k1 * 1e6, "ternary_gemm_ts": t_k2 * 1e6},
         "quant": quant,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": M_TOK * K_IN * 2,
                 "d2h_bytes_per_step": M_TOK * N_OUT * 2, "steps": e2e_steps,
@@ -386,10 +391,53 @@ def run_hbl(args):
     return 0
 
 
+def run_only(args):
+    """A single case with few launches, sized for profiler captures."""
+    import numpy as np
+    import torch
+
+    import hadamard_rotated_int4_b200 as hbl
+    from hadamard_rotated_int4_b200 import inputs
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    if args.only.startswith("quant"):
+        bits = int(args.only[-1])
+        X = torch.from_numpy(inputs.activations("quant").view(np.int16)).view(
+            torch.bfloat16).to(dev)
+        fn = lambda: hbl.norm_fwht_quant(X, bits)
+    else:
+        X = torch.from_numpy(inputs.activations("ffn_wdown").view(np.int16)).view(
+            torch.bfloat16).to(dev)
+        packed, alpha = hbl.pack_ternary(torch.from_numpy(inputs.weights("ffn_wdown")).to(dev))
+        if args.only == "forward":
+            ws = torch.empty(hbl.workspace_size(hbl.OP_HBITLINEAR_FORWARD, M_TOK, K_IN, N_OUT,
+                                                BITS), dtype=torch.uint8, device=dev)
+            fn = lambda: hbl.hbitlinear_forward(X, packed, alpha, BITS, ws=ws)
+        else:  # the forward's GEMM: interleaved one-byte INT4 codes
+            IL = hbl.ACT_INT4_I32
+            codes, scales, rowsum = hbl.norm_fwht_quant(X, IL)
+            fn = lambda: hbl.ternary_gemm(codes, scales, rowsum, IL, K_IN, packed, alpha)
+    for _ in range(args.warmup):
+        fn()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(args.steps):
+        fn()
+    b.record()
+    torch.cuda.synchronize()
+    print(json.dumps({"only": args.only, "steps": args.steps,
+                      "us_per_step": 1e3 * a.elapsed_time(b) / max(1, args.steps)}))
+    return 0
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
+    if args.only:
+        return run_only(args)
     return run_hbl(args)
 
 

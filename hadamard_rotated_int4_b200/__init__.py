@@ -25,6 +25,7 @@ STATUS_NAMES = {0: "HBL_OK", 1: "HBL_ERR_INVALID_ARG", 2: "HBL_ERR_SHAPE", 3: "H
                 4: "HBL_ERR_UNSUPPORTED_ARCH", 5: "HBL_ERR_WORKSPACE", 6: "HBL_ERR_CUDA",
                 7: "HBL_ERR_TIMEOUT"}
 OP_PACK_TERNARY, OP_TERNARY_GEMM, OP_HBITLINEAR_FORWARD, OP_HBITLINEAR_FORWARD_HOSTIO = 0, 1, 2, 3
+ACT_INT4_I32, ACT_INT8_I32 = 0x104, 0x108  # one byte per code, 32-row interleaved layout
 EXPORTS = ("hbl_status_string", "hbl_version", "hbl_set_gemm_path", "hbl_workspace_size",
            "hbl_pack_ternary", "hbl_norm_fwht", "hbl_norm_fwht_quant", "hbl_ternary_gemm",
            "hbl_hbitlinear_forward", "hbl_hbitlinear_forward_hostio",
@@ -109,7 +110,8 @@ def workspace_size(op, M, K, N, act_bits):
 
 
 def set_gemm_path(path):
-    """0 = automatic, 1 = tensor cores, 2 = CUDA-core GEMV (process-wide)."""
+    """0 = automatic, 1 = tensor cores (both operands in shared memory),
+    2 = CUDA-core GEMV, 3 = tensor cores with activations in TMEM (process-wide)."""
     _check(lib().hbl_set_gemm_path(int(path)), "set_gemm_path")
 
 
@@ -152,6 +154,8 @@ def norm_fwht(X, gain=None, norm_eps=1e-6, status=None):
 
 
 def codes_shape(M, K, act_bits):
+    if act_bits in (ACT_INT4_I32, ACT_INT8_I32):
+        return ((M + 31) // 32 * 32, K)
     return (M, K if act_bits == 8 else K // 2)
 
 
@@ -178,7 +182,7 @@ def ternary_gemm(codes, scales, rowsum, act_bits, K, W_packed, alpha, want_acc=F
                  out=None, status=None):
     import torch
 
-    M = codes.shape[0]
+    M = scales.shape[0]  # the interleaved layouts pad the codes buffer to 32 rows
     N = W_packed.shape[0]
     Y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16,
                                                 device=codes.device)

@@ -23,7 +23,7 @@ struct DevInfo {
     int sms = 0;
 };
 DevInfo g_dev[kMaxDevices];
-std::atomic<int> g_path{0};  // 0 auto, 1 tensor core, 2 CUDA-core GEMV
+std::atomic<int> g_path{0};  // 0 auto, 1 tensor core (SS), 2 CUDA-core GEMV, 3 tensor core (TS)
 
 bool is_pow2(int64_t v) { return v > 0 && (v & (v - 1)) == 0; }
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -59,9 +59,16 @@ hbl_status device(int* sms) {
 
 int codes_row_bytes(int K, int act_bits) { return act_bits == 8 ? K : K / 2; }
 
+// act_bits: 4 / 8 (row-major layouts) or HBL_ACT_INT{4,8}_I32 (interleaved bytes)
+bool act_valid(int a) {
+    return a == 4 || a == 8 || a == HBL_ACT_INT4_I32 || a == HBL_ACT_INT8_I32;
+}
+bool act_il(int a) { return a == HBL_ACT_INT4_I32 || a == HBL_ACT_INT8_I32; }
+int act_base(int a) { return a & 0xFF; }
+
 bool use_gemv(int64_t M) {
     const int path = g_path.load();
-    if (path == 1) return false;
+    if (path == 1 || path == 3) return false;
     if (path == 2) return true;
     return M <= gemv_max_m();
 }
@@ -77,7 +84,8 @@ size_t gemm_ws(int64_t M, int K, int N, int sms_guess) {
 constexpr int kSizingSms = 148;
 
 hbl_status run_gemm(const GemmArgs& a, void* ws, size_t ws_bytes, cudaStream_t s, int sms) {
-    if (!use_gemv(a.M)) return launch_gemm_tc(a, s, sms);
+    if (!use_gemv(a.M))
+        return g_path.load() == 1 ? launch_gemm_tc(a, s, sms) : launch_gemm_ts(a, s, sms);
     // CUDA-core path in chunks of up to gemv_max_m() tokens (workspace reused in order)
     const int64_t step = gemv_max_m();
     for (int64_t r0 = 0; r0 < a.M; r0 += step) {
@@ -135,7 +143,7 @@ const char* hbl_status_string(int status) {
 int hbl_version(void) { return 100; }
 
 int hbl_set_gemm_path(int path) {
-    if (path < 0 || path > 2) return HBL_ERR_INVALID_ARG;
+    if (path < 0 || path > 3) return HBL_ERR_INVALID_ARG;
     g_path.store(path);
     return HBL_OK;
 }
@@ -153,10 +161,11 @@ hbl_status hbl_workspace_size(int op, int M, int K, int N, int act_bits, size_t*
         case HBL_OP_HBITLINEAR_FORWARD:
         case HBL_OP_HBITLINEAR_FORWARD_HOSTIO: {
             if (M < 0 || check_k(K) != HBL_OK || check_n(N) != HBL_OK) return HBL_ERR_SHAPE;
-            if (act_bits != 4 && act_bits != 8) return HBL_ERR_INVALID_ARG;
-            size_t b = up256(gemm_ws(M, K, N, kSizingSms));
+            if (!act_valid(act_bits)) return HBL_ERR_INVALID_ARG;
+            if (op != HBL_OP_TERNARY_GEMM && act_il(act_bits)) return HBL_ERR_INVALID_ARG;
+            size_t b = act_il(act_bits) ? 0 : up256(gemm_ws(M, K, N, kSizingSms));
             if (op != HBL_OP_TERNARY_GEMM) {
-                b += up256((size_t)M * codes_row_bytes(K, act_bits));  // codes
+                b += up256((size_t)((M + 31) & ~31) * K);  // codes, one byte each, rows padded to 32
                 b += up256((size_t)M * 4) * 2;                         // scales, rowsum
             }
             if (op == HBL_OP_HBITLINEAR_FORWARD_HOSTIO) {
@@ -217,7 +226,7 @@ hbl_status hbl_norm_fwht_quant(const uint16_t* X, const float* gain, int M, int 
     (void)dev_status;
     hbl_status st = check_act_args(X, gain, M, K, norm_eps);
     if (st != HBL_OK) return st;
-    if (act_bits != 4 && act_bits != 8) return HBL_ERR_INVALID_ARG;
+    if (!act_valid(act_bits)) return HBL_ERR_INVALID_ARG;
     if (!finite_nonneg(quant_eps)) return HBL_ERR_INVALID_ARG;
     if (M == 0) return HBL_OK;
     if (!codes || !scales) return HBL_ERR_INVALID_ARG;
@@ -225,7 +234,8 @@ hbl_status hbl_norm_fwht_quant(const uint16_t* X, const float* gain, int M, int 
         return HBL_ERR_ALIGNMENT;
     int sms = 0;
     if ((st = device(&sms)) != HBL_OK) return st;
-    return launch_norm_fwht_quant(X, gain, M, K, norm_eps, quant_eps, act_bits, codes, scales,
+    const int mode = act_il(act_bits) ? (act_base(act_bits) == 4 ? 5 : 9) : act_bits;
+    return launch_norm_fwht_quant(X, gain, M, K, norm_eps, quant_eps, mode, codes, scales,
                                   rowsum, nullptr, static_cast<cudaStream_t>(stream), sms);
 }
 
@@ -233,7 +243,7 @@ hbl_status hbl_ternary_gemm(const void* codes, const float* scales, const int32_
                             int act_bits, int M, int K, const uint32_t* W_packed,
                             const float* alpha, int N, uint16_t* Y, int32_t* acc_out,
                             void* ws, size_t ws_bytes, int32_t* dev_status, void* stream) {
-    if (act_bits != 4 && act_bits != 8) return HBL_ERR_INVALID_ARG;
+    if (!act_valid(act_bits)) return HBL_ERR_INVALID_ARG;
     if (M < 0 || check_k(K) != HBL_OK || check_n(N) != HBL_OK) return HBL_ERR_SHAPE;
     if (M == 0) return HBL_OK;
     if (!codes || !scales || !rowsum || !W_packed || !alpha || !Y) return HBL_ERR_INVALID_ARG;
@@ -241,12 +251,17 @@ hbl_status hbl_ternary_gemm(const void* codes, const float* scales, const int32_
         !aligned16(alpha) || !aligned16(Y) || (acc_out && !aligned16(acc_out)) ||
         (dev_status && !aligned16(dev_status)))
         return HBL_ERR_ALIGNMENT;
-    const size_t need = gemm_ws(M, K, N, kSizingSms);
+    const size_t need = act_il(act_bits) ? 0 : gemm_ws(M, K, N, kSizingSms);
     if (need > 0 && (ws == nullptr || ws_bytes < need)) return HBL_ERR_WORKSPACE;
     if (ws && !aligned16(ws)) return HBL_ERR_ALIGNMENT;
     int sms = 0;
     hbl_status st = device(&sms);
     if (st != HBL_OK) return st;
+    if (act_il(act_bits)) {  // interleaved one-byte codes: the TMEM-activation kernel
+        GemmArgs a{codes, scales, rowsum, 8, M, K, W_packed, alpha, N, Y, acc_out, dev_status};
+        a.interleaved = true;
+        return launch_gemm_ts(a, static_cast<cudaStream_t>(stream), sms);
+    }
     GemmArgs a{codes, scales, rowsum, act_bits, M, K, W_packed, alpha, N, Y, acc_out, dev_status};
     return run_gemm(a, ws, ws_bytes, static_cast<cudaStream_t>(stream), sms);
 }
@@ -255,17 +270,25 @@ static hbl_status forward_impl(const uint16_t* X, const float* gain, int M, int 
                                const uint32_t* W_packed, const float* alpha, int act_bits,
                                float norm_eps, float quant_eps, uint16_t* Y, uint8_t* ws,
                                size_t ws_bytes, int32_t* dev_status, cudaStream_t s, int sms) {
-    const size_t cb = up256((size_t)M * codes_row_bytes(K, act_bits));
+    // For the default tensor-core kernel the codes stay in workspace one per
+    // byte (INT4 values too) in the 32-row interleaved layout, so the GEMM
+    // loads them coalesced and without widening; other back ends take the
+    // public row-major layouts.
+    const size_t cb = up256((size_t)((M + 31) & ~31) * K);
     const size_t sb = up256((size_t)M * 4);
     uint8_t* codes = ws;
     float* scales = reinterpret_cast<float*>(ws + cb);
     int32_t* rowsum = reinterpret_cast<int32_t*>(ws + cb + sb);
     uint8_t* gws = ws + cb + 2 * sb;
     const size_t gws_bytes = ws_bytes - (cb + 2 * sb);
-    hbl_status st = launch_norm_fwht_quant(X, gain, M, K, norm_eps, quant_eps, act_bits, codes,
+    const bool il = !use_gemv(M) && g_path.load() != 1;
+    const int k1_mode = il ? (act_bits == 4 ? 5 : 9) : act_bits;
+    hbl_status st = launch_norm_fwht_quant(X, gain, M, K, norm_eps, quant_eps, k1_mode, codes,
                                            scales, rowsum, nullptr, s, sms);
     if (st != HBL_OK) return st;
-    GemmArgs a{codes, scales, rowsum, act_bits, M, K, W_packed, alpha, N, Y, nullptr, dev_status};
+    GemmArgs a{codes, scales, rowsum, il ? 8 : act_bits, M, K, W_packed, alpha, N, Y, nullptr,
+               dev_status};
+    a.interleaved = il;
     return run_gemm(a, gws, gws_bytes, s, sms);
 }
 

@@ -12,7 +12,9 @@ namespace hbl {
 // Sets the dynamic shared-memory limit of `func` once per device (idempotent).
 bool smem_attr_once(const void* func, int bytes);
 
-// K1: mode 0 writes fp32 V, mode 4/8 writes INT4/INT8 codes + scales (+ rowsum).
+// K1: mode 0 writes fp32 V; modes 4 / 8 write INT4 (packed nibbles) / INT8 codes +
+// scales (+ rowsum); modes 5 / 9 write INT4 / INT8 codes one per byte in the
+// 32-row interleaved layout of the fused forward.
 hbl_status launch_norm_fwht_quant(const uint16_t* X, const float* gain, int64_t M, int K,
                                   float norm_eps, float quant_eps, int mode, void* codes,
                                   float* scales, int32_t* rowsum, float* V, cudaStream_t stream,
@@ -37,10 +39,13 @@ struct GemmArgs {
     uint16_t* Y;
     int32_t* acc_out;
     int32_t* dev_status;
+    bool interleaved = false;  // codes one per byte in the 32-row interleaved layout
 };
 
-// K2: tcgen05 tensor-core GEMM (TMEM accumulators), any M.
+// K2: tcgen05 tensor-core GEMM, both operands in shared memory, any M.
 hbl_status launch_gemm_tc(const GemmArgs& a, cudaStream_t stream, int num_sms);
+// K2b: tcgen05 tensor-core GEMM with the activations in TMEM, any M.
+hbl_status launch_gemm_ts(const GemmArgs& a, cudaStream_t stream, int num_sms);
 
 // K3: CUDA-core split-K GEMV for small M (M <= gemv_max_m()).
 int gemv_max_m();

@@ -207,11 +207,16 @@ __device__ __forceinline__ float stream_tree(F&& f) {
 
 // ---- the kernel -------------------------------------------------------------
 
-// MODE: 0 = write fp32 V (norm + transform only), 4 = INT4 codes, 8 = INT8 codes.
+// MODE: 0 = write fp32 V (norm + transform only), 4 = INT4 codes (packed nibbles),
+// 8 = INT8 codes (row-major); 5 / 9 = INT4 / INT8 codes one per byte in the
+// 32-row interleaved layout the fused forward's GEMM loads (16-code chunk c of
+// row m at byte (((m / 32) * (K / 16) + c) * 32 + m % 32) * 16).
 // GAIN: multiply by the per-channel RMSNorm gain (false: gain of one, exact skip).
 template <int L, int MODE, bool GAIN>
 __global__ void __launch_bounds__(Cfg<L>::kCtaThreads, Cfg<L>::kMinBlocks)
     norm_fwht_quant_kernel(Params p) {
+    constexpr bool kAbsmax = (MODE == 8 || MODE == 9);       // INT8 absmax statistic
+    constexpr bool kInterleaved = (MODE == 5 || MODE == 9);  // fused-forward code layout
     using C = Cfg<L>;
     using Y = Lay<L>;
     constexpr int R = C::R, T = C::T, W = C::W, K = C::K;
@@ -291,35 +296,39 @@ __global__ void __launch_bounds__(Cfg<L>::kCtaThreads, Cfg<L>::kMinBlocks)
     };
 
     const int64_t stride_groups = (int64_t)gridDim.x * C::kGroupsPerCta;
+    // Stage a group's bf16 rows in shared memory with coalesced 16-byte
+    // cp.async (zero-filled past M); also hint the group after it into L2.
+    auto issue_load = [&](int64_t g_rg) {
+        const int64_t g_row0 = g_rg * C::kRowsPerGroup;
+        if (g_row0 >= p.M) return;
+        const uint16_t* src0 = p.X + g_row0 * K;
+        const uint32_t wsw = stage_swz<C::kStageShift>((uint32_t)w);
+        static_for<0, R / 8>([&](auto ii) {
+            constexpr int i = decltype(ii)::value;
+            const int g = i * W + w;
+            const bool ok = g_row0 + ((g * 8) >> L) < p.M;
+            const uint32_t phys = stage_swz<C::kStageShift>((uint32_t)(i * W)) ^ wsw;
+            cp_async16(buf_s + phys * 16u, ok ? (const void*)(src0 + g * 8) : (const void*)p.X,
+                       ok ? 16 : 0);
+        });
+        cp_async_commit();
+        if (w == 0) {
+            const int64_t nrow0 = g_row0 + stride_groups * C::kRowsPerGroup;
+            if (nrow0 < p.M) {
+                int64_t nrows = p.M - nrow0;
+                if (nrows > C::kRowsPerGroup) nrows = C::kRowsPerGroup;
+                prefetch_l2_bulk(p.X + nrow0 * K, (uint32_t)(nrows * K * 2));
+            }
+        }
+    };
+
+    issue_load((int64_t)blockIdx.x * C::kGroupsPerCta + grp);
     for (int64_t rg = (int64_t)blockIdx.x * C::kGroupsPerCta + grp;; rg += stride_groups) {
         const int64_t row0 = rg * C::kRowsPerGroup;
         if (row0 >= p.M) break;
         const int64_t row = row0 + rig;
-
-        // ---- stage the group's bf16 rows in shared memory (coalesced)
-        {
-            const uint16_t* src0 = p.X + row0 * K;
-            const uint32_t wsw = stage_swz<C::kStageShift>((uint32_t)w);
-            static_for<0, R / 8>([&](auto ii) {
-                constexpr int i = decltype(ii)::value;
-                const int g = i * W + w;
-                const bool ok = row0 + ((g * 8) >> L) < p.M;
-                const uint32_t phys = stage_swz<C::kStageShift>((uint32_t)(i * W)) ^ wsw;
-                cp_async16(buf_s + phys * 16u, ok ? (const void*)(src0 + g * 8) : (const void*)p.X,
-                           ok ? 16 : 0);
-            });
-            cp_async_commit();
-            if (w == 0) {
-                const int64_t nrow0 = row0 + stride_groups * C::kRowsPerGroup;
-                if (nrow0 < p.M) {
-                    int64_t nrows = p.M - nrow0;
-                    if (nrows > C::kRowsPerGroup) nrows = C::kRowsPerGroup;
-                    prefetch_l2_bulk(p.X + nrow0 * K, (uint32_t)(nrows * K * 2));
-                }
-            }
-            cp_async_wait_all();
-            group_sync<T>(grp);
-        }
+        cp_async_wait_all();
+        group_sync<T>(grp);
 
         float2 d[R / 2];
         {
@@ -334,12 +343,13 @@ __global__ void __launch_bounds__(Cfg<L>::kCtaThreads, Cfg<L>::kMinBlocks)
             });
         }
         group_sync<T>(grp);  // staging buffer free again
+        if constexpr (P_LAST == 0) issue_load(rg + stride_groups);  // overlaps this row's work
 
-        // ---- RMSNorm: tree(x*x) over the row, ascending index order
+        // ---- RMSNorm: tree over the row in ascending index order; each leaf is
+        // x0*x0 + x1*x1 with one rounding (bf16 squares are exact in fp32)
         float ss = stream_tree<R / 2>([&](auto kk) {
             constexpr int k = decltype(kk)::value;
-            float2 q = mul2(d[k], d[k]);
-            return __fadd_rn(q.x, q.y);
+            return __fmaf_rn(d[k].x, d[k].x, __fmul_rn(d[k].y, d[k].y));
         });
         ss = row_sum(ss);
         const float ms = __fmul_rn(ss, 1.0f / (float)K);
@@ -400,6 +410,10 @@ __global__ void __launch_bounds__(Cfg<L>::kCtaThreads, Cfg<L>::kMinBlocks)
             });
         });
 
+        // the row buffer is free from here on: start the next group's load so it
+        // overlaps the rest of this row's work
+        if constexpr (P_LAST > 0) issue_load(rg + stride_groups);
+
         // ---- normalise by 1/sqrt(K)
         {
             const float2 c2 = make_float2(p.cK, p.cK);
@@ -425,7 +439,7 @@ __global__ void __launch_bounds__(Cfg<L>::kCtaThreads, Cfg<L>::kMinBlocks)
         } else {
             // ---- per-token statistic
             float stat;
-            if constexpr (MODE == 8) {
+            if constexpr (kAbsmax) {
                 float m = 0.f;
                 static_for<0, R / 2>([&](auto kk) {
                     constexpr int k = decltype(kk)::value;
@@ -491,21 +505,24 @@ __global__ void __launch_bounds__(Cfg<L>::kCtaThreads, Cfg<L>::kMinBlocks)
                 stat = __fmul_rn(x, 1.0f / (float)K);
             }
 
-            const float cq = (MODE == 8) ? 127.0f : p.s7;
+            const float cq = kAbsmax ? 127.0f : p.s7;
             const float inv = __fdiv_rn(cq, __fadd_rn(stat, p.quant_eps));
-            const float lo = (MODE == 8) ? -128.0f : -8.0f;
-            const float hi = (MODE == 8) ? 127.0f : 7.0f;
             const float2 inv2 = make_float2(inv, inv);
-            const float2 magic2 = make_float2(12582912.0f, 12582912.0f);  // 1.5 * 2^23
-
-            // codes: round-half-even via the 1.5*2^23 addition; the code is the
-            // low bits of the sum's bit pattern.  Packed word by word, run by run.
-            constexpr int RL = 1 << RUN;                       // elements per run
-            constexpr int BYTES = (MODE == 8) ? RL : RL / 2;   // code bytes per run
-            constexpr int EPW = (MODE == 8) ? 4 : (RL >= 8 ? 8 : 4);  // elements per word
+            // One rounding of the exact product v*inv to an integer: fma with
+            // 1.5*2^23 (+8 for packed INT4, making the stored nibble q + 8).
+            // |v*inv| <= 127 (INT8) or <= sqrt7*K (INT4), far below 2^22.
+            constexpr float kMagic = (MODE == 4) ? 12582920.0f : 12582912.0f;
+            constexpr int32_t kMagicBits = (MODE == 4) ? 0x4B400008 : 0x4B400000;
+            const float2 magic2 = make_float2(kMagic, kMagic);
+            // INT4 clamp on the integer bit pattern: q in [-8, 7]
+            constexpr int32_t kLoBits = kMagicBits - 8, kHiBits = kMagicBits + 7;
+            constexpr bool kPackNibbles = (MODE == 4);
+            constexpr int RL = 1 << RUN;                                 // elements per run
+            constexpr int BYTES = kPackNibbles ? RL / 2 : RL;            // code bytes per run
+            constexpr int EPW = kPackNibbles ? (RL >= 8 ? 8 : 4) : 4;    // elements per word
             constexpr int NWORD = RL / EPW;
             const bool row_ok = row < p.M;
-            uint8_t* crow = p.codes + row0 * (int64_t)((K * MODE) / 8);
+            uint8_t* crow = p.codes + row0 * (int64_t)(kPackNibbles ? K / 2 : K);
             uint32_t qsum = 0;
             static_for<0, R / RL>([&](auto mm) {
                 constexpr int m = decltype(mm)::value;
@@ -515,30 +532,44 @@ __global__ void __launch_bounds__(Cfg<L>::kCtaThreads, Cfg<L>::kMinBlocks)
                     uint32_t qv[EPW];
                     static_for<0, EPW / 2>([&](auto kk) {
                         constexpr int k = (m * RL + wi * EPW) / 2 + decltype(kk)::value;
-                        float2 y = mul2(d[k], inv2);
-                        y.x = fminf(fmaxf(y.x, lo), hi);
-                        y.y = fminf(fmaxf(y.y, lo), hi);
-                        y = add2(y, magic2);
-                        qv[2 * decltype(kk)::value] = __float_as_uint(y.x);
-                        qv[2 * decltype(kk)::value + 1] = __float_as_uint(y.y);
+                        const float2 y = __ffma2_rn(d[k], inv2, magic2);
+                        int32_t b0 = __float_as_int(y.x), b1 = __float_as_int(y.y);
+                        if constexpr (!kAbsmax) {  // INT8 codes never leave [-127, 127]
+                            b0 = min(max(b0, kLoBits), kHiBits);
+                            b1 = min(max(b1, kLoBits), kHiBits);
+                        }
+                        qv[2 * decltype(kk)::value] = (uint32_t)b0;
+                        qv[2 * decltype(kk)::value + 1] = (uint32_t)b1;
                     });
                     static_for<0, EPW>([&](auto ee) { qsum += qv[decltype(ee)::value]; });
-                    if constexpr (MODE == 8) {
+                    if constexpr (!kPackNibbles) {  // one byte per code: low byte = q
                         const uint32_t lo2 = __byte_perm(qv[0], qv[1], 0x0040);
                         const uint32_t hi2 = __byte_perm(qv[2], qv[3], 0x0040);
                         wv[wi] = __byte_perm(lo2, hi2, 0x5410);
-                    } else {
-                        uint32_t acc = 0;
-                        static_for<0, EPW>([&](auto ee) {
-                            constexpr int e = decltype(ee)::value;
-                            acc |= (qv[e] & 0xFu) << (4 * e);
-                        });
-                        wv[wi] = acc;
+                    } else {  // low nibble = q + 8; pairs by shift-add, bytes by permute
+                        const uint32_t p01 = (qv[1] << 4) + qv[0];
+                        const uint32_t p23 = (qv[3] << 4) + qv[2];
+                        const uint32_t lo2 = __byte_perm(p01, p23, 0x0040);
+                        if constexpr (EPW == 8) {
+                            const uint32_t p45 = (qv[5] << 4) + qv[4];
+                            const uint32_t p67 = (qv[7] << 4) + qv[6];
+                            const uint32_t hi2 = __byte_perm(p45, p67, 0x0040);
+                            wv[wi] = __byte_perm(lo2, hi2, 0x5410) ^ 0x88888888u;
+                        } else {
+                            wv[wi] = lo2 ^ 0x8888u;
+                        }
                     }
                 });
                 if (row_ok) {
                     constexpr uint32_t e0 = (uint32_t)Y::reg_off(P_LAST, m * RL);
-                    uint8_t* dst = crow + (((toff | e0) * MODE) >> 3);
+                    uint8_t* dst = crow + (kPackNibbles ? ((toff | e0) >> 1) : (toff | e0));
+                    if constexpr (kInterleaved) {
+                        // 32-row interleaved layout: 16-code chunk c of row m at
+                        // (((m / 32) * (K / 16) + c) * 32 + m % 32) * 16
+                        const uint32_t ein = (toff | e0) & (uint32_t)(K - 1);
+                        dst = p.codes + (((row >> 5) * (int64_t)(K >> 4) + (ein >> 4)) << 9) +
+                              ((row & 31) << 4) + (ein & 15u);
+                    }
                     if constexpr (BYTES == 2) {
                         *reinterpret_cast<uint16_t*>(dst) = (uint16_t)wv[0];
                     } else if constexpr (BYTES == 4) {
@@ -548,14 +579,15 @@ __global__ void __launch_bounds__(Cfg<L>::kCtaThreads, Cfg<L>::kMinBlocks)
                     } else {
                         static_for<0, BYTES / 16>([&](auto vv) {
                             constexpr int v = decltype(vv)::value;
-                            *reinterpret_cast<uint4*>(dst + 16 * v) =
+                            constexpr int step = kInterleaved ? 512 : 16;  // next 16-code chunk
+                            *reinterpret_cast<uint4*>(dst + step * v) =
                                 make_uint4(wv[4 * v], wv[4 * v + 1], wv[4 * v + 2], wv[4 * v + 3]);
                         });
                     }
                 }
             });
-            // sum of codes: each term is 0x4B400000 + q (mod 2^32)
-            int qs = (int)(qsum - (uint32_t)R * 0x4B400000u);
+            // sum of codes: each term is kMagicBits + q (mod 2^32)
+            int qs = (int)(qsum - (uint32_t)R * (uint32_t)kMagicBits);
             qs = row_isum(qs);
 
             if (row_ok) {

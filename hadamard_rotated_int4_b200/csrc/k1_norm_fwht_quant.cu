@@ -22,6 +22,10 @@ extern template hbl_status dispatch<0, false>(int, const Params&, cudaStream_t, 
 extern template hbl_status dispatch<0, true>(int, const Params&, cudaStream_t, int);
 extern template hbl_status dispatch<4, false>(int, const Params&, cudaStream_t, int);
 extern template hbl_status dispatch<4, true>(int, const Params&, cudaStream_t, int);
+extern template hbl_status dispatch<5, false>(int, const Params&, cudaStream_t, int);
+extern template hbl_status dispatch<5, true>(int, const Params&, cudaStream_t, int);
+extern template hbl_status dispatch<9, false>(int, const Params&, cudaStream_t, int);
+extern template hbl_status dispatch<9, true>(int, const Params&, cudaStream_t, int);
 extern template hbl_status dispatch<8, false>(int, const Params&, cudaStream_t, int);
 extern template hbl_status dispatch<8, true>(int, const Params&, cudaStream_t, int);
 }  // namespace k1
@@ -50,6 +54,10 @@ hbl_status launch_norm_fwht_quant(const uint16_t* X, const float* gain, int64_t 
                          : k1::dispatch<0, false>(L, prm, stream, num_sms);
         case 4: return g ? k1::dispatch<4, true>(L, prm, stream, num_sms)
                          : k1::dispatch<4, false>(L, prm, stream, num_sms);
+        case 5: return g ? k1::dispatch<5, true>(L, prm, stream, num_sms)
+                         : k1::dispatch<5, false>(L, prm, stream, num_sms);
+        case 9: return g ? k1::dispatch<9, true>(L, prm, stream, num_sms)
+                         : k1::dispatch<9, false>(L, prm, stream, num_sms);
         case 8: return g ? k1::dispatch<8, true>(L, prm, stream, num_sms)
                          : k1::dispatch<8, false>(L, prm, stream, num_sms);
         default: return HBL_ERR_INVALID_ARG;

@@ -77,12 +77,25 @@ HBL_API int hbl_version(void);
 
 /* Choice of ternary-GEMM back end (test and tuning aid; process-wide, not
  * synchronised with calls in flight on other threads):
- *   0 = automatic (CUDA-core split-K GEMV for M <= 8 tokens, tcgen05 tensor
- *       cores otherwise), 1 = always tensor cores, 2 = always the GEMV path
- *       (large M runs in chunks of 8 tokens).
+ *   0 = automatic (CUDA-core split-K GEMV for M <= 8 tokens, otherwise the
+ *       tcgen05 kernel with activations in tensor memory),
+ *   1 = tcgen05 with both operands in shared memory,
+ *   2 = always the GEMV path (large M runs in chunks of 8 tokens),
+ *   3 = always the tcgen05 kernel with activations in tensor memory.
  * hbl_workspace_size() answers for the path in force.  Returns HBL_OK or
  * HBL_ERR_INVALID_ARG.  This call has no counterpart on the BitNet v2 pages. */
 HBL_API int hbl_set_gemm_path(int path);
+
+/* act_bits also accepts these two values: the same INT4 / INT8 codes stored
+ * one byte per code (two's complement) in a 32-row interleaved layout.  Rows
+ * are padded to a multiple of 32 (the buffer holds ceil(M/32)*32*K bytes; the
+ * padding rows are neither written nor used), and the 16-code chunk c of row m
+ * starts at byte (((m / 32) * (K / 16) + c) * 32 + m % 32) * 16.  A warp that
+ * owns 32 consecutive rows reads each chunk as 512 contiguous bytes; the
+ * tensor-core GEMM takes this layout without widening, and
+ * hbl_hbitlinear_forward uses it internally.  hbl_ternary_gemm always runs its
+ * tcgen05 kernel for these layouts, whatever hbl_set_gemm_path says. */
+enum { HBL_ACT_INT4_I32 = 0x104, HBL_ACT_INT8_I32 = 0x108 };
 
 /* Operation identifiers for hbl_workspace_size(). */
 enum {

@@ -60,7 +60,7 @@ def test_workspace_sizes():
     try:
         M, K, N = 8192, 16384, 4096
         got = hbl.workspace_size(hbl.OP_HBITLINEAR_FORWARD, M, K, N, 4)
-        assert got == M * K // 2 + 2 * M * 4
+        assert got == M * K + 2 * M * 4  # codes one byte each inside the layer (M % 32 == 0)
         got8 = hbl.workspace_size(hbl.OP_HBITLINEAR_FORWARD, M, K, N, 8)
         assert got8 == M * K + 2 * M * 4
         hio = hbl.workspace_size(hbl.OP_HBITLINEAR_FORWARD_HOSTIO, M, K, N, 4)

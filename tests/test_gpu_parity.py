@@ -131,6 +131,56 @@ def test_quant_deterministic():
         assert torch.equal(c, c0) and torch.equal(s, s0) and torch.equal(r, r0)
 
 
+# ------------------------------------------- interleaved one-byte code layout
+
+def il_decode(buf, M, K):
+    """[ceil32(M), K] bytes in the 32-row interleaved layout -> int8 [M, K]."""
+    Mp = (M + 31) // 32 * 32
+    b = np.asarray(buf, dtype=np.uint8).reshape(Mp // 32, K // 16, 32, 16)
+    return b.transpose(0, 2, 1, 3).reshape(Mp, K)[:M].view(np.int8)
+
+
+def il_encode(q, K):
+    M = q.shape[0]
+    Mp = (M + 31) // 32 * 32
+    full = np.zeros((Mp, K), dtype=np.int8)
+    full[:M] = q
+    return np.ascontiguousarray(
+        full.view(np.uint8).reshape(Mp // 32, 32, K // 16, 16).transpose(0, 2, 1, 3)).reshape(Mp, K)
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("K", [16, 128, 256, 2048, 4096, 16384])
+def test_quant_interleaved_layout(bits, K):
+    M = 45
+    X = acts(M, K, seed=K + 1, kind="t")
+    flag = hbl.ACT_INT4_I32 if bits == 4 else hbl.ACT_INT8_I32
+    codes, scales, rowsum = hbl.norm_fwht_quant(to_dev_bf16(X), flag)
+    torch.cuda.synchronize()
+    wc, ws, wr = oracle.norm_fwht_quant(X, bits)
+    assert codes.shape == ((M + 31) // 32 * 32, K)
+    assert np.array_equal(il_decode(codes.cpu().numpy(), M, K), oracle.decode_codes(wc, K, bits))
+    assert np.array_equal(scales.cpu().numpy().view(np.uint32), ws.view(np.uint32))
+    assert np.array_equal(rowsum.cpu().numpy(), wr)
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("M,K,N", [(1, 16, 16), (45, 128, 272), (300, 4096, 256), (520, 2048, 400)])
+def test_gemm_interleaved_layout(bits, M, K, N):
+    codes, scales, rowsum, packed, alpha = make_gemm_case(M, K, N, bits, seed=M)
+    q = oracle.decode_codes(codes, K, bits)
+    flag = hbl.ACT_INT4_I32 if bits == 4 else hbl.ACT_INT8_I32
+    Y, acc = hbl.ternary_gemm(
+        torch.from_numpy(il_encode(q, K)).to(DEV), torch.from_numpy(scales).to(DEV),
+        torch.from_numpy(rowsum).to(DEV), flag, K,
+        torch.from_numpy(packed.view(np.int32)).to(DEV),
+        torch.from_numpy(np.array([alpha, 0, 0, 0], dtype=np.float32)).to(DEV), want_acc=True)
+    torch.cuda.synchronize()
+    wY, wacc = oracle.ternary_gemm(codes, scales, bits, K, packed, alpha)
+    assert np.array_equal(acc.cpu().numpy(), wacc)
+    assert np.array_equal(bf16_bits(Y), wY)
+
+
 # ------------------------------------------------------------ ternary pack
 
 @pytest.mark.parametrize("N,K", [(16, 16), (48, 256), (128, 256), (100, 2048), (4096, 4096),
@@ -168,7 +218,7 @@ def run_gemm(codes, scales, rowsum, bits, K, packed, alpha, path):
     return bf16_bits(Y), acc.cpu().numpy()
 
 
-@pytest.mark.parametrize("path", [1, 2])
+@pytest.mark.parametrize("path", [1, 2, 3])
 @pytest.mark.parametrize("bits", [4, 8])
 @pytest.mark.parametrize("M,K,N", [(1, 256, 128), (3, 16, 16), (8, 64, 48), (9, 128, 272),
                                    (127, 256, 256), (128, 512, 256), (129, 2048, 512),
@@ -189,8 +239,9 @@ def test_gemm_identity_weights(bits):
     K = 256
     codes, scales, rowsum, _, _ = make_gemm_case(130, K, 16, bits)
     pI = oracle.pack_codes(np.eye(K, dtype=np.int8))
-    Y, acc = run_gemm(codes, scales, rowsum, bits, K, pI, np.float32(1.0), 1)
-    assert np.array_equal(acc, oracle.decode_codes(codes, K, bits).astype(np.int32))
+    for path in (1, 3):
+        Y, acc = run_gemm(codes, scales, rowsum, bits, K, pI, np.float32(1.0), path)
+        assert np.array_equal(acc, oracle.decode_codes(codes, K, bits).astype(np.int32))
 
 
 # ------------------------------------------------------------ whole layer
@@ -211,7 +262,7 @@ def forward(X, packed, alpha, bits, path=0):
 def test_forward_tiny_workload(bits):
     X = inputs.activations("tiny")
     packed, alpha = oracle.pack_ternary(inputs.weights("tiny"))
-    for path in (0, 1, 2):
+    for path in (0, 1, 2, 3):
         Y = forward(X, packed, alpha, bits, path)
         assert np.array_equal(Y, oracle.hbitlinear_forward(X, packed, alpha, bits))
 
