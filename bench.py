@@ -315,6 +315,40 @@ def run_hbl(args):
                                "us": t * 1e6, "bytes": nbytes, "achieved_gbs": gbs,
                                "frac": gbs / pk["hbm_gbs"]}
     del qX
+
+    # ---- decode-batch sweep: T tokens through the whole layer, Wo 4096x4096 and
+    # W_down 4096x16384; weight copies rotate so the packed weights (4.2 / 16.8 MB)
+    # come from HBM (copies total > 2x L2)
+    decode = []
+    for shape, Kd in (("wo", 4096), ("wdown", 16384)):
+        Wd = torch.from_numpy(inputs.latent_weights(N_OUT, Kd, seed=7)).to(dev)
+        p0, a0 = hbl.pack_ternary(Wd)
+        del Wd
+        ncopy = max(2, int(2.2 * 126e6 // (N_OUT * Kd // 4)) + 1)
+        pcs = [p0.clone() for _ in range(ncopy)]
+        for T in inputs.DECODE_TOKENS:
+            Xt = torch.from_numpy(inputs.activations("decode_" + shape, M=T, K=Kd, seed=T).view(
+                np.int16)).view(torch.bfloat16).to(dev)
+            wsd = torch.empty(max(16, hbl.workspace_size(hbl.OP_HBITLINEAR_FORWARD, T, Kd, N_OUT,
+                                                         BITS)), dtype=torch.uint8, device=dev)
+            Yt = torch.empty((T, N_OUT), dtype=torch.bfloat16, device=dev)
+            for i in range(5):
+                hbl.hbitlinear_forward(Xt, pcs[i % ncopy], a0, BITS, ws=wsd, out=Yt)
+            iters = 200
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize()
+            a.record(stream)
+            for i in range(iters):
+                hbl.hbitlinear_forward(Xt, pcs[i % ncopy], a0, BITS, ws=wsd, out=Yt)
+            b.record(stream)
+            torch.cuda.synchronize()
+            t = a.elapsed_time(b) * 1e-3 / iters
+            wbytes = N_OUT * Kd // 4
+            decode.append({"shape": shape, "T": T, "K": Kd, "N": N_OUT, "us": t * 1e6,
+                           "tokens_per_s": T / t, "packed_w_gbs": wbytes / t / 1e9,
+                           "frac_hbm_on_packed_w": wbytes / t / 1e9 / pk["hbm_gbs"],
+                           "path": "gemv (dp4a split-K)" if T <= 8 else "gemm_ts"})
+        del pcs
     clocks = sampler.stop()
 
     # ---- end to end through the host-buffer call: H2D X, forward, D2H Y
@@ -370,6 +404,7 @@ def run_hbl(args):
         "roofline": roof,
         "kernels_us": {"norm_fwht_quant": t_k1 * 1e6, "ternary_gemm_ts": t_k2 * 1e6},
         "quant": quant,
+        "decode": decode,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": M_TOK * K_IN * 2,
                 "d2h_bytes_per_step": M_TOK * N_OUT * 2, "steps": e2e_steps,
                 "api": "hbl_hbitlinear_forward_hostio (pinned host buffers)"},

@@ -42,10 +42,16 @@ namespace k1 {
 constexpr int kRegLog = 7;
 constexpr int kRedFloats = 128;  // per-group cross-warp reduction scratch
 
+// log2 of the fp32 values each thread holds: 128 in general; 64 for K = 8192
+// and 16384, where it keeps two exchanges while doubling the resident warps.
+__host__ __device__ constexpr int reg_log(int L) {
+    return (L == 13 || L == 14) ? 6 : (L < kRegLog ? L : kRegLog);
+}
+
 template <int L>
 struct Cfg {
     static constexpr int K = 1 << L;
-    static constexpr int r = L < kRegLog ? L : kRegLog;
+    static constexpr int r = reg_log(L);
     static constexpr int R = 1 << r;           // values per thread
     static constexpr int t = L - r;            // thread bits of a row
     static constexpr int T = 1 << t;           // threads per row
@@ -55,26 +61,34 @@ struct Cfg {
     static constexpr int kCtaThreads = kGroupsPerCta * W;
     static constexpr int kLaneBits = t < 5 ? t : 5;
     static constexpr int kWarpBits = t > 5 ? t - 5 : 0;
-    static constexpr int kPasses = L <= kRegLog ? 0 : (L - kRegLog + 4) / 5;
+    static constexpr int kStagesPerPass = r - 2;  // index bits 0 and 1 stay in registers
+    static constexpr int kPasses = L <= r ? 0 : (L - r + kStagesPerPass - 1) / kStagesPerPass;
     static constexpr int kBufBytes = kRowsPerGroup * K * 4;  // fp32 row(s) of the group
     static constexpr int kStageShift = ilog2(R / 8);         // chunks per thread = R/8
     static constexpr int kSmemBytes = kGroupsPerCta * (kBufBytes + kRedFloats * 4);
     // 3 CTAs (12 warps) per SM where the register budget (170) suffices
-    static constexpr int kMinBlocks = kCtaThreads >= 256 ? 1 : ((L >= 8 && L != 12) ? 2 : 3);
+    static constexpr int kMinBlocks =
+        r == 6 ? (kCtaThreads >= 256 ? 2 : 4) : (kCtaThreads >= 256 ? 1 : ((L >= 8 && L != 12) ? 2 : 3));
 };
 
-// Layout p: 0 = natural, p >= 1 = pass p (stage base 7 + 5 (p - 1)).
+// Layout p: 0 = natural, p >= 1 = pass p (stage base r + (r - 2)(p - 1)).
 template <int L>
 struct Lay {
     using C = Cfg<L>;
+    __host__ __device__ static constexpr int pass_base(int p) {
+        return C::r + C::kStagesPerPass * (p - 1);
+    }
+    __host__ __device__ static constexpr int pass_count(int p) {
+        return (L - pass_base(p)) < C::kStagesPerPass ? (L - pass_base(p)) : C::kStagesPerPass;
+    }
     __host__ __device__ static constexpr uint32_t reg_mask(int p) {
         if (p == 0) return (1u << C::r) - 1u;
-        int b = kRegLog + 5 * (p - 1);
-        int n = (L - b) < 5 ? (L - b) : 5;
+        int b = pass_base(p);
+        int n = pass_count(p);
         uint32_t m = 3u;
         for (int s = b; s < b + n; ++s) m |= 1u << s;
         int cnt = 2 + n;
-        for (int f = 2; cnt < kRegLog; ++f)
+        for (int f = 2; cnt < C::r; ++f)
             if (!((m >> f) & 1u)) {
                 m |= 1u << f;
                 ++cnt;
@@ -402,8 +416,8 @@ __global__ void __launch_bounds__(Cfg<L>::kCtaThreads, Cfg<L>::kMinBlocks)
                 });
             }
             group_sync<T>(grp);
-            constexpr int b = kRegLog + 5 * (P - 1);
-            constexpr int n = (L - b) < 5 ? (L - b) : 5;
+            constexpr int b = Y::pass_base(P);
+            constexpr int n = Y::pass_count(P);
             static_for<0, n>([&](auto ss_) {
                 constexpr int s = b + decltype(ss_)::value;
                 stage_regs<R, Y::reg_bit_of(P, s)>(d);

@@ -74,10 +74,22 @@ __device__ __forceinline__ bool mbar_wait(uint32_t a, uint32_t parity) {
         if (gtime() - t0 > kTimeoutNs) return false;
     }
 }
+// Bounded wait that backs off with a short sleep between polls, so a waiting
+// lane does not take issue slots from the warps that share its scheduler.
+__device__ __forceinline__ bool mbar_wait_backoff(uint32_t a, uint32_t parity) {
+    if (mbar_try(a, parity)) return true;
+    const uint64_t t0 = gtime();
+    while (true) {
+        __nanosleep(64);
+        if (mbar_try(a, parity)) return true;
+        if (gtime() - t0 > kTimeoutNs) return false;
+    }
+}
 // Warp-uniform bounded wait: lane 0 waits, every lane gets its verdict.
+template <bool BACKOFF = false>
 __device__ __forceinline__ bool warp_wait(uint32_t a, uint32_t parity) {
     bool ok = true;
-    if ((threadIdx.x & 31) == 0) ok = mbar_wait(a, parity);
+    if ((threadIdx.x & 31) == 0) ok = BACKOFF ? mbar_wait_backoff(a, parity) : mbar_wait(a, parity);
     return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
 }
 __device__ __forceinline__ void tc_fence_before() {
@@ -207,6 +219,28 @@ __device__ __forceinline__ void load_stage(const ConvPtrs& cp, int K, int kb, Pa
     P.b = b;
 }
 
+// Loader for K % 128 == 0: no guards (rows past M or N read a valid row whose
+// results are never stored), running pointers, immediate offsets.
+template <int ABITS, bool IL>
+struct FastLoader {
+    const uint8_t* a;
+    const uint32_t* b;
+    __device__ __forceinline__ void load(Packed<ABITS>& P) {
+        if constexpr (ABITS == 8) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                P.a[i] = *reinterpret_cast<const uint4*>(a + (IL ? 512 * i : 16 * i));
+            a += IL ? 8 * 512 : BK;
+        } else {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) P.a[i] = *reinterpret_cast<const uint4*>(a + 16 * i);
+            a += BK / 2;
+        }
+        P.b = *reinterpret_cast<const uint4*>(b);
+        b += BK / 16;
+    }
+};
+
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
     asm volatile(
         "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
@@ -256,7 +290,7 @@ __device__ __forceinline__ void store_stage(uint32_t a_taddr, uint32_t sB, const
     }
 }
 
-template <int ABITS, bool IL>
+template <int ABITS, bool IL, bool FULLK>
 __global__ void __launch_bounds__(kThreads, 1) gemm_ts_kernel(Params p) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_s = smem_addr(smem_raw);
@@ -302,7 +336,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_ts_kernel(Params p) {
         bool ok = true;
         for (int kb = 0; kb < num_kb; ++kb) {
             const int s = kb % S;
-            if (!warp_wait(full_bar(s), (uint32_t)((kb / S) & 1))) {
+            if (!warp_wait<true>(full_bar(s), (uint32_t)((kb / S) & 1))) {
                 ok = false;
                 break;
             }
@@ -357,7 +391,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_ts_kernel(Params p) {
         auto stage = [&](int kb, const Packed<ABITS>& P) -> bool {
             const int s = kb % S;
             bool go = true;
-            if (kb >= S) go = warp_wait(empty_bar(s), (uint32_t)(((kb / S) - 1) & 1));
+            if (kb >= S) go = warp_wait<true>(empty_bar(s), (uint32_t)(((kb / S) - 1) & 1));
             go = go && (__shfl_sync(0xffffffffu, *abort_flag, 0) == 0);
             if (!go) return false;  // warp-uniform
             tc_fence_after();
@@ -369,19 +403,60 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_ts_kernel(Params p) {
             return true;
         };
         Packed<ABITS> P0, P1;
-        load_stage<ABITS, IL>(cp, p.K, 0, P0);
         bool ok = true;
-        for (int kb = 0; kb < num_kb; kb += 2) {
-            if (kb + 1 < num_kb) load_stage<ABITS, IL>(cp, p.K, kb + 1, P1);
-            if (!stage(kb, P0)) {
-                ok = false;
-                break;
+        if constexpr (FULLK) {
+            FastLoader<ABITS, IL> ld;
+            {
+                int64_t mm = m;
+                if constexpr (IL) {
+                    const int64_t mpad = (p.M + 31) & ~(int64_t)31;
+                    if (mm >= mpad) mm = mpad - 1;
+                    ld.a = p.codes + (((mm >> 5) * (int64_t)(p.K >> 4)) << 9) + ((mm & 31) << 4);
+                } else {
+                    if (mm >= p.M) mm = p.M - 1;
+                    ld.a = p.codes + mm * (int64_t)(ABITS == 8 ? p.K : p.K / 2);
+                }
+                const int nn = n < p.N ? n : p.N - 1;
+                ld.b = p.W + (int64_t)nn * (p.K / 16) + 4 * bh;
             }
-            if (kb + 1 >= num_kb) break;
-            if (kb + 2 < num_kb) load_stage<ABITS, IL>(cp, p.K, kb + 2, P0);
-            if (!stage(kb + 1, P1)) {
-                ok = false;
-                break;
+            // three stages of operands in flight in registers
+            Packed<ABITS> P2;
+            ld.load(P0);
+            if (num_kb > 1) ld.load(P1);
+            if (num_kb > 2) ld.load(P2);
+            for (int kb = 0; kb < num_kb; kb += 3) {
+                if (!stage(kb, P0)) {
+                    ok = false;
+                    break;
+                }
+                if (kb + 3 < num_kb) ld.load(P0);
+                if (kb + 1 >= num_kb) break;
+                if (!stage(kb + 1, P1)) {
+                    ok = false;
+                    break;
+                }
+                if (kb + 4 < num_kb) ld.load(P1);
+                if (kb + 2 >= num_kb) break;
+                if (!stage(kb + 2, P2)) {
+                    ok = false;
+                    break;
+                }
+                if (kb + 5 < num_kb) ld.load(P2);
+            }
+        } else {
+            load_stage<ABITS, IL>(cp, p.K, 0, P0);
+            for (int kb = 0; kb < num_kb; kb += 2) {
+                if (kb + 1 < num_kb) load_stage<ABITS, IL>(cp, p.K, kb + 1, P1);
+                if (!stage(kb, P0)) {
+                    ok = false;
+                    break;
+                }
+                if (kb + 1 >= num_kb) break;
+                if (kb + 2 < num_kb) load_stage<ABITS, IL>(cp, p.K, kb + 2, P0);
+                if (!stage(kb + 1, P1)) {
+                    ok = false;
+                    break;
+                }
             }
         }
         if (!ok && lane == 0) {
@@ -458,7 +533,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_ts_kernel(Params p) {
 
 template <int ABITS, bool IL>
 static hbl_status launch(const Params& prm, cudaStream_t stream) {
-    auto kern = gemm_ts_kernel<ABITS, IL>;
+    auto kern = (prm.K % BK == 0) ? gemm_ts_kernel<ABITS, IL, true>
+                                  : gemm_ts_kernel<ABITS, IL, false>;
     if (!smem_attr_once(reinterpret_cast<const void*>(kern), kSmemBytes)) return HBL_ERR_CUDA;
     dim3 grid((prm.N + BN - 1) / BN, (unsigned)((prm.M + BM - 1) / BM));
     kern<<<grid, kThreads, kSmemBytes, stream>>>(prm);
