@@ -334,20 +334,34 @@ def run_hbl(args):
             Yt = torch.empty((T, N_OUT), dtype=torch.bfloat16, device=dev)
             for i in range(5):
                 hbl.hbitlinear_forward(Xt, pcs[i % ncopy], a0, BITS, ws=wsd, out=Yt)
-            iters = 200
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             torch.cuda.synchronize()
+            # one CUDA graph holds one forward per weight copy; replays remove the
+            # host launch cost that would otherwise dominate a decode step
+            graph = torch.cuda.CUDAGraph()
+            cap = torch.cuda.Stream()
+            cap.wait_stream(stream)
+            with torch.cuda.stream(cap):
+                with torch.cuda.graph(graph, stream=cap):
+                    for i in range(ncopy):
+                        hbl.hbitlinear_forward(Xt, pcs[i], a0, BITS, ws=wsd, out=Yt)
+            stream.wait_stream(cap)
+            graph.replay()
+            torch.cuda.synchronize()
+            reps = max(3, 400 // ncopy)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record(stream)
-            for i in range(iters):
-                hbl.hbitlinear_forward(Xt, pcs[i % ncopy], a0, BITS, ws=wsd, out=Yt)
+            for _ in range(reps):
+                graph.replay()
             b.record(stream)
             torch.cuda.synchronize()
-            t = a.elapsed_time(b) * 1e-3 / iters
+            t = a.elapsed_time(b) * 1e-3 / (reps * ncopy)
+            del graph
             wbytes = N_OUT * Kd // 4
             decode.append({"shape": shape, "T": T, "K": Kd, "N": N_OUT, "us": t * 1e6,
                            "tokens_per_s": T / t, "packed_w_gbs": wbytes / t / 1e9,
                            "frac_hbm_on_packed_w": wbytes / t / 1e9 / pk["hbm_gbs"],
-                           "path": "gemv (dp4a split-K)" if T <= 8 else "gemm_ts"})
+                           "path": "gemv (dp4a split-K)" if T <= 8 else "gemm_ts split-K",
+                           "timing": "CUDA graph replay, one forward per weight copy"})
         del pcs
     clocks = sampler.stop()
 

@@ -74,7 +74,7 @@ bool use_gemv(int64_t M) {
 }
 
 size_t gemm_ws(int64_t M, int K, int N, int sms_guess) {
-    if (!use_gemv(M)) return 0;
+    if (!use_gemv(M)) return g_path.load() == 1 ? 0 : gemm_ts_workspace(M, K, N);
     const int64_t mchunk = M < gemv_max_m() ? M : gemv_max_m();
     return gemv_workspace(mchunk, K, N, sms_guess);
 }
@@ -85,7 +85,8 @@ constexpr int kSizingSms = 148;
 
 hbl_status run_gemm(const GemmArgs& a, void* ws, size_t ws_bytes, cudaStream_t s, int sms) {
     if (!use_gemv(a.M))
-        return g_path.load() == 1 ? launch_gemm_tc(a, s, sms) : launch_gemm_ts(a, s, sms);
+        return g_path.load() == 1 ? launch_gemm_tc(a, s, sms)
+                                  : launch_gemm_ts(a, ws, ws_bytes, s, sms);
     // CUDA-core path in chunks of up to gemv_max_m() tokens (workspace reused in order)
     const int64_t step = gemv_max_m();
     for (int64_t r0 = 0; r0 < a.M; r0 += step) {
@@ -163,7 +164,8 @@ hbl_status hbl_workspace_size(int op, int M, int K, int N, int act_bits, size_t*
             if (M < 0 || check_k(K) != HBL_OK || check_n(N) != HBL_OK) return HBL_ERR_SHAPE;
             if (!act_valid(act_bits)) return HBL_ERR_INVALID_ARG;
             if (op != HBL_OP_TERNARY_GEMM && act_il(act_bits)) return HBL_ERR_INVALID_ARG;
-            size_t b = act_il(act_bits) ? 0 : up256(gemm_ws(M, K, N, kSizingSms));
+            size_t b = act_il(act_bits) ? up256(gemm_ts_workspace(M, K, N))
+                                        : up256(gemm_ws(M, K, N, kSizingSms));
             if (op != HBL_OP_TERNARY_GEMM) {
                 b += up256((size_t)((M + 31) & ~31) * K);  // codes, one byte each, rows padded to 32
                 b += up256((size_t)M * 4) * 2;                         // scales, rowsum
@@ -251,7 +253,7 @@ hbl_status hbl_ternary_gemm(const void* codes, const float* scales, const int32_
         !aligned16(alpha) || !aligned16(Y) || (acc_out && !aligned16(acc_out)) ||
         (dev_status && !aligned16(dev_status)))
         return HBL_ERR_ALIGNMENT;
-    const size_t need = act_il(act_bits) ? 0 : gemm_ws(M, K, N, kSizingSms);
+    const size_t need = act_il(act_bits) ? gemm_ts_workspace(M, K, N) : gemm_ws(M, K, N, kSizingSms);
     if (need > 0 && (ws == nullptr || ws_bytes < need)) return HBL_ERR_WORKSPACE;
     if (ws && !aligned16(ws)) return HBL_ERR_ALIGNMENT;
     int sms = 0;
@@ -260,7 +262,7 @@ hbl_status hbl_ternary_gemm(const void* codes, const float* scales, const int32_
     if (act_il(act_bits)) {  // interleaved one-byte codes: the TMEM-activation kernel
         GemmArgs a{codes, scales, rowsum, 8, M, K, W_packed, alpha, N, Y, acc_out, dev_status};
         a.interleaved = true;
-        return launch_gemm_ts(a, static_cast<cudaStream_t>(stream), sms);
+        return launch_gemm_ts(a, ws, ws_bytes, static_cast<cudaStream_t>(stream), sms);
     }
     GemmArgs a{codes, scales, rowsum, act_bits, M, K, W_packed, alpha, N, Y, acc_out, dev_status};
     return run_gemm(a, ws, ws_bytes, static_cast<cudaStream_t>(stream), sms);

@@ -44,8 +44,16 @@ struct GemmArgs {
 
 // K2: tcgen05 tensor-core GEMM, both operands in shared memory, any M.
 hbl_status launch_gemm_tc(const GemmArgs& a, cudaStream_t stream, int num_sms);
-// K2b: tcgen05 tensor-core GEMM with the activations in TMEM, any M.
-hbl_status launch_gemm_ts(const GemmArgs& a, cudaStream_t stream, int num_sms);
+// K2b: tcgen05 tensor-core GEMM with the activations in TMEM, any M.  For
+// M <= 256 it splits K over CTAs and needs gemm_ts_workspace() bytes of ws.
+int gemm_ts_ksplit(int64_t M, int K, int N);
+size_t gemm_ts_workspace(int64_t M, int K, int N);
+hbl_status launch_gemm_ts(const GemmArgs& a, void* ws, size_t ws_bytes, cudaStream_t stream,
+                          int num_sms);
+// Sum int32 split-K partials [ksplit][M][N], subtract rowsum, dequantise to bf16.
+hbl_status launch_splitk_epilogue(const int32_t* part, int ksplit, int64_t M, int N,
+                                  const int32_t* rowsum, const float* scales, const float* alpha,
+                                  uint16_t* Y, int32_t* acc_out, cudaStream_t stream);
 
 // K3: CUDA-core split-K GEMV for small M (M <= gemv_max_m()).
 int gemv_max_m();

@@ -154,6 +154,8 @@ struct Params {
     uint16_t* Y;
     int32_t* acc_out;
     int32_t* status;
+    int32_t* part;  // split-K: raw int32 partials [gridDim.z][M][N] (null: full epilogue)
+    int kps;        // K-blocks per split
 };
 
 template <int ABITS>
@@ -308,7 +310,12 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_ts_kernel(Params p) {
     const int warp = tid >> 5, lane = tid & 31;
     const int n0 = blockIdx.x * BN;
     const int64_t m0 = (int64_t)blockIdx.y * BM;
-    const int num_kb = (p.K + BK - 1) / BK;
+    // this CTA's K-blocks: [kb0, kb0 + num_kb) of the whole K (split-K over grid.z)
+    const int num_kb_total = (p.K + BK - 1) / BK;
+    const int kb0 = (int)blockIdx.z * p.kps;
+    const int num_kb = min(p.kps, num_kb_total - kb0);
+    // rows of this tile that exist: one accumulator suffices when M - m0 <= 128
+    const int nacc = (p.M - m0 > 128) ? 2 : 1;
 
     if (tid == 0) {
         for (int s = 0; s < S; ++s) {
@@ -348,7 +355,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_ts_kernel(Params p) {
                     const uint64_t bd = sdesc(sB + 32 * k);
 #pragma unroll
                     for (int a = 0; a < 2; ++a)
-                        mma_ts(tmem + 128u * a, tmem + 256u + 32u * (2 * s + a) + 8u * k, bd,
+                        if (a < nacc)
+                            mma_ts(tmem + 128u * a, tmem + 256u + 32u * (2 * s + a) + 8u * k, bd,
                                (kb > 0 || k > 0) ? 1u : 0u);
                 }
                 mma_commit(empty_bar(s));
@@ -418,6 +426,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_ts_kernel(Params p) {
                 }
                 const int nn = n < p.N ? n : p.N - 1;
                 ld.b = p.W + (int64_t)nn * (p.K / 16) + 4 * bh;
+                ld.a += (int64_t)kb0 * (IL ? 8 * 512 : (ABITS == 8 ? BK : BK / 2));
+                ld.b += kb0 * (BK / 16);
             }
             // three stages of operands in flight in registers
             Packed<ABITS> P2;
@@ -444,15 +454,15 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_ts_kernel(Params p) {
                 if (kb + 5 < num_kb) ld.load(P2);
             }
         } else {
-            load_stage<ABITS, IL>(cp, p.K, 0, P0);
+            load_stage<ABITS, IL>(cp, p.K, kb0, P0);
             for (int kb = 0; kb < num_kb; kb += 2) {
-                if (kb + 1 < num_kb) load_stage<ABITS, IL>(cp, p.K, kb + 1, P1);
+                if (kb + 1 < num_kb) load_stage<ABITS, IL>(cp, p.K, kb0 + kb + 1, P1);
                 if (!stage(kb, P0)) {
                     ok = false;
                     break;
                 }
                 if (kb + 1 >= num_kb) break;
-                if (kb + 2 < num_kb) load_stage<ABITS, IL>(cp, p.K, kb + 2, P0);
+                if (kb + 2 < num_kb) load_stage<ABITS, IL>(cp, p.K, kb0 + kb + 2, P0);
                 if (!stage(kb + 1, P1)) {
                     ok = false;
                     break;
@@ -489,6 +499,19 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_ts_kernel(Params p) {
                     : "r"(taddr));
                 asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
                 const int nc = n0 + 32 * cc;
+                if (p.part != nullptr) {  // split-K: raw partial sums, reduced by a second kernel
+                    if (mok && nc < p.N) {
+                        int4* pd = reinterpret_cast<int4*>(
+                            p.part + ((int64_t)blockIdx.z * p.M + m) * p.N + nc);
+                        const int nq = (p.N - nc) >= 32 ? 8 : 4;
+#pragma unroll
+                        for (int e = 0; e < 8; ++e)
+                            if (e < nq)
+                                pd[e] = make_int4((int)v[4 * e], (int)v[4 * e + 1], (int)v[4 * e + 2],
+                                                  (int)v[4 * e + 3]);
+                    }
+                    continue;
+                }
                 if (mok && nc < p.N) {
                     uint32_t out[16];
 #pragma unroll
@@ -536,16 +559,41 @@ static hbl_status launch(const Params& prm, cudaStream_t stream) {
     auto kern = (prm.K % BK == 0) ? gemm_ts_kernel<ABITS, IL, true>
                                   : gemm_ts_kernel<ABITS, IL, false>;
     if (!smem_attr_once(reinterpret_cast<const void*>(kern), kSmemBytes)) return HBL_ERR_CUDA;
-    dim3 grid((prm.N + BN - 1) / BN, (unsigned)((prm.M + BM - 1) / BM));
+    const int num_kb = (prm.K + BK - 1) / BK;
+    dim3 grid((prm.N + BN - 1) / BN, (unsigned)((prm.M + BM - 1) / BM),
+              (unsigned)((num_kb + prm.kps - 1) / prm.kps));
     kern<<<grid, kThreads, kSmemBytes, stream>>>(prm);
     return cudaGetLastError() == cudaSuccess ? HBL_OK : HBL_ERR_CUDA;
 }
 
 }  // namespace k2b
 
-hbl_status launch_gemm_ts(const GemmArgs& a, cudaStream_t stream, int /*num_sms*/) {
+// Split factor over K for one-tile-high problems (M <= 256), so that a decode
+// batch still fills the GPU: about two CTAs per SM, at least 4 K-blocks each.
+int gemm_ts_ksplit(int64_t M, int K, int N) {
+    if (M > k2b::BM) return 1;
+    const int tiles = (N + k2b::BN - 1) / k2b::BN;
+    const int num_kb = (K + k2b::BK - 1) / k2b::BK;
+    int ks = 1;
+    while (tiles * ks * 2 <= 2 * 148 && num_kb / (ks * 2) >= 4) ks *= 2;
+    return ks;
+}
+
+size_t gemm_ts_workspace(int64_t M, int K, int N) {
+    const int ks = gemm_ts_ksplit(M, K, N);
+    return ks > 1 ? (((size_t)ks * (size_t)M * (size_t)N * 4 + 255) & ~(size_t)255) : 0;
+}
+
+hbl_status launch_gemm_ts(const GemmArgs& a, void* ws, size_t ws_bytes, cudaStream_t stream,
+                          int /*num_sms*/) {
     if (a.M == 0) return HBL_OK;
+    const int ks = gemm_ts_ksplit(a.M, a.K, a.N);
+    const int num_kb = (a.K + k2b::BK - 1) / k2b::BK;
+    if (ks > 1 && (ws == nullptr || ws_bytes < gemm_ts_workspace(a.M, a.K, a.N)))
+        return HBL_ERR_WORKSPACE;
     k2b::Params prm;
+    prm.part = ks > 1 ? static_cast<int32_t*>(ws) : nullptr;
+    prm.kps = (num_kb + ks - 1) / ks;
     prm.codes = static_cast<const uint8_t*>(a.codes);
     prm.scales = a.scales;
     prm.rowsum = a.rowsum;
@@ -557,9 +605,17 @@ hbl_status launch_gemm_ts(const GemmArgs& a, cudaStream_t stream, int /*num_sms*
     prm.Y = a.Y;
     prm.acc_out = a.acc_out;
     prm.status = a.dev_status;
-    if (a.interleaved) return k2b::launch<8, true>(prm, stream);
-    if (a.act_bits == 4) return k2b::launch<4, false>(prm, stream);
-    return k2b::launch<8, false>(prm, stream);
+    hbl_status st;
+    if (a.interleaved)
+        st = k2b::launch<8, true>(prm, stream);
+    else if (a.act_bits == 4)
+        st = k2b::launch<4, false>(prm, stream);
+    else
+        st = k2b::launch<8, false>(prm, stream);
+    if (st != HBL_OK || ks == 1) return st;
+    const int nsplit = (num_kb + prm.kps - 1) / prm.kps;  // grid.z: every split has K-blocks
+    return launch_splitk_epilogue(prm.part, nsplit, a.M, a.N, a.rowsum, a.scales, a.alpha, a.Y,
+                                  a.acc_out, stream);
 }
 
 }  // namespace hbl

@@ -159,6 +159,17 @@ static int choose_ksplit(int K, int N, int num_sms) {
 
 int gemv_max_m() { return k3::kMaxM; }
 
+hbl_status launch_splitk_epilogue(const int32_t* part, int ksplit, int64_t M, int N,
+                                  const int32_t* rowsum, const float* scales, const float* alpha,
+                                  uint16_t* Y, int32_t* acc_out, cudaStream_t stream) {
+    const int64_t total = M * N;
+    int64_t eb = (total + 255) / 256;
+    if (eb > 148 * 8) eb = 148 * 8;
+    k3::gemv_epilogue_kernel<<<(unsigned)eb, 256, 0, stream>>>(part, ksplit, (int)M, N, rowsum,
+                                                               scales, alpha, Y, acc_out);
+    return cudaGetLastError() == cudaSuccess ? HBL_OK : HBL_ERR_CUDA;
+}
+
 size_t gemv_workspace(int64_t M, int K, int N, int num_sms) {
     const int ks = k3::choose_ksplit(K, N, num_sms);
     return ((size_t)ks * (size_t)M * (size_t)N * 4 + 255) & ~(size_t)255;

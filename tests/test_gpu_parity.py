@@ -317,6 +317,34 @@ def test_decode_sweep(T, shape):
     assert np.array_equal(Y[rows], want)
 
 
+@pytest.mark.parametrize("T,K", [(1, 4096), (32, 16384), (300, 2048)])
+def test_forward_replays_from_cuda_graph(T, K):
+    # the forward launches only on the caller's stream, so it can be captured
+    X = inputs.activations("decode_wdown", M=T, K=K, seed=3)
+    packed, alpha = oracle.pack_ternary(inputs.latent_weights(512, K, seed=2))
+    Xd = to_dev_bf16(X)
+    Pd = torch.from_numpy(packed.view(np.int32)).to(DEV)
+    Ad = torch.from_numpy(np.array([alpha, 0, 0, 0], dtype=np.float32)).to(DEV)
+    ws = torch.empty(max(16, hbl.workspace_size(hbl.OP_HBITLINEAR_FORWARD, T, K, 512, 4)),
+                     dtype=torch.uint8, device=DEV)
+    Y = torch.empty((T, 512), dtype=torch.bfloat16, device=DEV)
+    hbl.hbitlinear_forward(Xd, Pd, Ad, 4, ws=ws, out=Y)  # warm-up outside capture
+    torch.cuda.synchronize()
+    Y.zero_()
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            hbl.hbitlinear_forward(Xd, Pd, Ad, 4, ws=ws, out=Y)
+    torch.cuda.current_stream().wait_stream(s)
+    g.replay()
+    torch.cuda.synchronize()
+    rows = np.arange(min(T, 6))
+    assert np.array_equal(bf16_bits(Y)[rows],
+                          oracle.hbitlinear_forward(X, packed, alpha, 4, rows=rows))
+
+
 def test_hostio_matches_device_forward():
     X = inputs.activations("tiny")
     packed, alpha = oracle.pack_ternary(inputs.weights("tiny"))
