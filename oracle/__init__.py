@@ -25,6 +25,17 @@ Pins (what fixes each function other than itself; see tests/test_oracle_pins.py)
                      identity weights give acc = q; all-ones weights give acc = rowsum
   bf16 conversion    torch's float32 -> bfloat16 rounding
   outlier invariant  INT4 reconstruction error lower after the transform
+  norm_transform     LayerNorm: balanced-row closed form, shift invariance on exact
+                     integer rows, torch.nn.functional.layer_norm in fp64; the
+                     (RMS, Hadamard) case equals norm_fwht's pins; no-Hadamard case:
+                     torch rms_norm / layer_norm in fp64
+  norm_quant         the quantiser pins above, applied to the pinned transforms;
+                     codes vs a torch fp64 evaluation away from rounding ties
+  rotate_weights     dense product with scipy's Hadamard matrix and the signs (fp64,
+                     1e-6); (x D H)(w D H)^T = x w^T; involution with the signs
+  kv_quant           brute force against Python's round-half-even per element;
+                     exact ties; max element -> 2^b - 1 or 1; zero row; packing
+                     against Python big-integer bit strings; round trip
 No function is left with parity unpinned.
 """
 import ctypes
@@ -69,6 +80,12 @@ def _load():
             "oracle_pack_ternary": (I, [P, I, I, F, P, P]),
             "oracle_ternary_gemm_rows": (I, [P, P, I, I, I, P, F, I, I, I, P, P]),
             "oracle_hbitlinear_forward_rows": (I, [P, P, I, I, I, P, F, I, F, F, I, I, P]),
+            "oracle_norm_transform": (I, [P, P, I, I, F, I, I, P]),
+            "oracle_norm_quant": (I, [P, P, I, I, F, F, I, I, I, P, P, P]),
+            "oracle_bitlinear_forward_rows": (I, [P, P, I, I, I, P, F, I, F, F, I, I, I, I, P]),
+            "oracle_rotate_weights": (I, [P, P, I, I, P]),
+            "oracle_kv_quant": (I, [P, I64, I, I, F, P, P]),
+            "oracle_kv_unpack": (I, [P, I64, I, I, P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(lib, name)
@@ -330,3 +347,131 @@ def hbitlinear_forward(X_bits, packed, alpha, act_bits, gain=None, norm_eps=1e-6
         with ThreadPoolExecutor(nt) as ex:
             list(ex.map(run, _split(M, nt)))
     return Y
+
+
+# ------------------------------------------------------------------ variants
+
+def norm_transform(X_bits, gain=None, norm_eps=1e-6, layernorm=False, hadamard=True,
+                   threads=None):
+    """fp32 V = T(N(X)): RMSNorm or LayerNorm, then the normalised FWHT or nothing."""
+    X_bits = _c(X_bits, np.uint16)
+    M, K = X_bits.shape
+    g = None if gain is None else _c(gain, np.float32)
+    V = np.empty((M, K), dtype=np.float32)
+    lib = _load()
+
+    def run(r):
+        a, b = r
+        _check(lib.oracle_norm_transform(_p(X_bits[a:b]), _p(g), b - a, K, norm_eps,
+                                         int(layernorm), int(hadamard), _p(V[a:b])),
+               "norm_transform")
+
+    if M:
+        nt = _threads(M, threads)
+        with ThreadPoolExecutor(nt) as ex:
+            list(ex.map(run, _split(M, nt)))
+    return V
+
+
+def norm_quant(X_bits, act_bits, gain=None, norm_eps=1e-6, quant_eps=1e-5, layernorm=False,
+               hadamard=True, threads=None):
+    X_bits = _c(X_bits, np.uint16)
+    M, K = X_bits.shape
+    g = None if gain is None else _c(gain, np.float32)
+    codes = np.empty((M, code_bytes_per_row(K, act_bits)), dtype=np.uint8)
+    scales = np.empty(M, dtype=np.float32)
+    rowsum = np.empty(M, dtype=np.int32)
+    lib = _load()
+
+    def run(r):
+        a, b = r
+        _check(lib.oracle_norm_quant(_p(X_bits[a:b]), _p(g), b - a, K, norm_eps, quant_eps,
+                                     act_bits, int(layernorm), int(hadamard), _p(codes[a:b]),
+                                     _p(scales[a:b]), _p(rowsum[a:b])), "norm_quant")
+
+    if M:
+        nt = _threads(M, threads)
+        with ThreadPoolExecutor(nt) as ex:
+            list(ex.map(run, _split(M, nt)))
+    return codes, scales, rowsum
+
+
+def bitlinear_forward(X_bits, packed, alpha, act_bits, gain=None, norm_eps=1e-6,
+                      quant_eps=1e-5, layernorm=False, hadamard=True, rows=None, threads=None):
+    """Y (bf16 bits) of the layer with the variant choices of norm_transform."""
+    X_bits = _c(X_bits, np.uint16)
+    if rows is not None:
+        X_bits = np.ascontiguousarray(X_bits[np.asarray(rows, dtype=np.int64)])
+    packed = _c(packed, np.uint32)
+    M, K = X_bits.shape
+    N = packed.shape[0]
+    g = None if gain is None else _c(gain, np.float32)
+    Y = np.empty((M, N), dtype=np.uint16)
+    lib = _load()
+
+    def run(r):
+        a, b = r
+        _check(lib.oracle_bitlinear_forward_rows(_p(X_bits), _p(g), M, K, N, _p(packed),
+                                                 float(alpha), act_bits, norm_eps, quant_eps,
+                                                 int(layernorm), int(hadamard), a, b, _p(Y)),
+               "bitlinear_forward")
+
+    if M:
+        nt = _threads(M, threads)
+        with ThreadPoolExecutor(nt) as ex:
+            list(ex.map(run, _split(M, nt)))
+    return Y
+
+
+def rotate_weights(W, signs=None, threads=None):
+    """W_rot = FWHT(W * signs) / sqrt(K) row by row (fp32)."""
+    W = _c(W, np.float32)
+    N, K = W.shape
+    s = None if signs is None else _c(signs, np.float32)
+    out = np.empty((N, K), dtype=np.float32)
+    lib = _load()
+
+    def run(r):
+        a, b = r
+        _check(lib.oracle_rotate_weights(_p(W[a:b]), _p(s), b - a, K, _p(out[a:b])),
+               "rotate_weights")
+
+    if N:
+        nt = _threads(N, threads)
+        with ThreadPoolExecutor(nt) as ex:
+            list(ex.map(run, _split(N, nt)))
+    return out
+
+
+def kv_code_bytes(D, bits):
+    return D // 32 * 4 * bits
+
+
+def kv_quant(X_bits, bits, eps=1e-5, threads=None):
+    """Packed unsigned codes [rows x D*bits/8] and fp32 scales [rows] per head row."""
+    X_bits = _c(X_bits, np.uint16)
+    D = X_bits.shape[-1]
+    flat = X_bits.reshape(-1, D)
+    rows = flat.shape[0]
+    codes = np.empty((rows, kv_code_bytes(D, bits)), dtype=np.uint8)
+    scales = np.empty(rows, dtype=np.float32)
+    lib = _load()
+
+    def run(r):
+        a, b = r
+        _check(lib.oracle_kv_quant(_p(flat[a:b]), b - a, D, int(bits), float(eps),
+                                   _p(codes[a:b]), _p(scales[a:b])), "kv_quant")
+
+    if rows:
+        nt = _threads(rows, threads)
+        with ThreadPoolExecutor(nt) as ex:
+            list(ex.map(run, _split(rows, nt)))
+    return codes, scales
+
+
+def kv_unpack(codes, D, bits):
+    codes = _c(codes, np.uint8)
+    rows = codes.shape[0]
+    u = np.empty((rows, D), dtype=np.uint8)
+    _check(_load().oracle_kv_unpack(_p(codes), rows, D, int(bits), _p(u)), "kv_unpack")
+    return u

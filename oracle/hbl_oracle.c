@@ -20,6 +20,13 @@
  *        a 4-bit activation takes one of 16 values.
  *   [P3] CSDN post "[论文品鉴] 1-bit LLM", section "掩码存储": ternary weights
  *        are stored by packing several values into one integer.
+ *   [P2-QKV] the same 0755model.com write-up, section "实验结果" (low-bit
+ *        attention, tables 2 and 3): Q, K and V states are quantised after RoPE,
+ *        per head, with absmax, directly to unsigned integers, no calibration;
+ *        a 3-bit KV cache is reported.
+ *   [P2-ABL] the same write-up, table 5 (Hadamard ablation): the rotation is
+ *        applied to weights and activations, or to activations only; section
+ *        on post-training baselines: QuaRot uses a randomised Hadamard transform.
  *
  * Arithmetic: IEEE binary32, round-to-nearest-even, no contraction (build with
  * -ffp-contract=off).  Where fp32 results depend on evaluation order the order
@@ -222,6 +229,55 @@ ORACLE_API int oracle_norm_fwht_f64(const uint16_t* X, const float* gain, int M,
     return 0;
 }
 
+/* ------------------------------------- variants: LayerNorm, no Hadamard [P2] */
+
+/* LayerNorm without bias, one row:
+ *   mu  = tree_sum(x) * (1/K);  d = x - mu;
+ *   var = tree_sum(d*d) * (1/K)   (leaves d0*d0 + d1*d1 with one rounding, as
+ *                                  in the RMS sum of squares);
+ *   u   = (d * (1 / sqrt(var + eps))) * g.
+ * [P2] writes the layer as LN(.) and glosses it as layer normalisation. */
+static void layernorm_row_f32(const uint16_t* xb, const float* gain, int K, float norm_eps,
+                              float* u, float* scratch) {
+    for (int k = 0; k < K; ++k) u[k] = oracle_bf16_to_f32(xb[k]);
+    float mu = tree_sum_f32(u, K) * (1.0f / (float)K);
+    for (int k = 0; k < K; ++k) u[k] = u[k] - mu;
+    if (K == 1) scratch[0] = u[0] * u[0];
+    for (int k = 0; k + 1 < K; k += 2) scratch[k / 2] = fmaf(u[k], u[k], u[k + 1] * u[k + 1]);
+    float var = tree_sum_f32(scratch, K == 1 ? 1 : K / 2) * (1.0f / (float)K);
+    float r = 1.0f / sqrtf(var + norm_eps);
+    for (int k = 0; k < K; ++k) {
+        float v = u[k] * r;
+        if (gain) v = v * gain[k];
+        u[k] = v;
+    }
+}
+
+/* V = T(N(X)): N = RMSNorm (layernorm == 0) or LayerNorm (layernorm != 0);
+ * T = the normalised Walsh-Hadamard transform (hadamard != 0) or the identity
+ * (the plain BitLinear of the layers without H).  norm_fwht is the case
+ * (layernorm, hadamard) = (0, 1). */
+ORACLE_API int oracle_norm_transform(const uint16_t* X, const float* gain, int M, int K,
+                                     float norm_eps, int layernorm, int hadamard, float* V) {
+    if (M < 0 || !is_pow2_i64(K)) return -1;
+    float* scratch = (float*)malloc(sizeof(float) * (size_t)K);
+    if (!scratch) return -2;
+    const float c = oracle_inv_sqrt_n(K);
+    for (int m = 0; m < M; ++m) {
+        float* v = V + (int64_t)m * K;
+        if (layernorm)
+            layernorm_row_f32(X + (int64_t)m * K, gain, K, norm_eps, v, scratch);
+        else
+            rmsnorm_row_f32(X + (int64_t)m * K, gain, K, norm_eps, v, scratch);
+        if (hadamard) {
+            oracle_fwht_f32(v, K);
+            for (int k = 0; k < K; ++k) v[k] = v[k] * c;
+        }
+    }
+    free(scratch);
+    return 0;
+}
+
 /* ------------------------------------------- activation quantisers [P2][P4] */
 
 /* Quantise fp32 rows V [M x K] per token.
@@ -323,6 +379,104 @@ ORACLE_API int oracle_norm_fwht_quant(const uint16_t* X, const float* gain, int 
     }
     free(v);
     return rc;
+}
+
+/* The activation half of a BitLinear layer with the variant choices above. */
+ORACLE_API int oracle_norm_quant(const uint16_t* X, const float* gain, int M, int K,
+                                 float norm_eps, float quant_eps, int act_bits, int layernorm,
+                                 int hadamard, uint8_t* codes, float* scales, int32_t* rowsum) {
+    if (M < 0 || !is_pow2_i64(K)) return -1;
+    float* v = (float*)malloc(sizeof(float) * (size_t)K);
+    if (!v) return -2;
+    int64_t cstride = act_bits == 8 ? K : K / 2;
+    int rc = 0;
+    for (int m = 0; m < M && rc == 0; ++m) {
+        rc = oracle_norm_transform(X + (int64_t)m * K, gain, 1, K, norm_eps, layernorm, hadamard,
+                                   v);
+        if (rc == 0)
+            rc = oracle_quantize_rows(v, 1, K, quant_eps, act_bits, codes + m * cstride,
+                                      scales + m, rowsum ? rowsum + m : NULL);
+    }
+    free(v);
+    return rc;
+}
+
+/* --------------------------------------- weight rotation [P2-ABL], offline */
+
+/* W_rot[n] = FWHT(W[n] * s) * (1/sqrt(K)) for every row n of W [N x K] fp32:
+ * the weights expressed in the rotated basis, so that for activations rotated
+ * by the same map, (x D H/sqrt(K)) . (w D H/sqrt(K)) = x . w (D = diag(s),
+ * H H^T = K I).  s (nullable, entries +-1) is the random sign vector of the
+ * randomised Hadamard transform; NULL means all ones.  Butterfly order and
+ * the final multiply are those of the activation transform. */
+ORACLE_API int oracle_rotate_weights(const float* W, const float* signs, int N, int K,
+                                     float* W_rot) {
+    if (N < 0 || !is_pow2_i64(K)) return -1;
+    const float c = oracle_inv_sqrt_n(K);
+    for (int64_t n = 0; n < N; ++n) {
+        float* w = W_rot + n * K;
+        for (int k = 0; k < K; ++k) w[k] = signs ? W[n * K + k] * signs[k] : W[n * K + k];
+        oracle_fwht_f32(w, K);
+        for (int k = 0; k < K; ++k) w[k] = w[k] * c;
+    }
+    return 0;
+}
+
+/* ------------------------------------------ QKV / KV-cache quantiser [P2-QKV] */
+
+/* Per-head absmax quantisation to unsigned b-bit integers (b in 2..8), for Q,
+ * K and V states after RoPE.  Each row of X [rows x D] bf16 is one head of one
+ * token.  The symmetric absmax quantiser of the INT8 activations, taken to b
+ * bits and offset into the unsigned range:
+ *   Qp = 2^(b-1) - 1;  gamma = max|x|;  inv = Qp / (gamma + eps)   (one division)
+ *   q = clip(round(x * inv), -Qp - 1, Qp)   (the exact product rounded once,
+ *                                            to nearest, ties to even)
+ *   u = q + 2^(b-1)  in [0, 2^b - 1];  scale = gamma / Qp;
+ *   dequantised x ~ (u - 2^(b-1)) * scale.
+ * Packing: groups of 32 consecutive codes of a row, each group 4*b bytes; code j
+ * of a group occupies bits [b*j, b*j + b) of the group read as one
+ * little-endian integer.  D must be a multiple of 32. */
+ORACLE_API int oracle_kv_quant(const uint16_t* X, int64_t rows, int D, int bits, float eps,
+                               uint8_t* codes, float* scales) {
+    if (rows < 0 || D <= 0 || D % 32 != 0 || bits < 2 || bits > 8) return -1;
+    const int qp = (1 << (bits - 1)) - 1;
+    const int64_t row_bytes = (int64_t)D / 32 * 4 * bits;
+    for (int64_t r = 0; r < rows; ++r) {
+        const uint16_t* x = X + r * D;
+        float g = 0.0f;
+        for (int k = 0; k < D; ++k) {
+            float a = fabsf(oracle_bf16_to_f32(x[k]));
+            if (a > g) g = a;
+        }
+        const float inv = (float)qp / (g + eps);
+        uint8_t* out = codes + r * row_bytes;
+        memset(out, 0, (size_t)row_bytes);
+        for (int k = 0; k < D; ++k) {
+            double y = (double)oracle_bf16_to_f32(x[k]) * (double)inv; /* exact */
+            int q = clip_round(y, -qp - 1, qp);
+            uint32_t u = (uint32_t)(q + (1 << (bits - 1)));
+            int64_t bit = (int64_t)(k / 32) * 32 * bits + (int64_t)(k % 32) * bits;
+            for (int i = 0; i < bits; ++i)
+                if ((u >> i) & 1u) out[(bit + i) / 8] |= (uint8_t)(1u << ((bit + i) % 8));
+        }
+        scales[r] = g / (float)qp;
+    }
+    return 0;
+}
+
+/* Unpacks kv_quant codes to their unsigned values u [rows x D]. */
+ORACLE_API int oracle_kv_unpack(const uint8_t* codes, int64_t rows, int D, int bits, uint8_t* u) {
+    if (rows < 0 || D <= 0 || D % 32 != 0 || bits < 2 || bits > 8) return -1;
+    const int64_t row_bytes = (int64_t)D / 32 * 4 * bits;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int k = 0; k < D; ++k) {
+            int64_t bit = (int64_t)(k / 32) * 32 * bits + (int64_t)(k % 32) * bits;
+            uint32_t v = 0;
+            for (int i = 0; i < bits; ++i)
+                v |= (uint32_t)((codes[r * row_bytes + (bit + i) / 8] >> ((bit + i) % 8)) & 1u) << i;
+            u[r * D + k] = (uint8_t)v;
+        }
+    return 0;
 }
 
 /* ------------------------------------------------ ternary weights [P2][P3] */
@@ -431,6 +585,30 @@ ORACLE_API int oracle_ternary_gemm(const uint8_t* codes, const float* scales, in
                                    int32_t* acc_out) {
     return oracle_ternary_gemm_rows(codes, scales, act_bits, M, K, packed, alpha, N, 0, M, Y,
                                     acc_out);
+}
+
+/* Whole layer for rows [m0, m1) with the variant choices of norm_transform:
+ * norm -> (Hadamard) -> quantise -> ternary matmul -> dequantise. */
+ORACLE_API int oracle_bitlinear_forward_rows(const uint16_t* X, const float* gain, int M, int K,
+                                             int N, const uint32_t* packed, float alpha,
+                                             int act_bits, float norm_eps, float quant_eps,
+                                             int layernorm, int hadamard, int m0, int m1,
+                                             uint16_t* Y) {
+    if (m0 < 0 || m1 > M || m0 > m1) return -1;
+    int rows = m1 - m0;
+    if (rows == 0) return 0;
+    int64_t cstride = act_bits == 8 ? K : K / 2;
+    uint8_t* codes = (uint8_t*)malloc((size_t)rows * (size_t)cstride);
+    float* scales = (float*)malloc(sizeof(float) * (size_t)rows);
+    if (!codes || !scales) { free(codes); free(scales); return -2; }
+    int rc = oracle_norm_quant(X + (int64_t)m0 * K, gain, rows, K, norm_eps, quant_eps, act_bits,
+                               layernorm, hadamard, codes, scales, NULL);
+    if (rc == 0)
+        rc = oracle_ternary_gemm(codes, scales, act_bits, rows, K, packed, alpha, N,
+                                 Y + (int64_t)m0 * N, NULL);
+    free(codes);
+    free(scales);
+    return rc;
 }
 
 /* Whole layer for rows [m0, m1): norm -> Hadamard -> quantise -> ternary matmul
