@@ -50,7 +50,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--kernel-iters", type=int, default=200,
                     help="iterations of the per-kernel timing loops")
-    ap.add_argument("--only", default=None, choices=["forward", "gemm", "quant4", "quant8"],
+    ap.add_argument("--only", default=None, choices=["forward", "gemm", "quant4", "quant8", "nohad4", "ln4",
+                                                      "rotate", "kv3", "kv4", "kv8"],
                     help="run only this case (a few launches, for profiler captures); prints a "
                          "short JSON line, not the benchmark line")
     return ap.parse_args()
@@ -265,30 +266,34 @@ def run_hbl(args):
     t_max_ms = hdist.max_over_ranks(t_dev_ms, dev)
     value = world * M_TOK * args.steps / (t_max_ms / 1e3)
 
-    # ---- per-kernel timing: the forward's two kernels through the two-call
-    # C-ABI path with the same (32-row interleaved, one byte per code) layout
-    IL = hbl.ACT_INT4_I32
-    codes = torch.empty(hbl.codes_shape(M_TOK, K_IN, IL), dtype=torch.uint8, device=dev)
+    # ---- per-kernel timing: the forward's kernels through the C ABI with the
+    # layouts the fused forward uses at this batch (one-byte INT4 codes for the
+    # TMA-fed GEMM; the packed weights expanded to signed bytes per call)
+    B8 = hbl.ACT_INT4_BYTES
+    codes = torch.empty(hbl.codes_shape(M_TOK, K_IN, B8), dtype=torch.uint8, device=dev)
     scales = torch.empty(M_TOK, dtype=torch.float32, device=dev)
     rowsum = torch.empty(M_TOK, dtype=torch.int32, device=dev)
-    gws = torch.empty(max(16, hbl.workspace_size(hbl.OP_TERNARY_GEMM, M_TOK, K_IN, N_OUT, IL)),
-                      dtype=torch.uint8, device=dev)
+    Ws = torch.empty((N_OUT, K_IN), dtype=torch.int8, device=dev)
     iters = max(args.kernel_iters, args.steps)
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(iters)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(iters)]
     for i in range(3):
-        hbl.norm_fwht_quant(Xd, IL, out=(codes, scales, rowsum))
-        hbl.ternary_gemm(codes, scales, rowsum, IL, K_IN, packed, alpha, ws=gws, out=Y)
+        hbl.norm_fwht_quant(Xd, B8, out=(codes, scales, rowsum))
+        hbl.expand_ternary(packed, K_IN, out=Ws)
+        hbl.ternary_gemm_s8w(codes, scales, B8, Ws, alpha, out=Y)
     torch.cuda.synchronize()
     for i in range(iters):
         evs[i][0].record(stream)
-        hbl.norm_fwht_quant(Xd, IL, out=(codes, scales, rowsum))
+        hbl.norm_fwht_quant(Xd, B8, out=(codes, scales, rowsum))
         evs[i][1].record(stream)
-        hbl.ternary_gemm(codes, scales, rowsum, IL, K_IN, packed, alpha, ws=gws, out=Y,
-                         status=status)
+        hbl.expand_ternary(packed, K_IN, out=Ws)
         evs[i][2].record(stream)
+        hbl.ternary_gemm_s8w(codes, scales, B8, Ws, alpha, out=Y, status=status)
+        evs[i][3].record(stream)
     torch.cuda.synchronize()
     t_k1 = statistics.mean(e[0].elapsed_time(e[1]) for e in evs) * 1e-3
-    t_k2 = statistics.mean(e[1].elapsed_time(e[2]) for e in evs) * 1e-3
+    t_kx = statistics.mean(e[1].elapsed_time(e[2]) for e in evs) * 1e-3
+    t_k2 = statistics.mean(e[2].elapsed_time(e[3]) for e in evs) * 1e-3
+    del Ws
 
     # ---- quant workload: 8192 x 4096, a4 and a8, 4 rotating inputs (256 MB > L2)
     qX = [torch.from_numpy(inputs.activations("quant", seed=s).view(np.int16)).view(
@@ -363,6 +368,58 @@ def run_hbl(args):
                            "path": "gemv (dp4a split-K)" if T <= 8 else "gemm_ts split-K",
                            "timing": "CUDA graph replay, one forward per weight copy"})
         del pcs
+
+    # ---- the other rows of the hot path, each against the HBM roofline
+    def ev_time(fn, n, iters):
+        for i in range(3):
+            fn(i % n)
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for i in range(iters):
+            fn(i % n)
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) * 1e-3 / iters
+
+    others = {}
+    # BitLinear variants (no Hadamard / LayerNorm) on the quant workload, a4 packed
+    qX = [torch.from_numpy(inputs.activations("quant", seed=s).view(np.int16)).view(
+        torch.bfloat16).to(dev) for s in range(4)]
+    qc = torch.empty((QM, QK // 2), dtype=torch.uint8, device=dev)
+    qs = torch.empty(QM, dtype=torch.float32, device=dev)
+    qr = torch.empty(QM, dtype=torch.int32, device=dev)
+    for name, fl in (("no_hadamard", hbl.NORM_NO_HADAMARD), ("layernorm", hbl.NORM_LAYERNORM),
+                     ("layernorm_no_hadamard", hbl.NORM_LAYERNORM | hbl.NORM_NO_HADAMARD)):
+        t = ev_time(lambda i: hbl.norm_quant(qX[i], 4, fl, out=(qc, qs, qr)), 4, 40)
+        nbytes = QM * QK * 2 + QM * QK // 2 + 8 * QM
+        others["norm_quant_a4_" + name] = {
+            "workload": "quant 8192 x 4096, a4 packed", "us": t * 1e6, "bytes": nbytes,
+            "achieved_gbs": nbytes / t / 1e9, "frac": nbytes / t / 1e9 / pk["hbm_gbs"]}
+    del qX
+    # offline weight rotation of W_down (4096 x 16384 fp32, 268 MB in and out), random signs
+    Wd = torch.from_numpy(W).to(dev)
+    sg = torch.from_numpy(inputs.random_signs(K_IN)).to(dev)
+    Wr = torch.empty_like(Wd)
+    t = ev_time(lambda i: hbl.rotate_weights(Wd, sg, out=Wr), 1, 10)
+    nbytes = 2 * N_OUT * K_IN * 4
+    others["rotate_weights"] = {"workload": "W_down 4096 x 16384 fp32, random signs",
+                                "us": t * 1e6, "bytes": nbytes, "achieved_gbs": nbytes / t / 1e9,
+                                "frac": nbytes / t / 1e9 / pk["hbm_gbs"]}
+    del Wd, Wr
+    # QKV / KV-cache quantiser: 8192 tokens x 96 heads x 128 (201 MB bf16)
+    QX = torch.from_numpy(inputs.qkv_states().view(np.int16)).view(torch.bfloat16).to(dev)
+    rows = QX.numel() // 128
+    ksc = torch.empty(rows, dtype=torch.float32, device=dev)
+    for kb in (3, 4, 8):
+        kc = torch.empty((rows, 128 * kb // 8), dtype=torch.uint8, device=dev)
+        t = ev_time(lambda i: hbl.kv_quant(QX, kb, out=(kc, ksc)), 1, 20)
+        nbytes = rows * 128 * 2 + rows * 128 * kb // 8 + rows * 4
+        others["kv_quant_%dbit" % kb] = {
+            "workload": "qkv 8192 x 96 x 128 after RoPE", "us": t * 1e6, "bytes": nbytes,
+            "achieved_gbs": nbytes / t / 1e9, "frac": nbytes / t / 1e9 / pk["hbm_gbs"]}
+        del kc
+    del QX
     clocks = sampler.stop()
 
     # ---- end to end through the host-buffer call: H2D X, forward, D2H Y
@@ -390,12 +447,13 @@ def run_hbl(args):
     if t_k2 >= t_k1:
         achieved = ops / t_k2 / 1e12
         peak = 2.0 * pk["bf16_tflops_sustained"]
-        roof = {"bound": "tensor", "kernel": "gemm_ts (tcgen05 kind::i8, activations in TMEM)",
+        roof = {"bound": "tensor",
+                "kernel": "gemm_tma (TMA-fed tcgen05 kind::i8, accumulators in TMEM)",
                 "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                 "peak_note": "int8 dense = %s sustained bf16 %.1f TFLOP/s x 2 (nominal "
                              "int8:bf16 ratio)" % (pk["source"], pk["bf16_tflops_sustained"]),
-                "traffic": recorded_traffic("gemm_ts_a4_ffn_wdown",
-                                            source_hash("k2b_ternary_gemm_ts.cu")),
+                "traffic": recorded_traffic("gemm_tma_a4_ffn_wdown",
+                                            source_hash("k2c_gemm_tma.cu")),
                 "us_per_launch": t_k2 * 1e6}
     else:
         nbytes = M_TOK * K_IN * 2 + M_TOK * K_IN + 8 * M_TOK  # one-byte codes in the forward
@@ -416,13 +474,15 @@ def run_hbl(args):
                    else "single GPU",
                    "l2": "inputs larger than L2 (X 268 MB per step)"},
         "roofline": roof,
-        "kernels_us": {"norm_fwht_quant": t_k1 * 1e6, "ternary_gemm_ts": t_k2 * 1e6},
+        "kernels_us": {"norm_fwht_quant": t_k1 * 1e6, "expand_ternary": t_kx * 1e6,
+                       "gemm_tma": t_k2 * 1e6},
         "quant": quant,
         "decode": decode,
+        "others": others,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": M_TOK * K_IN * 2,
                 "d2h_bytes_per_step": M_TOK * N_OUT * 2, "steps": e2e_steps,
                 "api": "hbl_hbitlinear_forward_hostio (pinned host buffers)"},
-        "gpu_launches": 2 * args.steps,
+        "gpu_launches": 3 * args.steps,  # K1, weight expansion, GEMM per forward
         "clocks": clocks,
         "device_status": st,
         "peaks": pk,
@@ -455,6 +515,20 @@ def run_only(args):
         X = torch.from_numpy(inputs.activations("quant").view(np.int16)).view(
             torch.bfloat16).to(dev)
         fn = lambda: hbl.norm_fwht_quant(X, bits)
+    elif args.only in ("nohad4", "ln4"):
+        X = torch.from_numpy(inputs.activations("quant").view(np.int16)).view(
+            torch.bfloat16).to(dev)
+        fl = hbl.NORM_NO_HADAMARD if args.only == "nohad4" else hbl.NORM_LAYERNORM
+        fn = lambda: hbl.norm_quant(X, 4, fl)
+    elif args.only == "rotate":
+        Wd = torch.from_numpy(inputs.weights("ffn_wdown")).to(dev)
+        sg = torch.from_numpy(inputs.random_signs(K_IN)).to(dev)
+        Wr = torch.empty_like(Wd)
+        fn = lambda: hbl.rotate_weights(Wd, sg, out=Wr)
+    elif args.only.startswith("kv"):
+        QX = torch.from_numpy(inputs.qkv_states().view(np.int16)).view(torch.bfloat16).to(dev)
+        kb = int(args.only[2:])
+        fn = lambda: hbl.kv_quant(QX, kb)
     else:
         X = torch.from_numpy(inputs.activations("ffn_wdown").view(np.int16)).view(
             torch.bfloat16).to(dev)
@@ -463,10 +537,11 @@ def run_only(args):
             ws = torch.empty(hbl.workspace_size(hbl.OP_HBITLINEAR_FORWARD, M_TOK, K_IN, N_OUT,
                                                 BITS), dtype=torch.uint8, device=dev)
             fn = lambda: hbl.hbitlinear_forward(X, packed, alpha, BITS, ws=ws)
-        else:  # the forward's GEMM: interleaved one-byte INT4 codes
-            IL = hbl.ACT_INT4_I32
-            codes, scales, rowsum = hbl.norm_fwht_quant(X, IL)
-            fn = lambda: hbl.ternary_gemm(codes, scales, rowsum, IL, K_IN, packed, alpha)
+        else:  # the forward's GEMM: one-byte INT4 codes, expanded weights
+            B8 = hbl.ACT_INT4_BYTES
+            codes, scales, rowsum = hbl.norm_fwht_quant(X, B8)
+            Ws = hbl.expand_ternary(packed, K_IN)
+            fn = lambda: hbl.ternary_gemm_s8w(codes, scales, B8, Ws, alpha)
     for _ in range(args.warmup):
         fn()
     torch.cuda.synchronize()

@@ -13,6 +13,11 @@ Names follow include/hbl.h:
   hbitlinear_forward(X, W_packed, alpha, act_bits)                   -> Y bf16 [M, N]
   hbitlinear_forward_hostio(X_host, W_packed, alpha, act_bits, Y_host, ws)
   ternary_gemv_noalloc(codes, scales, rowsum, act_bits, K, W_packed, alpha)  -> Y (, acc)
+  norm_transform(X, flags)                -> V fp32 [M, K]       (variants: NORM_* flags)
+  norm_quant(X, act_bits, flags)          -> (codes, scales, rowsum)
+  bitlinear_forward(X, W_packed, alpha, act_bits, flags)            -> Y bf16 [M, N]
+  rotate_weights(W, signs)                -> W_rot fp32 [N, K]
+  kv_quant(X, bits)                       -> (codes uint8 [rows, D*bits/8], scales fp32 [rows])
 """
 import ctypes
 import os
@@ -26,10 +31,14 @@ STATUS_NAMES = {0: "HBL_OK", 1: "HBL_ERR_INVALID_ARG", 2: "HBL_ERR_SHAPE", 3: "H
                 7: "HBL_ERR_TIMEOUT"}
 OP_PACK_TERNARY, OP_TERNARY_GEMM, OP_HBITLINEAR_FORWARD, OP_HBITLINEAR_FORWARD_HOSTIO = 0, 1, 2, 3
 ACT_INT4_I32, ACT_INT8_I32 = 0x104, 0x108  # one byte per code, 32-row interleaved layout
+ACT_INT4_BYTES = 0x204                      # INT4 codes one byte each, row-major
+NORM_LAYERNORM, NORM_NO_HADAMARD = 1, 2     # variant flags of norm_transform / norm_quant / bitlinear_forward
 EXPORTS = ("hbl_status_string", "hbl_version", "hbl_set_gemm_path", "hbl_workspace_size",
            "hbl_pack_ternary", "hbl_norm_fwht", "hbl_norm_fwht_quant", "hbl_ternary_gemm",
            "hbl_hbitlinear_forward", "hbl_hbitlinear_forward_hostio",
-           "hbl_ternary_gemv_noalloc")
+           "hbl_ternary_gemv_noalloc", "hbl_norm_transform", "hbl_norm_quant",
+           "hbl_bitlinear_forward", "hbl_rotate_weights", "hbl_kv_quant",
+           "hbl_expand_ternary", "hbl_ternary_gemm_s8w")
 
 _lib = None
 
@@ -72,6 +81,21 @@ def lib():
         L.hbl_hbitlinear_forward_hostio.argtypes = [P, P, I, I, I, P, P, I, F, F, P, P, SZ, P, P]
         L.hbl_ternary_gemv_noalloc.restype = I
         L.hbl_ternary_gemv_noalloc.argtypes = [P, P, P, I, I, I, P, P, I, P, P, P, P]
+        U, I64 = ctypes.c_uint, ctypes.c_int64
+        L.hbl_norm_transform.restype = I
+        L.hbl_norm_transform.argtypes = [P, P, I, I, F, U, P, P, P]
+        L.hbl_norm_quant.restype = I
+        L.hbl_norm_quant.argtypes = [P, P, I, I, F, F, I, U, P, P, P, P, P]
+        L.hbl_bitlinear_forward.restype = I
+        L.hbl_bitlinear_forward.argtypes = [P, P, I, I, I, P, P, I, U, F, F, P, P, SZ, P, P]
+        L.hbl_rotate_weights.restype = I
+        L.hbl_rotate_weights.argtypes = [P, P, I, I, P, P, P]
+        L.hbl_kv_quant.restype = I
+        L.hbl_kv_quant.argtypes = [P, I64, I, I, F, P, P, P, P]
+        L.hbl_expand_ternary.restype = I
+        L.hbl_expand_ternary.argtypes = [P, I, I, P, P, P]
+        L.hbl_ternary_gemm_s8w.restype = I
+        L.hbl_ternary_gemm_s8w.argtypes = [P, P, I, I, I, P, P, I, P, P, P, P]
         _lib = L
     return _lib
 
@@ -110,8 +134,9 @@ def workspace_size(op, M, K, N, act_bits):
 
 
 def set_gemm_path(path):
-    """0 = automatic, 1 = tensor cores (both operands in shared memory),
-    2 = CUDA-core GEMV, 3 = tensor cores with activations in TMEM (process-wide)."""
+    """0 = automatic, 1 = tensor cores (both operands staged by threads),
+    2 = CUDA-core GEMV, 3 = tensor cores with activations in TMEM, 4 = TMA-fed
+    tensor cores for one-byte codes (process-wide)."""
     _check(lib().hbl_set_gemm_path(int(path)), "set_gemm_path")
 
 
@@ -156,7 +181,7 @@ def norm_fwht(X, gain=None, norm_eps=1e-6, status=None):
 def codes_shape(M, K, act_bits):
     if act_bits in (ACT_INT4_I32, ACT_INT8_I32):
         return ((M + 31) // 32 * 32, K)
-    return (M, K if act_bits == 8 else K // 2)
+    return (M, K // 2 if act_bits == 4 else K)
 
 
 def norm_fwht_quant(X, act_bits, gain=None, norm_eps=1e-6, quant_eps=1e-5, out=None,
@@ -210,7 +235,9 @@ def ternary_gemv_noalloc(codes, scales, rowsum, act_bits, K, W_packed, alpha, wa
     _check(lib().hbl_ternary_gemv_noalloc(_ptr(codes), _ptr(scales), _ptr(rowsum),
                                           int(act_bits), M, K, _ptr(W_packed), _ptr(alpha), N,
                                           _ptr(Y), _ptr(acc), _ptr(status), _stream()),
-           "hbl_ternary_gemv_noalloc")
+           "hbl_ternary_gemv_noalloc", "hbl_norm_transform", "hbl_norm_quant",
+           "hbl_bitlinear_forward", "hbl_rotate_weights", "hbl_kv_quant",
+           "hbl_expand_ternary", "hbl_ternary_gemm_s8w")
     return (Y, acc) if want_acc else Y
 
 
@@ -242,3 +269,117 @@ def hbitlinear_forward_hostio(X_host, W_packed, alpha, act_bits, Y_host, ws, gai
                                                ws.numel(), _ptr(status), _stream()),
            "hbl_hbitlinear_forward_hostio")
     return Y_host
+
+
+# ------------------------------------------------------------------ variants
+
+def norm_transform(X, flags=0, gain=None, norm_eps=1e-6, status=None):
+    """hbl_norm_transform: V = T(N(X)) with NORM_LAYERNORM / NORM_NO_HADAMARD flags."""
+    import torch
+
+    _dev(X, torch.bfloat16, "X")
+    M, K = X.shape
+    V = torch.empty((M, K), dtype=torch.float32, device=X.device)
+    _check(lib().hbl_norm_transform(_ptr(X), _ptr(gain), M, K, float(norm_eps), int(flags),
+                                    _ptr(V), _ptr(status), _stream()), "hbl_norm_transform")
+    return V
+
+
+def norm_quant(X, act_bits, flags=0, gain=None, norm_eps=1e-6, quant_eps=1e-5, out=None,
+               status=None):
+    import torch
+
+    _dev(X, torch.bfloat16, "X")
+    M, K = X.shape
+    if out is None:
+        codes = torch.empty(codes_shape(M, K, act_bits), dtype=torch.uint8, device=X.device)
+        scales = torch.empty(max(M, 4), dtype=torch.float32, device=X.device)
+        rowsum = torch.empty(max(M, 4), dtype=torch.int32, device=X.device)
+    else:
+        codes, scales, rowsum = out
+    _check(lib().hbl_norm_quant(_ptr(X), _ptr(gain), M, K, float(norm_eps), float(quant_eps),
+                                int(act_bits), int(flags), _ptr(codes), _ptr(scales),
+                                _ptr(rowsum), _ptr(status), _stream()), "hbl_norm_quant")
+    return codes, scales[:M], rowsum[:M]
+
+
+def bitlinear_forward(X, W_packed, alpha, act_bits, flags=0, gain=None, norm_eps=1e-6,
+                      quant_eps=1e-5, ws=None, out=None, status=None):
+    import torch
+
+    _dev(X, torch.bfloat16, "X")
+    M, K = X.shape
+    N = W_packed.shape[0]
+    Y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=X.device)
+    if ws is None:
+        ws = _workspace(workspace_size(OP_HBITLINEAR_FORWARD, M, K, N, act_bits), X.device)
+    _check(lib().hbl_bitlinear_forward(_ptr(X), _ptr(gain), M, K, N, _ptr(W_packed),
+                                       _ptr(alpha), int(act_bits), int(flags), float(norm_eps),
+                                       float(quant_eps), _ptr(Y), _ptr(ws), ws.numel(),
+                                       _ptr(status), _stream()), "hbl_bitlinear_forward")
+    return Y
+
+
+def rotate_weights(W, signs=None, out=None, status=None):
+    """hbl_rotate_weights: W_rot = FWHT(W * signs) / sqrt(K) per row (out may be W)."""
+    import torch
+
+    _dev(W, torch.float32, "W")
+    N, K = W.shape
+    if signs is not None:
+        _dev(signs, torch.float32, "signs")
+    Wr = out if out is not None else torch.empty_like(W)
+    _check(lib().hbl_rotate_weights(_ptr(W), _ptr(signs), N, K, _ptr(Wr), _ptr(status),
+                                    _stream()), "hbl_rotate_weights")
+    return Wr
+
+
+def kv_code_bytes(D, bits):
+    return D * bits // 8
+
+
+def kv_quant(X, bits, eps=1e-5, out=None, status=None):
+    """hbl_kv_quant over the last dimension (one head of one token per row)."""
+    import torch
+
+    _dev(X, torch.bfloat16, "X")
+    D = X.shape[-1]
+    rows = X.numel() // D if D else 0
+    if out is None:
+        codes = torch.empty((rows, kv_code_bytes(D, bits)), dtype=torch.uint8, device=X.device)
+        scales = torch.empty(max(rows, 4), dtype=torch.float32, device=X.device)
+    else:
+        codes, scales = out
+    _check(lib().hbl_kv_quant(_ptr(X), rows, D, int(bits), float(eps), _ptr(codes),
+                              _ptr(scales), _ptr(status), _stream()), "hbl_kv_quant")
+    return codes, scales[:rows]
+
+
+# ------------------------------------------------------- expanded weights
+
+def expand_ternary(W_packed, K, out=None, status=None):
+    """hbl_expand_ternary: packed 2-bit weights -> int8 t in {-1, 0, 1} [N, K]."""
+    import torch
+
+    N = W_packed.shape[0]
+    Ws = out if out is not None else torch.empty((N, K), dtype=torch.int8,
+                                                 device=W_packed.device)
+    _check(lib().hbl_expand_ternary(_ptr(W_packed), N, K, _ptr(Ws), _ptr(status), _stream()),
+           "hbl_expand_ternary")
+    return Ws
+
+
+def ternary_gemm_s8w(codes, scales, act_bits, W_s8, alpha, want_acc=False, out=None,
+                     status=None):
+    """hbl_ternary_gemm_s8w: the TMA-fed tensor-core GEMM on expanded weights."""
+    import torch
+
+    M = scales.shape[0]
+    N, K = W_s8.shape
+    Y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16,
+                                                device=codes.device)
+    acc = torch.empty((M, N), dtype=torch.int32, device=codes.device) if want_acc else None
+    _check(lib().hbl_ternary_gemm_s8w(_ptr(codes), _ptr(scales), int(act_bits), M, K, _ptr(W_s8),
+                                      _ptr(alpha), N, _ptr(Y), _ptr(acc), _ptr(status),
+                                      _stream()), "hbl_ternary_gemm_s8w")
+    return (Y, acc) if want_acc else Y

@@ -23,7 +23,7 @@ struct DevInfo {
     int sms = 0;
 };
 DevInfo g_dev[kMaxDevices];
-std::atomic<int> g_path{0};  // 0 auto, 1 tensor core (SS), 2 CUDA-core GEMV, 3 tensor core (TS)
+std::atomic<int> g_path{0};  // 0 auto, 1 SS tcgen05, 2 CUDA-core GEMV, 3 TS tcgen05, 4 TMA tcgen05
 
 bool is_pow2(int64_t v) { return v > 0 && (v & (v - 1)) == 0; }
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -57,37 +57,75 @@ hbl_status device(int* sms) {
     return HBL_OK;
 }
 
-int codes_row_bytes(int K, int act_bits) { return act_bits == 8 ? K : K / 2; }
-
-// act_bits: 4 / 8 (row-major layouts) or HBL_ACT_INT{4,8}_I32 (interleaved bytes)
+// act_bits: 4 / 8 (row-major), HBL_ACT_INT4_BYTES (INT4 values one byte each,
+// row-major) or HBL_ACT_INT{4,8}_I32 (interleaved bytes)
 bool act_valid(int a) {
-    return a == 4 || a == 8 || a == HBL_ACT_INT4_I32 || a == HBL_ACT_INT8_I32;
+    return a == 4 || a == 8 || a == HBL_ACT_INT4_BYTES || a == HBL_ACT_INT4_I32 ||
+           a == HBL_ACT_INT8_I32;
 }
 bool act_il(int a) { return a == HBL_ACT_INT4_I32 || a == HBL_ACT_INT8_I32; }
 int act_base(int a) { return a & 0xFF; }
+// bits each code occupies in memory (row-major layouts): 4 for packed nibbles, else 8
+int act_width(int a) { return a == 4 ? 4 : 8; }
+int codes_row_bytes(int K, int act_bits) { return act_width(act_bits) == 4 ? K / 2 : K; }
 
-bool use_gemv(int64_t M) {
+// Ternary-GEMM back ends.
+enum class Back { GEMV, SS, TS, TMA };
+
+// Batches above this many tokens take the TMA-fed kernel (automatic choice).
+constexpr int64_t kTmaMinM = 257;
+
+// The back end for M tokens; `bytes`: the codes are (or can be made) one byte each.
+Back pick(int64_t M, int K, bool bytes) {
     const int path = g_path.load();
-    if (path == 1 || path == 3) return false;
-    if (path == 2) return true;
-    return M <= gemv_max_m();
+    if (path == 1) return Back::SS;
+    if (path == 2) return Back::GEMV;
+    if (path == 3) return Back::TS;
+    if (path == 4) return (bytes && K >= 128) ? Back::TMA : Back::TS;
+    if (M <= gemv_max_m()) return Back::GEMV;
+    if (bytes && K >= 128 && M >= kTmaMinM) return Back::TMA;
+    return Back::TS;
 }
 
-size_t gemm_ws(int64_t M, int K, int N, int sms_guess) {
-    if (!use_gemv(M)) return g_path.load() == 1 ? 0 : gemm_ts_workspace(M, K, N);
-    const int64_t mchunk = M < gemv_max_m() ? M : gemv_max_m();
-    return gemv_workspace(mchunk, K, N, sms_guess);
+size_t backend_ws(Back b, int64_t M, int K, int N) {
+    switch (b) {
+        case Back::SS: return 0;
+        case Back::TS: return gemm_ts_workspace(M, K, N);
+        case Back::TMA: return gemm_tma_workspace(K, N);
+        case Back::GEMV:
+        default: {
+            if (gemv_rows_supported(K)) return 0;  // the row GEMV needs no scratch
+            const int64_t mchunk = M < gemv_max_m() ? M : gemv_max_m();
+            return gemv_workspace(mchunk, K, N, 148);
+        }
+    }
 }
 
 // SM count for sizing when no device is queried yet (workspace queries must
 // not need a GPU): the split factor only grows with SM count, so size for 148.
 constexpr int kSizingSms = 148;
 
-hbl_status run_gemm(const GemmArgs& a, void* ws, size_t ws_bytes, cudaStream_t s, int sms) {
-    if (!use_gemv(a.M))
-        return g_path.load() == 1 ? launch_gemm_tc(a, s, sms)
-                                  : launch_gemm_ts(a, ws, ws_bytes, s, sms);
-    // CUDA-core path in chunks of up to gemv_max_m() tokens (workspace reused in order)
+hbl_status run_gemm(Back b, const GemmArgs& a, void* ws, size_t ws_bytes, cudaStream_t s,
+                    int sms) {
+    if (b == Back::SS) return launch_gemm_tc(a, s, sms);
+    if (b == Back::TS) return launch_gemm_ts(a, ws, ws_bytes, s, sms);
+    if (b == Back::TMA) return launch_gemm_tma(a, ws, ws_bytes, s, sms);
+    if (gemv_rows_supported(a.K)) {  // row GEMV in chunks of up to gemv_rows_max_m(K) tokens
+        const int64_t step = gemv_rows_max_m(a.K);
+        for (int64_t r0 = 0; r0 < a.M; r0 += step) {
+            GemmArgs c = a;
+            c.M = (a.M - r0) < step ? (a.M - r0) : step;
+            c.codes = static_cast<const uint8_t*>(a.codes) + r0 * codes_row_bytes(a.K, a.act_bits);
+            c.scales = a.scales + r0;
+            c.rowsum = a.rowsum + r0;
+            c.Y = a.Y + r0 * a.N;
+            c.acc_out = a.acc_out ? a.acc_out + r0 * a.N : nullptr;
+            hbl_status st = launch_gemv_rows(c, a.pdl, s);
+            if (st != HBL_OK) return st;
+        }
+        return HBL_OK;
+    }
+    // split-K CUDA-core path in chunks of up to gemv_max_m() tokens (workspace reused in order)
     const int64_t step = gemv_max_m();
     for (int64_t r0 = 0; r0 < a.M; r0 += step) {
         GemmArgs c = a;
@@ -101,6 +139,30 @@ hbl_status run_gemm(const GemmArgs& a, void* ws, size_t ws_bytes, cudaStream_t s
         if (st != HBL_OK) return st;
     }
     return HBL_OK;
+}
+
+// The fused forward's choice: back end, K1 mode and the codes layout it feeds.
+struct FwdPlan {
+    Back back;
+    int k1_mode;
+    int gemm_act_bits;  // value width the GEMM reads (4 or 8)
+    bool interleaved;
+};
+FwdPlan forward_plan(int64_t M, int K, int act_bits) {
+    FwdPlan f;
+    f.back = pick(M, K, true);
+    f.interleaved = f.back == Back::TS;
+    if (f.back == Back::TMA) {
+        f.k1_mode = act_bits == 4 ? 6 : 8;
+        f.gemm_act_bits = 8;
+    } else if (f.back == Back::TS) {
+        f.k1_mode = act_bits == 4 ? 5 : 9;
+        f.gemm_act_bits = 8;
+    } else {
+        f.k1_mode = act_bits;
+        f.gemm_act_bits = act_bits;
+    }
+    return f;
 }
 
 }  // namespace
@@ -144,7 +206,7 @@ const char* hbl_status_string(int status) {
 int hbl_version(void) { return 100; }
 
 int hbl_set_gemm_path(int path) {
-    if (path < 0 || path > 3) return HBL_ERR_INVALID_ARG;
+    if (path < 0 || path > 4) return HBL_ERR_INVALID_ARG;
     g_path.store(path);
     return HBL_OK;
 }
@@ -163,9 +225,15 @@ hbl_status hbl_workspace_size(int op, int M, int K, int N, int act_bits, size_t*
         case HBL_OP_HBITLINEAR_FORWARD_HOSTIO: {
             if (M < 0 || check_k(K) != HBL_OK || check_n(N) != HBL_OK) return HBL_ERR_SHAPE;
             if (!act_valid(act_bits)) return HBL_ERR_INVALID_ARG;
-            if (op != HBL_OP_TERNARY_GEMM && act_il(act_bits)) return HBL_ERR_INVALID_ARG;
-            size_t b = act_il(act_bits) ? up256(gemm_ts_workspace(M, K, N))
-                                        : up256(gemm_ws(M, K, N, kSizingSms));
+            if (op != HBL_OP_TERNARY_GEMM && act_bits != 4 && act_bits != 8)
+                return HBL_ERR_INVALID_ARG;
+            size_t b;
+            if (op == HBL_OP_TERNARY_GEMM)
+                b = act_il(act_bits) ? up256(gemm_ts_workspace(M, K, N))
+                                     : up256(backend_ws(pick(M, K, act_width(act_bits) == 8), M,
+                                                        K, N));
+            else
+                b = up256(backend_ws(forward_plan(M, K, act_bits).back, M, K, N));
             if (op != HBL_OP_TERNARY_GEMM) {
                 b += up256((size_t)((M + 31) & ~31) * K);  // codes, one byte each, rows padded to 32
                 b += up256((size_t)M * 4) * 2;                         // scales, rowsum
@@ -194,6 +262,13 @@ hbl_status hbl_pack_ternary(const float* W, int N, int K, float eps, uint32_t* W
     if (st != HBL_OK) return st;
     return launch_pack_ternary(W, N, K, eps, W_packed, alpha, ws,
                                static_cast<cudaStream_t>(stream), sms);
+}
+
+// K1 mode writing the codes layout `act_bits` names.
+static int k1_mode_of(int act_bits) {
+    if (act_il(act_bits)) return act_base(act_bits) == 4 ? 5 : 9;
+    if (act_bits == HBL_ACT_INT4_BYTES) return 6;
+    return act_bits;
 }
 
 // Scalars and shapes first; pointers only matter when there is work (M > 0).
@@ -236,9 +311,9 @@ hbl_status hbl_norm_fwht_quant(const uint16_t* X, const float* gain, int M, int 
         return HBL_ERR_ALIGNMENT;
     int sms = 0;
     if ((st = device(&sms)) != HBL_OK) return st;
-    const int mode = act_il(act_bits) ? (act_base(act_bits) == 4 ? 5 : 9) : act_bits;
-    return launch_norm_fwht_quant(X, gain, M, K, norm_eps, quant_eps, mode, codes, scales,
-                                  rowsum, nullptr, static_cast<cudaStream_t>(stream), sms);
+    return launch_norm_fwht_quant(X, gain, M, K, norm_eps, quant_eps, k1_mode_of(act_bits),
+                                  codes, scales, rowsum, nullptr,
+                                  static_cast<cudaStream_t>(stream), sms);
 }
 
 hbl_status hbl_ternary_gemm(const void* codes, const float* scales, const int32_t* rowsum,
@@ -253,25 +328,24 @@ hbl_status hbl_ternary_gemm(const void* codes, const float* scales, const int32_
         !aligned16(alpha) || !aligned16(Y) || (acc_out && !aligned16(acc_out)) ||
         (dev_status && !aligned16(dev_status)))
         return HBL_ERR_ALIGNMENT;
-    const size_t need = act_il(act_bits) ? gemm_ts_workspace(M, K, N) : gemm_ws(M, K, N, kSizingSms);
+    const Back bk = act_il(act_bits) ? Back::TS : pick(M, K, act_width(act_bits) == 8);
+    const size_t need = backend_ws(bk, M, K, N);
     if (need > 0 && (ws == nullptr || ws_bytes < need)) return HBL_ERR_WORKSPACE;
     if (ws && !aligned16(ws)) return HBL_ERR_ALIGNMENT;
     int sms = 0;
     hbl_status st = device(&sms);
     if (st != HBL_OK) return st;
-    if (act_il(act_bits)) {  // interleaved one-byte codes: the TMEM-activation kernel
-        GemmArgs a{codes, scales, rowsum, 8, M, K, W_packed, alpha, N, Y, acc_out, dev_status};
-        a.interleaved = true;
-        return launch_gemm_ts(a, ws, ws_bytes, static_cast<cudaStream_t>(stream), sms);
-    }
-    GemmArgs a{codes, scales, rowsum, act_bits, M, K, W_packed, alpha, N, Y, acc_out, dev_status};
-    return run_gemm(a, ws, ws_bytes, static_cast<cudaStream_t>(stream), sms);
+    GemmArgs a{codes, scales, rowsum, act_width(act_bits), M, K, W_packed, alpha, N, Y, acc_out,
+               dev_status};
+    a.interleaved = act_il(act_bits);  // interleaved one-byte codes: the TMEM-activation kernel
+    return run_gemm(bk, a, ws, ws_bytes, static_cast<cudaStream_t>(stream), sms);
 }
 
 static hbl_status forward_impl(const uint16_t* X, const float* gain, int M, int K, int N,
                                const uint32_t* W_packed, const float* alpha, int act_bits,
                                float norm_eps, float quant_eps, uint16_t* Y, uint8_t* ws,
-                               size_t ws_bytes, int32_t* dev_status, cudaStream_t s, int sms) {
+                               size_t ws_bytes, int32_t* dev_status, cudaStream_t s, int sms,
+                               unsigned variant = 0) {
     // For the default tensor-core kernel the codes stay in workspace one per
     // byte (INT4 values too) in the 32-row interleaved layout, so the GEMM
     // loads them coalesced and without widening; other back ends take the
@@ -283,15 +357,15 @@ static hbl_status forward_impl(const uint16_t* X, const float* gain, int M, int 
     int32_t* rowsum = reinterpret_cast<int32_t*>(ws + cb + sb);
     uint8_t* gws = ws + cb + 2 * sb;
     const size_t gws_bytes = ws_bytes - (cb + 2 * sb);
-    const bool il = !use_gemv(M) && g_path.load() != 1;
-    const int k1_mode = il ? (act_bits == 4 ? 5 : 9) : act_bits;
-    hbl_status st = launch_norm_fwht_quant(X, gain, M, K, norm_eps, quant_eps, k1_mode, codes,
-                                           scales, rowsum, nullptr, s, sms);
+    const FwdPlan f = forward_plan(M, K, act_bits);
+    hbl_status st = launch_norm_fwht_quant(X, gain, M, K, norm_eps, quant_eps, f.k1_mode, codes,
+                                           scales, rowsum, nullptr, s, sms, variant);
     if (st != HBL_OK) return st;
-    GemmArgs a{codes, scales, rowsum, il ? 8 : act_bits, M, K, W_packed, alpha, N, Y, nullptr,
+    GemmArgs a{codes, scales, rowsum, f.gemm_act_bits, M, K, W_packed, alpha, N, Y, nullptr,
                dev_status};
-    a.interleaved = il;
-    return run_gemm(a, gws, gws_bytes, s, sms);
+    a.interleaved = f.interleaved;
+    a.pdl = true;  // right after K1 on the same stream
+    return run_gemm(f.back, a, gws, gws_bytes, s, sms);
 }
 
 static hbl_status check_forward(const uint16_t* X, const float* gain, int M, int K, int N,
@@ -358,6 +432,122 @@ hbl_status hbl_hbitlinear_forward_hostio(const uint16_t* X_host, const float* ga
     return HBL_OK;
 }
 
+static bool flags_valid(unsigned f) {
+    return (f & ~(unsigned)(HBL_NORM_LAYERNORM | HBL_NORM_NO_HADAMARD)) == 0;
+}
+
+hbl_status hbl_norm_transform(const uint16_t* X, const float* gain, int M, int K, float norm_eps,
+                              unsigned flags, float* V, int32_t* dev_status, void* stream) {
+    (void)dev_status;
+    if (!flags_valid(flags)) return HBL_ERR_INVALID_ARG;
+    hbl_status st = check_act_args(X, gain, M, K, norm_eps);
+    if (st != HBL_OK) return st;
+    if (M == 0) return HBL_OK;
+    if (!V) return HBL_ERR_INVALID_ARG;
+    if (!aligned16(V)) return HBL_ERR_ALIGNMENT;
+    int sms = 0;
+    if ((st = device(&sms)) != HBL_OK) return st;
+    return launch_norm_fwht_quant(X, gain, M, K, norm_eps, 0.f, 0, nullptr, nullptr, nullptr, V,
+                                  static_cast<cudaStream_t>(stream), sms, flags);
+}
+
+hbl_status hbl_norm_quant(const uint16_t* X, const float* gain, int M, int K, float norm_eps,
+                          float quant_eps, int act_bits, unsigned flags, void* codes,
+                          float* scales, int32_t* rowsum, int32_t* dev_status, void* stream) {
+    (void)dev_status;
+    if (!flags_valid(flags)) return HBL_ERR_INVALID_ARG;
+    hbl_status st = check_act_args(X, gain, M, K, norm_eps);
+    if (st != HBL_OK) return st;
+    if (!act_valid(act_bits)) return HBL_ERR_INVALID_ARG;
+    if (!finite_nonneg(quant_eps)) return HBL_ERR_INVALID_ARG;
+    if (M == 0) return HBL_OK;
+    if (!codes || !scales) return HBL_ERR_INVALID_ARG;
+    if (!aligned16(codes) || !aligned16(scales) || (rowsum && !aligned16(rowsum)))
+        return HBL_ERR_ALIGNMENT;
+    int sms = 0;
+    if ((st = device(&sms)) != HBL_OK) return st;
+    return launch_norm_fwht_quant(X, gain, M, K, norm_eps, quant_eps, k1_mode_of(act_bits),
+                                  codes, scales, rowsum, nullptr,
+                                  static_cast<cudaStream_t>(stream), sms, flags);
+}
+
+hbl_status hbl_bitlinear_forward(const uint16_t* X, const float* gain, int M, int K, int N,
+                                 const uint32_t* W_packed, const float* alpha, int act_bits,
+                                 unsigned flags, float norm_eps, float quant_eps, uint16_t* Y,
+                                 void* ws, size_t ws_bytes, int32_t* dev_status, void* stream) {
+    if (!flags_valid(flags)) return HBL_ERR_INVALID_ARG;
+    hbl_status st = check_forward(X, gain, M, K, N, W_packed, alpha, act_bits, norm_eps,
+                                  quant_eps, Y, ws, ws_bytes, dev_status,
+                                  HBL_OP_HBITLINEAR_FORWARD, false);
+    if (st != HBL_OK) return st;
+    if (M == 0) return HBL_OK;
+    int sms = 0;
+    if ((st = device(&sms)) != HBL_OK) return st;
+    return forward_impl(X, gain, M, K, N, W_packed, alpha, act_bits, norm_eps, quant_eps, Y,
+                        static_cast<uint8_t*>(ws), ws_bytes, dev_status,
+                        static_cast<cudaStream_t>(stream), sms, flags);
+}
+
+hbl_status hbl_rotate_weights(const float* W, const float* signs, int N, int K, float* W_rot,
+                              int32_t* dev_status, void* stream) {
+    (void)dev_status;
+    if (N < 0 || check_k(K) != HBL_OK) return HBL_ERR_SHAPE;
+    if (N == 0) return HBL_OK;
+    if (!W || !W_rot) return HBL_ERR_INVALID_ARG;
+    if (!aligned16(W) || !aligned16(W_rot) || (signs && !aligned16(signs)))
+        return HBL_ERR_ALIGNMENT;
+    int sms = 0;
+    hbl_status st = device(&sms);
+    if (st != HBL_OK) return st;
+    return launch_rotate_weights(W, signs, N, K, W_rot, static_cast<cudaStream_t>(stream), sms);
+}
+
+hbl_status hbl_kv_quant(const uint16_t* X, int64_t rows, int D, int bits, float eps,
+                        uint8_t* codes, float* scales, int32_t* dev_status, void* stream) {
+    (void)dev_status;
+    if (!finite_nonneg(eps)) return HBL_ERR_INVALID_ARG;
+    if (bits != 2 && bits != 3 && bits != 4 && bits != 8) return HBL_ERR_INVALID_ARG;
+    if (rows < 0 || (D != 32 && D != 64 && D != 128 && D != 256)) return HBL_ERR_SHAPE;
+    if (rows == 0) return HBL_OK;
+    if (!X || !codes || !scales) return HBL_ERR_INVALID_ARG;
+    if (!aligned16(X) || !aligned16(codes) || !aligned16(scales)) return HBL_ERR_ALIGNMENT;
+    int sms = 0;
+    hbl_status st = device(&sms);
+    if (st != HBL_OK) return st;
+    return launch_kv_quant(X, rows, D, bits, eps, codes, scales,
+                           static_cast<cudaStream_t>(stream), sms);
+}
+
+hbl_status hbl_expand_ternary(const uint32_t* W_packed, int N, int K, int8_t* W_s8,
+                              int32_t* dev_status, void* stream) {
+    (void)dev_status;
+    if (N < 0 || check_k(K) != HBL_OK) return HBL_ERR_SHAPE;
+    if (N == 0) return HBL_OK;
+    if (!W_packed || !W_s8) return HBL_ERR_INVALID_ARG;
+    if (!aligned16(W_packed) || !aligned16(W_s8)) return HBL_ERR_ALIGNMENT;
+    int sms = 0;
+    hbl_status st = device(&sms);
+    if (st != HBL_OK) return st;
+    return launch_expand_ternary(W_packed, N, K, W_s8, static_cast<cudaStream_t>(stream), sms);
+}
+
+hbl_status hbl_ternary_gemm_s8w(const void* codes, const float* scales, int act_bits, int M,
+                                int K, const int8_t* W_s8, const float* alpha, int N, uint16_t* Y,
+                                int32_t* acc_out, int32_t* dev_status, void* stream) {
+    if (act_bits != 8 && act_bits != HBL_ACT_INT4_BYTES) return HBL_ERR_INVALID_ARG;
+    if (M < 0 || check_k(K) != HBL_OK || K < 128 || check_n(N) != HBL_OK) return HBL_ERR_SHAPE;
+    if (M == 0) return HBL_OK;
+    if (!codes || !scales || !W_s8 || !alpha || !Y) return HBL_ERR_INVALID_ARG;
+    if (!aligned16(codes) || !aligned16(scales) || !aligned16(W_s8) || !aligned16(alpha) ||
+        !aligned16(Y) || (acc_out && !aligned16(acc_out)) ||
+        (dev_status && !aligned16(dev_status)))
+        return HBL_ERR_ALIGNMENT;
+    int sms = 0;
+    hbl_status st = device(&sms);
+    if (st != HBL_OK) return st;
+    GemmArgs a{codes, scales, nullptr, 8, M, K, nullptr, alpha, N, Y, acc_out, dev_status};
+    return launch_gemm_tma_s8w(a, W_s8, static_cast<cudaStream_t>(stream), sms);
+}
 
 // Allocation-free ternary GEMV: the CUDA-core split-K path with its partial
 // sums in the library's fixed 2 MiB device array instead of caller workspace.

@@ -86,6 +86,20 @@ __device__ __forceinline__ void sts128(uint32_t addr, uint4 v) {
                  : "memory");
 }
 
+// ------------------------------------------------------------ dependent launch
+
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialisation may start while the previous kernel on the stream is still
+// running; it must call pdl_wait() before reading anything that kernel (or any
+// earlier work) produced.  pdl_wait() is a no-op for a normal launch.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Lets the next kernel on the stream (if launched as a dependent) start early.
+// No memory clobber: the dependent's pdl_wait() still waits for this whole grid
+// to finish and its writes to be visible, so no ordering is needed here.
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;");
+}
+
 // ------------------------------------------------------------ fp32x2 (sm_100)
 
 __device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }

@@ -12,13 +12,42 @@ namespace hbl {
 // Sets the dynamic shared-memory limit of `func` once per device (idempotent).
 bool smem_attr_once(const void* func, int bytes);
 
+// Launch with programmatic stream serialisation (the kernel must pdl_wait()
+// before reading inputs).  Returns HBL_ERR_CUDA on failure.
+template <class... KArgs, class... Args>
+hbl_status launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                      cudaStream_t stream, Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...) == cudaSuccess ? HBL_OK
+                                                                                         : HBL_ERR_CUDA;
+}
+
 // K1: mode 0 writes fp32 V; modes 4 / 8 write INT4 (packed nibbles) / INT8 codes +
-// scales (+ rowsum); modes 5 / 9 write INT4 / INT8 codes one per byte in the
-// 32-row interleaved layout of the fused forward.
+// scales (+ rowsum); mode 6 writes INT4 codes one per byte, row-major;
+// modes 5 / 9 write INT4 / INT8 codes one per byte in the
+// 32-row interleaved layout of the fused forward.  variant: HBL_NORM_* bits
+// (LayerNorm instead of RMSNorm, no Hadamard transform).
 hbl_status launch_norm_fwht_quant(const uint16_t* X, const float* gain, int64_t M, int K,
                                   float norm_eps, float quant_eps, int mode, void* codes,
                                   float* scales, int32_t* rowsum, float* V, cudaStream_t stream,
-                                  int num_sms);
+                                  int num_sms, unsigned variant = 0);
+
+// K4: offline weight rotation W_rot[n] = FWHT(W[n] * signs) * c_K (in place allowed).
+hbl_status launch_rotate_weights(const float* W, const float* signs, int N, int K, float* W_rot,
+                                 cudaStream_t stream, int num_sms);
+
+// K5: per-head absmax quantiser of Q/K/V states to unsigned `bits`-bit codes.
+hbl_status launch_kv_quant(const uint16_t* X, int64_t rows, int D, int bits, float eps,
+                           uint8_t* codes, float* scales, cudaStream_t stream, int num_sms);
 
 // K0: absmean ternarisation + 2-bit packing (K a power of two).
 size_t pack_ternary_workspace(int N, int K);
@@ -39,7 +68,10 @@ struct GemmArgs {
     uint16_t* Y;
     int32_t* acc_out;
     int32_t* dev_status;
-    bool interleaved = false;  // codes one per byte in the 32-row interleaved layout
+    bool interleaved = false;
+    // launched right after the activation kernel of the fused forward: the
+    // weights (not produced by that kernel) may be read before the dependency wait
+    bool pdl = false;  // codes one per byte in the 32-row interleaved layout
 };
 
 // K2: tcgen05 tensor-core GEMM, both operands in shared memory, any M.
@@ -56,6 +88,26 @@ hbl_status launch_splitk_epilogue(const int32_t* part, int ksplit, int64_t M, in
                                   uint16_t* Y, int32_t* acc_out, cudaStream_t stream);
 
 // K3: CUDA-core split-K GEMV for small M (M <= gemv_max_m()).
+// TMA-fed tcgen05 GEMM for large batches: codes one byte each, row-major;
+// the packed weights are expanded to signed bytes in workspace (N*K bytes).
+size_t gemm_tma_workspace(int K, int N);
+hbl_status launch_gemm_tma(const GemmArgs& a, void* ws, size_t ws_bytes, cudaStream_t stream,
+                           int num_sms);
+// The two halves of launch_gemm_tma: packed 2-bit weights -> signed bytes
+// [N x K], and the GEMM on already expanded weights (a.W_packed unused).
+hbl_status launch_expand_ternary(const uint32_t* W_packed, int N, int K, int8_t* W_s8,
+                                 cudaStream_t stream, int num_sms);
+hbl_status launch_gemm_tma_s8w(const GemmArgs& a, const int8_t* W_s8, cudaStream_t stream,
+                               int num_sms);
+
+// Row GEMV (one weight row per warp over the whole K, epilogue fused, no
+// workspace) for M <= gemv_rows_max_m(K) tokens and 2048 <= K <= 32768.
+// pdl_after_producer: launched as a programmatic dependent of the kernel that
+// wrote the codes; the weights are then loaded before the dependency wait.
+bool gemv_rows_supported(int K);
+int gemv_rows_max_m(int K);
+hbl_status launch_gemv_rows(const GemmArgs& a, bool pdl_after_producer, cudaStream_t stream);
+
 int gemv_max_m();
 size_t gemv_workspace(int64_t M, int K, int N, int num_sms);
 hbl_status launch_gemv(const GemmArgs& a, void* ws, size_t ws_bytes, cudaStream_t stream,

@@ -42,6 +42,11 @@ namespace k1 {
 constexpr int kRegLog = 7;
 constexpr int kRedFloats = 128;  // per-group cross-warp reduction scratch
 
+// Kernel variant bits (template parameter FL).
+constexpr int kFlGain = 1;
+constexpr int kFlNoHadamard = 2;
+constexpr int kFlLayerNorm = 4;
+
 // log2 of the fp32 values each thread holds: 128 in general; 64 for K = 8192
 // and 16384, where it keeps two exchanges while doubling the resident warps.
 __host__ __device__ constexpr int reg_log(int L) {
@@ -222,19 +227,26 @@ __device__ __forceinline__ float stream_tree(F&& f) {
 // ---- the kernel -------------------------------------------------------------
 
 // MODE: 0 = write fp32 V (norm + transform only), 4 = INT4 codes (packed nibbles),
-// 8 = INT8 codes (row-major); 5 / 9 = INT4 / INT8 codes one per byte in the
+// 6 = INT4 codes one per byte (row-major), 8 = INT8 codes (row-major);
+// 5 / 9 = INT4 / INT8 codes one per byte in the
 // 32-row interleaved layout the fused forward's GEMM loads (16-code chunk c of
 // row m at byte (((m / 32) * (K / 16) + c) * 32 + m % 32) * 16).
-// GAIN: multiply by the per-channel RMSNorm gain (false: gain of one, exact skip).
-template <int L, int MODE, bool GAIN>
+// FL: kFlGain = multiply by the per-channel gain (else a gain of one, exact
+// skip); kFlNoHadamard = no transform (the plain BitLinear of the layers
+// without H: the codes are those of the normalised row itself); kFlLayerNorm =
+// subtract the row mean first (LayerNorm without bias) instead of RMSNorm.
+template <int L, int MODE, int FL>
 __global__ void __launch_bounds__(Cfg<L>::kCtaThreads, Cfg<L>::kMinBlocks)
     norm_fwht_quant_kernel(Params p) {
     constexpr bool kAbsmax = (MODE == 8 || MODE == 9);       // INT8 absmax statistic
     constexpr bool kInterleaved = (MODE == 5 || MODE == 9);  // fused-forward code layout
+    constexpr bool GAIN = (FL & kFlGain) != 0;
+    constexpr bool kHadamard = (FL & kFlNoHadamard) == 0;
+    constexpr bool kLayerNorm = (FL & kFlLayerNorm) != 0;
     using C = Cfg<L>;
     using Y = Lay<L>;
     constexpr int R = C::R, T = C::T, W = C::W, K = C::K;
-    constexpr int P_LAST = C::kPasses;
+    constexpr int P_LAST = kHadamard ? C::kPasses : 0;  // final layout (natural without H)
     extern __shared__ __align__(128) uint8_t smem[];
 
     const int tid = threadIdx.x;
@@ -336,6 +348,9 @@ __global__ void __launch_bounds__(Cfg<L>::kCtaThreads, Cfg<L>::kMinBlocks)
         }
     };
 
+    // One row group per thread (small M, e.g. decode): let the next kernel
+    // start its prologue (weight prefetch) while this one works.
+    if ((int64_t)gridDim.x * C::kGroupsPerCta * C::kRowsPerGroup >= p.M) pdl_launch_dependents();
     issue_load((int64_t)blockIdx.x * C::kGroupsPerCta + grp);
     for (int64_t rg = (int64_t)blockIdx.x * C::kGroupsPerCta + grp;; rg += stride_groups) {
         const int64_t row0 = rg * C::kRowsPerGroup;
@@ -359,8 +374,23 @@ __global__ void __launch_bounds__(Cfg<L>::kCtaThreads, Cfg<L>::kMinBlocks)
         group_sync<T>(grp);  // staging buffer free again
         if constexpr (P_LAST == 0) issue_load(rg + stride_groups);  // overlaps this row's work
 
-        // ---- RMSNorm: tree over the row in ascending index order; each leaf is
-        // x0*x0 + x1*x1 with one rounding (bf16 squares are exact in fp32)
+        // ---- LayerNorm: mean by the same tree (leaves x0 + x1), subtracted first
+        if constexpr (kLayerNorm) {
+            float sx = stream_tree<R / 2>([&](auto kk) {
+                constexpr int k = decltype(kk)::value;
+                return __fadd_rn(d[k].x, d[k].y);
+            });
+            sx = row_sum(sx);
+            const float mu = __fmul_rn(sx, 1.0f / (float)K);
+            const float2 mu2 = make_float2(mu, mu);
+            static_for<0, R / 2>([&](auto kk) {
+                constexpr int k = decltype(kk)::value;
+                d[k] = sub2(d[k], mu2);
+            });
+        }
+        // ---- RMS of the row (of x - mean for LayerNorm): tree over the row in
+        // ascending index order; each leaf is d0*d0 + d1*d1 with one rounding
+        // (for RMSNorm of bf16 inputs the squares are exact in fp32)
         float ss = stream_tree<R / 2>([&](auto kk) {
             constexpr int k = decltype(kk)::value;
             return __fmaf_rn(d[k].x, d[k].x, __fmul_rn(d[k].y, d[k].y));
@@ -386,7 +416,8 @@ __global__ void __launch_bounds__(Cfg<L>::kCtaThreads, Cfg<L>::kMinBlocks)
         }
 
         // ---- Walsh-Hadamard butterflies: natural layout, stages 0..r-1
-        static_for<0, C::r>([&](auto rr) { stage_regs<R, decltype(rr)::value>(d); });
+        if constexpr (kHadamard)
+            static_for<0, C::r>([&](auto rr) { stage_regs<R, decltype(rr)::value>(d); });
 
         // ---- exchanges through shared memory, one per pass
         static_for<1, P_LAST + 1>([&](auto pp) {
@@ -429,7 +460,7 @@ __global__ void __launch_bounds__(Cfg<L>::kCtaThreads, Cfg<L>::kMinBlocks)
         if constexpr (P_LAST > 0) issue_load(rg + stride_groups);
 
         // ---- normalise by 1/sqrt(K)
-        {
+        if constexpr (kHadamard) {
             const float2 c2 = make_float2(p.cK, p.cK);
             static_for<0, R / 2>([&](auto kk) {
                 constexpr int k = decltype(kk)::value;
@@ -520,7 +551,10 @@ __global__ void __launch_bounds__(Cfg<L>::kCtaThreads, Cfg<L>::kMinBlocks)
             }
 
             const float cq = kAbsmax ? 127.0f : p.s7;
-            const float inv = __fdiv_rn(cq, __fadd_rn(stat, p.quant_eps));
+            // (a zero row with quant_eps = 0: inv = 0, so every code is 0)
+            const float den = __fadd_rn(stat, p.quant_eps);
+            const bool pos = den > 0.f;
+            const float inv = __fdiv_rn(pos ? cq : 0.f, pos ? den : 1.f);
             const float2 inv2 = make_float2(inv, inv);
             // One rounding of the exact product v*inv to an integer: fma with
             // 1.5*2^23 (+8 for packed INT4, making the stored nibble q + 8).
@@ -614,10 +648,10 @@ __global__ void __launch_bounds__(Cfg<L>::kCtaThreads, Cfg<L>::kMinBlocks)
     }
 }
 
-template <int L, int MODE, bool GAIN>
+template <int L, int MODE, int FL>
 static hbl_status launch_one(const Params& prm, cudaStream_t stream, int num_sms) {
     using C = Cfg<L>;
-    auto kern = norm_fwht_quant_kernel<L, MODE, GAIN>;
+    auto kern = norm_fwht_quant_kernel<L, MODE, FL>;
     if (!smem_attr_once(reinterpret_cast<const void*>(kern), C::kSmemBytes)) return HBL_ERR_CUDA;
     const int64_t groups = (prm.M + C::kRowsPerGroup - 1) / C::kRowsPerGroup;
     const int64_t ctas_needed = (groups + C::kGroupsPerCta - 1) / C::kGroupsPerCta;
@@ -628,21 +662,21 @@ static hbl_status launch_one(const Params& prm, cudaStream_t stream, int num_sms
     return cudaGetLastError() == cudaSuccess ? HBL_OK : HBL_ERR_CUDA;
 }
 
-template <int MODE, bool GAIN>
+template <int MODE, int FL>
 hbl_status dispatch(int L, const Params& prm, cudaStream_t s, int sms) {
     switch (L) {
-        case 4: return launch_one<4, MODE, GAIN>(prm, s, sms);
-        case 5: return launch_one<5, MODE, GAIN>(prm, s, sms);
-        case 6: return launch_one<6, MODE, GAIN>(prm, s, sms);
-        case 7: return launch_one<7, MODE, GAIN>(prm, s, sms);
-        case 8: return launch_one<8, MODE, GAIN>(prm, s, sms);
-        case 9: return launch_one<9, MODE, GAIN>(prm, s, sms);
-        case 10: return launch_one<10, MODE, GAIN>(prm, s, sms);
-        case 11: return launch_one<11, MODE, GAIN>(prm, s, sms);
-        case 12: return launch_one<12, MODE, GAIN>(prm, s, sms);
-        case 13: return launch_one<13, MODE, GAIN>(prm, s, sms);
-        case 14: return launch_one<14, MODE, GAIN>(prm, s, sms);
-        case 15: return launch_one<15, MODE, GAIN>(prm, s, sms);
+        case 4: return launch_one<4, MODE, FL>(prm, s, sms);
+        case 5: return launch_one<5, MODE, FL>(prm, s, sms);
+        case 6: return launch_one<6, MODE, FL>(prm, s, sms);
+        case 7: return launch_one<7, MODE, FL>(prm, s, sms);
+        case 8: return launch_one<8, MODE, FL>(prm, s, sms);
+        case 9: return launch_one<9, MODE, FL>(prm, s, sms);
+        case 10: return launch_one<10, MODE, FL>(prm, s, sms);
+        case 11: return launch_one<11, MODE, FL>(prm, s, sms);
+        case 12: return launch_one<12, MODE, FL>(prm, s, sms);
+        case 13: return launch_one<13, MODE, FL>(prm, s, sms);
+        case 14: return launch_one<14, MODE, FL>(prm, s, sms);
+        case 15: return launch_one<15, MODE, FL>(prm, s, sms);
         default: return HBL_ERR_SHAPE;
     }
 }

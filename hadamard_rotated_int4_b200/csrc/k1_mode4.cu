@@ -1,10 +1,10 @@
 // k1_mode4.cu -- instantiations of the fused norm + transform + quantisation
-// kernel for mode 4 (INT4 codes), with and without a gain vector.
+// kernel for mode 4: RMSNorm + Hadamard, with and without a gain vector.
 #include "k1_impl.cuh"
 
 namespace hbl {
 namespace k1 {
-template hbl_status dispatch<4, false>(int, const Params&, cudaStream_t, int);
-template hbl_status dispatch<4, true>(int, const Params&, cudaStream_t, int);
+template hbl_status dispatch<4, 0>(int, const Params&, cudaStream_t, int);
+template hbl_status dispatch<4, kFlGain>(int, const Params&, cudaStream_t, int);
 }  // namespace k1
 }  // namespace hbl

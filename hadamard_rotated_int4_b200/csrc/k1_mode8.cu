@@ -1,10 +1,10 @@
 // k1_mode8.cu -- instantiations of the fused norm + transform + quantisation
-// kernel for mode 8 (INT8 codes), with and without a gain vector.
+// kernel for mode 8: RMSNorm + Hadamard, with and without a gain vector.
 #include "k1_impl.cuh"
 
 namespace hbl {
 namespace k1 {
-template hbl_status dispatch<8, false>(int, const Params&, cudaStream_t, int);
-template hbl_status dispatch<8, true>(int, const Params&, cudaStream_t, int);
+template hbl_status dispatch<8, 0>(int, const Params&, cudaStream_t, int);
+template hbl_status dispatch<8, kFlGain>(int, const Params&, cudaStream_t, int);
 }  // namespace k1
 }  // namespace hbl

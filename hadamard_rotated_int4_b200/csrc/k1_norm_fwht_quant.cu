@@ -9,7 +9,7 @@
 namespace hbl {
 namespace k1 {
 struct Params;
-template <int MODE, bool GAIN>
+template <int MODE, int FL>
 hbl_status dispatch(int L, const Params& prm, cudaStream_t s, int sms);
 }  // namespace k1
 }  // namespace hbl
@@ -18,22 +18,43 @@ hbl_status dispatch(int L, const Params& prm, cudaStream_t s, int sms);
 
 namespace hbl {
 namespace k1 {
-extern template hbl_status dispatch<0, false>(int, const Params&, cudaStream_t, int);
-extern template hbl_status dispatch<0, true>(int, const Params&, cudaStream_t, int);
-extern template hbl_status dispatch<4, false>(int, const Params&, cudaStream_t, int);
-extern template hbl_status dispatch<4, true>(int, const Params&, cudaStream_t, int);
-extern template hbl_status dispatch<5, false>(int, const Params&, cudaStream_t, int);
-extern template hbl_status dispatch<5, true>(int, const Params&, cudaStream_t, int);
-extern template hbl_status dispatch<9, false>(int, const Params&, cudaStream_t, int);
-extern template hbl_status dispatch<9, true>(int, const Params&, cudaStream_t, int);
-extern template hbl_status dispatch<8, false>(int, const Params&, cudaStream_t, int);
-extern template hbl_status dispatch<8, true>(int, const Params&, cudaStream_t, int);
+#define HBL_K1_EXTERN(MODE)                                                                      \
+    extern template hbl_status dispatch<MODE, 0>(int, const Params&, cudaStream_t, int);        \
+    extern template hbl_status dispatch<MODE, 1>(int, const Params&, cudaStream_t, int);        \
+    extern template hbl_status dispatch<MODE, 2>(int, const Params&, cudaStream_t, int);        \
+    extern template hbl_status dispatch<MODE, 3>(int, const Params&, cudaStream_t, int);        \
+    extern template hbl_status dispatch<MODE, 4>(int, const Params&, cudaStream_t, int);        \
+    extern template hbl_status dispatch<MODE, 5>(int, const Params&, cudaStream_t, int);        \
+    extern template hbl_status dispatch<MODE, 6>(int, const Params&, cudaStream_t, int);        \
+    extern template hbl_status dispatch<MODE, 7>(int, const Params&, cudaStream_t, int);
+HBL_K1_EXTERN(0)
+HBL_K1_EXTERN(4)
+HBL_K1_EXTERN(5)
+HBL_K1_EXTERN(6)
+HBL_K1_EXTERN(8)
+HBL_K1_EXTERN(9)
+#undef HBL_K1_EXTERN
+
+template <int MODE>
+static hbl_status by_flags(int fl, int L, const Params& prm, cudaStream_t s, int sms) {
+    switch (fl) {
+        case 0: return dispatch<MODE, 0>(L, prm, s, sms);
+        case 1: return dispatch<MODE, 1>(L, prm, s, sms);
+        case 2: return dispatch<MODE, 2>(L, prm, s, sms);
+        case 3: return dispatch<MODE, 3>(L, prm, s, sms);
+        case 4: return dispatch<MODE, 4>(L, prm, s, sms);
+        case 5: return dispatch<MODE, 5>(L, prm, s, sms);
+        case 6: return dispatch<MODE, 6>(L, prm, s, sms);
+        case 7: return dispatch<MODE, 7>(L, prm, s, sms);
+        default: return HBL_ERR_INVALID_ARG;
+    }
+}
 }  // namespace k1
 
 hbl_status launch_norm_fwht_quant(const uint16_t* X, const float* gain, int64_t M, int K,
                                   float norm_eps, float quant_eps, int mode, void* codes,
                                   float* scales, int32_t* rowsum, float* V, cudaStream_t stream,
-                                  int num_sms) {
+                                  int num_sms, unsigned variant) {
     if (M == 0) return HBL_OK;
     k1::Params prm;
     prm.X = X;
@@ -48,18 +69,16 @@ hbl_status launch_norm_fwht_quant(const uint16_t* X, const float* gain, int64_t 
     prm.rowsum = rowsum;
     prm.V = V;
     const int L = ilog2((unsigned)K);
-    const bool g = gain != nullptr;
+    const int fl = (gain != nullptr ? k1::kFlGain : 0) |
+                   ((variant & HBL_NORM_NO_HADAMARD) ? k1::kFlNoHadamard : 0) |
+                   ((variant & HBL_NORM_LAYERNORM) ? k1::kFlLayerNorm : 0);
     switch (mode) {
-        case 0: return g ? k1::dispatch<0, true>(L, prm, stream, num_sms)
-                         : k1::dispatch<0, false>(L, prm, stream, num_sms);
-        case 4: return g ? k1::dispatch<4, true>(L, prm, stream, num_sms)
-                         : k1::dispatch<4, false>(L, prm, stream, num_sms);
-        case 5: return g ? k1::dispatch<5, true>(L, prm, stream, num_sms)
-                         : k1::dispatch<5, false>(L, prm, stream, num_sms);
-        case 9: return g ? k1::dispatch<9, true>(L, prm, stream, num_sms)
-                         : k1::dispatch<9, false>(L, prm, stream, num_sms);
-        case 8: return g ? k1::dispatch<8, true>(L, prm, stream, num_sms)
-                         : k1::dispatch<8, false>(L, prm, stream, num_sms);
+        case 0: return k1::by_flags<0>(fl, L, prm, stream, num_sms);
+        case 4: return k1::by_flags<4>(fl, L, prm, stream, num_sms);
+        case 5: return k1::by_flags<5>(fl, L, prm, stream, num_sms);
+        case 6: return k1::by_flags<6>(fl, L, prm, stream, num_sms);
+        case 8: return k1::by_flags<8>(fl, L, prm, stream, num_sms);
+        case 9: return k1::by_flags<9>(fl, L, prm, stream, num_sms);
         default: return HBL_ERR_INVALID_ARG;
     }
 }

@@ -292,7 +292,10 @@ __device__ __forceinline__ void store_stage(uint32_t a_taddr, uint32_t sB, const
     }
 }
 
-template <int ABITS, bool IL, bool FULLK>
+// SMALL: a single tile of tokens (M <= 256, decode batches): split-K over
+// grid.z, one accumulator when M <= 128, and the weights prefetched into L2
+// before the dependency wait.  The large-M instantiation keeps none of these.
+template <int ABITS, bool IL, bool FULLK, bool SMALL>
 __global__ void __launch_bounds__(kThreads, 1) gemm_ts_kernel(Params p) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_s = smem_addr(smem_raw);
@@ -312,10 +315,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_ts_kernel(Params p) {
     const int64_t m0 = (int64_t)blockIdx.y * BM;
     // this CTA's K-blocks: [kb0, kb0 + num_kb) of the whole K (split-K over grid.z)
     const int num_kb_total = (p.K + BK - 1) / BK;
-    const int kb0 = (int)blockIdx.z * p.kps;
-    const int num_kb = min(p.kps, num_kb_total - kb0);
+    const int kb0 = SMALL ? (int)blockIdx.z * p.kps : 0;
+    const int num_kb = SMALL ? min(p.kps, num_kb_total - kb0) : num_kb_total;
     // rows of this tile that exist: one accumulator suffices when M - m0 <= 128
-    const int nacc = (p.M - m0 > 128) ? 2 : 1;
+    const int nacc = (!SMALL || p.M - m0 > 128) ? 2 : 1;
 
     if (tid == 0) {
         for (int s = 0; s < S; ++s) {
@@ -333,6 +336,17 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_ts_kernel(Params p) {
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
+    // Packed weights of this CTA into L2 while the previous kernel finishes
+    // (a hint: it reads nothing into registers), then wait for its outputs.
+    // (K >= 64 keeps every row start and length a multiple of 16 bytes.)
+    if (SMALL && tid >= 32 && tid < 32 + BN && p.K >= 64 && num_kb > 0) {
+        const int n = n0 + tid - 32;
+        if (n < p.N) {
+            const int k_lo = kb0 * BK, k_hi = min((kb0 + num_kb) * BK, p.K);
+            prefetch_l2_bulk(p.W + (int64_t)n * (p.K / 16) + k_lo / 16, (uint32_t)(k_hi - k_lo) / 4);
+        }
+    }
+    pdl_wait();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -426,8 +440,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_ts_kernel(Params p) {
                 }
                 const int nn = n < p.N ? n : p.N - 1;
                 ld.b = p.W + (int64_t)nn * (p.K / 16) + 4 * bh;
-                ld.a += (int64_t)kb0 * (IL ? 8 * 512 : (ABITS == 8 ? BK : BK / 2));
-                ld.b += kb0 * (BK / 16);
+                if constexpr (SMALL) {
+                    ld.a += (int64_t)kb0 * (IL ? 8 * 512 : (ABITS == 8 ? BK : BK / 2));
+                    ld.b += kb0 * (BK / 16);
+                }
             }
             // three stages of operands in flight in registers
             Packed<ABITS> P2;
@@ -499,7 +515,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_ts_kernel(Params p) {
                     : "r"(taddr));
                 asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
                 const int nc = n0 + 32 * cc;
-                if (p.part != nullptr) {  // split-K: raw partial sums, reduced by a second kernel
+                if (SMALL && p.part != nullptr) {  // split-K: raw partial sums, reduced by a second kernel
                     if (mok && nc < p.N) {
                         int4* pd = reinterpret_cast<int4*>(
                             p.part + ((int64_t)blockIdx.z * p.M + m) * p.N + nc);
@@ -556,14 +572,16 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_ts_kernel(Params p) {
 
 template <int ABITS, bool IL>
 static hbl_status launch(const Params& prm, cudaStream_t stream) {
-    auto kern = (prm.K % BK == 0) ? gemm_ts_kernel<ABITS, IL, true>
-                                  : gemm_ts_kernel<ABITS, IL, false>;
+    const bool full = prm.K % BK == 0, small = prm.M <= BM;
+    auto kern = full ? (small ? gemm_ts_kernel<ABITS, IL, true, true>
+                              : gemm_ts_kernel<ABITS, IL, true, false>)
+                     : (small ? gemm_ts_kernel<ABITS, IL, false, true>
+                              : gemm_ts_kernel<ABITS, IL, false, false>);
     if (!smem_attr_once(reinterpret_cast<const void*>(kern), kSmemBytes)) return HBL_ERR_CUDA;
     const int num_kb = (prm.K + BK - 1) / BK;
     dim3 grid((prm.N + BN - 1) / BN, (unsigned)((prm.M + BM - 1) / BM),
               (unsigned)((num_kb + prm.kps - 1) / prm.kps));
-    kern<<<grid, kThreads, kSmemBytes, stream>>>(prm);
-    return cudaGetLastError() == cudaSuccess ? HBL_OK : HBL_ERR_CUDA;
+    return launch_pdl(kern, grid, dim3(kThreads), kSmemBytes, stream, prm);
 }
 
 }  // namespace k2b

@@ -53,6 +53,11 @@ __global__ void __launch_bounds__(kWarps * 32)
     const int n0 = blockIdx.x * kRowsPerCta;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
+    // this CTA's weight slice into L2 while the previous kernel finishes, then wait
+    if (tid < kRowsPerCta && n0 + tid < N && klen >= 64)
+        prefetch_l2_bulk(Wp + (int64_t)(n0 + tid) * (K / 16) + k0 / 16, (uint32_t)(klen / 4));
+    pdl_wait();
+
     // stage activations [MT][klen] as int8 (rows >= M zero)
     const int chunks = klen / 16;  // 16 int8 per chunk
     for (int c = tid; c < MT * chunks; c += blockDim.x) {
@@ -130,6 +135,7 @@ __global__ void gemv_epilogue_kernel(const int32_t* __restrict__ part, int kspli
                                      const float* __restrict__ scales,
                                      const float* __restrict__ alpha, uint16_t* __restrict__ Y,
                                      int32_t* __restrict__ acc_out) {
+    pdl_wait();
     const float a = *alpha;
     const int64_t total = (int64_t)M * N;
     for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
@@ -165,9 +171,8 @@ hbl_status launch_splitk_epilogue(const int32_t* part, int ksplit, int64_t M, in
     const int64_t total = M * N;
     int64_t eb = (total + 255) / 256;
     if (eb > 148 * 8) eb = 148 * 8;
-    k3::gemv_epilogue_kernel<<<(unsigned)eb, 256, 0, stream>>>(part, ksplit, (int)M, N, rowsum,
-                                                               scales, alpha, Y, acc_out);
-    return cudaGetLastError() == cudaSuccess ? HBL_OK : HBL_ERR_CUDA;
+    return launch_pdl(k3::gemv_epilogue_kernel, dim3((unsigned)eb), dim3(256), 0, stream, part,
+                      ksplit, (int)M, N, rowsum, scales, alpha, Y, acc_out);
 }
 
 size_t gemv_workspace(int64_t M, int K, int N, int num_sms) {
@@ -195,9 +200,9 @@ hbl_status launch_gemv(const GemmArgs& a, void* ws, size_t ws_bytes, cudaStream_
         if (smem > 48 * 1024 &&                                                                 \
             !smem_attr_once(reinterpret_cast<const void*>(k3::gemv_kernel<MT>), (int)smem))     \
             return HBL_ERR_CUDA;                                                                \
-        k3::gemv_kernel<MT><<<grid, k3::kWarps * 32, smem, stream>>>(codes, a.act_bits, M, a.K, \
-                                                                     a.W_packed, a.N, kslice,   \
-                                                                     part);                     \
+        if (launch_pdl(k3::gemv_kernel<MT>, grid, dim3(k3::kWarps * 32), smem, stream, codes,    \
+                       a.act_bits, M, a.K, a.W_packed, a.N, kslice, part) != HBL_OK)             \
+            return HBL_ERR_CUDA;                                                                \
         break;
     switch (mt) {
         HBL_GEMV_CASE(1)
@@ -210,9 +215,9 @@ hbl_status launch_gemv(const GemmArgs& a, void* ws, size_t ws_bytes, cudaStream_
     const int64_t total = a.M * a.N;
     int64_t eb = (total + 255) / 256;
     if (eb > (int64_t)num_sms * 8) eb = (int64_t)num_sms * 8;
-    k3::gemv_epilogue_kernel<<<(unsigned)eb, 256, 0, stream>>>(part, ks, M, a.N, a.rowsum,
-                                                               a.scales, a.alpha, a.Y, a.acc_out);
-    return cudaGetLastError() == cudaSuccess ? HBL_OK : HBL_ERR_CUDA;
+    return launch_pdl(k3::gemv_epilogue_kernel, dim3((unsigned)eb), dim3(256), 0, stream,
+                      (const int32_t*)part, ks, M, a.N, a.rowsum, a.scales, a.alpha, a.Y,
+                      a.acc_out);
 }
 
 

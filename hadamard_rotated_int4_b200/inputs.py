@@ -19,6 +19,11 @@ Workloads (tokens x in-features -> out-features):
   ffn_wdown  8192 x 16384 -> 4096, silu(a)*b with a, b ~ N(0,1), 1% channels x 40
   decode     T x 4096 -> 4096 (attn_wo recipe) and T x 16384 -> 4096 (ffn_wdown
              recipe), T in {1, 8, 32, 128, 256}
+  qkv        Q, K, V states after RoPE for the KV-cache quantiser: 8192 tokens x
+             (3 x 32) heads x 128, N(0,1) times a per-(token, head) log-normal
+             magnitude (sigma 0.5), with 2% of the head dimensions (the same for
+             every token) x 8, standing in for the outlier dimensions of keys
+  signs      +-1 fp32 vector (fair coin) for the randomised Hadamard transform
 """
 import numpy as np
 
@@ -99,3 +104,25 @@ def weights(name, seed=0, N=None, K=None):
     N = w.get("N") if N is None else N
     K = w.get("K") if K is None else K
     return latent_weights(N, K, seed)
+
+
+QKV = dict(T=8192, H=96, D=128)  # 7B-like: 32 query + 32 key + 32 value heads of 128
+
+
+def qkv_states(T=None, H=None, D=None, seed=0, frac=0.02, mult=8.0):
+    """bf16 bit patterns [T x H x D] of attention states after RoPE."""
+    T = QKV["T"] if T is None else T
+    H = QKV["H"] if H is None else H
+    D = QKV["D"] if D is None else D
+    rng = np.random.default_rng(seed + 7919)
+    x = rng.standard_normal((T, H, D), dtype=np.float32)
+    mag = np.exp(rng.standard_normal((T, H, 1)) * 0.5).astype(np.float32)
+    x *= mag
+    dims = outlier_channels(rng, D, count=max(1, int(round(frac * D))))
+    x[:, :, dims] *= np.float32(mult)
+    return _to_bf16_bits(x)
+
+
+def random_signs(K, seed=0):
+    rng = np.random.default_rng(seed + 104729)
+    return np.where(rng.random(K) < 0.5, -1.0, 1.0).astype(np.float32)

@@ -77,11 +77,16 @@ HBL_API int hbl_version(void);
 
 /* Choice of ternary-GEMM back end (test and tuning aid; process-wide, not
  * synchronised with calls in flight on other threads):
- *   0 = automatic (CUDA-core split-K GEMV for M <= 8 tokens, otherwise the
- *       tcgen05 kernel with activations in tensor memory),
- *   1 = tcgen05 with both operands in shared memory,
+ *   0 = automatic: CUDA-core GEMV for M <= 8 tokens (one weight row per warp
+ *       for K >= 2048, split-K below); the tcgen05 kernel with activations in
+ *       tensor memory (split over K for M <= 256) up to 256 tokens; above that
+ *       the TMA-fed tcgen05 kernel when the codes are one byte each (it expands
+ *       the packed weights to signed bytes in workspace first),
+ *   1 = tcgen05 with both operands staged in shared memory by threads,
  *   2 = always the GEMV path (large M runs in chunks of 8 tokens),
- *   3 = always the tcgen05 kernel with activations in tensor memory.
+ *   3 = always the tcgen05 kernel with activations in tensor memory,
+ *   4 = the TMA-fed tcgen05 kernel whenever the codes are one byte each and
+ *       K >= 128 (else as 3).
  * hbl_workspace_size() answers for the path in force.  Returns HBL_OK or
  * HBL_ERR_INVALID_ARG.  This call has no counterpart on the BitNet v2 pages. */
 HBL_API int hbl_set_gemm_path(int path);
@@ -96,6 +101,12 @@ HBL_API int hbl_set_gemm_path(int path);
  * hbl_hbitlinear_forward uses it internally.  hbl_ternary_gemm always runs its
  * tcgen05 kernel for these layouts, whatever hbl_set_gemm_path says. */
 enum { HBL_ACT_INT4_I32 = 0x104, HBL_ACT_INT8_I32 = 0x108 };
+
+/* act_bits may also be HBL_ACT_INT4_BYTES: INT4 codes stored one byte each
+ * (two's complement), row-major [M x K], like the INT8 layout.  The TMA-fed
+ * tensor-core GEMM (large batches) reads one-byte codes; hbl_hbitlinear_forward
+ * uses this layout internally for INT4 batches above 256 tokens. */
+enum { HBL_ACT_INT4_BYTES = 0x204 };
 
 /* Operation identifiers for hbl_workspace_size(). */
 enum {
@@ -180,6 +191,98 @@ HBL_API hbl_status hbl_hbitlinear_forward_hostio(const uint16_t* X_host, const f
                                          const float* alpha, int act_bits, float norm_eps,
                                          float quant_eps, uint16_t* Y_host, void* ws,
                                          size_t ws_bytes, int32_t* dev_status, void* stream);
+
+/* ---------------------------------------------------------------- variants
+ * BitNet v2 uses H-BitLinear only at Wo and W_down; its other linear layers are
+ * the plain BitLinear: the same normalise -> quantise -> ternary matmul without
+ * the Hadamard transform (write-up on 0755model.com, section "BitNet v2：原生4位
+ * 激活": all linears except the embeddings are fine-tuned to 4-bit activations).
+ * The layer expression there writes the normalisation as LN and glosses it as
+ * layer normalisation, while the architecture uses RMS normalisation; both are
+ * offered.  Flags (bitwise or):
+ *   HBL_NORM_LAYERNORM:   LayerNorm without bias instead of RMSNorm:
+ *       mu = tree_sum(x) * (1/K);  d = x - mu;
+ *       r = 1 / sqrt(tree_sum(d*d) * (1/K) + norm_eps);  u = (d * r) * gain
+ *       (tree sums as for RMSNorm; the leaves of the d*d sum are
+ *        d0*d0 + d1*d1 with one rounding).
+ *   HBL_NORM_NO_HADAMARD: no transform: the codes quantise u itself.
+ * flags = 0 is exactly the H-BitLinear path of the calls above.  Other bits
+ * return HBL_ERR_INVALID_ARG.  Shapes and layouts as above (K a power of two). */
+enum { HBL_NORM_LAYERNORM = 1, HBL_NORM_NO_HADAMARD = 2 };
+
+/* hbl_norm_fwht with variant flags: V = T(N(x)) fp32 [M x K]. */
+HBL_API hbl_status hbl_norm_transform(const uint16_t* X, const float* gain, int M, int K,
+                                      float norm_eps, unsigned flags, float* V,
+                                      int32_t* dev_status, void* stream);
+
+/* hbl_norm_fwht_quant with variant flags (act_bits 4, 8, or the interleaved
+ * HBL_ACT_INT*_I32 layouts). */
+HBL_API hbl_status hbl_norm_quant(const uint16_t* X, const float* gain, int M, int K,
+                                  float norm_eps, float quant_eps, int act_bits, unsigned flags,
+                                  void* codes, float* scales, int32_t* rowsum,
+                                  int32_t* dev_status, void* stream);
+
+/* The whole BitLinear / H-BitLinear layer with variant flags; workspace as for
+ * HBL_OP_HBITLINEAR_FORWARD. */
+HBL_API hbl_status hbl_bitlinear_forward(const uint16_t* X, const float* gain, int M, int K,
+                                         int N, const uint32_t* W_packed, const float* alpha,
+                                         int act_bits, unsigned flags, float norm_eps,
+                                         float quant_eps, uint16_t* Y, void* ws, size_t ws_bytes,
+                                         int32_t* dev_status, void* stream);
+
+/* Offline weight rotation (BitNet v2 write-up, table 5: the Hadamard rotation
+ * applied to weights and activations; the QuaRot baseline there uses a
+ * randomised Hadamard transform H . diag(s)):
+ *   W_rot[n] = ((W[n] * s) . H_K) * c_K      for every row n,
+ * with the butterfly order and c_K of hbl_norm_fwht.  Then
+ * (x D H c_K) . (w D H c_K) = x . w for D = diag(s), so rotated weights pair with
+ * activations normalised with gain' = gain * s (hbl_norm_* with that gain: the
+ * product with +-1 is exact) and transformed as usual.  Ternarise W_rot with
+ * hbl_pack_ternary.
+ * W: fp32 [N x K] device; signs: fp32 [K] of +-1 or NULL (all ones; the plain
+ * transform); W_rot: fp32 [N x K] out, may be W itself (in place).
+ * K: power of two in [16, 32768]; N >= 0. */
+HBL_API hbl_status hbl_rotate_weights(const float* W, const float* signs, int N, int K,
+                                      float* W_rot, int32_t* dev_status, void* stream);
+
+/* Per-head absmax quantiser of Q, K, V states after RoPE, to unsigned integers
+ * (BitNet v2 write-up, section "实验结果", tables 2 and 3: QKV heads quantised
+ * with absmax directly to unsigned integers, no calibration; 3-bit KV cache).
+ * One row = one head of one token, D values:
+ *   Qp = 2^(bits-1) - 1;  gamma = max|x|;  inv = Qp / (gamma + eps)  (one division)
+ *   q = clip(rhe(x * inv), -Qp-1, Qp);  u = q + 2^(bits-1);  scales[row] = gamma / Qp
+ * (the INT8 activation quantiser taken to `bits` bits and offset into the
+ * unsigned range; dequantise as (u - 2^(bits-1)) * scale).
+ * X: bf16 [rows x D] (e.g. [tokens x heads x D]); bits in {2, 3, 4, 8};
+ * D in {32, 64, 128, 256}; eps >= 0 finite.
+ * codes: [rows x D*bits/8] bytes out: each group of 32 consecutive codes of a
+ * row is 4*bits bytes, code j of the group at bits [bits*j, bits*j + bits) of
+ * the group read as a little-endian integer.  scales: fp32 [rows] out. */
+HBL_API hbl_status hbl_kv_quant(const uint16_t* X, int64_t rows, int D, int bits, float eps,
+                                uint8_t* codes, float* scales, int32_t* dev_status, void* stream);
+
+/* --------------------------------------------------- expanded-weight GEMM
+ * For large token batches the tensor-core GEMM reads the ternary weights as
+ * one signed byte each (tcgen05 has no integer MMA narrower than 8 bits);
+ * hbl_ternary_gemm and hbl_hbitlinear_forward expand the packed weights into
+ * workspace on every call.  A caller that keeps the expanded copy (N*K bytes,
+ * 4x the packed size) can skip that step with these two calls.  No
+ * counterpart on the BitNet v2 pages: a deployment aid.
+ *
+ * hbl_expand_ternary: W_s8[n][k] = t[n][k] in {-1, 0, +1} (int8, row-major
+ * [N x K]) from W_packed (layout above).  K as for the layer; N >= 0. */
+HBL_API hbl_status hbl_expand_ternary(const uint32_t* W_packed, int N, int K, int8_t* W_s8,
+                                      int32_t* dev_status, void* stream);
+
+/* The TMA-fed tensor-core GEMM on expanded weights:
+ *   Y[m][n] = bf16_rne((float)(sum_k q[m][k] * W_s8[n][k]) * (alpha * scales[m]))
+ * codes: one byte per code, row-major [M x K]: act_bits 8 (INT8) or
+ * HBL_ACT_INT4_BYTES.  K >= 128 (a power of two as above).  acc_out: int32
+ * [M x N] or NULL.  No workspace; no rowsum needed (the weights are signed). */
+HBL_API hbl_status hbl_ternary_gemm_s8w(const void* codes, const float* scales, int act_bits,
+                                        int M, int K, const int8_t* W_s8, const float* alpha,
+                                        int N, uint16_t* Y, int32_t* acc_out,
+                                        int32_t* dev_status, void* stream);
 
 /* Allocation-free ternary GEMV (no counterpart on the BitNet v2 pages; it is a
  * deployment aid).  Same arguments, layouts and results as hbl_ternary_gemm

@@ -280,7 +280,9 @@ ORACLE_API int oracle_norm_transform(const uint16_t* X, const float* gain, int M
 
 /* ------------------------------------------- activation quantisers [P2][P4] */
 
-/* Quantise fp32 rows V [M x K] per token.
+/* Quantise fp32 rows V [M x K] per token.  A zero row with eps = 0 would divide
+ * by zero; inv is then taken as 0, so the row quantises to zeros (scale 0), as
+ * it does for any eps > 0.
  *   act_bits = 8 (absmax):  gamma = max|v|;  q = clip(round(v * (127/(gamma+eps))), -128, 127);
  *                           scale = gamma / 127.
  *   act_bits = 4 (absmean): beta = tree_sum(|v|) * (1/K);
@@ -314,13 +316,13 @@ ORACLE_API int oracle_quantize_rows(const float* V, int M, int K, float quant_ep
         if (act_bits == 8) {
             float g = 0.0f;
             for (int k = 0; k < K; ++k) { float a = fabsf(v[k]); if (a > g) g = a; }
-            inv = 127.0f / (g + quant_eps);
+            inv = (g + quant_eps) > 0.0f ? 127.0f / (g + quant_eps) : 0.0f;
             scale = g / 127.0f;
             lo = -128; hi = 127;
         } else {
             for (int k = 0; k < K; ++k) absv[k] = fabsf(v[k]);
             float beta = tree_sum_f32(absv, K) * (1.0f / (float)K);
-            inv = s7 / (beta + quant_eps);
+            inv = (beta + quant_eps) > 0.0f ? s7 / (beta + quant_eps) : 0.0f;
             scale = beta / s7;
             lo = -8; hi = 7;
         }
@@ -424,7 +426,8 @@ ORACLE_API int oracle_rotate_weights(const float* W, const float* signs, int N, 
 
 /* ------------------------------------------ QKV / KV-cache quantiser [P2-QKV] */
 
-/* Per-head absmax quantisation to unsigned b-bit integers (b in 2..8), for Q,
+/* Per-head absmax quantisation to unsigned b-bit integers (b in 2..8)
+ * (inv = 0 when gamma + eps == 0, as in quantize_rows) for Q,
  * K and V states after RoPE.  Each row of X [rows x D] bf16 is one head of one
  * token.  The symmetric absmax quantiser of the INT8 activations, taken to b
  * bits and offset into the unsigned range:
@@ -448,7 +451,7 @@ ORACLE_API int oracle_kv_quant(const uint16_t* X, int64_t rows, int D, int bits,
             float a = fabsf(oracle_bf16_to_f32(x[k]));
             if (a > g) g = a;
         }
-        const float inv = (float)qp / (g + eps);
+        const float inv = (g + eps) > 0.0f ? (float)qp / (g + eps) : 0.0f;
         uint8_t* out = codes + r * row_bytes;
         memset(out, 0, (size_t)row_bytes);
         for (int k = 0; k < D; ++k) {

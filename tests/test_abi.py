@@ -56,9 +56,9 @@ def test_workspace_sizes():
     # pack: one float per weight row (rounded to 256 B)
     assert hbl.workspace_size(hbl.OP_PACK_TERNARY, 0, 4096, 100, 0) == 512
     # forward: codes + scales + rowsum, each 256-aligned (tensor-core path: no GEMM scratch)
+    M, K, N = 8192, 16384, 4096
     hbl.set_gemm_path(1)
     try:
-        M, K, N = 8192, 16384, 4096
         got = hbl.workspace_size(hbl.OP_HBITLINEAR_FORWARD, M, K, N, 4)
         assert got == M * K + 2 * M * 4  # codes one byte each inside the layer (M % 32 == 0)
         got8 = hbl.workspace_size(hbl.OP_HBITLINEAR_FORWARD, M, K, N, 8)
@@ -68,8 +68,15 @@ def test_workspace_sizes():
         assert hbl.workspace_size(hbl.OP_TERNARY_GEMM, M, K, N, 4) == 0
     finally:
         hbl.set_gemm_path(0)
-    # small M uses the split-K GEMV, which needs integer partials
-    assert hbl.workspace_size(hbl.OP_TERNARY_GEMM, 1, 16384, 4096, 4) > 0
+    # automatic choice at this batch: the TMA-fed GEMM, plus N*K bytes of expanded weights
+    auto = hbl.workspace_size(hbl.OP_HBITLINEAR_FORWARD, M, K, N, 4)
+    assert auto == M * K + 2 * M * 4 + N * K
+    assert hbl.workspace_size(hbl.OP_TERNARY_GEMM, M, K, N, hbl.ACT_INT4_BYTES) == N * K
+    assert hbl.workspace_size(hbl.OP_TERNARY_GEMM, M, K, N, 8) == N * K
+    # small M: the row GEMV (K >= 2048) needs no scratch; below that the split-K
+    # GEMV needs integer partials
+    assert hbl.workspace_size(hbl.OP_TERNARY_GEMM, 1, 16384, 4096, 4) == 0
+    assert hbl.workspace_size(hbl.OP_TERNARY_GEMM, 8, 1024, 4096, 4) > 0
 
 
 @pytest.mark.parametrize("K", [0, 8, 24, 100, 65536])
@@ -118,3 +125,44 @@ def test_binding_rejects_non_cuda_tensors():
 
     with pytest.raises(TypeError):
         hbl.norm_fwht_quant(torch.zeros(4, 256, dtype=torch.bfloat16), 4)
+
+
+def test_variant_rotation_and_kv_validation():
+    lib = hbl.lib()
+    # variant flags: only HBL_NORM_LAYERNORM | HBL_NORM_NO_HADAMARD
+    assert lib.hbl_norm_transform(A, NUL, 4, 256, 1e-6, 4, B, NUL, NUL) == 1
+    assert lib.hbl_norm_quant(A, NUL, 4, 256, 1e-6, 1e-5, 4, 8, B, C, D, NUL, NUL) == 1
+    assert lib.hbl_norm_quant(A, NUL, 4, 100, 1e-6, 1e-5, 4, 2, B, C, D, NUL, NUL) == 2
+    assert lib.hbl_norm_quant(A, NUL, 0, 256, 1e-6, 1e-5, 4, 3, B, C, D, NUL, NUL) == 0
+    fwd = lib.hbl_bitlinear_forward
+    assert fwd(A, NUL, 64, 256, 64, B, C, 4, 16, 1e-6, 1e-5, D, E, 1 << 20, NUL, NUL) == 1
+    assert fwd(A, NUL, 64, 256, 64, B, C, 4, 2, 1e-6, 1e-5, D, E, 16, NUL, NUL) == 5
+    # rotation: K rule, alignment, N == 0 is a no-op
+    assert lib.hbl_rotate_weights(A, NUL, 8, 100, B, NUL, NUL) == 2
+    assert lib.hbl_rotate_weights(A, NUL, -1, 256, B, NUL, NUL) == 2
+    assert lib.hbl_rotate_weights(MIS, NUL, 8, 256, B, NUL, NUL) == 3
+    assert lib.hbl_rotate_weights(A, MIS, 8, 256, B, NUL, NUL) == 3
+    assert lib.hbl_rotate_weights(A, NUL, 0, 256, B, NUL, NUL) == 0
+    # KV quantiser: bits, head size, eps, alignment, empty
+    kv = lib.hbl_kv_quant
+    assert kv(A, 10, 128, 5, 1e-5, B, C, NUL, NUL) == 1
+    assert kv(A, 10, 128, 3, -1.0, B, C, NUL, NUL) == 1
+    assert kv(A, 10, 96, 3, 1e-5, B, C, NUL, NUL) == 2
+    assert kv(A, -1, 128, 3, 1e-5, B, C, NUL, NUL) == 2
+    assert kv(MIS, 10, 128, 3, 1e-5, B, C, NUL, NUL) == 3
+    assert kv(A, 10, 128, 3, 1e-5, NUL, C, NUL, NUL) == 1
+    assert kv(A, 0, 128, 3, 1e-5, B, C, NUL, NUL) == 0
+
+
+def test_expanded_weight_calls_validation():
+    lib = hbl.lib()
+    assert lib.hbl_expand_ternary(A, 8, 100, B, NUL, NUL) == 2
+    assert lib.hbl_expand_ternary(A, 0, 256, B, NUL, NUL) == 0
+    assert lib.hbl_expand_ternary(MIS, 8, 256, B, NUL, NUL) == 3
+    s8w = lib.hbl_ternary_gemm_s8w
+    assert s8w(A, B, 4, 16, 256, C, D, 64, E, NUL, NUL, NUL) == 1    # packed nibbles refused
+    assert s8w(A, B, 8, 16, 64, C, D, 64, E, NUL, NUL, NUL) == 2     # K < 128
+    assert s8w(A, B, 0x204, 16, 256, C, D, 40, E, NUL, NUL, NUL) == 2
+    assert s8w(A, B, 8, 0, 256, C, D, 64, E, NUL, NUL, NUL) == 0
+    assert lib.hbl_set_gemm_path(4) == 0 and lib.hbl_set_gemm_path(0) == 0
+    assert lib.hbl_set_gemm_path(5) == 1

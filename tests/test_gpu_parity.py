@@ -235,6 +235,43 @@ def test_gemm_paths(path, bits, M, K, N):
 
 
 @pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("M,K,N", [(1, 128, 16), (45, 256, 272), (128, 512, 256),
+                                   (300, 4096, 400), (1000, 2048, 512), (257, 16384, 4096)])
+def test_gemm_tma_one_byte_codes(bits, M, K, N):
+    # the TMA-fed kernel reads one byte per code: INT8 row-major, or INT4 values
+    # one byte each (HBL_ACT_INT4_BYTES)
+    codes, scales, rowsum, packed, alpha = make_gemm_case(M, K, N, bits, seed=M + K)
+    q = oracle.decode_codes(codes, K, bits)
+    act = 8 if bits == 8 else hbl.ACT_INT4_BYTES
+    hbl.set_gemm_path(4)
+    try:
+        Y, acc = hbl.ternary_gemm(
+            torch.from_numpy(q.view(np.uint8).copy()).to(DEV), torch.from_numpy(scales).to(DEV),
+            torch.from_numpy(rowsum).to(DEV), act, K,
+            torch.from_numpy(packed.view(np.int32)).to(DEV),
+            torch.from_numpy(np.array([alpha, 0, 0, 0], dtype=np.float32)).to(DEV),
+            want_acc=True)
+        torch.cuda.synchronize()
+    finally:
+        hbl.set_gemm_path(0)
+    wY, wacc = oracle.ternary_gemm(codes, scales, bits, K, packed, alpha)
+    assert np.array_equal(acc.cpu().numpy(), wacc)
+    assert np.array_equal(bf16_bits(Y), wY)
+
+
+@pytest.mark.parametrize("K", [16, 256, 4096, 16384])
+def test_quant_int4_one_byte_layout(K):
+    X = acts(45, K, seed=K + 7, kind="t")
+    codes, scales, rowsum = hbl.norm_fwht_quant(to_dev_bf16(X), hbl.ACT_INT4_BYTES)
+    torch.cuda.synchronize()
+    wc, ws, wr = oracle.norm_fwht_quant(X, 4)
+    assert codes.shape == (45, K)
+    assert np.array_equal(codes.cpu().numpy().view(np.int8), oracle.decode_codes(wc, K, 4))
+    assert np.array_equal(scales.cpu().numpy().view(np.uint32), ws.view(np.uint32))
+    assert np.array_equal(rowsum.cpu().numpy(), wr)
+
+
+@pytest.mark.parametrize("bits", [4, 8])
 def test_gemm_identity_weights(bits):
     K = 256
     codes, scales, rowsum, _, _ = make_gemm_case(130, K, 16, bits)
@@ -262,7 +299,7 @@ def forward(X, packed, alpha, bits, path=0):
 def test_forward_tiny_workload(bits):
     X = inputs.activations("tiny")
     packed, alpha = oracle.pack_ternary(inputs.weights("tiny"))
-    for path in (0, 1, 2, 3):
+    for path in (0, 1, 2, 3, 4):
         Y = forward(X, packed, alpha, bits, path)
         assert np.array_equal(Y, oracle.hbitlinear_forward(X, packed, alpha, bits))
 
