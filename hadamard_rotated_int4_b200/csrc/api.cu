@@ -87,6 +87,10 @@ Back pick(int64_t M, int K, bool bytes) {
     return Back::TS;
 }
 
+// The GEMV back end uses the row GEMV when K allows it and the tokens fit one
+// launch; otherwise the split-K GEMV (8-token chunks).
+bool rows_gemv(int64_t M, int K) { return gemv_rows_supported(K) && M <= gemv_rows_max_m(K); }
+
 size_t backend_ws(Back b, int64_t M, int K, int N) {
     switch (b) {
         case Back::SS: return 0;
@@ -94,7 +98,7 @@ size_t backend_ws(Back b, int64_t M, int K, int N) {
         case Back::TMA: return gemm_tma_workspace(K, N);
         case Back::GEMV:
         default: {
-            if (gemv_rows_supported(K)) return 0;  // the row GEMV needs no scratch
+            if (rows_gemv(M, K)) return 0;  // the row GEMV needs no scratch
             const int64_t mchunk = M < gemv_max_m() ? M : gemv_max_m();
             return gemv_workspace(mchunk, K, N, 148);
         }
@@ -110,7 +114,7 @@ hbl_status run_gemm(Back b, const GemmArgs& a, void* ws, size_t ws_bytes, cudaSt
     if (b == Back::SS) return launch_gemm_tc(a, s, sms);
     if (b == Back::TS) return launch_gemm_ts(a, ws, ws_bytes, s, sms);
     if (b == Back::TMA) return launch_gemm_tma(a, ws, ws_bytes, s, sms);
-    if (gemv_rows_supported(a.K)) {  // row GEMV in chunks of up to gemv_rows_max_m(K) tokens
+    if (rows_gemv(a.M, a.K)) {  // row GEMV in chunks of up to gemv_rows_max_m(K) tokens
         const int64_t step = gemv_rows_max_m(a.K);
         for (int64_t r0 = 0; r0 < a.M; r0 += step) {
             GemmArgs c = a;

@@ -169,9 +169,10 @@ static hbl_status launch_l(const GemmArgs& a, bool pre, cudaStream_t stream) {
 
 }  // namespace k3b
 
-// Tokens one launch of the row GEMV takes at this K (shared memory holds
-// M x K int8 activations, at most 128 KB).
-int gemv_rows_max_m(int K) { return K >= 32768 ? 4 : 8; }
+// Tokens one launch of the row GEMV takes at this K: the CTA stages M x K int8
+// activations in shared memory; up to 64 KB keeps three or more CTAs (24 warps
+// of weight loads in flight) per SM.  Larger token counts go to the split-K GEMV.
+int gemv_rows_max_m(int K) { return K >= 16384 ? (K >= 32768 ? 2 : 4) : 8; }
 
 bool gemv_rows_supported(int K) { return K >= 2048 && K <= 32768; }
 
