@@ -223,21 +223,25 @@ __device__ __forceinline__ void load_stage(const ConvPtrs& cp, int K, int kb, Pa
 
 // Loader for K % 128 == 0: no guards (rows past M or N read a valid row whose
 // results are never stored), running pointers, immediate offsets.
+// a_on = false (warp-uniform): this warp's token rows are all past M, so its
+// activation loads are skipped (the MMA rows they would feed are never stored).
 template <int ABITS, bool IL>
 struct FastLoader {
     const uint8_t* a;
     const uint32_t* b;
+    bool a_on;
     __device__ __forceinline__ void load(Packed<ABITS>& P) {
-        if constexpr (ABITS == 8) {
+        if (a_on) {
+            if constexpr (ABITS == 8) {
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-                P.a[i] = *reinterpret_cast<const uint4*>(a + (IL ? 512 * i : 16 * i));
-            a += IL ? 8 * 512 : BK;
-        } else {
+                for (int i = 0; i < 8; ++i)
+                    P.a[i] = *reinterpret_cast<const uint4*>(a + (IL ? 512 * i : 16 * i));
+            } else {
 #pragma unroll
-            for (int i = 0; i < 4; ++i) P.a[i] = *reinterpret_cast<const uint4*>(a + 16 * i);
-            a += BK / 2;
+                for (int i = 0; i < 4; ++i) P.a[i] = *reinterpret_cast<const uint4*>(a + 16 * i);
+            }
         }
+        a += ABITS == 8 ? (IL ? 8 * 512 : BK) : BK / 2;
         P.b = *reinterpret_cast<const uint4*>(b);
         b += BK / 16;
     }
@@ -259,7 +263,7 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
 
 template <int ABITS>
 __device__ __forceinline__ void store_stage(uint32_t a_taddr, uint32_t sB, const uint32_t (&boff)[4],
-                                            const Packed<ABITS>& P) {
+                                            const Packed<ABITS>& P, bool a_on) {
     uint32_t av[32];
     if constexpr (ABITS == 8) {
 #pragma unroll
@@ -281,7 +285,7 @@ __device__ __forceinline__ void store_stage(uint32_t a_taddr, uint32_t sB, const
             }
         }
     }
-    tmem_st32(a_taddr, av);
+    if (a_on) tmem_st32(a_taddr, av);  // warp-uniform
     const uint32_t wv[4] = {P.b.x, P.b.y, P.b.z, P.b.w};
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
@@ -391,6 +395,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_ts_kernel(Params p) {
         const int acc = (warp - 1) >> 2;         // accumulator 0 or 1
         const int trow = 128 * acc + 32 * q + lane;  // token row within the tile
         const int64_t m = m0 + trow;
+        // one-tile batches: warps whose 32 rows all lie past M skip their
+        // activation loads and TMEM stores (warp-uniform)
+        const bool a_on = !SMALL || (m0 + 128 * acc + 32 * q < p.M);
         const int br = ct >> 1, bh = ct & 1;     // weight row / half of this thread's chunk
         const int n = n0 + br;
         const uint32_t lane_base = (uint32_t)(32 * q) << 16;
@@ -417,7 +424,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_ts_kernel(Params p) {
             go = go && (__shfl_sync(0xffffffffu, *abort_flag, 0) == 0);
             if (!go) return false;  // warp-uniform
             tc_fence_after();
-            store_stage<ABITS>(a_col0 + 64u * s, base_s + s * kBStageBytes, boff, P);
+            store_stage<ABITS>(a_col0 + 64u * s, base_s + s * kBStageBytes, boff, P, a_on);
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
             tc_fence_before();
@@ -428,6 +435,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_ts_kernel(Params p) {
         bool ok = true;
         if constexpr (FULLK) {
             FastLoader<ABITS, IL> ld;
+            ld.a_on = a_on;
             {
                 int64_t mm = m;
                 if constexpr (IL) {

@@ -21,8 +21,8 @@
 // Tile 128 tokens x 256 weight rows, K in stages of 128 bytes (one 128-byte
 // swizzled row per token / weight row: the TMA SWIZZLE_128B pattern is the
 // K-major layout the MMA descriptors name), 4 stages (48 KB each).  Persistent
-// CTAs walk the tiles in token-block-major order, so the blocks in flight share
-// their weight tiles in L2.  TMEM holds two 128 x 256 int32 accumulators: the
+// CTAs walk the tiles in groups of 8 weight blocks, token blocks in order within
+// a group, so a group's weights stay in L2 while the activations stream past.  TMEM holds two 128 x 256 int32 accumulators: the
 // epilogue drains one while the MMAs fill the other.  Every wait is bounded by
 // the global timer; on expiry the kernel records HBL_ERR_TIMEOUT and stops,
 // letting its own TMA loads and MMAs land before it frees TMEM and exits.
@@ -139,6 +139,7 @@ __device__ __forceinline__ void tma_load(uint32_t dst, const CUtensorMap* map, i
 struct Params {
     int64_t M;
     int N, K;
+    int tiles_m;    // token tiles
     const float* scales;
     const float* alpha;
     uint16_t* Y;
@@ -147,6 +148,20 @@ struct Params {
     int tiles_n;    // weight-row tiles
     int64_t tiles;  // total tiles
 };
+
+// Tile t -> (token block, weight block).  Weight blocks go in groups of kGroup
+// (kGroup x 4 MB of expanded weights at K = 16384); within a group the token
+// blocks run in order, so the group's weights stay in L2 while the
+// activations stream past, and a wave of 148 tiles spans ~18 token blocks.
+constexpr int kGroup = 8;
+__device__ __forceinline__ void tile_coords(const Params& p, int64_t t, int& mb, int& nb) {
+    const int64_t per_group = (int64_t)p.tiles_m * kGroup;
+    const int g = (int)(t / per_group);
+    const int gw = min(kGroup, p.tiles_n - g * kGroup);
+    const int64_t idx = t - (int64_t)g * per_group;
+    mb = (int)(idx / gw);
+    nb = g * kGroup + (int)(idx % gw);
+}
 
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_tma_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -204,7 +219,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t it = 0;
             bool ok = true;
             for (int64_t t = blockIdx.x; t < p.tiles && ok; t += gridDim.x) {
-                const int mb = (int)(t / p.tiles_n), nb = (int)(t % p.tiles_n);
+                int mb, nb;
+                tile_coords(p, t, mb, nb);
                 for (int kb = 0; kb < num_kb; ++kb, ++it) {
                     const int s = (int)(it % S);
                     if (it >= (uint32_t)S &&
@@ -285,7 +301,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 break;
             }
             tc_fence_after();
-            const int mb = (int)(t / p.tiles_n), nb = (int)(t % p.tiles_n);
+            int mb, nb;
+            tile_coords(p, t, mb, nb);
             const int64_t m = (int64_t)mb * BM + 32 * q + lane;
             const bool mok = m < p.M;
             const float sc = mok ? __fmul_rn(alpha, p.scales[m]) : 0.f;
@@ -428,7 +445,8 @@ hbl_status launch_gemm_tma_s8w(const GemmArgs& a, const int8_t* W_s8, cudaStream
     prm.acc_out = a.acc_out;
     prm.status = a.dev_status;
     prm.tiles_n = (a.N + k2c::BN - 1) / k2c::BN;
-    prm.tiles = ((a.M + k2c::BM - 1) / k2c::BM) * (int64_t)prm.tiles_n;
+    prm.tiles_m = (int)((a.M + k2c::BM - 1) / k2c::BM);
+    prm.tiles = (int64_t)prm.tiles_m * prm.tiles_n;
     if (!smem_attr_once(reinterpret_cast<const void*>(k2c::gemm_tma_kernel), k2c::kSmemBytes))
         return HBL_ERR_CUDA;
     const int64_t grid = prm.tiles < num_sms ? prm.tiles : num_sms;

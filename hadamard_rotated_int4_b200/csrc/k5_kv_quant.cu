@@ -22,6 +22,8 @@
 // loads in flight.
 #include <cuda_runtime.h>
 
+#include <type_traits>
+
 #include "hbl_internal.cuh"
 #include "hbl_launch.h"
 
@@ -75,21 +77,24 @@ __global__ void __launch_bounds__(kThreads) kv_quant_kernel(const uint16_t* __re
             for (int o = 1; o < LPR; o <<= 1) g = fmaxf(g, __shfl_xor_sync(0xffffffffu, g, o));
             const float den = __fadd_rn(g, eps);
             const float inv = den > 0.f ? __fdiv_rn(qp, den) : 0.f;
-            // 8 codes of this lane, code i at bits [B*i, B*i + B)
-            uint64_t bits = 0;
+            // 8 codes of this lane, code i at bits [B*i, B*i + B).  No clamp is
+            // needed: |x| <= gamma, so |x * inv| <= Qp * gamma / (gamma + eps)
+            // up to the rounding of inv (well under half a unit), and rounding
+            // to the nearest integer stays within [-Qp, Qp].
+            using Word = typename std::conditional<(8 * B <= 32), uint32_t, uint64_t>::type;
+            Word bits = 0;
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
-                int32_t b = __float_as_int(__fmaf_rn(x[i], inv, 12582912.0f));
-                b = min(max(b, kMagicBits - QP - 1), kMagicBits + QP);
+                const int32_t b = __float_as_int(__fmaf_rn(x[i], inv, 12582912.0f));
                 const uint32_t code = (uint32_t)(b - kMagicBits + (QP + 1));
-                bits |= (uint64_t)code << (B * i);
+                bits |= (Word)code << (B * i);
             }
             const bool ok = row < rows;
             uint8_t* dst = codes + row * ROW_BYTES;
             if constexpr (B == 8) {
                 if (ok)
                     *reinterpret_cast<uint2*>(dst + li * 8) =
-                        make_uint2((uint32_t)bits, (uint32_t)(bits >> 32));
+                        make_uint2((uint32_t)bits, (uint32_t)((uint64_t)bits >> 32));
             } else if constexpr (B == 4) {
                 if (ok) *reinterpret_cast<uint32_t*>(dst + li * 4) = (uint32_t)bits;
             } else if constexpr (B == 2) {  // 16 bits per lane: even lanes write pairs
