@@ -38,7 +38,7 @@ EXPORTS = ("hbl_status_string", "hbl_version", "hbl_set_gemm_path", "hbl_workspa
            "hbl_hbitlinear_forward", "hbl_hbitlinear_forward_hostio",
            "hbl_ternary_gemv_noalloc", "hbl_norm_transform", "hbl_norm_quant",
            "hbl_bitlinear_forward", "hbl_rotate_weights", "hbl_kv_quant",
-           "hbl_expand_ternary", "hbl_ternary_gemm_s8w")
+           "hbl_expand_ternary", "hbl_ternary_gemm_s8w", "hbl_selftest_bounded_wait")
 
 _lib = None
 
@@ -96,6 +96,8 @@ def lib():
         L.hbl_expand_ternary.argtypes = [P, I, I, P, P, P]
         L.hbl_ternary_gemm_s8w.restype = I
         L.hbl_ternary_gemm_s8w.argtypes = [P, P, I, I, I, P, P, I, P, P, P, P]
+        L.hbl_selftest_bounded_wait.restype = I
+        L.hbl_selftest_bounded_wait.argtypes = [I, I, P, P]
         _lib = L
     return _lib
 
@@ -237,7 +239,7 @@ def ternary_gemv_noalloc(codes, scales, rowsum, act_bits, K, W_packed, alpha, wa
                                           _ptr(Y), _ptr(acc), _ptr(status), _stream()),
            "hbl_ternary_gemv_noalloc", "hbl_norm_transform", "hbl_norm_quant",
            "hbl_bitlinear_forward", "hbl_rotate_weights", "hbl_kv_quant",
-           "hbl_expand_ternary", "hbl_ternary_gemm_s8w")
+           "hbl_expand_ternary", "hbl_ternary_gemm_s8w", "hbl_selftest_bounded_wait")
     return (Y, acc) if want_acc else Y
 
 
@@ -383,3 +385,9 @@ def ternary_gemm_s8w(codes, scales, act_bits, W_s8, alpha, want_acc=False, out=N
                                       _ptr(alpha), N, _ptr(Y), _ptr(acc), _ptr(status),
                                       _stream()), "hbl_ternary_gemm_s8w")
     return (Y, acc) if want_acc else Y
+
+
+def selftest_bounded_wait(arrive, timeout_us, status):
+    """hbl_selftest_bounded_wait: the bounded-wait failure path on one probe kernel."""
+    _check(lib().hbl_selftest_bounded_wait(int(bool(arrive)), int(timeout_us), _ptr(status),
+                                           _stream()), "hbl_selftest_bounded_wait")

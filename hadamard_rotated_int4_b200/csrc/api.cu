@@ -553,6 +553,18 @@ hbl_status hbl_ternary_gemm_s8w(const void* codes, const float* scales, int act_
     return launch_gemm_tma_s8w(a, W_s8, static_cast<cudaStream_t>(stream), sms);
 }
 
+hbl_status hbl_selftest_bounded_wait(int arrive, int timeout_us, int32_t* dev_status,
+                                     void* stream) {
+    if (dev_status == nullptr) return HBL_ERR_INVALID_ARG;
+    if (timeout_us < 1 || timeout_us > 1000000) return HBL_ERR_INVALID_ARG;
+    if (!aligned16(dev_status)) return HBL_ERR_ALIGNMENT;
+    int sms = 0;
+    hbl_status st = device(&sms);
+    if (st != HBL_OK) return st;
+    return launch_bounded_wait_probe(arrive, timeout_us, dev_status,
+                                     static_cast<cudaStream_t>(stream));
+}
+
 // Allocation-free ternary GEMV: the CUDA-core split-K path with its partial
 // sums in the library's fixed 2 MiB device array instead of caller workspace.
 hbl_status hbl_ternary_gemv_noalloc(const void* codes, const float* scales,

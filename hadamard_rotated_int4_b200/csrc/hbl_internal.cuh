@@ -43,6 +43,45 @@ __device__ __forceinline__ void report_status(int32_t* st, int code) {
 // wait that can never be satisfied returns an error instead of hanging.
 constexpr uint32_t kSpinLimit = 1u << 22;
 
+// ------------------------------------------------------------ bounded waits
+
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+    return t;
+}
+__device__ __forceinline__ void mbar_init_count(uint32_t a, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(a), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_one(uint32_t a) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(a) : "memory");
+}
+// true once the phase of the given parity has completed
+__device__ __forceinline__ bool mbar_test_parity(uint32_t a, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n.reg .pred p;\n"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+        "selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(a), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// Waits for an mbarrier phase for at most limit_ns of global time; SLEEP backs
+// off between polls.  Returns false on expiry (the caller reports
+// HBL_ERR_TIMEOUT and unwinds instead of hanging).
+template <bool SLEEP>
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t a, uint32_t parity, uint64_t limit_ns) {
+    if (mbar_test_parity(a, parity)) return true;
+    const uint64_t t0 = global_ns();
+    while (true) {
+        if constexpr (SLEEP) __nanosleep(64);
+        if (mbar_test_parity(a, parity)) return true;
+        if (global_ns() - t0 > limit_ns) return false;
+    }
+}
+
 // ------------------------------------------------------------ memory
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {

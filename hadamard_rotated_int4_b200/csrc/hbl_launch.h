@@ -49,6 +49,10 @@ hbl_status launch_rotate_weights(const float* W, const float* signs, int N, int 
 hbl_status launch_kv_quant(const uint16_t* X, int64_t rows, int D, int bits, float eps,
                            uint8_t* codes, float* scales, cudaStream_t stream, int num_sms);
 
+// Self-test of the bounded-wait failure path (see k9_selftest.cu).
+hbl_status launch_bounded_wait_probe(int arrive, int timeout_us, int32_t* status,
+                                     cudaStream_t stream);
+
 // K0: absmean ternarisation + 2-bit packing (K a power of two).
 size_t pack_ternary_workspace(int N, int K);
 hbl_status launch_pack_ternary(const float* W, int N, int K, float eps, uint32_t* W_packed,

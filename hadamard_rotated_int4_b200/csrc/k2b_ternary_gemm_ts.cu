@@ -42,48 +42,25 @@ constexpr int kThreads = 32 * (1 + kConvWarps);
 constexpr uint32_t kTmemCols = 512;
 constexpr int kBStageBytes = BN * BK;  // 16 KB
 constexpr int kSmemBytes = S * kBStageBytes + 256 + 1024;
+// One-tile batches stream the packed weights through a per-thread cp.async ring
+// of kWRing K-blocks (each thread copies, and later reads, its own 16-byte chunk
+// of every K-block), so kWRing x 4 KB per CTA are in flight instead of the
+// three K-blocks the register prefetch holds: decode is bound by this stream.
+constexpr int kWRing = 8;
+constexpr int kWRingBytes = kWRing * 256 * 16;
+constexpr int kSmemBytesSmall = kSmemBytes + kWRingBytes;
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 
-__device__ __forceinline__ uint64_t gtime() {
-    uint64_t t;
-    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
-    return t;
-}
-__device__ __forceinline__ void mbar_init(uint32_t a, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(a), "r"(count) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint32_t a) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(a) : "memory");
-}
-__device__ __forceinline__ bool mbar_try(uint32_t a, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n.reg .pred p;\n"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
-        "selp.u32 %0, 1, 0, p;\n}\n"
-        : "=r"(ok)
-        : "r"(a), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
+// mbarrier helpers over the library's bounded wait (kTimeoutNs of global time)
+__device__ __forceinline__ void mbar_init(uint32_t a, uint32_t count) { mbar_init_count(a, count); }
+__device__ __forceinline__ void mbar_arrive(uint32_t a) { mbar_arrive_one(a); }
 __device__ __forceinline__ bool mbar_wait(uint32_t a, uint32_t parity) {
-    if (mbar_try(a, parity)) return true;
-    const uint64_t t0 = gtime();
-    while (true) {
-        if (mbar_try(a, parity)) return true;
-        if (gtime() - t0 > kTimeoutNs) return false;
-    }
+    return mbar_wait_bounded<false>(a, parity, kTimeoutNs);
 }
-// Bounded wait that backs off with a short sleep between polls, so a waiting
-// lane does not take issue slots from the warps that share its scheduler.
+// Backs off with a short sleep between polls, so a waiting lane does not take
+// issue slots from the warps that share its scheduler.
 __device__ __forceinline__ bool mbar_wait_backoff(uint32_t a, uint32_t parity) {
-    if (mbar_try(a, parity)) return true;
-    const uint64_t t0 = gtime();
-    while (true) {
-        __nanosleep(64);
-        if (mbar_try(a, parity)) return true;
-        if (gtime() - t0 > kTimeoutNs) return false;
-    }
+    return mbar_wait_bounded<true>(a, parity, kTimeoutNs);
 }
 // Warp-uniform bounded wait: lane 0 waits, every lane gets its verdict.
 template <bool BACKOFF = false>
@@ -225,7 +202,8 @@ __device__ __forceinline__ void load_stage(const ConvPtrs& cp, int K, int kb, Pa
 // results are never stored), running pointers, immediate offsets.
 // a_on = false (warp-uniform): this warp's token rows are all past M, so its
 // activation loads are skipped (the MMA rows they would feed are never stored).
-template <int ABITS, bool IL>
+// B_ON = false: the packed weights come through the cp.async ring instead.
+template <int ABITS, bool IL, bool B_ON = true>
 struct FastLoader {
     const uint8_t* a;
     const uint32_t* b;
@@ -242,8 +220,10 @@ struct FastLoader {
             }
         }
         a += ABITS == 8 ? (IL ? 8 * 512 : BK) : BK / 2;
-        P.b = *reinterpret_cast<const uint4*>(b);
-        b += BK / 16;
+        if constexpr (B_ON) {
+            P.b = *reinterpret_cast<const uint4*>(b);
+            b += BK / 16;
+        }
     }
 };
 
@@ -263,7 +243,7 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
 
 template <int ABITS>
 __device__ __forceinline__ void store_stage(uint32_t a_taddr, uint32_t sB, const uint32_t (&boff)[4],
-                                            const Packed<ABITS>& P, bool a_on) {
+                                            const Packed<ABITS>& P, uint4 bw, bool a_on) {
     uint32_t av[32];
     if constexpr (ABITS == 8) {
 #pragma unroll
@@ -286,7 +266,7 @@ __device__ __forceinline__ void store_stage(uint32_t a_taddr, uint32_t sB, const
         }
     }
     if (a_on) tmem_st32(a_taddr, av);  // warp-uniform
-    const uint32_t wv[4] = {P.b.x, P.b.y, P.b.z, P.b.w};
+    const uint32_t wv[4] = {bw.x, bw.y, bw.z, bw.w};
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
         const uint32_t w = wv[j];
@@ -416,6 +396,19 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_ts_kernel(Params p) {
         for (int j = 0; j < 4; ++j) boff[j] = sw128(br, 4 * bh + j);
         const uint32_t a_col0 = tmem + lane_base + 256u + 32u * acc;
 
+        // one-tile batches: this thread's packed-weight chunks through the ring
+        constexpr bool WRING = SMALL && FULLK;
+        const uint32_t wring_s = base_s + S * kBStageBytes + 256 + (uint32_t)ct * 16u;
+        const uint32_t* wsrc = p.W + (int64_t)(n < p.N ? n : p.N - 1) * (p.K / 16) + 4 * bh +
+                               (int64_t)kb0 * (BK / 16);
+        auto wslot = [&](int j) { return wring_s + (uint32_t)((j % kWRing) * 256 * 16); };
+        auto wissue = [&](int j) {  // one commit group per K-block (empty past the end)
+            if (j < num_kb) cp_async16(wslot(j), wsrc + (int64_t)j * (BK / 16), 16);
+            cp_async_commit();
+        };
+        if constexpr (WRING)
+            for (int j = 0; j < kWRing - 1; ++j) wissue(j);
+
         // one stage: wait for the slot, write A to TMEM and B to shared memory, signal
         auto stage = [&](int kb, const Packed<ABITS>& P) -> bool {
             const int s = kb % S;
@@ -423,8 +416,16 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_ts_kernel(Params p) {
             if (kb >= S) go = warp_wait<true>(empty_bar(s), (uint32_t)(((kb / S) - 1) & 1));
             go = go && (__shfl_sync(0xffffffffu, *abort_flag, 0) == 0);
             if (!go) return false;  // warp-uniform
+            uint4 bw;
+            if constexpr (WRING) {
+                wissue(kb + kWRing - 1);
+                asm volatile("cp.async.wait_group %0;" ::"n"(kWRing - 1) : "memory");
+                bw = lds128(wslot(kb));
+            } else {
+                bw = P.b;
+            }
             tc_fence_after();
-            store_stage<ABITS>(a_col0 + 64u * s, base_s + s * kBStageBytes, boff, P, a_on);
+            store_stage<ABITS>(a_col0 + 64u * s, base_s + s * kBStageBytes, boff, P, bw, a_on);
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
             tc_fence_before();
@@ -434,7 +435,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_ts_kernel(Params p) {
         Packed<ABITS> P0, P1;
         bool ok = true;
         if constexpr (FULLK) {
-            FastLoader<ABITS, IL> ld;
+            FastLoader<ABITS, IL, !(SMALL && FULLK)> ld;
             ld.a_on = a_on;
             {
                 int64_t mm = m;
@@ -493,6 +494,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_ts_kernel(Params p) {
                 }
             }
         }
+        if constexpr (SMALL && FULLK) cp_async_wait_all();  // no copy outlives the CTA
         if (!ok && lane == 0) {
             *abort_flag = 1;
             report_status(p.status, HBL_ERR_TIMEOUT);
@@ -585,11 +587,12 @@ static hbl_status launch(const Params& prm, cudaStream_t stream) {
                               : gemm_ts_kernel<ABITS, IL, true, false>)
                      : (small ? gemm_ts_kernel<ABITS, IL, false, true>
                               : gemm_ts_kernel<ABITS, IL, false, false>);
-    if (!smem_attr_once(reinterpret_cast<const void*>(kern), kSmemBytes)) return HBL_ERR_CUDA;
+    const int smem = (full && small) ? kSmemBytesSmall : kSmemBytes;
+    if (!smem_attr_once(reinterpret_cast<const void*>(kern), smem)) return HBL_ERR_CUDA;
     const int num_kb = (prm.K + BK - 1) / BK;
     dim3 grid((prm.N + BN - 1) / BN, (unsigned)((prm.M + BM - 1) / BM),
               (unsigned)((num_kb + prm.kps - 1) / prm.kps));
-    return launch_pdl(kern, grid, dim3(kThreads), kSmemBytes, stream, prm);
+    return launch_pdl(kern, grid, dim3(kThreads), smem, stream, prm);
 }
 
 }  // namespace k2b

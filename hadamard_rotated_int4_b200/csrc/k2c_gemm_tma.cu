@@ -58,42 +58,16 @@ constexpr uint64_t kTimeoutNs = 2000000000ull;
 constexpr uint32_t kIdesc = (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
                             ((uint32_t)(BM >> 4) << 24);
 
-__device__ __forceinline__ uint64_t gtime() {
-    uint64_t t;
-    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
-    return t;
-}
-__device__ __forceinline__ void mbar_init(uint32_t a, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(a), "r"(count) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint32_t a) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(a) : "memory");
-}
+// mbarrier helpers over the library's bounded wait (kTimeoutNs of global time)
+__device__ __forceinline__ void mbar_init(uint32_t a, uint32_t count) { mbar_init_count(a, count); }
+__device__ __forceinline__ void mbar_arrive(uint32_t a) { mbar_arrive_one(a); }
 __device__ __forceinline__ void mbar_expect_tx(uint32_t a, uint32_t bytes) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(a), "r"(bytes)
                  : "memory");
 }
-__device__ __forceinline__ bool mbar_try(uint32_t a, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n.reg .pred p;\n"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
-        "selp.u32 %0, 1, 0, p;\n}\n"
-        : "=r"(ok)
-        : "r"(a), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-// Bounded wait (global timer); SLEEP backs off between polls.
 template <bool SLEEP>
 __device__ __forceinline__ bool mbar_wait(uint32_t a, uint32_t parity) {
-    if (mbar_try(a, parity)) return true;
-    const uint64_t t0 = gtime();
-    while (true) {
-        if constexpr (SLEEP) __nanosleep(64);
-        if (mbar_try(a, parity)) return true;
-        if (gtime() - t0 > kTimeoutNs) return false;
-    }
+    return mbar_wait_bounded<SLEEP>(a, parity, kTimeoutNs);
 }
 __device__ __forceinline__ void tc_fence_before() {
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");

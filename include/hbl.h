@@ -284,6 +284,17 @@ HBL_API hbl_status hbl_ternary_gemm_s8w(const void* codes, const float* scales, 
                                         int N, uint16_t* Y, int32_t* acc_out,
                                         int32_t* dev_status, void* stream);
 
+/* Self-test of the failure path (no counterpart on the pages).  Every
+ * pipelined kernel here waits on mbarriers with a bound on global time and, if
+ * the bound runs out, records HBL_ERR_TIMEOUT in dev_status and returns
+ * instead of hanging.  This launches one probe kernel running the same bounded
+ * wait on a barrier that receives its arrival first (arrive != 0: dev_status
+ * stays 0) or never (arrive == 0: after timeout_us microseconds dev_status
+ * becomes HBL_ERR_TIMEOUT).  dev_status: device int32 (required); timeout_us
+ * in [1, 1000000]. */
+HBL_API hbl_status hbl_selftest_bounded_wait(int arrive, int timeout_us, int32_t* dev_status,
+                                             void* stream);
+
 /* Allocation-free ternary GEMV (no counterpart on the BitNet v2 pages; it is a
  * deployment aid).  Same arguments, layouts and results as hbl_ternary_gemm
  * run on its CUDA-core split-K path, but without a workspace argument: the

@@ -166,3 +166,10 @@ def test_expanded_weight_calls_validation():
     assert s8w(A, B, 8, 0, 256, C, D, 64, E, NUL, NUL, NUL) == 0
     assert lib.hbl_set_gemm_path(4) == 0 and lib.hbl_set_gemm_path(0) == 0
     assert lib.hbl_set_gemm_path(5) == 1
+
+
+def test_selftest_validation():
+    lib = hbl.lib()
+    assert lib.hbl_selftest_bounded_wait(0, 100, NUL, NUL) == 1
+    assert lib.hbl_selftest_bounded_wait(0, 0, A, NUL) == 1
+    assert lib.hbl_selftest_bounded_wait(0, 100, MIS, NUL) == 3

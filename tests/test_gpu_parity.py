@@ -406,3 +406,18 @@ def test_status_word_stays_clear():
     hbl.hbitlinear_forward(X, packed, alpha, 4, status=st)
     torch.cuda.synchronize()
     assert int(st[0].item()) == 0
+
+
+@pytest.mark.parametrize("arrive", [True, False])
+def test_bounded_wait_reports_timeout_and_context_survives(arrive):
+    # a wait that nothing satisfies runs out and reports HBL_ERR_TIMEOUT (7);
+    # the context stays usable for the next launch
+    st = hbl.new_status(DEV)
+    hbl.selftest_bounded_wait(arrive, 2000, st)
+    torch.cuda.synchronize()
+    assert int(st[0].item()) == (0 if arrive else 7)
+    X = to_dev_bf16(acts(3, 256, seed=1))
+    codes, scales, rowsum = hbl.norm_fwht_quant(X, 4)
+    torch.cuda.synchronize()
+    wc, _, _ = oracle.norm_fwht_quant(acts(3, 256, seed=1), 4)
+    assert np.array_equal(codes.cpu().numpy(), wc)
