@@ -163,9 +163,27 @@ def cpu_baseline(X_bits, packed, alpha, target_s=15.0):
         oracle.hbitlinear_forward(X_bits[:rows], packed, alpha, BITS, threads=threads)
         dt = time.perf_counter() - t0
     used = min(threads, rows)
+    # the same oracle on one core, a few rows (a second figure for scale)
+    r1 = 2
+    t1 = time.perf_counter()
+    oracle.hbitlinear_forward(X_bits[:r1], packed, alpha, BITS, threads=1)
+    d1 = time.perf_counter() - t1
     return {"value": rows / dt, "unit": UNIT, "cores": used, "kind": "oracle",
+            "value_1core": r1 / d1, "cpu_model": cpu_model(),
             "sample": "%d of the 8192 token rows of the ffn_wdown workload (full K, full N), "
-                      "scalar C oracle, rows split over %d threads, %.1f s" % (rows, used, dt)}
+                      "scalar C oracle, rows split over %d threads, %.1f s; value_1core: %d rows "
+                      "on one thread, %.1f s" % (rows, used, dt, r1, d1)}
+
+
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
 
 
 def run_reference(args):

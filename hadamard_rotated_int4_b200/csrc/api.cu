@@ -407,6 +407,41 @@ hbl_status hbl_hbitlinear_forward(const uint16_t* X, const float* gain, int M, i
                         static_cast<cudaStream_t>(stream), sms);
 }
 
+namespace {
+// Per-device copy streams and events of the host-buffer forward: the input
+// copies, the layer and the output copies of consecutive row chunks overlap.
+constexpr int kMaxChunks = 8;
+struct CopyLanes {
+    cudaStream_t in = nullptr, out = nullptr;
+    cudaEvent_t start = nullptr, done = nullptr;
+    cudaEvent_t in_ev[kMaxChunks] = {}, fwd_ev[kMaxChunks] = {};
+    bool ready = false;
+};
+CopyLanes g_lanes[kMaxDevices];
+std::mutex g_lanes_mu;
+
+hbl_status copy_lanes(CopyLanes** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return HBL_ERR_CUDA;
+    CopyLanes& c = g_lanes[dev];
+    if (!c.ready) {
+        const unsigned ef = cudaEventDisableTiming;
+        if (cudaStreamCreateWithFlags(&c.in, cudaStreamNonBlocking) != cudaSuccess ||
+            cudaStreamCreateWithFlags(&c.out, cudaStreamNonBlocking) != cudaSuccess ||
+            cudaEventCreateWithFlags(&c.start, ef) != cudaSuccess ||
+            cudaEventCreateWithFlags(&c.done, ef) != cudaSuccess)
+            return HBL_ERR_CUDA;
+        for (int i = 0; i < kMaxChunks; ++i)
+            if (cudaEventCreateWithFlags(&c.in_ev[i], ef) != cudaSuccess ||
+                cudaEventCreateWithFlags(&c.fwd_ev[i], ef) != cudaSuccess)
+                return HBL_ERR_CUDA;
+        c.ready = true;
+    }
+    *out = &c;
+    return HBL_OK;
+}
+}  // namespace
+
 hbl_status hbl_hbitlinear_forward_hostio(const uint16_t* X_host, const float* gain, int M,
                                          int K, int N, const uint32_t* W_packed,
                                          const float* alpha, int act_bits, float norm_eps,
@@ -426,13 +461,67 @@ hbl_status hbl_hbitlinear_forward_hostio(const uint16_t* X_host, const float* ga
     uint16_t* Yd = reinterpret_cast<uint16_t*>(w8 + xb);
     uint8_t* fws = w8 + xb + yb;
     const size_t fws_bytes = ws_bytes - xb - yb;
-    if (cudaMemcpyAsync(Xd, X_host, (size_t)M * K * 2, cudaMemcpyHostToDevice, s) != cudaSuccess)
-        return HBL_ERR_CUDA;
-    st = forward_impl(Xd, gain, M, K, N, W_packed, alpha, act_bits, norm_eps, quant_eps, Yd, fws,
-                      fws_bytes, dev_status, s, sms);
-    if (st != HBL_OK) return st;
-    if (cudaMemcpyAsync(Y_host, Yd, (size_t)M * N * 2, cudaMemcpyDeviceToHost, s) != cudaSuccess)
-        return HBL_ERR_CUDA;
+    const FwdPlan plan = forward_plan(M, K, act_bits);
+    // Batches on the TMA-fed GEMM run in row chunks of at least kTmaMinM rows
+    // (so every chunk keeps that plan and fits its workspace): chunk c's input
+    // copy, its layer and chunk c-1's output copy overlap on three streams.
+    const int nch = plan.back == Back::TMA
+                        ? (int)((int64_t)M / kTmaMinM < kMaxChunks ? (int64_t)M / kTmaMinM
+                                                                    : kMaxChunks)
+                        : 1;
+    if (nch <= 1) {
+        if (cudaMemcpyAsync(Xd, X_host, (size_t)M * K * 2, cudaMemcpyHostToDevice, s) !=
+            cudaSuccess)
+            return HBL_ERR_CUDA;
+        st = forward_impl(Xd, gain, M, K, N, W_packed, alpha, act_bits, norm_eps, quant_eps, Yd,
+                          fws, fws_bytes, dev_status, s, sms);
+        if (st != HBL_OK) return st;
+        if (cudaMemcpyAsync(Y_host, Yd, (size_t)M * N * 2, cudaMemcpyDeviceToHost, s) !=
+            cudaSuccess)
+            return HBL_ERR_CUDA;
+        return HBL_OK;
+    }
+    std::lock_guard<std::mutex> lock(g_lanes_mu);  // the lanes' events are shared
+    CopyLanes* c = nullptr;
+    if ((st = copy_lanes(&c)) != HBL_OK) return st;
+    // workspace of one chunk: codes (rows padded to 32), scales, rowsum, then the
+    // expanded weights (written once, shared by the chunks)
+    const int64_t rows = ((int64_t)M + nch - 1) / nch;
+    const size_t cb = up256((size_t)((rows + 31) & ~31) * K), sb = up256((size_t)rows * 4);
+    uint8_t* codes = fws;
+    float* scales = reinterpret_cast<float*>(fws + cb);
+    int32_t* rowsum = reinterpret_cast<int32_t*>(fws + cb + sb);
+    int8_t* wexp = reinterpret_cast<int8_t*>(fws + cb + 2 * sb);
+    if (cb + 2 * sb + gemm_tma_workspace(K, N) > fws_bytes) return HBL_ERR_WORKSPACE;
+#define HBL_CK(x) \
+    if ((x) != cudaSuccess) return HBL_ERR_CUDA
+    HBL_CK(cudaEventRecord(c->start, s));
+    HBL_CK(cudaStreamWaitEvent(c->in, c->start, 0));
+    HBL_CK(cudaStreamWaitEvent(c->out, c->start, 0));
+    if ((st = launch_expand_ternary(W_packed, N, K, wexp, s, sms)) != HBL_OK) return st;
+    for (int i = 0; i < nch; ++i) {
+        const int64_t r0 = (int64_t)i * rows;
+        const int64_t mc = ((int64_t)M - r0) < rows ? ((int64_t)M - r0) : rows;
+        if (mc <= 0) break;
+        HBL_CK(cudaMemcpyAsync(Xd + r0 * K, X_host + r0 * K, (size_t)mc * K * 2,
+                               cudaMemcpyHostToDevice, c->in));
+        HBL_CK(cudaEventRecord(c->in_ev[i], c->in));
+        HBL_CK(cudaStreamWaitEvent(s, c->in_ev[i], 0));
+        if ((st = launch_norm_fwht_quant(Xd + r0 * K, gain, mc, K, norm_eps, quant_eps,
+                                         plan.k1_mode, codes, scales, rowsum, nullptr, s, sms)) !=
+            HBL_OK)
+            return st;
+        GemmArgs a{codes, scales, rowsum, plan.gemm_act_bits, mc, K, W_packed, alpha, N,
+                   Yd + r0 * N, nullptr, dev_status};
+        if ((st = launch_gemm_tma_s8w(a, wexp, s, sms)) != HBL_OK) return st;
+        HBL_CK(cudaEventRecord(c->fwd_ev[i], s));
+        HBL_CK(cudaStreamWaitEvent(c->out, c->fwd_ev[i], 0));
+        HBL_CK(cudaMemcpyAsync(Y_host + r0 * N, Yd + r0 * N, (size_t)mc * N * 2,
+                               cudaMemcpyDeviceToHost, c->out));
+    }
+    HBL_CK(cudaEventRecord(c->done, c->out));
+    HBL_CK(cudaStreamWaitEvent(s, c->done, 0));  // later work on `stream` follows the copies
+#undef HBL_CK
     return HBL_OK;
 }
 

@@ -589,12 +589,14 @@ __global__ void __launch_bounds__(Cfg<L>::kCtaThreads, Cfg<L>::kMinBlocks)
                         qv[2 * decltype(kk)::value] = (uint32_t)b0;
                         qv[2 * decltype(kk)::value + 1] = (uint32_t)b1;
                     });
-                    static_for<0, EPW>([&](auto ee) { qsum += qv[decltype(ee)::value]; });
                     if constexpr (!kPackNibbles) {  // one byte per code: low byte = q
                         const uint32_t lo2 = __byte_perm(qv[0], qv[1], 0x0040);
                         const uint32_t hi2 = __byte_perm(qv[2], qv[3], 0x0040);
                         wv[wi] = __byte_perm(lo2, hi2, 0x5410);
-                    } else {  // low nibble = q + 8; pairs by shift-add, bytes by permute
+                        // rowsum: the four signed bytes summed by one dp4a
+                        qsum = (uint32_t)__dp4a((int)wv[wi], 0x01010101, (int)qsum);
+                    } else {
+                        static_for<0, EPW>([&](auto ee) { qsum += qv[decltype(ee)::value]; });  // low nibble = q + 8; pairs by shift-add, bytes by permute
                         const uint32_t p01 = (qv[1] << 4) + qv[0];
                         const uint32_t p23 = (qv[3] << 4) + qv[2];
                         const uint32_t lo2 = __byte_perm(p01, p23, 0x0040);
@@ -634,8 +636,9 @@ __global__ void __launch_bounds__(Cfg<L>::kCtaThreads, Cfg<L>::kMinBlocks)
                     }
                 }
             });
-            // sum of codes: each term is kMagicBits + q (mod 2^32)
-            int qs = (int)(qsum - (uint32_t)R * (uint32_t)kMagicBits);
+            // sum of codes: packed nibbles added kMagicBits + q per code (mod 2^32);
+            // one-byte codes were summed directly
+            int qs = kPackNibbles ? (int)(qsum - (uint32_t)R * (uint32_t)kMagicBits) : (int)qsum;
             qs = row_isum(qs);
 
             if (row_ok) {

@@ -42,13 +42,6 @@ constexpr int kThreads = 32 * (1 + kConvWarps);
 constexpr uint32_t kTmemCols = 512;
 constexpr int kBStageBytes = BN * BK;  // 16 KB
 constexpr int kSmemBytes = S * kBStageBytes + 256 + 1024;
-// One-tile batches stream the packed weights through a per-thread cp.async ring
-// of kWRing K-blocks (each thread copies, and later reads, its own 16-byte chunk
-// of every K-block), so kWRing x 4 KB per CTA are in flight instead of the
-// three K-blocks the register prefetch holds: decode is bound by this stream.
-constexpr int kWRing = 8;
-constexpr int kWRingBytes = kWRing * 256 * 16;
-constexpr int kSmemBytesSmall = kSmemBytes + kWRingBytes;
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 
 // mbarrier helpers over the library's bounded wait (kTimeoutNs of global time)
@@ -202,8 +195,7 @@ __device__ __forceinline__ void load_stage(const ConvPtrs& cp, int K, int kb, Pa
 // results are never stored), running pointers, immediate offsets.
 // a_on = false (warp-uniform): this warp's token rows are all past M, so its
 // activation loads are skipped (the MMA rows they would feed are never stored).
-// B_ON = false: the packed weights come through the cp.async ring instead.
-template <int ABITS, bool IL, bool B_ON = true>
+template <int ABITS, bool IL>
 struct FastLoader {
     const uint8_t* a;
     const uint32_t* b;
@@ -220,10 +212,8 @@ struct FastLoader {
             }
         }
         a += ABITS == 8 ? (IL ? 8 * 512 : BK) : BK / 2;
-        if constexpr (B_ON) {
-            P.b = *reinterpret_cast<const uint4*>(b);
-            b += BK / 16;
-        }
+        P.b = *reinterpret_cast<const uint4*>(b);
+        b += BK / 16;
     }
 };
 
@@ -243,7 +233,7 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
 
 template <int ABITS>
 __device__ __forceinline__ void store_stage(uint32_t a_taddr, uint32_t sB, const uint32_t (&boff)[4],
-                                            const Packed<ABITS>& P, uint4 bw, bool a_on) {
+                                            const Packed<ABITS>& P, bool a_on) {
     uint32_t av[32];
     if constexpr (ABITS == 8) {
 #pragma unroll
@@ -266,7 +256,7 @@ __device__ __forceinline__ void store_stage(uint32_t a_taddr, uint32_t sB, const
         }
     }
     if (a_on) tmem_st32(a_taddr, av);  // warp-uniform
-    const uint32_t wv[4] = {bw.x, bw.y, bw.z, bw.w};
+    const uint32_t wv[4] = {P.b.x, P.b.y, P.b.z, P.b.w};
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
         const uint32_t w = wv[j];
@@ -396,19 +386,6 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_ts_kernel(Params p) {
         for (int j = 0; j < 4; ++j) boff[j] = sw128(br, 4 * bh + j);
         const uint32_t a_col0 = tmem + lane_base + 256u + 32u * acc;
 
-        // one-tile batches: this thread's packed-weight chunks through the ring
-        constexpr bool WRING = SMALL && FULLK;
-        const uint32_t wring_s = base_s + S * kBStageBytes + 256 + (uint32_t)ct * 16u;
-        const uint32_t* wsrc = p.W + (int64_t)(n < p.N ? n : p.N - 1) * (p.K / 16) + 4 * bh +
-                               (int64_t)kb0 * (BK / 16);
-        auto wslot = [&](int j) { return wring_s + (uint32_t)((j % kWRing) * 256 * 16); };
-        auto wissue = [&](int j) {  // one commit group per K-block (empty past the end)
-            if (j < num_kb) cp_async16(wslot(j), wsrc + (int64_t)j * (BK / 16), 16);
-            cp_async_commit();
-        };
-        if constexpr (WRING)
-            for (int j = 0; j < kWRing - 1; ++j) wissue(j);
-
         // one stage: wait for the slot, write A to TMEM and B to shared memory, signal
         auto stage = [&](int kb, const Packed<ABITS>& P) -> bool {
             const int s = kb % S;
@@ -416,16 +393,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_ts_kernel(Params p) {
             if (kb >= S) go = warp_wait<true>(empty_bar(s), (uint32_t)(((kb / S) - 1) & 1));
             go = go && (__shfl_sync(0xffffffffu, *abort_flag, 0) == 0);
             if (!go) return false;  // warp-uniform
-            uint4 bw;
-            if constexpr (WRING) {
-                wissue(kb + kWRing - 1);
-                asm volatile("cp.async.wait_group %0;" ::"n"(kWRing - 1) : "memory");
-                bw = lds128(wslot(kb));
-            } else {
-                bw = P.b;
-            }
             tc_fence_after();
-            store_stage<ABITS>(a_col0 + 64u * s, base_s + s * kBStageBytes, boff, P, bw, a_on);
+            store_stage<ABITS>(a_col0 + 64u * s, base_s + s * kBStageBytes, boff, P, a_on);
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
             tc_fence_before();
@@ -435,7 +404,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_ts_kernel(Params p) {
         Packed<ABITS> P0, P1;
         bool ok = true;
         if constexpr (FULLK) {
-            FastLoader<ABITS, IL, !(SMALL && FULLK)> ld;
+            FastLoader<ABITS, IL> ld;
             ld.a_on = a_on;
             {
                 int64_t mm = m;
@@ -494,7 +463,6 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_ts_kernel(Params p) {
                 }
             }
         }
-        if constexpr (SMALL && FULLK) cp_async_wait_all();  // no copy outlives the CTA
         if (!ok && lane == 0) {
             *abort_flag = 1;
             report_status(p.status, HBL_ERR_TIMEOUT);
@@ -587,7 +555,7 @@ static hbl_status launch(const Params& prm, cudaStream_t stream) {
                               : gemm_ts_kernel<ABITS, IL, true, false>)
                      : (small ? gemm_ts_kernel<ABITS, IL, false, true>
                               : gemm_ts_kernel<ABITS, IL, false, false>);
-    const int smem = (full && small) ? kSmemBytesSmall : kSmemBytes;
+    const int smem = kSmemBytes;
     if (!smem_attr_once(reinterpret_cast<const void*>(kern), smem)) return HBL_ERR_CUDA;
     const int num_kb = (prm.K + BK - 1) / BK;
     dim3 grid((prm.N + BN - 1) / BN, (unsigned)((prm.M + BM - 1) / BM),
@@ -598,13 +566,14 @@ static hbl_status launch(const Params& prm, cudaStream_t stream) {
 }  // namespace k2b
 
 // Split factor over K for one-tile-high problems (M <= 256), so that a decode
-// batch still fills the GPU: about two CTAs per SM, at least 4 K-blocks each.
+// batch still fills the GPU in one wave (one CTA per SM: the kernel holds all
+// of TMEM), at least 8 K-blocks per CTA.
 int gemm_ts_ksplit(int64_t M, int K, int N) {
     if (M > k2b::BM) return 1;
     const int tiles = (N + k2b::BN - 1) / k2b::BN;
     const int num_kb = (K + k2b::BK - 1) / k2b::BK;
     int ks = 1;
-    while (tiles * ks * 2 <= 2 * 148 && num_kb / (ks * 2) >= 4) ks *= 2;
+    while (tiles * ks * 2 <= 148 && num_kb / (ks * 2) >= 8) ks *= 2;
     return ks;
 }
 

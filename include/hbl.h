@@ -181,8 +181,15 @@ HBL_API hbl_status hbl_hbitlinear_forward(const uint16_t* X, const float* gain, 
                                   size_t ws_bytes, int32_t* dev_status, void* stream);
 
 /* The whole layer with HOST activations in and HOST outputs out: copies X_host
- * to the device, runs hbl_hbitlinear_forward, copies Y back to Y_host, all on
- * `stream` (asynchronous; pinned host memory makes the copies asynchronous).
+ * to the device, runs hbl_hbitlinear_forward, copies Y back to Y_host
+ * (asynchronous; pinned host memory makes the copies asynchronous).  Ordered
+ * as if everything ran on `stream`: it starts after the work already queued on
+ * `stream`, and work queued on `stream` afterwards starts after Y_host is
+ * written.  Batches above 513 tokens run in up to 8 row chunks whose input
+ * copies, layer and output copies overlap; for that the library keeps two
+ * copy streams and a few events per device, created on the first such call
+ * and kept until exit (they are not memory).  Concurrent calls of this
+ * function on one device are serialised while they enqueue.
  * X_host: bf16 [M x K] host; Y_host: bf16 [M x N] host, out.
  * ws: >= hbl_workspace_size(HBL_OP_HBITLINEAR_FORWARD_HOSTIO, M, K, N, act_bits)
  * bytes of device memory (it holds the device copies of X and Y as well). */

@@ -399,6 +399,30 @@ def test_hostio_matches_device_forward():
                           oracle.hbitlinear_forward(X, packed, alpha, 4))
 
 
+@pytest.mark.parametrize("M,bits", [(1000, 4), (2600, 8), (8192, 4)])
+def test_hostio_chunked_pipeline(M, bits):
+    # batches above 513 tokens run in overlapped row chunks (ragged last chunk);
+    # the result must equal the device-buffer forward bit for bit, and work
+    # queued on the stream afterwards must see Y on the host
+    K, N = 2048, 512
+    X = inputs.activations("attn_wo", M=M, K=K, seed=M)
+    W = torch.from_numpy(inputs.latent_weights(N, K, seed=M)).to(DEV)
+    packed, alpha = hbl.pack_ternary(W)
+    ws = torch.empty(hbl.workspace_size(hbl.OP_HBITLINEAR_FORWARD_HOSTIO, M, K, N, bits),
+                     dtype=torch.uint8, device=DEV)
+    Xh = torch.from_numpy(X.view(np.int16).copy()).view(torch.bfloat16).pin_memory()
+    Yh = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
+    Yh.fill_(0)
+    hbl.hbitlinear_forward_hostio(Xh, packed, alpha, bits, Yh, ws)
+    Yd = hbl.hbitlinear_forward(Xh.to(DEV), packed, alpha, bits)
+    torch.cuda.synchronize()
+    assert torch.equal(Yh.view(torch.int16), Yd.cpu().view(torch.int16))
+    rows = np.array([0, 1, M // 2, M - 1])
+    want = oracle.hbitlinear_forward(X, packed.cpu().numpy().view(np.uint32),
+                                     alpha.cpu().numpy()[0], bits, rows=rows)
+    assert np.array_equal(Yh.view(torch.int16).numpy().view(np.uint16)[rows], want)
+
+
 def test_status_word_stays_clear():
     st = hbl.new_status(DEV)
     X = to_dev_bf16(acts(200, 2048, seed=1))
