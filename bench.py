@@ -153,15 +153,13 @@ def cpu_baseline(X_bits, packed, alpha, target_s=15.0):
 
     threads = os.cpu_count() or 1
     rows = min(threads, 64)
-    t0 = time.perf_counter()
-    oracle.hbitlinear_forward(X_bits[:rows], packed, alpha, BITS, threads=threads)
-    dt = time.perf_counter() - t0
-    if dt < target_s / 3:
-        scale = max(1, int(target_s / max(dt, 1e-3)))
-        rows = min(M_TOK, rows * scale)
+    while True:  # grow the sample until it takes about target_s (or covers the workload)
         t0 = time.perf_counter()
         oracle.hbitlinear_forward(X_bits[:rows], packed, alpha, BITS, threads=threads)
         dt = time.perf_counter() - t0
+        if dt >= target_s / 2 or rows >= M_TOK:
+            break
+        rows = min(M_TOK, max(rows * 2, int(rows * target_s / max(dt, 1e-3))))
     used = min(threads, rows)
     # the same oracle on one core, a few rows (a second figure for scale)
     r1 = 2
@@ -383,8 +381,9 @@ def run_hbl(args):
             decode.append({"shape": shape, "T": T, "K": Kd, "N": N_OUT, "us": t * 1e6,
                            "tokens_per_s": T / t, "packed_w_gbs": wbytes / t / 1e9,
                            "frac_hbm_on_packed_w": wbytes / t / 1e9 / pk["hbm_gbs"],
-                           "path": ("row GEMV (one weight row per warp, PDL after K1)" if T <= 8
-                                    else "gemm_ts (TMEM activations, split-K)"),
+                           "path": ("row GEMV (weight rows per warp, PDL after K1)"
+                                    if T <= (4 if Kd >= 16384 else 8)
+                                    else "gemm_ts (TMEM activations, one-wave split-K)"),
                            "timing": "CUDA graph replay, one forward per weight copy"})
         del pcs
 

@@ -72,6 +72,10 @@ int codes_row_bytes(int K, int act_bits) { return act_width(act_bits) == 4 ? K /
 // Ternary-GEMM back ends.
 enum class Back { GEMV, SS, TS, TMA };
 
+// The GEMV back end uses the row GEMV when K allows it and the tokens fit one
+// launch; otherwise the split-K GEMV (8-token chunks).
+bool rows_gemv(int64_t M, int K) { return gemv_rows_supported(K) && M <= gemv_rows_max_m(K); }
+
 // Batches above this many tokens take the TMA-fed kernel (automatic choice).
 constexpr int64_t kTmaMinM = 257;
 
@@ -82,14 +86,13 @@ Back pick(int64_t M, int K, bool bytes) {
     if (path == 2) return Back::GEMV;
     if (path == 3) return Back::TS;
     if (path == 4) return (bytes && K >= 128) ? Back::TMA : Back::TS;
-    if (M <= gemv_max_m()) return Back::GEMV;
+    // CUDA cores for a few tokens: the row GEMV where it takes the batch in one
+    // launch; past that at K >= 16384 the tensor-core kernel is faster than the
+    // split-K GEMV
+    if (M <= gemv_max_m() && (rows_gemv(M, K) || K < 16384)) return Back::GEMV;
     if (bytes && K >= 128 && M >= kTmaMinM) return Back::TMA;
     return Back::TS;
 }
-
-// The GEMV back end uses the row GEMV when K allows it and the tokens fit one
-// launch; otherwise the split-K GEMV (8-token chunks).
-bool rows_gemv(int64_t M, int K) { return gemv_rows_supported(K) && M <= gemv_rows_max_m(K); }
 
 size_t backend_ws(Back b, int64_t M, int K, int N) {
     switch (b) {

@@ -46,7 +46,9 @@ __device__ __forceinline__ uint2 widen_nibbles(uint32_t w) {
 }
 
 // L = log2 K (>= 11), MT = token capacity (1, 2, 4, 8), PRE = weights loaded
-// before the programmatic-dependency wait.
+// before the programmatic-dependency wait.  Each warp owns RPW consecutive
+// weight rows (RPW = 2 for two or more tokens: every activation word read from
+// shared memory then feeds two rows, halving that traffic).
 template <int L, int MT, bool PRE>
 __global__ void __launch_bounds__(kWarps * 32)
     gemv_rows_kernel(const uint8_t* __restrict__ codes, int act_bits, int M,
@@ -54,25 +56,26 @@ __global__ void __launch_bounds__(kWarps * 32)
                      const float* __restrict__ scales, const float* __restrict__ alpha,
                      uint16_t* __restrict__ Y, int32_t* __restrict__ acc_out) {
     constexpr int K = 1 << L;
-    constexpr int CH = K / 2048;  // 16-byte weight chunks per lane
+    constexpr int CH = K / 2048;  // 16-byte weight chunks per lane per row
     constexpr int NC = K / 64;    // 16-byte chunks per weight row
+    constexpr int RPW = MT >= 2 ? 2 : 1;
     extern __shared__ __align__(16) uint8_t sact[];  // [MT][4][NC] x 16 B
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int n = blockIdx.x * kWarps + warp;
-    const bool nok = n < N;
-    const uint4* wrow =
-        reinterpret_cast<const uint4*>(Wp + (int64_t)(nok ? n : N - 1) * (K / 16));
+    const int nb = (blockIdx.x * kWarps + warp) * RPW;  // first row of this warp
 
-    uint4 w[CH];
-    if constexpr (PRE) {
+    uint4 w[RPW][CH];
+    auto load_w = [&]() {
 #pragma unroll
-        for (int i = 0; i < CH; ++i) w[i] = __ldg(wrow + lane + 32 * i);
-    }
+        for (int r = 0; r < RPW; ++r) {
+            const int n = min(nb + r, N - 1);  // rows past N read a valid row, never stored
+            const uint4* wrow = reinterpret_cast<const uint4*>(Wp + (int64_t)n * (K / 16));
+#pragma unroll
+            for (int i = 0; i < CH; ++i) w[r][i] = __ldg(wrow + lane + 32 * i);
+        }
+    };
+    if constexpr (PRE) load_w();
     pdl_wait();
-    if constexpr (!PRE) {
-#pragma unroll
-        for (int i = 0; i < CH; ++i) w[i] = __ldg(wrow + lane + 32 * i);
-    }
+    if constexpr (!PRE) load_w();
 
     // stage activations: item = (m, piece p, chunk c) with c fastest, so the
     // shared-memory stores of a warp are consecutive 16-byte words; the
@@ -95,51 +98,65 @@ __global__ void __launch_bounds__(kWarps * 32)
     }
     __syncthreads();
 
-    int acc[MT];
+    int acc[RPW][MT];
 #pragma unroll
-    for (int m = 0; m < MT; ++m) acc[m] = 0;
+    for (int r = 0; r < RPW; ++r)
+#pragma unroll
+        for (int m = 0; m < MT; ++m) acc[r][m] = 0;
 #pragma unroll
     for (int i = 0; i < CH; ++i) {
         const int c = lane + 32 * i;
-        const uint32_t wv[4] = {w[i].x, w[i].y, w[i].z, w[i].w};
 #pragma unroll
         for (int m = 0; m < MT; ++m) {
 #pragma unroll
             for (int p = 0; p < 4; ++p) {
                 const uint4 a = *reinterpret_cast<const uint4*>(
                     sact + ((size_t)(m * 4 + p) * NC + c) * 16);
-                int s = acc[m];
-                s = dp4a_su((int)a.x, wv[p] & 0x03030303u, s);
-                s = dp4a_su((int)a.y, (wv[p] >> 2) & 0x03030303u, s);
-                s = dp4a_su((int)a.z, (wv[p] >> 4) & 0x03030303u, s);
-                s = dp4a_su((int)a.w, (wv[p] >> 6) & 0x03030303u, s);
-                acc[m] = s;
+#pragma unroll
+                for (int r = 0; r < RPW; ++r) {
+                    const uint32_t wp = p == 0 ? w[r][i].x
+                                      : p == 1 ? w[r][i].y
+                                      : p == 2 ? w[r][i].z
+                                               : w[r][i].w;
+                    int s = acc[r][m];
+                    s = dp4a_su((int)a.x, wp & 0x03030303u, s);
+                    s = dp4a_su((int)a.y, (wp >> 2) & 0x03030303u, s);
+                    s = dp4a_su((int)a.z, (wp >> 4) & 0x03030303u, s);
+                    s = dp4a_su((int)a.w, (wp >> 6) & 0x03030303u, s);
+                    acc[r][m] = s;
+                }
             }
         }
     }
 #pragma unroll
-    for (int m = 0; m < MT; ++m)
-#pragma unroll
-        for (int b = 16; b >= 1; b >>= 1) acc[m] += __shfl_xor_sync(0xffffffffu, acc[m], b);
-
-    if (nok) {
-        const float a = *alpha;
+    for (int r = 0; r < RPW; ++r)
 #pragma unroll
         for (int m = 0; m < MT; ++m)
-            if (lane == m && m < M) {
-                const int s = acc[m] - rowsum[m];
+#pragma unroll
+            for (int b = 16; b >= 1; b >>= 1)
+                acc[r][m] += __shfl_xor_sync(0xffffffffu, acc[r][m], b);
+
+    const float a = *alpha;
+#pragma unroll
+    for (int r = 0; r < RPW; ++r)
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+            const int n = nb + r;
+            if (lane == r * MT + m && m < M && n < N) {
+                const int s = acc[r][m] - rowsum[m];
                 if (acc_out != nullptr) acc_out[(int64_t)m * N + n] = s;
                 const float y = __fmul_rn((float)s, __fmul_rn(a, scales[m]));
                 Y[(int64_t)m * N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(y));
             }
-    }
+        }
 }
 
 template <int L, int MT>
 static hbl_status launch_mt(const GemmArgs& a, bool pre, cudaStream_t stream) {
     constexpr int K = 1 << L;
+    constexpr int RPW = MT >= 2 ? 2 : 1;
     const size_t smem = (size_t)MT * K;
-    const dim3 grid((unsigned)((a.N + kWarps - 1) / kWarps)), block(kWarps * 32);
+    const dim3 grid((unsigned)((a.N + kWarps * RPW - 1) / (kWarps * RPW))), block(kWarps * 32);
     const uint8_t* codes = static_cast<const uint8_t*>(a.codes);
     const int M = (int)a.M;
     if (pre) {
