@@ -296,7 +296,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_ts_kernel(Params p) {
 
     if (tid == 0) {
         for (int s = 0; s < S; ++s) {
-            mbar_init(full_bar(s), 32 * kConvWarps);
+            mbar_init(full_bar(s), kConvWarps);  // one arrival per converter warp
             mbar_init(empty_bar(s), 1);
         }
         mbar_init(acc_bar, 1);
@@ -398,7 +398,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_ts_kernel(Params p) {
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
             tc_fence_before();
-            mbar_arrive(full_bar(s));
+            __syncwarp();  // the warp's shared and TMEM writes are ordered before lane 0's arrive
+            if (lane == 0) mbar_arrive(full_bar(s));
             return true;
         };
         Packed<ABITS> P0, P1;
