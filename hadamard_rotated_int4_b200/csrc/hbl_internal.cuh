@@ -143,14 +143,10 @@ __device__ __forceinline__ void pdl_launch_dependents() {
 
 __device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
 __device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+// a - b as one packed fma: b * (-1) + a rounds the exact a - b once, so it is
+// bit-identical to an IEEE subtraction.
 __device__ __forceinline__ float2 sub2(float2 a, float2 b) {
-    unsigned long long ra, rb, rd;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(ra) : "f"(a.x), "f"(a.y));
-    asm("mov.b64 %0, {%1, %2};" : "=l"(rb) : "f"(b.x), "f"(b.y));
-    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(rd) : "l"(ra), "l"(rb));
-    float2 d;
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(d.x), "=f"(d.y) : "l"(rd));
-    return d;
+    return __ffma2_rn(b, make_float2(-1.0f, -1.0f), a);
 }
 
 // bf16 pair (low half = first element) -> two fp32 (exact widening).

@@ -445,3 +445,29 @@ def test_bounded_wait_reports_timeout_and_context_survives(arrive):
     torch.cuda.synchronize()
     wc, _, _ = oracle.norm_fwht_quant(acts(3, 256, seed=1), 4)
     assert np.array_equal(codes.cpu().numpy(), wc)
+
+
+@pytest.mark.parametrize("N,K", [(16, 256), (272, 2048), (4096, 16384)])
+def test_expand_ternary_matches_unpacked_codes(N, K):
+    W = inputs.latent_weights(N, K, seed=N)
+    packed, _ = oracle.pack_ternary(W)
+    Ws = hbl.expand_ternary(torch.from_numpy(packed.view(np.int32)).to(DEV), K)
+    torch.cuda.synchronize()
+    assert np.array_equal(Ws.cpu().numpy(), oracle.unpack_codes(packed, K))
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("M,K,N", [(1, 128, 16), (300, 4096, 400), (1030, 2048, 512)])
+def test_gemm_on_kept_expanded_weights(bits, M, K, N):
+    codes, scales, rowsum, packed, alpha = make_gemm_case(M, K, N, bits, seed=M + 3)
+    q = oracle.decode_codes(codes, K, bits)
+    Ws = hbl.expand_ternary(torch.from_numpy(packed.view(np.int32)).to(DEV), K)
+    act = 8 if bits == 8 else hbl.ACT_INT4_BYTES
+    Y, acc = hbl.ternary_gemm_s8w(
+        torch.from_numpy(q.view(np.uint8).copy()).to(DEV), torch.from_numpy(scales).to(DEV), act,
+        Ws, torch.from_numpy(np.array([alpha, 0, 0, 0], dtype=np.float32)).to(DEV),
+        want_acc=True)
+    torch.cuda.synchronize()
+    wY, wacc = oracle.ternary_gemm(codes, scales, bits, K, packed, alpha)
+    assert np.array_equal(acc.cpu().numpy(), wacc)
+    assert np.array_equal(bf16_bits(Y), wY)
