@@ -133,6 +133,7 @@ struct Packed {
     static constexpr int kA = ABITS == 8 ? 8 : 4;  // 16-byte chunks of this row per stage
     uint4 a[kA];
     uint4 b;
+    uint4 b2;  // second 16-byte weight chunk (HALF: each thread owns a whole 128-weight row piece)
 };
 
 // Per-thread constants of the converter loop.
@@ -195,7 +196,7 @@ __device__ __forceinline__ void load_stage(const ConvPtrs& cp, int K, int kb, Pa
 // results are never stored), running pointers, immediate offsets.
 // a_on = false (warp-uniform): this warp's token rows are all past M, so its
 // activation loads are skipped (the MMA rows they would feed are never stored).
-template <int ABITS, bool IL>
+template <int ABITS, bool IL, bool TWO = false>
 struct FastLoader {
     const uint8_t* a;
     const uint32_t* b;
@@ -213,6 +214,7 @@ struct FastLoader {
         }
         a += ABITS == 8 ? (IL ? 8 * 512 : BK) : BK / 2;
         P.b = *reinterpret_cast<const uint4*>(b);
+        if constexpr (TWO) P.b2 = *reinterpret_cast<const uint4*>(b + 4);
         b += BK / 16;
     }
 };
@@ -231,9 +233,10 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
         : "memory");
 }
 
-template <int ABITS>
+template <int ABITS, bool TWO = false>
 __device__ __forceinline__ void store_stage(uint32_t a_taddr, uint32_t sB, const uint32_t (&boff)[4],
-                                            const Packed<ABITS>& P, bool a_on) {
+                                            const uint32_t (&boff2)[4], const Packed<ABITS>& P,
+                                            bool a_on) {
     uint32_t av[32];
     if constexpr (ABITS == 8) {
 #pragma unroll
@@ -264,12 +267,26 @@ __device__ __forceinline__ void store_stage(uint32_t a_taddr, uint32_t sB, const
                make_uint4(w & 0x03030303u, (w >> 2) & 0x03030303u, (w >> 4) & 0x03030303u,
                           (w >> 6) & 0x03030303u));
     }
+    if constexpr (TWO) {
+        const uint32_t wv2[4] = {P.b2.x, P.b2.y, P.b2.z, P.b2.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const uint32_t w = wv2[j];
+            sts128(sB + boff2[j],
+                   make_uint4(w & 0x03030303u, (w >> 2) & 0x03030303u, (w >> 4) & 0x03030303u,
+                              (w >> 6) & 0x03030303u));
+        }
+    }
 }
 
 // SMALL: a single tile of tokens (M <= 256, decode batches): split-K over
 // grid.z, one accumulator when M <= 128, and the weights prefetched into L2
 // before the dependency wait.  The large-M instantiation keeps none of these.
-template <int ABITS, bool IL, bool FULLK, bool SMALL>
+// HALF (SMALL, M <= 128, K % 128 == 0): only the four converter warps of the
+// one accumulator run; each thread converts a whole 32-byte piece of its
+// weight row per stage, so the per-stage synchronisation is paid by half as
+// many warps.
+template <int ABITS, bool IL, bool FULLK, bool SMALL, bool HALF = false>
 __global__ void __launch_bounds__(kThreads, 1) gemm_ts_kernel(Params p) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_s = smem_addr(smem_raw);
@@ -292,11 +309,11 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_ts_kernel(Params p) {
     const int kb0 = SMALL ? (int)blockIdx.z * p.kps : 0;
     const int num_kb = SMALL ? min(p.kps, num_kb_total - kb0) : num_kb_total;
     // rows of this tile that exist: one accumulator suffices when M - m0 <= 128
-    const int nacc = (!SMALL || p.M - m0 > 128) ? 2 : 1;
+    const int nacc = HALF ? 1 : ((!SMALL || p.M - m0 > 128) ? 2 : 1);
 
     if (tid == 0) {
         for (int s = 0; s < S; ++s) {
-            mbar_init(full_bar(s), kConvWarps);  // one arrival per converter warp
+            mbar_init(full_bar(s), HALF ? kConvWarps / 2 : kConvWarps);  // one per converter warp
             mbar_init(empty_bar(s), 1);
         }
         mbar_init(acc_bar, 1);
@@ -358,6 +375,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_ts_kernel(Params p) {
         if (lane == 0) mma_commit(acc_bar);
         __syncwarp();
         if (!warp_wait(acc_bar, 0) && lane == 0) report_status(p.status, HBL_ERR_TIMEOUT);
+    } else if (HALF && warp > kConvWarps / 2) {
+        // ---------------- HALF: the second accumulator's warps have nothing to do
     } else {
         // ---------------- converters, then epilogue
         const int ct = tid - 32;                 // 0..255
@@ -368,7 +387,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_ts_kernel(Params p) {
         // one-tile batches: warps whose 32 rows all lie past M skip their
         // activation loads and TMEM stores (warp-uniform)
         const bool a_on = !SMALL || (m0 + 128 * acc + 32 * q < p.M);
-        const int br = ct >> 1, bh = ct & 1;     // weight row / half of this thread's chunk
+        // weight row / half of this thread's 16-byte chunk (HALF: both halves)
+        const int br = HALF ? ct : (ct >> 1), bh = HALF ? 0 : (ct & 1);
         const int n = n0 + br;
         const uint32_t lane_base = (uint32_t)(32 * q) << 16;
         ConvPtrs cp;
@@ -381,9 +401,12 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_ts_kernel(Params p) {
         }
         cp.b = (n < p.N) ? p.W + (int64_t)n * (p.K / 16) : nullptr;
         cp.bh = bh;
-        uint32_t boff[4];
+        uint32_t boff[4], boff2[4];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) boff[j] = sw128(br, 4 * bh + j);
+        for (int j = 0; j < 4; ++j) {
+            boff[j] = sw128(br, 4 * bh + j);
+            boff2[j] = sw128(br, 4 + j);
+        }
         const uint32_t a_col0 = tmem + lane_base + 256u + 32u * acc;
 
         // one stage: wait for the slot, write A to TMEM and B to shared memory, signal
@@ -394,7 +417,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_ts_kernel(Params p) {
             go = go && (__shfl_sync(0xffffffffu, *abort_flag, 0) == 0);
             if (!go) return false;  // warp-uniform
             tc_fence_after();
-            store_stage<ABITS>(a_col0 + 64u * s, base_s + s * kBStageBytes, boff, P, a_on);
+            store_stage<ABITS, HALF>(a_col0 + 64u * s, base_s + s * kBStageBytes, boff, boff2, P,
+                                     a_on);
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
             tc_fence_before();
@@ -405,7 +429,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_ts_kernel(Params p) {
         Packed<ABITS> P0, P1;
         bool ok = true;
         if constexpr (FULLK) {
-            FastLoader<ABITS, IL> ld;
+            FastLoader<ABITS, IL, HALF> ld;
             ld.a_on = a_on;
             {
                 int64_t mm = m;
@@ -551,8 +575,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_ts_kernel(Params p) {
 
 template <int ABITS, bool IL>
 static hbl_status launch(const Params& prm, cudaStream_t stream) {
-    const bool full = prm.K % BK == 0, small = prm.M <= BM;
-    auto kern = full ? (small ? gemm_ts_kernel<ABITS, IL, true, true>
+    const bool full = prm.K % BK == 0, small = prm.M <= BM, half = small && prm.M <= 128;
+    auto kern = full ? (small ? (half ? gemm_ts_kernel<ABITS, IL, true, true, true>
+                                      : gemm_ts_kernel<ABITS, IL, true, true>)
                               : gemm_ts_kernel<ABITS, IL, true, false>)
                      : (small ? gemm_ts_kernel<ABITS, IL, false, true>
                               : gemm_ts_kernel<ABITS, IL, false, false>);
