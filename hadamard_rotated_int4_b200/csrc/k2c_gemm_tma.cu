@@ -10,7 +10,8 @@
 // with q one byte per code (INT8 values, or INT4 values in [-8, 7]) row-major,
 // and t in {-1, 0, +1} one signed byte per weight, row-major [N x K].  The
 // library's packed 2-bit weights are expanded to that form in workspace by
-// expand_kernel below (N*K bytes written, N*K/4 read) before the GEMM.
+// the expansion kernel (k2d_expand_ternary.cu: N*K bytes written, N*K/4 read)
+// before the GEMM.
 //
 // There is no narrower integer MMA than 8 bits in tcgen05, so the weights must
 // reach shared memory as bytes; expanding them once per call in HBM (67 MB for
@@ -342,21 +343,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-// Packed 2-bit codes (16 per word; weight j of a word at bits 8(j%4) + 2(j/4),
-// code t + 1) -> one signed byte t per weight, row-major [N x K].  Bytes 4i..4i+3
-// of a word's 16 are ((w >> 2i) & 0x03030303) - 1 per byte.
-__global__ void expand_kernel(const uint32_t* __restrict__ Wp, int64_t words,
-                              uint4* __restrict__ out) {
-    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < words;
-         i += (int64_t)gridDim.x * blockDim.x) {
-        const uint32_t w = Wp[i];
-        out[i] = make_uint4(__vsub4(w & 0x03030303u, 0x01010101u),
-                            __vsub4((w >> 2) & 0x03030303u, 0x01010101u),
-                            __vsub4((w >> 4) & 0x03030303u, 0x01010101u),
-                            __vsub4((w >> 6) & 0x03030303u, 0x01010101u));
-    }
-}
-
 // cuTensorMapEncodeTiled through the runtime's driver entry point (the library
 // links the CUDA runtime statically and not libcuda directly).
 static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -390,17 +376,6 @@ static bool make_map(CUtensorMap* map, const void* ptr, int64_t rows, int K, int
 }  // namespace k2c
 
 size_t gemm_tma_workspace(int K, int N) { return ((size_t)N * (size_t)K + 255) & ~(size_t)255; }
-
-hbl_status launch_expand_ternary(const uint32_t* W_packed, int N, int K, int8_t* W_s8,
-                                 cudaStream_t stream, int num_sms) {
-    const int64_t words = (int64_t)N * (K / 16);
-    if (words == 0) return HBL_OK;
-    int64_t blocks = (words + 255) / 256;
-    if (blocks > (int64_t)num_sms * 8) blocks = (int64_t)num_sms * 8;
-    k2c::expand_kernel<<<(unsigned)blocks, 256, 0, stream>>>(W_packed, words,
-                                                             reinterpret_cast<uint4*>(W_s8));
-    return cudaGetLastError() == cudaSuccess ? HBL_OK : HBL_ERR_CUDA;
-}
 
 hbl_status launch_gemm_tma_s8w(const GemmArgs& a, const int8_t* W_s8, cudaStream_t stream,
                                int num_sms) {

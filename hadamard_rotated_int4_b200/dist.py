@@ -47,3 +47,25 @@ def sum_over_ranks(value, device=None):
                      device=device if device is not None else "cpu")
     dist.all_reduce(t, op=dist.ReduceOp.SUM)
     return float(t.item())
+
+
+def gather_rows(Y_local, M, group=None):
+    """All-gather of row shards (the shard_rows split of M rows) into one [M, N]
+    tensor on every rank: the optional step for a caller that wants the whole
+    output on each device.  The layer itself needs no collective.  Shards may
+    differ by one row, so each is padded to the largest before the all-gather
+    (NCCL on GPUs, gloo on CPU) and the padding is dropped afterwards."""
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size(group) == 1:
+        return Y_local
+    world = dist.get_world_size(group)
+    spans = [shard_rows(M, world, r) for r in range(world)]
+    rows = max(b - a for a, b in spans)
+    pad = torch.zeros((rows,) + tuple(Y_local.shape[1:]), dtype=Y_local.dtype,
+                      device=Y_local.device)
+    pad[: Y_local.shape[0]] = Y_local
+    parts = [torch.empty_like(pad) for _ in range(world)]
+    dist.all_gather(parts, pad, group=group)
+    return torch.cat([parts[r][: b - a] for r, (a, b) in enumerate(spans)])

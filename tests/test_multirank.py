@@ -40,7 +40,10 @@ def _worker(rank, world, port, q):
         tsum = hdist.sum_over_ranks(1.0)
         gathered = [None] * world
         dist.all_gather_object(gathered, (lo, hi, Y))
-        q.put((rank, tmax, tsum, gathered))
+        # the optional output gather (bf16 bit patterns widened to int32: the
+        # gloo backend has no 16-bit integer type; NCCL takes bf16 directly)
+        Yall = hdist.gather_rows(torch.from_numpy(Y.astype(np.int32)), X.shape[0])
+        q.put((rank, tmax, tsum, gathered, Yall.numpy().astype(np.uint16)))
     finally:
         dist.destroy_process_group()
 
@@ -76,7 +79,8 @@ def test_two_rank_gloo_sharded_layer_and_timing():
     X = inputs.activations("tiny")
     packed, alpha = oracle.pack_ternary(inputs.weights("tiny"))
     full = oracle.hbitlinear_forward(X, packed, alpha, 4, threads=1)
-    for rank, tmax, tsum, gathered in results:
+    for rank, tmax, tsum, gathered, Yall in results:
         assert tmax == 2.5 and tsum == 2.0
         Ycat = np.concatenate([g[2] for g in sorted(gathered, key=lambda g: g[0])])
         assert np.array_equal(Ycat, full)
+        assert np.array_equal(Yall, full)  # the optional output all-gather
