@@ -471,3 +471,16 @@ def test_gemm_on_kept_expanded_weights(bits, M, K, N):
     wY, wacc = oracle.ternary_gemm(codes, scales, bits, K, packed, alpha)
     assert np.array_equal(acc.cpu().numpy(), wacc)
     assert np.array_equal(bf16_bits(Y), wY)
+
+
+@pytest.mark.parametrize("M", [1, 3, 300])
+def test_forward_at_the_largest_K(M):
+    # K = 32768 (the largest transform): row GEMV (1 token), tensor-core kernel
+    # with activations in TMEM (3), TMA-fed GEMM (300); sampled rows vs the oracle
+    K, N = 32768, 256
+    X = inputs.student_t_acts(M, K, seed=M)
+    W = inputs.latent_weights(N, K, seed=M)
+    packed, alpha = oracle.pack_ternary(W)
+    Y = forward(X, packed, alpha, 4)
+    rows = np.arange(M) if M <= 3 else np.array([0, 1, 150, M - 1])
+    assert np.array_equal(Y[rows], oracle.hbitlinear_forward(X, packed, alpha, 4, rows=rows))
