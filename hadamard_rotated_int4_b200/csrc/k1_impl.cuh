@@ -565,6 +565,10 @@ __global__ void __launch_bounds__(Cfg<L>::kCtaThreads, Cfg<L>::kMinBlocks)
             // INT4 clamp on the integer bit pattern: q in [-8, 7]
             constexpr int32_t kLoBits = kMagicBits - 8, kHiBits = kMagicBits + 7;
             constexpr bool kPackNibbles = (MODE == 4);
+            // ... or on int16 halves where |q| < 2^15 is guaranteed (K <= 8192)
+            constexpr bool kClamp16 = !kAbsmax && L <= 13;
+            constexpr uint32_t kLo2 = kPackNibbles ? 0x00000000u : 0xFFF8FFF8u;
+            constexpr uint32_t kHi2 = kPackNibbles ? 0x000F000Fu : 0x00070007u;
             constexpr int RL = 1 << RUN;                                 // elements per run
             constexpr int BYTES = kPackNibbles ? RL / 2 : RL;            // code bytes per run
             constexpr int EPW = kPackNibbles ? (RL >= 8 ? 8 : 4) : 4;    // elements per word
@@ -577,36 +581,71 @@ __global__ void __launch_bounds__(Cfg<L>::kCtaThreads, Cfg<L>::kMinBlocks)
                 uint32_t wv[NWORD];
                 static_for<0, NWORD>([&](auto ww) {
                     constexpr int wi = decltype(ww)::value;
-                    uint32_t qv[EPW];
-                    static_for<0, EPW / 2>([&](auto kk) {
-                        constexpr int k = (m * RL + wi * EPW) / 2 + decltype(kk)::value;
-                        const float2 y = __ffma2_rn(d[k], inv2, magic2);
-                        int32_t b0 = __float_as_int(y.x), b1 = __float_as_int(y.y);
-                        if constexpr (!kAbsmax) {  // INT8 codes never leave [-127, 127]
-                            b0 = min(max(b0, kLoBits), kHiBits);
-                            b1 = min(max(b1, kLoBits), kHiBits);
+                    if constexpr (kClamp16) {
+                        // INT4 at K <= 8192: |q| <= sqrt7 * K < 2^15, so the low 16
+                        // bits of each rounded pattern hold q (+8 for nibbles)
+                        // exactly; pairs of codes are clamped as int16 halves
+                        uint32_t pr[EPW / 2];
+                        static_for<0, EPW / 2>([&](auto kk) {
+                            constexpr int k = (m * RL + wi * EPW) / 2 + decltype(kk)::value;
+                            const float2 y = __ffma2_rn(d[k], inv2, magic2);
+                            uint32_t h = __byte_perm(__float_as_uint(y.x),
+                                                     __float_as_uint(y.y), 0x5410);
+                            asm("min.s16x2 %0, %0, %1;" : "+r"(h) : "r"(kHi2));
+                            asm("max.s16x2 %0, %0, %1;" : "+r"(h) : "r"(kLo2));
+                            pr[decltype(kk)::value] = h;
+                        });
+                        if constexpr (!kPackNibbles) {  // bytes q0..q3
+                            wv[wi] = __byte_perm(pr[0], pr[1], 0x6420);
+                            qsum = (uint32_t)__dp4a((int)wv[wi], 0x01010101, (int)qsum);
+                        } else {  // byte = (q_odd + 8) << 4 | (q_even + 8), then q's nibbles
+                            uint32_t by[EPW / 2];
+                            static_for<0, EPW / 2>([&](auto kk) {
+                                constexpr int i = decltype(kk)::value;
+                                qsum = (uint32_t)__dp2a_lo((int)pr[i], 0x0101, (int)qsum);
+                                by[i] = pr[i] | (pr[i] >> 12);
+                            });
+                            const uint32_t lo2 = __byte_perm(by[0], by[1], 0x0040);
+                            if constexpr (EPW == 8) {
+                                const uint32_t hi2 = __byte_perm(by[2], by[3], 0x0040);
+                                wv[wi] = __byte_perm(lo2, hi2, 0x5410) ^ 0x88888888u;
+                            } else {
+                                wv[wi] = lo2 ^ 0x8888u;
+                            }
                         }
-                        qv[2 * decltype(kk)::value] = (uint32_t)b0;
-                        qv[2 * decltype(kk)::value + 1] = (uint32_t)b1;
-                    });
-                    if constexpr (!kPackNibbles) {  // one byte per code: low byte = q
-                        const uint32_t lo2 = __byte_perm(qv[0], qv[1], 0x0040);
-                        const uint32_t hi2 = __byte_perm(qv[2], qv[3], 0x0040);
-                        wv[wi] = __byte_perm(lo2, hi2, 0x5410);
-                        // rowsum: the four signed bytes summed by one dp4a
-                        qsum = (uint32_t)__dp4a((int)wv[wi], 0x01010101, (int)qsum);
                     } else {
-                        static_for<0, EPW>([&](auto ee) { qsum += qv[decltype(ee)::value]; });  // low nibble = q + 8; pairs by shift-add, bytes by permute
-                        const uint32_t p01 = (qv[1] << 4) + qv[0];
-                        const uint32_t p23 = (qv[3] << 4) + qv[2];
-                        const uint32_t lo2 = __byte_perm(p01, p23, 0x0040);
-                        if constexpr (EPW == 8) {
-                            const uint32_t p45 = (qv[5] << 4) + qv[4];
-                            const uint32_t p67 = (qv[7] << 4) + qv[6];
-                            const uint32_t hi2 = __byte_perm(p45, p67, 0x0040);
-                            wv[wi] = __byte_perm(lo2, hi2, 0x5410) ^ 0x88888888u;
+                        uint32_t qv[EPW];
+                        static_for<0, EPW / 2>([&](auto kk) {
+                            constexpr int k = (m * RL + wi * EPW) / 2 + decltype(kk)::value;
+                            const float2 y = __ffma2_rn(d[k], inv2, magic2);
+                            int32_t b0 = __float_as_int(y.x), b1 = __float_as_int(y.y);
+                            if constexpr (!kAbsmax) {  // INT8 codes never leave [-127, 127]
+                                b0 = min(max(b0, kLoBits), kHiBits);
+                                b1 = min(max(b1, kLoBits), kHiBits);
+                            }
+                            qv[2 * decltype(kk)::value] = (uint32_t)b0;
+                            qv[2 * decltype(kk)::value + 1] = (uint32_t)b1;
+                        });
+                        if constexpr (!kPackNibbles) {  // one byte per code: low byte = q
+                            const uint32_t lo2 = __byte_perm(qv[0], qv[1], 0x0040);
+                            const uint32_t hi2 = __byte_perm(qv[2], qv[3], 0x0040);
+                            wv[wi] = __byte_perm(lo2, hi2, 0x5410);
+                            // rowsum: the four signed bytes summed by one dp4a
+                            qsum = (uint32_t)__dp4a((int)wv[wi], 0x01010101, (int)qsum);
                         } else {
-                            wv[wi] = lo2 ^ 0x8888u;
+                            // low nibble = q + 8; pairs by shift-add, bytes by permute
+                            static_for<0, EPW>([&](auto ee) { qsum += qv[decltype(ee)::value]; });
+                            const uint32_t p01 = (qv[1] << 4) + qv[0];
+                            const uint32_t p23 = (qv[3] << 4) + qv[2];
+                            const uint32_t lo2 = __byte_perm(p01, p23, 0x0040);
+                            if constexpr (EPW == 8) {
+                                const uint32_t p45 = (qv[5] << 4) + qv[4];
+                                const uint32_t p67 = (qv[7] << 4) + qv[6];
+                                const uint32_t hi2 = __byte_perm(p45, p67, 0x0040);
+                                wv[wi] = __byte_perm(lo2, hi2, 0x5410) ^ 0x88888888u;
+                            } else {
+                                wv[wi] = lo2 ^ 0x8888u;
+                            }
                         }
                     }
                 });
@@ -636,9 +675,11 @@ __global__ void __launch_bounds__(Cfg<L>::kCtaThreads, Cfg<L>::kMinBlocks)
                     }
                 }
             });
-            // sum of codes: packed nibbles added kMagicBits + q per code (mod 2^32);
-            // one-byte codes were summed directly
-            int qs = kPackNibbles ? (int)(qsum - (uint32_t)R * (uint32_t)kMagicBits) : (int)qsum;
+            // sum of codes: packed nibbles added kMagicBits + q per code (mod 2^32),
+            // or q + 8 per code on the int16 path; one-byte codes were summed directly
+            int qs = !kPackNibbles ? (int)qsum
+                     : kClamp16    ? (int)qsum - 8 * R
+                                   : (int)(qsum - (uint32_t)R * (uint32_t)kMagicBits);
             qs = row_isum(qs);
 
             if (row_ok) {
