@@ -353,6 +353,13 @@ static hbl_status forward_impl(const uint16_t* X, const float* gain, int M, int 
                                float norm_eps, float quant_eps, uint16_t* Y, uint8_t* ws,
                                size_t ws_bytes, int32_t* dev_status, cudaStream_t s, int sms,
                                unsigned variant = 0) {
+    // Decode batches: one kernel quantises and multiplies (no workspace used);
+    // a forced GEMM path keeps the two-kernel forward.
+    if (g_path.load() == 0 && decode_fused_supported(M, K, N, act_bits, variant, sms)) {
+        DecodeArgs d{X, gain, M, K, N, W_packed, alpha, act_bits, norm_eps, quant_eps, Y,
+                     dev_status};
+        return launch_decode_fused(d, s, sms);
+    }
     // For the default tensor-core kernel the codes stay in workspace one per
     // byte (INT4 values too) in the 32-row interleaved layout, so the GEMM
     // loads them coalesced and without widening; other back ends take the

@@ -41,6 +41,26 @@ hbl_status launch_norm_fwht_quant(const uint16_t* X, const float* gain, int64_t 
                                   float* scales, int32_t* rowsum, float* V, cudaStream_t stream,
                                   int num_sms, unsigned variant = 0);
 
+// K6: the whole forward of a decode batch in one kernel (quantiser and ternary
+// GEMV fused; see k6_decode_fused.cuh).  Supported for M <= 16384 / K tokens
+// (K = 4096 / 8192 / 16384), RMSNorm + transform (no variant bits), when the
+// CTA's shared memory fits (decode_fused_supported).
+struct DecodeArgs {
+    const uint16_t* X;
+    const float* gain;
+    int M, K, N;
+    const uint32_t* W_packed;
+    const float* alpha;
+    int act_bits;
+    float norm_eps, quant_eps;
+    uint16_t* Y;
+    int32_t* status;
+};
+// Weight rows per CTA for N rows: spread evenly over at most num_sms CTAs.
+int decode_fused_rows(int N, int num_sms);
+bool decode_fused_supported(int M, int K, int N, int act_bits, unsigned variant, int num_sms);
+hbl_status launch_decode_fused(const DecodeArgs& d, cudaStream_t stream, int num_sms);
+
 // K4: offline weight rotation W_rot[n] = FWHT(W[n] * signs) * c_K (in place allowed).
 hbl_status launch_rotate_weights(const float* W, const float* signs, int N, int K, float* W_rot,
                                  cudaStream_t stream, int num_sms);

@@ -53,10 +53,10 @@ __host__ __device__ constexpr int reg_log(int L) {
     return (L == 13 || L == 14) ? 6 : (L < kRegLog ? L : kRegLog);
 }
 
-template <int L>
+template <int L, int RLOG = reg_log(L)>
 struct Cfg {
     static constexpr int K = 1 << L;
-    static constexpr int r = reg_log(L);
+    static constexpr int r = RLOG;
     static constexpr int R = 1 << r;           // values per thread
     static constexpr int t = L - r;            // thread bits of a row
     static constexpr int T = 1 << t;           // threads per row
@@ -77,9 +77,9 @@ struct Cfg {
 };
 
 // Layout p: 0 = natural, p >= 1 = pass p (stage base r + (r - 2)(p - 1)).
-template <int L>
+template <int L, int RLOG = reg_log(L)>
 struct Lay {
-    using C = Cfg<L>;
+    using C = Cfg<L, RLOG>;
     __host__ __device__ static constexpr int pass_base(int p) {
         return C::r + C::kStagesPerPass * (p - 1);
     }
@@ -162,6 +162,37 @@ struct Params {
     float* scales;
     int32_t* rowsum;
     float* V;
+    // used only by an extension (Ext below) that consumes the codes in-kernel
+    const uint32_t* W;
+    const float* alpha;
+    uint16_t* Y;
+    int32_t* status;
+    int N, rows;
+};
+
+// Kernel extension points.  The plain kernel (NoExt) quantises rows spread
+// over the grid into global memory.  An extension (the one-kernel decode
+// forward) sets its own block shape and values per thread, keeps codes (one
+// byte each, row-major), scales and row sums in its shared memory, runs
+// `prologue` before the rows,
+// `staged` (thread 0) once the first row is in shared memory, and `finish`
+// after the rows, with the whole block.
+struct NoExt {
+    static constexpr bool kOn = false;
+    template <int L>
+    __host__ __device__ static constexpr int threads() { return Cfg<L>::kCtaThreads; }
+    template <int L>
+    __host__ __device__ static constexpr int min_blocks() { return Cfg<L>::kMinBlocks; }
+    template <int L>
+    __host__ __device__ static constexpr int rlog() { return reg_log(L); }
+    template <int L>
+    __host__ __device__ static constexpr int groups() { return Cfg<L>::kGroupsPerCta; }
+    static __device__ uint8_t* codes() { return nullptr; }
+    static __device__ float* scales() { return nullptr; }
+    static __device__ int32_t* rowsum() { return nullptr; }
+    static __device__ void prologue(const Params&) {}
+    static __device__ void staged(const Params&) {}
+    static __device__ void finish(const Params&) {}
 };
 
 template <int T>
@@ -235,19 +266,22 @@ __device__ __forceinline__ float stream_tree(F&& f) {
 // skip); kFlNoHadamard = no transform (the plain BitLinear of the layers
 // without H: the codes are those of the normalised row itself); kFlLayerNorm =
 // subtract the row mean first (LayerNorm without bias) instead of RMSNorm.
-template <int L, int MODE, int FL>
-__global__ void __launch_bounds__(Cfg<L>::kCtaThreads, Cfg<L>::kMinBlocks)
+template <int L, int MODE, int FL, class Ext = NoExt>
+__global__ void __launch_bounds__(Ext::template threads<L>(), Ext::template min_blocks<L>())
     norm_fwht_quant_kernel(Params p) {
     constexpr bool kAbsmax = (MODE == 8 || MODE == 9);       // INT8 absmax statistic
     constexpr bool kInterleaved = (MODE == 5 || MODE == 9);  // fused-forward code layout
     constexpr bool GAIN = (FL & kFlGain) != 0;
     constexpr bool kHadamard = (FL & kFlNoHadamard) == 0;
     constexpr bool kLayerNorm = (FL & kFlLayerNorm) != 0;
-    using C = Cfg<L>;
-    using Y = Lay<L>;
+    constexpr int RLOG = Ext::template rlog<L>();
+    constexpr int GPC = Ext::template groups<L>();  // row groups per block
+    using C = Cfg<L, RLOG>;
+    using Y = Lay<L, RLOG>;
     constexpr int R = C::R, T = C::T, W = C::W, K = C::K;
     constexpr int P_LAST = kHadamard ? C::kPasses : 0;  // final layout (natural without H)
     extern __shared__ __align__(128) uint8_t smem[];
+    if constexpr (Ext::kOn) Ext::prologue(p);
 
     const int tid = threadIdx.x;
     const int grp = tid / W;
@@ -258,8 +292,7 @@ __global__ void __launch_bounds__(Cfg<L>::kCtaThreads, Cfg<L>::kMinBlocks)
     const int wig = w >> 5;                      // warp within the row (T > 32)
     uint8_t* buf = smem + grp * C::kBufBytes;
     const uint32_t buf_s = smem_addr(buf);
-    float* red = reinterpret_cast<float*>(smem + C::kGroupsPerCta * C::kBufBytes) +
-                 grp * kRedFloats;
+    float* red = reinterpret_cast<float*>(smem + GPC * C::kBufBytes) + grp * kRedFloats;
 
     // thread part of the element index in layout P (plus the row offset)
     auto thr_off = [&](auto pp) -> uint32_t {
@@ -321,7 +354,11 @@ __global__ void __launch_bounds__(Cfg<L>::kCtaThreads, Cfg<L>::kMinBlocks)
         return x;
     };
 
-    const int64_t stride_groups = (int64_t)gridDim.x * C::kGroupsPerCta;
+    // an extension's block does all rows itself, with threads [0, GPC W)
+    const int64_t stride_groups = (int64_t)(Ext::kOn ? 1u : gridDim.x) * GPC;
+    const int64_t rg_first = (!Ext::kOn || tid < GPC * W)
+                                 ? (int64_t)(Ext::kOn ? 0u : blockIdx.x) * GPC + grp
+                                 : p.M;
     // Stage a group's bf16 rows in shared memory with coalesced 16-byte
     // cp.async (zero-filled past M); also hint the group after it into L2.
     auto issue_load = [&](int64_t g_rg) {
@@ -350,14 +387,17 @@ __global__ void __launch_bounds__(Cfg<L>::kCtaThreads, Cfg<L>::kMinBlocks)
 
     // One row group per thread (small M, e.g. decode): let the next kernel
     // start its prologue (weight prefetch) while this one works.
-    if ((int64_t)gridDim.x * C::kGroupsPerCta * C::kRowsPerGroup >= p.M) pdl_launch_dependents();
-    issue_load((int64_t)blockIdx.x * C::kGroupsPerCta + grp);
-    for (int64_t rg = (int64_t)blockIdx.x * C::kGroupsPerCta + grp;; rg += stride_groups) {
+    if (!Ext::kOn && stride_groups * C::kRowsPerGroup >= p.M) pdl_launch_dependents();
+    issue_load(rg_first);
+    for (int64_t rg = rg_first;; rg += stride_groups) {
         const int64_t row0 = rg * C::kRowsPerGroup;
         if (row0 >= p.M) break;
         const int64_t row = row0 + rig;
         cp_async_wait_all();
         group_sync<T>(grp);
+        if constexpr (Ext::kOn) {
+            if (rg == rg_first && tid == 0) Ext::staged(p);
+        }
 
         float2 d[R / 2];
         {
@@ -574,7 +614,8 @@ __global__ void __launch_bounds__(Cfg<L>::kCtaThreads, Cfg<L>::kMinBlocks)
             constexpr int EPW = kPackNibbles ? (RL >= 8 ? 8 : 4) : 4;    // elements per word
             constexpr int NWORD = RL / EPW;
             const bool row_ok = row < p.M;
-            uint8_t* crow = p.codes + row0 * (int64_t)(kPackNibbles ? K / 2 : K);
+            uint8_t* crow = (Ext::kOn ? Ext::codes() : p.codes) +
+                            row0 * (int64_t)(kPackNibbles ? K / 2 : K);
             uint32_t qsum = 0;
             static_for<0, R / RL>([&](auto mm) {
                 constexpr int m = decltype(mm)::value;
@@ -684,12 +725,16 @@ __global__ void __launch_bounds__(Cfg<L>::kCtaThreads, Cfg<L>::kMinBlocks)
 
             if (row_ok) {
                 if (j == 0) {
-                    p.scales[row] = __fdiv_rn(stat, cq);
-                    if (p.rowsum != nullptr) p.rowsum[row] = qs;
+                    (Ext::kOn ? Ext::scales() : p.scales)[row] = __fdiv_rn(stat, cq);
+                    if constexpr (Ext::kOn)
+                        Ext::rowsum()[row] = qs;
+                    else if (p.rowsum != nullptr)
+                        p.rowsum[row] = qs;
                 }
             }
         }
     }
+    if constexpr (Ext::kOn) Ext::finish(p);
 }
 
 template <int L, int MODE, int FL>

@@ -77,7 +77,8 @@ HBL_API int hbl_version(void);
 
 /* Choice of ternary-GEMM back end (test and tuning aid; process-wide, not
  * synchronised with calls in flight on other threads):
- *   0 = automatic: CUDA-core GEMV for M <= 8 tokens (one weight row per warp
+ *   0 = automatic (and, in hbl_hbitlinear_forward, the one-kernel decode
+ *       forward where it applies): CUDA-core GEMV for M <= 8 tokens (one weight row per warp
  *       for K >= 2048, split-K below); the tcgen05 kernel with activations in
  *       tensor memory (split over K for M <= 256) up to 256 tokens; above that
  *       the TMA-fed tcgen05 kernel when the codes are one byte each (it expands
@@ -173,6 +174,10 @@ HBL_API hbl_status hbl_ternary_gemm(const void* codes, const float* scales, cons
                             void* ws, size_t ws_bytes, int32_t* dev_status, void* stream);
 
 /* The whole layer: hbl_norm_fwht_quant into workspace, then hbl_ternary_gemm.
+ * Decode batches (M <= 16384 / K tokens at K = 4096 / 8192 / 16384, while the
+ * packed weight rows of one SM's share fit its shared memory, GEMM path 0) run
+ * both steps in one kernel instead: every CTA quantises the M rows itself
+ * while its weight rows stream in; the results are the same values.
  * X: bf16 [M x K]; Y: bf16 [M x N] out; other arguments as above.
  * ws: >= hbl_workspace_size(HBL_OP_HBITLINEAR_FORWARD, M, K, N, act_bits). */
 HBL_API hbl_status hbl_hbitlinear_forward(const uint16_t* X, const float* gain, int M, int K, int N,

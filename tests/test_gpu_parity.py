@@ -283,12 +283,13 @@ def test_gemm_identity_weights(bits):
 
 # ------------------------------------------------------------ whole layer
 
-def forward(X, packed, alpha, bits, path=0):
+def forward(X, packed, alpha, bits, path=0, gain=None):
     hbl.set_gemm_path(path)
     try:
         Y = hbl.hbitlinear_forward(
             to_dev_bf16(X), torch.from_numpy(packed.view(np.int32)).to(DEV),
-            torch.from_numpy(np.array([alpha, 0, 0, 0], dtype=np.float32)).to(DEV), bits)
+            torch.from_numpy(np.array([alpha, 0, 0, 0], dtype=np.float32)).to(DEV), bits,
+            gain=None if gain is None else torch.from_numpy(gain).to(DEV))
         torch.cuda.synchronize()
     finally:
         hbl.set_gemm_path(0)
@@ -352,6 +353,50 @@ def test_decode_sweep(T, shape):
     rows = np.arange(T) if T <= 8 else np.concatenate([np.arange(4), [T - 1]])
     want = oracle.hbitlinear_forward(X, packed, alpha, 4, rows=rows)
     assert np.array_equal(Y[rows], want)
+
+
+# one-kernel decode forward (M <= 16384 / K tokens at K = 4096 / 8192 / 16384
+# where the CTA's weight rows fit shared memory) against the oracle and
+# against the two-kernel forward (GEMM path 2: K1, then the row GEMV).  N (a
+# multiple of 16) spans fewer rows than SMs, ragged splits over the SMs and the
+# largest split that fits; the other (M, K) pairs take the two-kernel forward.
+@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("K,N", [(4096, 4096), (4096, 1008), (4096, 16384), (8192, 304),
+                                 (8192, 4096), (16384, 112), (16384, 4096)])
+@pytest.mark.parametrize("M", [1, 2, 3, 4])
+def test_decode_one_kernel_forward(bits, K, N, M):
+    X = acts(M, K, seed=M + K, kind="t" if M % 2 else "gauss")
+    W = inputs.latent_weights(N, K, seed=N + M)
+    packed, alpha = oracle.pack_ternary(W)
+    want = oracle.hbitlinear_forward(X, packed, alpha, bits)
+    assert np.array_equal(forward(X, packed, alpha, bits), want)
+    assert np.array_equal(forward(X, packed, alpha, bits, path=2), want)
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("M,K", [(1, 4096), (2, 8192), (4, 4096), (1, 16384)])
+def test_decode_one_kernel_forward_with_gain(bits, M, K):
+    X = acts(M, K, seed=5)
+    g = np.random.default_rng(K).uniform(0.25, 2.0, K).astype(np.float32)
+    W = inputs.latent_weights(512, K, seed=9)
+    packed, alpha = oracle.pack_ternary(W)
+    want = oracle.hbitlinear_forward(X, packed, alpha, bits, gain=g)
+    assert np.array_equal(forward(X, packed, alpha, bits, gain=g), want)
+
+
+def test_decode_one_kernel_edge_rows():
+    # zero, constant and single-spike rows (the transform of a spike is flat;
+    # of a Hadamard row, a spike) next to a normal row, M = 4
+    K, N = 4096, 704
+    X = np.zeros((4, K), dtype=np.uint16)
+    X[1] = np.float32(0.75).view(np.uint32) >> 16
+    X[2, 77] = np.float32(-3.0).view(np.uint32) >> 16
+    X[3] = acts(1, K, seed=11)[0]
+    W = inputs.latent_weights(N, K, seed=3)
+    packed, alpha = oracle.pack_ternary(W)
+    for bits in (4, 8):
+        assert np.array_equal(forward(X, packed, alpha, bits),
+                              oracle.hbitlinear_forward(X, packed, alpha, bits))
 
 
 @pytest.mark.parametrize("T,K", [(1, 4096), (32, 16384), (300, 2048)])
