@@ -51,7 +51,8 @@ def parse():
     ap.add_argument("--kernel-iters", type=int, default=200,
                     help="iterations of the per-kernel timing loops")
     ap.add_argument("--only", default=None, choices=["forward", "gemm", "quant4", "quant8", "nohad4", "ln4",
-                                                      "rotate", "kv3", "kv4", "kv8"],
+                                                      "rotate", "kv3", "kv4", "kv8", "decode_wo",
+                                                      "decode_wdown"],
                     help="run only this case (a few launches, for profiler captures); prints a "
                          "short JSON line, not the benchmark line")
     return ap.parse_args()
@@ -381,7 +382,9 @@ def run_hbl(args):
             decode.append({"shape": shape, "T": T, "K": Kd, "N": N_OUT, "us": t * 1e6,
                            "tokens_per_s": T / t, "packed_w_gbs": wbytes / t / 1e9,
                            "frac_hbm_on_packed_w": wbytes / t / 1e9 / pk["hbm_gbs"],
-                           "path": ("row GEMV (weight rows per warp, PDL after K1)"
+                           "path": ("one kernel (quantiser in every CTA, weights by bulk copy)"
+                                    if T <= 16384 // Kd
+                                    else "row GEMV (weight rows per warp, PDL after K1)"
                                     if T <= (4 if Kd >= 16384 else 8)
                                     else "gemm_ts (TMEM activations, one-wave split-K)"),
                            "timing": "CUDA graph replay, one forward per weight copy"})
@@ -550,6 +553,14 @@ def run_only(args):
         QX = torch.from_numpy(inputs.qkv_states().view(np.int16)).view(torch.bfloat16).to(dev)
         kb = int(args.only[2:])
         fn = lambda: hbl.kv_quant(QX, kb)
+    elif args.only.startswith("decode"):  # one token through W_o or W_down
+        Kd = 4096 if args.only == "decode_wo" else 16384
+        Xt = torch.from_numpy(inputs.activations(args.only, M=1, K=Kd, seed=1).view(
+            np.int16)).view(torch.bfloat16).to(dev)
+        pd, ad = hbl.pack_ternary(torch.from_numpy(inputs.latent_weights(N_OUT, Kd, seed=7)).to(dev))
+        wsd = torch.empty(max(16, hbl.workspace_size(hbl.OP_HBITLINEAR_FORWARD, 1, Kd, N_OUT,
+                                                     BITS)), dtype=torch.uint8, device=dev)
+        fn = lambda: hbl.hbitlinear_forward(Xt, pd, ad, BITS, ws=wsd)
     else:
         X = torch.from_numpy(inputs.activations("ffn_wdown").view(np.int16)).view(
             torch.bfloat16).to(dev)

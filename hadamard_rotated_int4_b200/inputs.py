@@ -80,7 +80,7 @@ WORKLOADS = {
     "ffn_wdown": dict(M=8192, K=16384, N=4096),
 }
 
-DECODE_TOKENS = (1, 8, 32, 128, 256)
+DECODE_TOKENS = (1, 2, 4, 8, 32, 128, 256)
 
 
 def activations(name, seed=0, M=None, K=None):
