@@ -17,6 +17,8 @@ namespace hbl {
 
 template <int I>
 using ic = std::integral_constant<int, I>;
+template <bool B>
+using ic_bool = std::integral_constant<bool, B>;
 
 template <int Begin, int End, class F>
 __device__ __forceinline__ void static_for(F&& f) {

@@ -162,6 +162,9 @@ struct Params {
     float* scales;
     int32_t* rowsum;
     float* V;
+    // INT4 at K >= 16384: rows with norm_eps-free energy (sum x^2 >= 2^-100)
+    // and den > thr16 have every |q| < 2^15 (see the quantisation below)
+    float thr16;
     // used only by an extension (Ext below) that consumes the codes in-kernel
     const uint32_t* W;
     const float* alpha;
@@ -169,6 +172,12 @@ struct Params {
     int32_t* status;
     int N, rows;
 };
+
+// den above this keeps every INT4 |q| below 2^15 at K >= 16384 without a gain
+// (Params::thr16): sqrt(7 K) (1 + 2^-8) / 32767, rounded up.
+inline float thr16_for(int K) {
+    return nextafterf((float)(sqrt(7.0 * K) * (1.0 + 1.0 / 256) / 32767.0), INFINITY);
+}
 
 // Kernel extension points.  The plain kernel (NoExt) quantises rows spread
 // over the grid into global memory.  An extension (the one-kernel decode
@@ -436,6 +445,7 @@ __global__ void __launch_bounds__(Ext::template threads<L>(), Ext::template min_
             return __fmaf_rn(d[k].x, d[k].x, __fmul_rn(d[k].y, d[k].y));
         });
         ss = row_sum(ss);
+        [[maybe_unused]] const bool ss_ok = ss >= 0x1p-100f;
         const float ms = __fmul_rn(ss, 1.0f / (float)K);
         const float rn = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, p.norm_eps)));
         {
@@ -605,8 +615,14 @@ __global__ void __launch_bounds__(Ext::template threads<L>(), Ext::template min_
             // INT4 clamp on the integer bit pattern: q in [-8, 7]
             constexpr int32_t kLoBits = kMagicBits - 8, kHiBits = kMagicBits + 7;
             constexpr bool kPackNibbles = (MODE == 4);
-            // ... or on int16 halves where |q| < 2^15 is guaranteed (K <= 8192)
-            constexpr bool kClamp16 = !kAbsmax && L <= 13;
+            // ... or on int16 halves where |q| < 2^15 is guaranteed: always for
+            // K <= 8192 (|q| <= sqrt7 K); for larger K without a gain, on rows
+            // where max|v| <= ||v|| <= sqrt(K) (1 + 2^-8) bounds |q| by
+            // sqrt(7 K) (1 + 2^-8) / den < 2^15 - 1, i.e. den > thr16 (||u||^2 =
+            // r^2 sum x^2 <= K up to rounding, the transform is orthonormal; the
+            // sum x^2 >= 2^-100 test keeps squares out of the subnormal range)
+            constexpr bool kClamp16Static = !kAbsmax && L <= 13;
+            constexpr bool kClamp16Dyn = !kAbsmax && L >= 14 && !GAIN;
             constexpr uint32_t kLo2 = kPackNibbles ? 0x00000000u : 0xFFF8FFF8u;
             constexpr uint32_t kHi2 = kPackNibbles ? 0x000F000Fu : 0x00070007u;
             constexpr int RL = 1 << RUN;                                 // elements per run
@@ -616,6 +632,9 @@ __global__ void __launch_bounds__(Ext::template threads<L>(), Ext::template min_
             const bool row_ok = row < p.M;
             uint8_t* crow = (Ext::kOn ? Ext::codes() : p.codes) +
                             row0 * (int64_t)(kPackNibbles ? K / 2 : K);
+            // codes of the thread's runs, stored; returns the sum of its codes
+            auto quant_runs = [&](auto c16) -> int {
+            constexpr bool kClamp16 = decltype(c16)::value;
             uint32_t qsum = 0;
             static_for<0, R / RL>([&](auto mm) {
                 constexpr int m = decltype(mm)::value;
@@ -718,9 +737,19 @@ __global__ void __launch_bounds__(Ext::template threads<L>(), Ext::template min_
             });
             // sum of codes: packed nibbles added kMagicBits + q per code (mod 2^32),
             // or q + 8 per code on the int16 path; one-byte codes were summed directly
-            int qs = !kPackNibbles ? (int)qsum
-                     : kClamp16    ? (int)qsum - 8 * R
-                                   : (int)(qsum - (uint32_t)R * (uint32_t)kMagicBits);
+            return !kPackNibbles ? (int)qsum
+                   : kClamp16    ? (int)qsum - 8 * R
+                                 : (int)(qsum - (uint32_t)R * (uint32_t)kMagicBits);
+            };
+            int qs;
+            if constexpr (kClamp16Dyn) {
+                if (ss_ok && den > p.thr16)  // uniform over the row
+                    qs = quant_runs(ic_bool<true>{});
+                else
+                    qs = quant_runs(ic_bool<false>{});
+            } else {
+                qs = quant_runs(ic_bool<kClamp16Static>{});
+            }
             qs = row_isum(qs);
 
             if (row_ok) {

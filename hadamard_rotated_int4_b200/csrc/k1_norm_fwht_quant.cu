@@ -64,6 +64,7 @@ hbl_status launch_norm_fwht_quant(const uint16_t* X, const float* gain, int64_t 
     prm.quant_eps = quant_eps;
     prm.cK = (float)(1.0 / sqrt((double)K));
     prm.s7 = (float)sqrt(7.0);
+    prm.thr16 = k1::thr16_for(K);
     prm.codes = static_cast<uint8_t*>(codes);
     prm.scales = scales;
     prm.rowsum = rowsum;

@@ -268,6 +268,7 @@ hbl_status launch(const DecodeArgs& d, cudaStream_t stream, int num_sms) {
     p.quant_eps = d.quant_eps;
     p.cK = (float)(1.0 / sqrt((double)(1 << L)));
     p.s7 = (float)sqrt(7.0);
+    p.thr16 = k1::thr16_for(1 << L);
     p.W = d.W_packed;
     p.alpha = d.alpha;
     p.Y = d.Y;

@@ -110,6 +110,52 @@ def test_quant_edge_rows(bits):
     check_quant(X, bits)
 
 
+def hadamard_row_bits(K, k, scale=1.0):
+    # bf16 bits of scale * (row k of the Sylvester Hadamard matrix): its
+    # transform is a single spike of height scale * sqrt(K)
+    i = np.arange(K)
+    par = np.array([bin(int(k) & int(t)).count("1") & 1 for t in i])
+    v = np.where(par == 1, -scale, scale).astype(np.float32)
+    return (v.view(np.uint32) >> 16).astype(np.uint16)
+
+
+@pytest.mark.parametrize("K", [16384, 32768])
+def test_quant_int4_large_k_spiky_rows(K):
+    # INT4 codes at K >= 16384 are clamped as int16 pairs on rows whose
+    # statistic bounds |q| below 2^15, else on 32-bit patterns: spike rows
+    # (|q| would reach sqrt7 K), near-spikes on both sides of the bound,
+    # normal rows; packed nibbles, one byte per code, interleaved bytes
+    rng = np.random.default_rng(K)
+    X = acts(8, K, seed=3)
+    X[0] = hadamard_row_bits(K, 5)
+    X[1] = hadamard_row_bits(K, 77, scale=-3.0)
+    h = (hadamard_row_bits(K, 9).astype(np.uint32) << 16).view(np.float32)
+    for r, eps in ((2, 0.02), (3, 0.1), (4, 0.5)):
+        v = (h + eps * rng.standard_normal(K)).astype(np.float32)
+        X[r] = (v.view(np.uint32) >> 16).astype(np.uint16)
+    X[5] = 0
+    wc, ws, wr = oracle.norm_fwht_quant(X, 4)
+    want_q = oracle.decode_codes(wc, K, 4)
+    for bits in (4, hbl.ACT_INT4_BYTES, hbl.ACT_INT4_I32):
+        codes, scales, rowsum = hbl.norm_fwht_quant(to_dev_bf16(X), bits)
+        assert np.array_equal(scales.cpu().numpy().view(np.uint32), ws.view(np.uint32))
+        assert np.array_equal(rowsum.cpu().numpy()[:8], wr)
+        got = codes.cpu().numpy()
+        if bits == 4:
+            assert np.array_equal(got, wc)
+        elif bits == hbl.ACT_INT4_BYTES:
+            assert np.array_equal(got.view(np.int8).astype(np.int32), want_q)
+        else:
+            assert np.array_equal(il_decode(got, 8, K).astype(np.int32), want_q)
+    # the same rows through the one-kernel decode forward (one token)
+    if K == 16384:
+        W = inputs.latent_weights(512, K, seed=1)
+        packed, alpha = oracle.pack_ternary(W)
+        for r in range(6):
+            assert np.array_equal(forward(X[r:r + 1], packed, alpha, 4),
+                                  oracle.hbitlinear_forward(X[r:r + 1], packed, alpha, 4))
+
+
 def test_quant_workloads_full_size():
     # quant workload (8192 x 4096, Student-t, 1% channels x 20), both widths
     X = inputs.activations("quant")
