@@ -69,6 +69,21 @@ def peaks():
             "source": "fallback"}
 
 
+SM_MAX_MHZ = 1965.0  # B200 clocks.max.sm
+
+
+def fp32_view(elements, L, t, sms, clock_mhz):
+    """K1 against the FP32 lanes instead of HBM: per element L butterfly
+    add/subs, the square and its tree add, the products by 1/rms and 1/sqrt(K),
+    the |v| (or max) tree step and the quantising FMA = L + 6 operations; peak =
+    SMs x 128 FP32 lanes x the maximum SM clock."""
+    ops = float(elements) * (L + 6)
+    peak = sms * 128 * clock_mhz * 1e6 / 1e12
+    ach = ops / t / 1e12
+    return {"bound": "alu", "unit": "Tops/s (fp32)", "ops": ops, "achieved": ach, "peak": peak,
+            "frac": ach / peak, "peak_note": "%d SMs x 128 fp32 lanes x %.0f MHz" % (sms, clock_mhz)}
+
+
 class ClockSampler:
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -253,6 +268,7 @@ def run_hbl(args):
         torch.cuda.synchronize()
 
     pk = peaks()
+    n_sms = torch.cuda.get_device_properties(dev).multi_processor_count
     # ---- inputs: each rank its own 8192-token batch; the same weights everywhere
     X_bits = inputs.activations("ffn_wdown", seed=rank)
     W = inputs.weights("ffn_wdown")
@@ -335,7 +351,8 @@ def run_hbl(args):
         gbs = nbytes / t / 1e9
         quant["a%d" % bits] = {"workload": "quant 8192 x 4096 Student-t nu=3, 1% channels x20",
                                "us": t * 1e6, "bytes": nbytes, "achieved_gbs": gbs,
-                               "frac": gbs / pk["hbm_gbs"]}
+                               "frac": gbs / pk["hbm_gbs"],
+                               "alu_view": fp32_view(QM * QK, 12, t, n_sms, SM_MAX_MHZ)}
     del qX
 
     # ---- decode-batch sweep: T tokens through the whole layer, Wo 4096x4096 and
@@ -500,6 +517,11 @@ def run_hbl(args):
         "roofline": roof,
         "kernels_us": {"norm_fwht_quant": t_k1 * 1e6, "expand_ternary": t_kx * 1e6,
                        "gemm_tma": t_k2 * 1e6},
+        "norm_fwht_quant_views": {
+            "hbm": {"bytes": M_TOK * K_IN * 3 + 8 * M_TOK,
+                    "achieved_gbs": (M_TOK * K_IN * 3 + 8 * M_TOK) / t_k1 / 1e9,
+                    "frac": (M_TOK * K_IN * 3 + 8 * M_TOK) / t_k1 / 1e9 / pk["hbm_gbs"]},
+            "alu": fp32_view(M_TOK * K_IN, 14, t_k1, n_sms, SM_MAX_MHZ)},
         "quant": quant,
         "decode": decode,
         "others": others,
