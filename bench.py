@@ -401,6 +401,9 @@ def run_hbl(args):
                            "frac_hbm_on_packed_w": wbytes / t / 1e9 / pk["hbm_gbs"],
                            "path": ("one kernel (quantiser in every CTA, weights by bulk copy)"
                                     if T <= 16384 // Kd
+                                    else "K1 + GEMV half of the one-kernel forward (weights "
+                                         "bulk-copied under K1)"
+                                    if Kd == 16384 and T <= 4
                                     else "row GEMV (weight rows per warp, PDL after K1)"
                                     if T <= (4 if Kd >= 16384 else 8)
                                     else "gemm_ts (TMEM activations, one-wave split-K)"),

@@ -371,6 +371,17 @@ static hbl_status forward_impl(const uint16_t* X, const float* gain, int M, int 
     int32_t* rowsum = reinterpret_cast<int32_t*>(ws + cb + sb);
     uint8_t* gws = ws + cb + 2 * sb;
     const size_t gws_bytes = ws_bytes - (cb + 2 * sb);
+    // Other decode batches of up to 4 tokens at K = 16384: K1 (one byte per
+    // code, row-major), then the one-kernel forward's GEMV half, its weight
+    // rows streaming into shared memory under K1.
+    if (g_path.load() == 0 && decode_gemv_supported(M, K, N, sms)) {
+        hbl_status st = launch_norm_fwht_quant(X, gain, M, K, norm_eps, quant_eps,
+                                               act_bits == 4 ? 6 : 8, codes, scales, rowsum,
+                                               nullptr, s, sms, variant);
+        if (st != HBL_OK) return st;
+        GemvArgs g{codes, scales, rowsum, M, K, N, W_packed, alpha, Y, dev_status};
+        return launch_decode_gemv(g, s, sms);
+    }
     const FwdPlan f = forward_plan(M, K, act_bits);
     hbl_status st = launch_norm_fwht_quant(X, gain, M, K, norm_eps, quant_eps, f.k1_mode, codes,
                                            scales, rowsum, nullptr, s, sms, variant);

@@ -58,6 +58,23 @@ struct DecodeArgs {
 };
 // Weight rows per CTA for N rows: spread evenly over at most num_sms CTAs.
 int decode_fused_rows(int N, int num_sms);
+
+// K6's GEMV half alone, after K1 (programmatic dependent launch; the weight
+// rows stream into shared memory under K1): codes one byte each, row-major
+// [M][K]; M <= 4 at K = 16384, when the CTA's weight rows fit its shared
+// memory (decode_gemv_supported).
+struct GemvArgs {
+    const uint8_t* codes;
+    const float* scales;
+    const int32_t* rowsum;
+    int M, K, N;
+    const uint32_t* W_packed;
+    const float* alpha;
+    uint16_t* Y;
+    int32_t* status;
+};
+bool decode_gemv_supported(int M, int K, int N, int num_sms);
+hbl_status launch_decode_gemv(const GemvArgs& g, cudaStream_t stream, int num_sms);
 bool decode_fused_supported(int M, int K, int N, int act_bits, unsigned variant, int num_sms);
 hbl_status launch_decode_fused(const DecodeArgs& d, cudaStream_t stream, int num_sms);
 

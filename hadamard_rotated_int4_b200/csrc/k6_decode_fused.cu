@@ -1,5 +1,6 @@
-// k6_decode_fused.cu -- host entry of the fused decode forward (the kernel is
-// in k6_decode_fused.cuh, instantiated per K in k6_decode_l*.cu).
+// k6_decode_fused.cu -- host entries of the decode kernels: the one-kernel
+// forward and its GEMV half (the kernels are in k6_decode_fused.cuh,
+// instantiated per K in k6_decode_l*.cu).
 #include <cuda_runtime.h>
 
 #include "hbl_internal.cuh"
@@ -13,6 +14,8 @@ hbl_status launch_l14(const DecodeArgs& d, cudaStream_t s, int sms);
 int smem_l12(int N, int MT, int sms);
 int smem_l13(int N, int MT, int sms);
 int smem_l14(int N, int MT, int sms);
+hbl_status launch_gemv_l14(const GemvArgs& g, cudaStream_t s, int sms);
+int gemv_smem_l14(int N, int MT, int sms);
 }  // namespace k6
 
 int decode_fused_rows(int N, int num_sms) {
@@ -43,6 +46,29 @@ bool decode_fused_supported(int M, int K, int N, int act_bits, unsigned variant,
         default: return false;
     }
     return bytes <= optin;
+}
+
+static int optin_smem() {
+    int dev = 0, optin = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
+            cudaSuccess)
+        return 0;
+    return optin;
+}
+
+// Used at K = 16384 only: at smaller K a lane's slice of a row is short, the
+// shuffle reductions outweigh the dp4a work, and K1 + the row GEMV is faster
+// (K = 8192, 4 tokens: 12.8 vs 10.4 us).
+bool decode_gemv_supported(int M, int K, int N, int num_sms) {
+    if (M < 1 || M > 4 || N < 1 || K != 16384) return false;
+    return k6::gemv_smem_l14(N, token_capacity(M), num_sms) <= optin_smem();
+}
+
+hbl_status launch_decode_gemv(const GemvArgs& g, cudaStream_t stream, int num_sms) {
+    if (g.M == 0) return HBL_OK;
+    if (g.K != 16384) return HBL_ERR_SHAPE;
+    return k6::launch_gemv_l14(g, stream, num_sms);
 }
 
 hbl_status launch_decode_fused(const DecodeArgs& d, cudaStream_t stream, int num_sms) {

@@ -46,10 +46,11 @@ constexpr uint32_t kCopyChunk = 32768;  // bytes per bulk copy
 
 __host__ __device__ constexpr int up128(int x) { return (x + 127) & ~127; }
 
-// Launch shape for K = 2^L and token capacity MT: GPC K1 row groups of T
-// threads (64 values each); the GEMV phase's warps cover KSEG elements of a
-// row, KSPLIT of them per row, RG row groups.
-template <int L, int MT>
+// Launch shape for K = 2^L and token capacity MT.  Q: the quantiser runs in
+// the kernel (GPC K1 row groups of T threads, 64 values each); otherwise the
+// codes come from global memory.  The GEMV phase's warps cover KSEG elements
+// of a row, KSPLIT warps per row, RG row groups.
+template <int L, int MT, bool Q = true>
 struct Shape {
     static constexpr int NT = 256;
     static constexpr int NW = NT / 32;
@@ -57,14 +58,18 @@ struct Shape {
     static constexpr int T = 1 << (L - RLOG);
     static constexpr int GPC = MT < NT / T ? MT : NT / T;
     using C = k1::Cfg<L, RLOG>;
-    static constexpr int WPL = 8 / MT;  // packed words per lane per row
+    // packed words per lane per row: 8 / MT (32 code registers), at least
+    // enough for NW warps to cover a row
+    static constexpr int WPL = (8 / MT) > ((1 << L) / (512 * NW)) ? (8 / MT)
+                                                                  : ((1 << L) / (512 * NW));
     static constexpr int KSEG = 512 * WPL;
     static constexpr int KSPLIT = (1 << L) / KSEG;
     static constexpr int RG = NW / KSPLIT;
-    // shared memory: K1 row buffers, codes [MT][K], scales [4] + rowsum [4],
-    // mbarrier + flag, partial sums [rows][KSPLIT][MT], packed weight rows
-    static constexpr int kCodes = up128(GPC * (C::kBufBytes + k1::kRedFloats * 4));
-    static constexpr int kScales = kCodes + MT * (1 << L);
+    // shared memory: [K1 row buffers, codes [MT][K]] (Q only), scales [4] +
+    // rowsum [4], mbarrier + flag, partial sums [rows][KSPLIT][MT], packed
+    // weight rows
+    static constexpr int kCodes = Q ? up128(GPC * (C::kBufBytes + k1::kRedFloats * 4)) : 0;
+    static constexpr int kScales = kCodes + (Q ? MT * (1 << L) : 0);
     static constexpr int kRowsum = kScales + 16;
     static constexpr int kBar = kScales + 32;
     static constexpr int kPart = kBar + 16;
@@ -74,8 +79,9 @@ struct Shape {
     __host__ __device__ static constexpr int total(int rows) {
         return weights(rows) + rows * ((1 << L) / 4);
     }
-    static_assert(C::T == T && C::kRowsPerGroup == 1 && GPC * T <= NT, "K1 grouping");
+    static_assert(!Q || (C::T == T && C::kRowsPerGroup == 1 && GPC * T <= NT), "K1 grouping");
     static_assert(KSPLIT >= 1 && KSPLIT <= NW && NW % KSPLIT == 0, "GEMV split");
+    static_assert(WPL == 2 || WPL == 4 || WPL == 8, "lane words");
 };
 
 __device__ __forceinline__ int dp4a_su(uint32_t a, uint32_t b, int c) {
@@ -98,6 +104,146 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
         : "memory");
 }
 
+__device__ __forceinline__ uint8_t* dyn_smem() {
+    extern __shared__ __align__(128) uint8_t dyn[];
+    return dyn;
+}
+
+// CTA blockIdx.x's weight rows [n0, n0 + rows): at most p.rows, fewer in the last CTA.
+__device__ __forceinline__ int cta_rows(const k1::Params& p) {
+    return min(p.rows, p.N - (int)blockIdx.x * p.rows);  // >= 1 by the grid size
+}
+
+// Thread 0: the mbarrier the weights complete on.
+template <class S>
+__device__ __forceinline__ void init_weight_barrier(uint8_t* sm) {
+    mbar_init_count(smem_addr(sm + S::kBar), 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+// Thread 0: bulk copies of the CTA's packed weight rows into shared memory.
+template <class S, int L>
+__device__ __forceinline__ void issue_weights(const k1::Params& p, uint8_t* sm) {
+    constexpr int K = 1 << L;
+    const uint32_t bar = smem_addr(sm + S::kBar);
+    const uint32_t bytes = (uint32_t)cta_rows(p) * (K / 4);
+    mbar_expect_tx(bar, bytes);
+    const uint8_t* src =
+        reinterpret_cast<const uint8_t*>(p.W + (int64_t)blockIdx.x * p.rows * (K / 16));
+    const uint32_t dst = smem_addr(sm + S::weights(p.rows));
+    for (uint32_t off = 0; off < bytes; off += kCopyChunk)
+        bulk_load(dst + off, src + off, min(kCopyChunk, bytes - off), bar);
+}
+
+// The GEMV over the CTA's weight rows (in shared memory once the mbarrier
+// completes) and the dequantising epilogue.  codes: one byte per code,
+// row-major [M][K] (shared or global memory); sc / rs: scales and row sums.
+template <class S, int L, int MT>
+__device__ __forceinline__ void gemv_phase(const k1::Params& p, uint8_t* sm,
+                                           const uint8_t* codes, const float* sc,
+                                           const int32_t* rs) {
+    constexpr int K = 1 << L;
+    constexpr int NT = S::NT, WPL = S::WPL, KSEG = S::KSEG, KSPLIT = S::KSPLIT, RG = S::RG;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int n0 = blockIdx.x * p.rows;
+    const int rows = cta_rows(p);
+    const int M = (int)p.M;
+    volatile int* flag = reinterpret_cast<volatile int*>(sm + S::kBar + 8);
+
+    // warp = (row group, K segment); lane word j covers elements e(j) .. +15
+    // of the segment: 16-byte chunks lane + 32 i (WPL >= 4) or the 8-byte
+    // piece `lane` (WPL = 2), so the shared-memory reads of a warp are
+    // consecutive
+    const int seg = warp % KSPLIT, rgp = warp / KSPLIT;
+    auto elem = [&](int j) -> int {
+        return WPL >= 4 ? seg * KSEG + 64 * (lane + 32 * (j / 4)) + 16 * (j % 4)
+                        : seg * KSEG + 32 * lane + 16 * j;
+    };
+    uint32_t a[MT][4 * WPL];
+#pragma unroll
+    for (int m = 0; m < MT; ++m)
+#pragma unroll
+        for (int j = 0; j < WPL; ++j) {
+            const uint4 v = *reinterpret_cast<const uint4*>(codes + m * K + elem(j));
+            a[m][4 * j] = v.x;
+            a[m][4 * j + 1] = v.y;
+            a[m][4 * j + 2] = v.z;
+            a[m][4 * j + 3] = v.w;
+        }
+    if (tid == 0)
+        *flag = mbar_wait_bounded<false>(smem_addr(sm + S::kBar), 0, kTimeoutNs) ? 1 : 0;
+    __syncthreads();
+    if (*flag == 0) {
+        if (tid == 0) report_status(p.status, HBL_ERR_TIMEOUT);
+        return;
+    }
+    const uint8_t* wsm = sm + S::weights(p.rows);
+    int32_t* part = reinterpret_cast<int32_t*>(sm + S::kPart);
+    // two rows of the row group per step (independent chains overlap)
+    for (int r0 = rgp; r0 < rows; r0 += 2 * RG) {
+        uint32_t wd[2][WPL];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int r = r0 + u * RG;
+            const uint8_t* wr = wsm + (r < rows ? r : r0) * (K / 4);
+#pragma unroll
+            for (int j = 0; j < WPL; j += (WPL >= 4 ? 4 : 2)) {
+                if constexpr (WPL >= 4) {
+                    const uint4 t = *reinterpret_cast<const uint4*>(wr + elem(j) / 4);
+                    wd[u][j] = t.x, wd[u][j + 1] = t.y, wd[u][j + 2] = t.z, wd[u][j + 3] = t.w;
+                } else {
+                    const uint2 t = *reinterpret_cast<const uint2*>(wr + elem(j) / 4);
+                    wd[u][j] = t.x, wd[u][j + 1] = t.y;
+                }
+            }
+        }
+        int v[2][MT];
+#pragma unroll
+        for (int u = 0; u < 2; ++u)
+#pragma unroll
+            for (int m = 0; m < MT; ++m) {
+                int s0 = 0, s1 = 0, s2 = 0, s3 = 0;
+#pragma unroll
+                for (int j = 0; j < WPL; ++j) {
+                    s0 = dp4a_su(a[m][4 * j + 0], wd[u][j] & 0x03030303u, s0);
+                    s1 = dp4a_su(a[m][4 * j + 1], wd[u][j] & 0x0C0C0C0Cu, s1);
+                    s2 = dp4a_su(a[m][4 * j + 2], wd[u][j] & 0x30303030u, s2);
+                    s3 = dp4a_su(a[m][4 * j + 3], wd[u][j] & 0xC0C0C0C0u, s3);
+                }
+                v[u][m] = s0 + (s1 >> 2) + (s2 >> 4) + (s3 >> 6);
+            }
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1)
+#pragma unroll
+            for (int u = 0; u < 2; ++u)
+#pragma unroll
+                for (int m = 0; m < MT; ++m) v[u][m] += __shfl_xor_sync(0xffffffffu, v[u][m], o);
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int r = r0 + u * RG;
+            if (lane < MT && r < rows) {
+                int x = v[u][0];
+#pragma unroll
+                for (int m = 1; m < MT; ++m) x = lane == m ? v[u][m] : x;
+                part[(r * KSPLIT + seg) * MT + lane] = x;
+            }
+        }
+    }
+    __syncthreads();
+
+    // sum over the K segments, dequantise, store
+    const float al = *p.alpha;
+    for (int vi = tid; vi < rows * MT; vi += NT) {
+        const int m = vi % MT, r = vi / MT;
+        if (m >= M) continue;
+        int s = -rs[m];
+#pragma unroll
+        for (int g = 0; g < KSPLIT; ++g) s += part[(r * KSPLIT + g) * MT + m];
+        const float y = __fmul_rn((float)s, __fmul_rn(al, sc[m]));
+        p.Y[(int64_t)m * p.N + n0 + r] = __bfloat16_as_ushort(__float2bfloat16_rn(y));
+    }
+}
+
 // The one-kernel decode forward as an extension of K1's kernel template.
 template <int L, int MT>
 struct DecodeExt {
@@ -112,151 +258,43 @@ struct DecodeExt {
     template <int>
     __host__ __device__ static constexpr int groups() { return S::GPC; }
 
-    static __device__ uint8_t* smem() {
-        extern __shared__ __align__(128) uint8_t dyn[];
-        return dyn;
-    }
-    static __device__ uint8_t* codes() { return smem() + S::kCodes; }
-    static __device__ float* scales() { return reinterpret_cast<float*>(smem() + S::kScales); }
+    static __device__ uint8_t* codes() { return dyn_smem() + S::kCodes; }
+    static __device__ float* scales() { return reinterpret_cast<float*>(dyn_smem() + S::kScales); }
     static __device__ int32_t* rowsum() {
-        return reinterpret_cast<int32_t*>(smem() + S::kRowsum);
+        return reinterpret_cast<int32_t*>(dyn_smem() + S::kRowsum);
     }
-    static __device__ int nrows(const k1::Params& p) {
-        return min(p.rows, p.N - (int)blockIdx.x * p.rows);  // >= 1 by the grid size
-    }
-
     // 1a. token rows into L2 ahead of the weight traffic; the weights' mbarrier
     static __device__ void prologue(const k1::Params& p) {
         if (threadIdx.x == 0) {
             prefetch_l2_bulk(p.X, (uint32_t)(p.M * (1 << L) * 2));
-            mbar_init_count(smem_addr(smem() + S::kBar), 1);
-            asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+            init_weight_barrier<S>(dyn_smem());
         }
     }
     // 1b. (thread 0, first row staged) the CTA's packed weight rows -> shared memory
-    static __device__ void staged(const k1::Params& p) {
-        constexpr int K = 1 << L;
-        const uint32_t bar = smem_addr(smem() + S::kBar);
-        const uint32_t bytes = (uint32_t)nrows(p) * (K / 4);
-        mbar_expect_tx(bar, bytes);
-        const uint8_t* src =
-            reinterpret_cast<const uint8_t*>(p.W + (int64_t)blockIdx.x * p.rows * (K / 16));
-        const uint32_t dst = smem_addr(smem() + S::weights(p.rows));
-        for (uint32_t off = 0; off < bytes; off += kCopyChunk)
-            bulk_load(dst + off, src + off, min(kCopyChunk, bytes - off), bar);
-    }
-
+    static __device__ void staged(const k1::Params& p) { issue_weights<S, L>(p, dyn_smem()); }
     // 3-4. after the rows: the GEMV over this CTA's weight rows and the epilogue
     static __device__ void finish(const k1::Params& p) {
-        constexpr int K = 1 << L;
-        constexpr int NT = S::NT, WPL = S::WPL, KSEG = S::KSEG, KSPLIT = S::KSPLIT, RG = S::RG;
-        uint8_t* sm = smem();
-        const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-        const int n0 = blockIdx.x * p.rows;
-        const int rows = nrows(p);
-        const int M = (int)p.M;
-        volatile int* flag = reinterpret_cast<volatile int*>(sm + S::kBar + 8);
         __syncthreads();  // codes, scales, row sums complete
-        if (tid == 0)
-            *flag = mbar_wait_bounded<false>(smem_addr(sm + S::kBar), 0, kTimeoutNs) ? 1 : 0;
-        __syncthreads();
-        if (*flag == 0) {
-            if (tid == 0) report_status(p.status, HBL_ERR_TIMEOUT);
-            return;
-        }
-
-        // warp = (row group, K segment); lane word j covers elements e(j) .. +15
-        // of the segment: 16-byte chunks lane + 32 i (WPL >= 4) or the 8-byte
-        // piece `lane` (WPL = 2), so the shared-memory reads of a warp are
-        // consecutive
-        const int seg = warp % KSPLIT, rgp = warp / KSPLIT;
-        auto elem = [&](int j) -> int {
-            return WPL >= 4 ? seg * KSEG + 64 * (lane + 32 * (j / 4)) + 16 * (j % 4)
-                            : seg * KSEG + 32 * lane + 16 * j;
-        };
-        uint32_t a[MT][4 * WPL];
-#pragma unroll
-        for (int m = 0; m < MT; ++m)
-#pragma unroll
-            for (int j = 0; j < WPL; ++j) {
-                const uint4 v =
-                    *reinterpret_cast<const uint4*>(sm + S::kCodes + m * K + elem(j));
-                a[m][4 * j] = v.x;
-                a[m][4 * j + 1] = v.y;
-                a[m][4 * j + 2] = v.z;
-                a[m][4 * j + 3] = v.w;
-            }
-        const uint8_t* wsm = sm + S::weights(p.rows);
-        int32_t* part = reinterpret_cast<int32_t*>(sm + S::kPart);
-        // two rows of the row group per step (independent chains overlap)
-        for (int r0 = rgp; r0 < rows; r0 += 2 * RG) {
-            uint32_t wd[2][WPL];
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                const int r = r0 + u * RG;
-                const uint8_t* wr = wsm + (r < rows ? r : r0) * (K / 4);
-#pragma unroll
-                for (int j = 0; j < WPL; j += (WPL >= 4 ? 4 : 2)) {
-                    if constexpr (WPL >= 4) {
-                        const uint4 t = *reinterpret_cast<const uint4*>(wr + elem(j) / 4);
-                        wd[u][j] = t.x, wd[u][j + 1] = t.y, wd[u][j + 2] = t.z,
-                        wd[u][j + 3] = t.w;
-                    } else {
-                        const uint2 t = *reinterpret_cast<const uint2*>(wr + elem(j) / 4);
-                        wd[u][j] = t.x, wd[u][j + 1] = t.y;
-                    }
-                }
-            }
-            int v[2][MT];
-#pragma unroll
-            for (int u = 0; u < 2; ++u)
-#pragma unroll
-                for (int m = 0; m < MT; ++m) {
-                    int s0 = 0, s1 = 0, s2 = 0, s3 = 0;
-#pragma unroll
-                    for (int j = 0; j < WPL; ++j) {
-                        s0 = dp4a_su(a[m][4 * j + 0], wd[u][j] & 0x03030303u, s0);
-                        s1 = dp4a_su(a[m][4 * j + 1], wd[u][j] & 0x0C0C0C0Cu, s1);
-                        s2 = dp4a_su(a[m][4 * j + 2], wd[u][j] & 0x30303030u, s2);
-                        s3 = dp4a_su(a[m][4 * j + 3], wd[u][j] & 0xC0C0C0C0u, s3);
-                    }
-                    v[u][m] = s0 + (s1 >> 2) + (s2 >> 4) + (s3 >> 6);
-                }
-#pragma unroll
-            for (int o = 16; o >= 1; o >>= 1)
-#pragma unroll
-                for (int u = 0; u < 2; ++u)
-#pragma unroll
-                    for (int m = 0; m < MT; ++m)
-                        v[u][m] += __shfl_xor_sync(0xffffffffu, v[u][m], o);
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                const int r = r0 + u * RG;
-                if (lane < MT && r < rows) {
-                    int x = v[u][0];
-#pragma unroll
-                    for (int m = 1; m < MT; ++m) x = lane == m ? v[u][m] : x;
-                    part[(r * KSPLIT + seg) * MT + lane] = x;
-                }
-            }
-        }
-        __syncthreads();
-
-        // sum over the K segments, dequantise, store
-        const float al = *p.alpha;
-        const float* sc = scales();
-        const int32_t* rs = rowsum();
-        for (int vi = tid; vi < rows * MT; vi += NT) {
-            const int m = vi % MT, r = vi / MT;
-            if (m >= M) continue;
-            int s = -rs[m];
-#pragma unroll
-            for (int g = 0; g < KSPLIT; ++g) s += part[(r * KSPLIT + g) * MT + m];
-            const float y = __fmul_rn((float)s, __fmul_rn(al, sc[m]));
-            p.Y[(int64_t)m * p.N + n0 + r] = __bfloat16_as_ushort(__float2bfloat16_rn(y));
-        }
+        gemv_phase<S, L, MT>(p, dyn_smem(), codes(), scales(), rowsum());
     }
 };
+
+// The GEMV half alone, for decode batches K6 does not take (M <= 4): launched
+// as a programmatic dependent of K1, it starts its weight rows' bulk copies
+// before the dependency wait (the weights are not K1's output), then reads
+// K1's codes (one byte each, row-major), scales and row sums from global
+// memory.
+template <int L, int MT>
+__global__ void __launch_bounds__(256, 1) decode_gemv_kernel(const __grid_constant__ k1::Params p) {
+    using S = Shape<L, MT, false>;
+    uint8_t* sm = dyn_smem();
+    if (threadIdx.x == 0) {
+        init_weight_barrier<S>(sm);
+        issue_weights<S, L>(p, sm);
+    }
+    pdl_wait();
+    gemv_phase<S, L, MT>(p, sm, p.codes, p.scales, p.rowsum);
+}
 
 template <int L, int MT, int MODE, int FL>
 hbl_status launch(const DecodeArgs& d, cudaStream_t stream, int num_sms) {
@@ -285,6 +323,41 @@ hbl_status launch(const DecodeArgs& d, cudaStream_t stream, int num_sms) {
 
 // Token capacities: up to 2^(14 - L) (one K1 row group per token): 1, 2, 4
 // at K = 4096, 1, 2 at K = 8192, 1 at K = 16384.
+template <int L, int MT>
+hbl_status launch_gemv(const GemvArgs& g, cudaStream_t stream, int num_sms) {
+    k1::Params p = {};
+    p.M = g.M;
+    p.codes = const_cast<uint8_t*>(g.codes);
+    p.scales = const_cast<float*>(g.scales);
+    p.rowsum = const_cast<int32_t*>(g.rowsum);
+    p.W = g.W_packed;
+    p.alpha = g.alpha;
+    p.Y = g.Y;
+    p.status = g.status;
+    p.N = g.N;
+    p.rows = decode_fused_rows(g.N, num_sms);
+    const int smem = Shape<L, MT, false>::total(p.rows);
+    auto kern = decode_gemv_kernel<L, MT>;
+    if (!smem_attr_once(reinterpret_cast<const void*>(kern), smem)) return HBL_ERR_CUDA;
+    const unsigned grid = (unsigned)((g.N + p.rows - 1) / p.rows);
+    return launch_pdl(kern, dim3(grid), dim3(256), (size_t)smem, stream, p);
+}
+
+template <int L>
+int gemv_smem_bytes(int N, int MT, int num_sms) {
+    const int rows = decode_fused_rows(N, num_sms);
+    if (MT == 1) return Shape<L, 1, false>::total(rows);
+    if (MT == 2) return Shape<L, 2, false>::total(rows);
+    return Shape<L, 4, false>::total(rows);
+}
+
+template <int L>
+hbl_status launch_gemv_l(const GemvArgs& g, cudaStream_t s, int sms) {
+    if (g.M <= 1) return launch_gemv<L, 1>(g, s, sms);
+    if (g.M <= 2) return launch_gemv<L, 2>(g, s, sms);
+    return launch_gemv<L, 4>(g, s, sms);
+}
+
 template <int L>
 int smem_bytes(int N, int MT, int num_sms) {
     const int rows = decode_fused_rows(N, num_sms);

@@ -1,4 +1,4 @@
-// k6_decode_l12.cu -- instantiations of the fused decode forward for K = 2^12.
+// k6_decode_l12.cu -- instantiations of the one-kernel decode forward for K = 2^12.
 #include "k6_decode_fused.cuh"
 
 namespace hbl {

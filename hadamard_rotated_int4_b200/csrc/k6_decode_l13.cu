@@ -1,4 +1,4 @@
-// k6_decode_l13.cu -- instantiations of the fused decode forward for K = 2^13.
+// k6_decode_l13.cu -- instantiations of the one-kernel decode forward for K = 2^13.
 #include "k6_decode_fused.cuh"
 
 namespace hbl {

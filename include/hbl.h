@@ -177,7 +177,10 @@ HBL_API hbl_status hbl_ternary_gemm(const void* codes, const float* scales, cons
  * Decode batches (M <= 16384 / K tokens at K = 4096 / 8192 / 16384, while the
  * packed weight rows of one SM's share fit its shared memory, GEMM path 0) run
  * both steps in one kernel instead: every CTA quantises the M rows itself
- * while its weight rows stream in; the results are the same values.
+ * while its weight rows stream in; up to 4 tokens at K = 16384 run
+ * hbl_norm_fwht_quant followed by that kernel's GEMV half, whose weight rows
+ * stream into shared memory during the quantiser.  The results are the same
+ * values on every path.
  * X: bf16 [M x K]; Y: bf16 [M x N] out; other arguments as above.
  * ws: >= hbl_workspace_size(HBL_OP_HBITLINEAR_FORWARD, M, K, N, act_bits). */
 HBL_API hbl_status hbl_hbitlinear_forward(const uint16_t* X, const float* gain, int M, int K, int N,
