@@ -230,7 +230,10 @@ def run_reference(args):
         "ms_per_step": 1e3 * dt / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "s8", "data": "synthetic",
         "config": {"workload": WORKLOAD, "M": M_TOK, "K": K_IN, "N": N_OUT, "act_bits": BITS,
-                   "parallelism": "replicas by token rows (no collective)"},
+                   "global_batch": args.gpus * M_TOK,
+                   "parallelism": "replicas by token rows (no collective)" if args.gpus > 1
+                   else "single GPU",
+                   "l2": "inputs larger than L2 (X 268 MB per step)"},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": used, "kind": "oracle",
                          "sample": "each step: %d token rows of the ffn_wdown workload (full K "
                                    "and N), scalar C oracle over %d threads" % (rows_per_step,
