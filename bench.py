@@ -406,7 +406,7 @@ def run_hbl(args):
                                     if T <= 16384 // Kd
                                     else "K1 + GEMV half of the one-kernel forward (weights "
                                          "bulk-copied under K1)"
-                                    if Kd == 16384 and T <= 4
+                                    if Kd == 16384 and T <= 8
                                     else "row GEMV (weight rows per warp, PDL after K1)"
                                     if T <= (4 if Kd >= 16384 else 8)
                                     else "gemm_ts (TMEM activations, one-wave split-K)"),

@@ -371,7 +371,7 @@ static hbl_status forward_impl(const uint16_t* X, const float* gain, int M, int 
     int32_t* rowsum = reinterpret_cast<int32_t*>(ws + cb + sb);
     uint8_t* gws = ws + cb + 2 * sb;
     const size_t gws_bytes = ws_bytes - (cb + 2 * sb);
-    // Other decode batches of up to 4 tokens at K = 16384: K1 (one byte per
+    // Other decode batches of up to 8 tokens at K = 16384: K1 (one byte per
     // code, row-major), then the one-kernel forward's GEMV half, its weight
     // rows streaming into shared memory under K1.
     if (g_path.load() == 0 && decode_gemv_supported(M, K, N, sms)) {

@@ -61,7 +61,7 @@ int decode_fused_rows(int N, int num_sms);
 
 // K6's GEMV half alone, after K1 (programmatic dependent launch; the weight
 // rows stream into shared memory under K1): codes one byte each, row-major
-// [M][K]; M <= 4 at K = 16384, when the CTA's weight rows fit its shared
+// [M][K]; M <= 8 at K = 16384, when the CTA's weight rows fit its shared
 // memory (decode_gemv_supported).
 struct GemvArgs {
     const uint8_t* codes;

@@ -61,8 +61,8 @@ static int optin_smem() {
 // shuffle reductions outweigh the dp4a work, and K1 + the row GEMV is faster
 // (K = 8192, 4 tokens: 12.8 vs 10.4 us).
 bool decode_gemv_supported(int M, int K, int N, int num_sms) {
-    if (M < 1 || M > 4 || N < 1 || K != 16384) return false;
-    return k6::gemv_smem_l14(N, token_capacity(M), num_sms) <= optin_smem();
+    if (M < 1 || M > 8 || N < 1 || K != 16384) return false;
+    return k6::gemv_smem_l14(N, M <= 4 ? token_capacity(M) : 8, num_sms) <= optin_smem();
 }
 
 hbl_status launch_decode_gemv(const GemvArgs& g, cudaStream_t stream, int num_sms) {

@@ -59,9 +59,10 @@ struct Shape {
     static constexpr int GPC = MT < NT / T ? MT : NT / T;
     using C = k1::Cfg<L, RLOG>;
     // packed words per lane per row: 8 / MT (32 code registers), at least
-    // enough for NW warps to cover a row
+    // enough for NW warps to cover a row (then MT * 4 * WPL code registers)
     static constexpr int WPL = (8 / MT) > ((1 << L) / (512 * NW)) ? (8 / MT)
                                                                   : ((1 << L) / (512 * NW));
+    static_assert(MT * 4 * WPL <= 128, "code registers");
     static constexpr int KSEG = 512 * WPL;
     static constexpr int KSPLIT = (1 << L) / KSEG;
     static constexpr int RG = NW / KSPLIT;
@@ -279,7 +280,7 @@ struct DecodeExt {
     }
 };
 
-// The GEMV half alone, for decode batches K6 does not take (M <= 4): launched
+// The GEMV half alone, for decode batches K6 does not take (M <= 8): launched
 // as a programmatic dependent of K1, it starts its weight rows' bulk copies
 // before the dependency wait (the weights are not K1's output), then reads
 // K1's codes (one byte each, row-major), scales and row sums from global
@@ -348,14 +349,17 @@ int gemv_smem_bytes(int N, int MT, int num_sms) {
     const int rows = decode_fused_rows(N, num_sms);
     if (MT == 1) return Shape<L, 1, false>::total(rows);
     if (MT == 2) return Shape<L, 2, false>::total(rows);
-    return Shape<L, 4, false>::total(rows);
+    if (MT == 4) return Shape<L, 4, false>::total(rows);
+    return Shape<L, 8, false>::total(rows);
 }
 
+// Token capacities 1, 2, 4, 8 (8: the codes take 128 registers per lane).
 template <int L>
 hbl_status launch_gemv_l(const GemvArgs& g, cudaStream_t s, int sms) {
     if (g.M <= 1) return launch_gemv<L, 1>(g, s, sms);
     if (g.M <= 2) return launch_gemv<L, 2>(g, s, sms);
-    return launch_gemv<L, 4>(g, s, sms);
+    if (g.M <= 4) return launch_gemv<L, 4>(g, s, sms);
+    return launch_gemv<L, 8>(g, s, sms);
 }
 
 template <int L>

@@ -177,7 +177,7 @@ HBL_API hbl_status hbl_ternary_gemm(const void* codes, const float* scales, cons
  * Decode batches (M <= 16384 / K tokens at K = 4096 / 8192 / 16384, while the
  * packed weight rows of one SM's share fit its shared memory, GEMM path 0) run
  * both steps in one kernel instead: every CTA quantises the M rows itself
- * while its weight rows stream in; up to 4 tokens at K = 16384 run
+ * while its weight rows stream in; up to 8 tokens at K = 16384 run
  * hbl_norm_fwht_quant followed by that kernel's GEMV half, whose weight rows
  * stream into shared memory during the quantiser.  The results are the same
  * values on every path.

@@ -405,11 +405,12 @@ def test_decode_sweep(T, shape):
 # where the CTA's weight rows fit shared memory) against the oracle and
 # against the two-kernel forward (GEMM path 2: K1, then the row GEMV).  N (a
 # multiple of 16) spans fewer rows than SMs, ragged splits over the SMs and the
-# largest split that fits; the other (M, K) pairs take the two-kernel forward.
+# largest split that fits; the other (M, K) pairs take K1 and then the same
+# kernel's GEMV half (K = 16384, up to 8 tokens) or the row GEMV.
 @pytest.mark.parametrize("bits", [4, 8])
 @pytest.mark.parametrize("K,N", [(4096, 4096), (4096, 1008), (4096, 16384), (8192, 304),
                                  (8192, 4096), (16384, 112), (16384, 4096)])
-@pytest.mark.parametrize("M", [1, 2, 3, 4])
+@pytest.mark.parametrize("M", [1, 2, 3, 4, 6, 8])
 def test_decode_one_kernel_forward(bits, K, N, M):
     X = acts(M, K, seed=M + K, kind="t" if M % 2 else "gauss")
     W = inputs.latent_weights(N, K, seed=N + M)
