@@ -47,10 +47,12 @@ constexpr int kFlGain = 1;
 constexpr int kFlNoHadamard = 2;
 constexpr int kFlLayerNorm = 4;
 
-// log2 of the fp32 values each thread holds: 128 in general; 64 for K = 8192
-// and 16384, where it keeps two exchanges while doubling the resident warps.
+// log2 of the fp32 values each thread holds: 128 in general (K = 16384: four
+// warps per row, three rows per SM, 149 us on 8192 rows against 169 us with
+// 64 values and eight warps per row); 64 for K = 8192, where it keeps two
+// exchanges while doubling the resident warps.
 __host__ __device__ constexpr int reg_log(int L) {
-    return (L == 13 || L == 14) ? 6 : (L < kRegLog ? L : kRegLog);
+    return (L == 13) ? 6 : (L < kRegLog ? L : kRegLog);
 }
 
 template <int L, int RLOG = reg_log(L)>
@@ -73,7 +75,8 @@ struct Cfg {
     static constexpr int kSmemBytes = kGroupsPerCta * (kBufBytes + kRedFloats * 4);
     // 3 CTAs (12 warps) per SM where the register budget (170) suffices
     static constexpr int kMinBlocks =
-        r == 6 ? (kCtaThreads >= 256 ? 2 : 4) : (kCtaThreads >= 256 ? 1 : ((L >= 8 && L != 12) ? 2 : 3));
+        r == 6 ? (kCtaThreads >= 256 ? 2 : 4)
+               : (kCtaThreads >= 256 ? 1 : ((L >= 8 && L != 12 && L != 14) ? 2 : 3));
 };
 
 // Layout p: 0 = natural, p >= 1 = pass p (stage base r + (r - 2)(p - 1)).
