@@ -206,6 +206,18 @@ struct NoExt {
     static __device__ void staged(const Params&) {}
     static __device__ void finish(const Params&) {}
 };
+// The plain kernel with 2^RL values per thread instead of reg_log(L).
+template <int RL>
+struct NoExtR : NoExt {
+    template <int L>
+    __host__ __device__ static constexpr int threads() { return Cfg<L, RL>::kCtaThreads; }
+    template <int L>
+    __host__ __device__ static constexpr int min_blocks() { return Cfg<L, RL>::kMinBlocks; }
+    template <int L>
+    __host__ __device__ static constexpr int rlog() { return RL; }
+    template <int L>
+    __host__ __device__ static constexpr int groups() { return Cfg<L, RL>::kGroupsPerCta; }
+};
 
 template <int T>
 __device__ __forceinline__ void group_sync(int grp) {
@@ -769,10 +781,10 @@ __global__ void __launch_bounds__(Ext::template threads<L>(), Ext::template min_
     if constexpr (Ext::kOn) Ext::finish(p);
 }
 
-template <int L, int MODE, int FL>
-static hbl_status launch_one(const Params& prm, cudaStream_t stream, int num_sms) {
-    using C = Cfg<L>;
-    auto kern = norm_fwht_quant_kernel<L, MODE, FL>;
+template <int L, int MODE, int FL, class Ext>
+static hbl_status launch_cfg(const Params& prm, cudaStream_t stream, int num_sms) {
+    using C = Cfg<L, Ext::template rlog<L>()>;
+    auto kern = norm_fwht_quant_kernel<L, MODE, FL, Ext>;
     if (!smem_attr_once(reinterpret_cast<const void*>(kern), C::kSmemBytes)) return HBL_ERR_CUDA;
     const int64_t groups = (prm.M + C::kRowsPerGroup - 1) / C::kRowsPerGroup;
     const int64_t ctas_needed = (groups + C::kGroupsPerCta - 1) / C::kGroupsPerCta;
@@ -781,6 +793,16 @@ static hbl_status launch_one(const Params& prm, cudaStream_t stream, int num_sms
     if (grid < 1) grid = 1;
     kern<<<(unsigned)grid, C::kCtaThreads, C::kSmemBytes, stream>>>(prm);
     return cudaGetLastError() == cudaSuccess ? HBL_OK : HBL_ERR_CUDA;
+}
+
+template <int L, int MODE, int FL>
+static hbl_status launch_one(const Params& prm, cudaStream_t stream, int num_sms) {
+    // K = 16384 with at most one row per CTA: latency per row decides, and 64
+    // values per thread (eight warps per row) finish a row sooner
+    if constexpr (L == 14)
+        if (prm.M <= (int64_t)num_sms * Cfg<L>::kMinBlocks)
+            return launch_cfg<L, MODE, FL, NoExtR<6>>(prm, stream, num_sms);
+    return launch_cfg<L, MODE, FL, NoExt>(prm, stream, num_sms);
 }
 
 template <int MODE, int FL>
