@@ -156,6 +156,20 @@ def test_quant_int4_large_k_spiky_rows(K):
                                   oracle.hbitlinear_forward(X[r:r + 1], packed, alpha, 4))
 
 
+@pytest.mark.parametrize("K", [8192, 16384])
+def test_quant_many_rows_large_k(K):
+    # more rows than three per SM: at K = 16384 the 128-values-per-thread
+    # launch (fewer rows take the 64-values one, covered above)
+    X = acts(1000, K, seed=K, kind="t")
+    for bits in (4, 8):
+        check_quant(X, bits)
+    codes, scales, rowsum = hbl.norm_fwht_quant(to_dev_bf16(X), hbl.ACT_INT4_BYTES)
+    wc, ws, wr = oracle.norm_fwht_quant(X, 4)
+    assert np.array_equal(codes.cpu().numpy().view(np.int8).astype(np.int32),
+                          oracle.decode_codes(wc, K, 4))
+    assert np.array_equal(scales.cpu().numpy().view(np.uint32), ws.view(np.uint32))
+
+
 def test_quant_workloads_full_size():
     # quant workload (8192 x 4096, Student-t, 1% channels x 20), both widths
     X = inputs.activations("quant")
