@@ -20,10 +20,11 @@
 //     kernel), writing one code byte per element into shared memory.  Latency
 //     sets the shape: 64 values per thread (K / 64 threads per row, two
 //     shared-memory exchanges), one row group per token;
-//  3. a warp covers KSEG = 4096 / M' elements of a weight row (M' = token
-//     capacity): each lane keeps the codes of its 8 / M' packed words per token
-//     in registers and, for each row of the warp's row group, reads those
-//     words once from shared memory.  The four 2-bit fields g of a packed byte
+//  3. a warp covers KSEG = 512 * WPL elements of a weight row, WPL = the
+//     larger of 8 / M' (M' = token capacity) and K / 4096 packed words per
+//     lane: each lane keeps the codes of its WPL words per token in registers
+//     and, for each row of the warp's row group, reads those words once from
+//     shared memory.  The four 2-bit fields g of a packed byte
 //     are masked in place (value c * 4^g, c = t + 1 in {0, 1, 2}) and summed by
 //     dp4a into four accumulators that exact shifts bring back to one sum of
 //     q * c, reduced over the lanes by xor shuffles;
