@@ -150,19 +150,13 @@ ORACLE_API float oracle_sqrt7(void) { return (float)sqrt(7.0); }
  * description uses RMS normalisation without bias; the RMS reading is taken. */
 static void rmsnorm_row_f32(const uint16_t* xb, const float* gain, int K, float norm_eps,
                             float* u, float* scratch) {
-    /* Leaves of the tree are pairs: x0*x0 + x1*x1 with one rounding.  For bf16
-     * inputs each square is exact in binary32 (8-bit significands), so this
-     * equals rounding the two squares first whenever they do not underflow. */
-    if (K == 1) {
-        float x = oracle_bf16_to_f32(xb[0]);
-        scratch[0] = x * x;
+    /* The plain reading of "sum of x^2": every square x*x is one binary32
+     * multiply (rounded), and the K squares are summed by the pairwise tree. */
+    for (int k = 0; k < K; ++k) {
+        float x = oracle_bf16_to_f32(xb[k]);
+        scratch[k] = x * x;
     }
-    for (int k = 0; k + 1 < K; k += 2) {
-        float x0 = oracle_bf16_to_f32(xb[k]);
-        float x1 = oracle_bf16_to_f32(xb[k + 1]);
-        scratch[k / 2] = fmaf(x0, x0, x1 * x1);
-    }
-    float ss = tree_sum_f32(scratch, K == 1 ? 1 : K / 2);
+    float ss = tree_sum_f32(scratch, K);
     float ms = ss * (1.0f / (float)K);
     float r = 1.0f / sqrtf(ms + norm_eps);
     for (int k = 0; k < K; ++k) {
@@ -233,7 +227,7 @@ ORACLE_API int oracle_norm_fwht_f64(const uint16_t* X, const float* gain, int M,
 
 /* LayerNorm without bias, one row:
  *   mu  = tree_sum(x) * (1/K);  d = x - mu;
- *   var = tree_sum(d*d) * (1/K)   (leaves d0*d0 + d1*d1 with one rounding, as
+ *   var = tree_sum(d*d) * (1/K)   (every square d*d rounded to binary32, as
  *                                  in the RMS sum of squares);
  *   u   = (d * (1 / sqrt(var + eps))) * g.
  * [P2] writes the layer as LN(.) and glosses it as layer normalisation. */
@@ -242,9 +236,8 @@ static void layernorm_row_f32(const uint16_t* xb, const float* gain, int K, floa
     for (int k = 0; k < K; ++k) u[k] = oracle_bf16_to_f32(xb[k]);
     float mu = tree_sum_f32(u, K) * (1.0f / (float)K);
     for (int k = 0; k < K; ++k) u[k] = u[k] - mu;
-    if (K == 1) scratch[0] = u[0] * u[0];
-    for (int k = 0; k + 1 < K; k += 2) scratch[k / 2] = fmaf(u[k], u[k], u[k + 1] * u[k + 1]);
-    float var = tree_sum_f32(scratch, K == 1 ? 1 : K / 2) * (1.0f / (float)K);
+    for (int k = 0; k < K; ++k) scratch[k] = u[k] * u[k];
+    float var = tree_sum_f32(scratch, K) * (1.0f / (float)K);
     float r = 1.0f / sqrtf(var + norm_eps);
     for (int k = 0; k < K; ++k) {
         float v = u[k] * r;
@@ -554,16 +547,17 @@ ORACLE_API int oracle_pack_ternary(const float* W, int N, int K, float eps, uint
 
 /* acc[m][n] = sum_k q[m][k] * t[n][k]   (exact, int64, must fit int32);
  * y[m][n]   = bf16_rne( (float)acc * (alpha * scale[m]) ).
+ * t: the ternary values int8 [N x K] (unpacked once by the caller).
  * Rows m in [m0, m1) only (callers split rows across threads). */
-ORACLE_API int oracle_ternary_gemm_rows(const uint8_t* codes, const float* scales, int act_bits,
-                                        int M, int K, const uint32_t* packed, float alpha, int N,
-                                        int m0, int m1, uint16_t* Y, int32_t* acc_out) {
-    if (M < 0 || K <= 0 || K % 16 != 0 || N <= 0) return -1;
+ORACLE_API int oracle_ternary_gemm_rows_t(const uint8_t* codes, const float* scales,
+                                          int act_bits, int M, int K, const int8_t* t,
+                                          float alpha, int N, int m0, int m1, uint16_t* Y,
+                                          int32_t* acc_out) {
+    if (M < 0 || K <= 0 || N <= 0) return -1;
     if (m0 < 0 || m1 > M || m0 > m1) return -1;
-    int8_t* t = (int8_t*)malloc((size_t)N * (size_t)K);
     int8_t* q = (int8_t*)malloc((size_t)K);
-    if (!t || !q) { free(t); free(q); return -2; }
-    int rc = oracle_unpack_codes(packed, N, K, t);
+    if (!q) return -2;
+    int rc = 0;
     int64_t cstride = act_bits == 8 ? K : K / 2;
     for (int64_t m = m0; m < m1 && rc == 0; ++m) {
         rc = oracle_decode_codes(codes + m * cstride, 1, K, act_bits, q);
@@ -578,8 +572,23 @@ ORACLE_API int oracle_ternary_gemm_rows(const uint8_t* codes, const float* scale
             if (Y) Y[m * N + n] = oracle_f32_to_bf16((float)s * sc);
         }
     }
-    free(t);
     free(q);
+    return rc;
+}
+
+/* The same from the packed weights (unpacked here). */
+ORACLE_API int oracle_ternary_gemm_rows(const uint8_t* codes, const float* scales, int act_bits,
+                                        int M, int K, const uint32_t* packed, float alpha, int N,
+                                        int m0, int m1, uint16_t* Y, int32_t* acc_out) {
+    if (M < 0 || K <= 0 || K % 16 != 0 || N <= 0) return -1;
+    if (m0 < 0 || m1 > M || m0 > m1) return -1;
+    int8_t* t = (int8_t*)malloc((size_t)N * (size_t)K);
+    if (!t) return -2;
+    int rc = oracle_unpack_codes(packed, N, K, t);
+    if (rc == 0)
+        rc = oracle_ternary_gemm_rows_t(codes, scales, act_bits, M, K, t, alpha, N, m0, m1, Y,
+                                        acc_out);
+    free(t);
     return rc;
 }
 
@@ -615,11 +624,12 @@ ORACLE_API int oracle_bitlinear_forward_rows(const uint16_t* X, const float* gai
 }
 
 /* Whole layer for rows [m0, m1): norm -> Hadamard -> quantise -> ternary matmul
- * -> dequantise.  Y is [M x N] bf16 bits; only rows [m0, m1) are written. */
-ORACLE_API int oracle_hbitlinear_forward_rows(const uint16_t* X, const float* gain, int M, int K,
-                                              int N, const uint32_t* packed, float alpha,
-                                              int act_bits, float norm_eps, float quant_eps,
-                                              int m0, int m1, uint16_t* Y) {
+ * -> dequantise.  Y is [M x N] bf16 bits; only rows [m0, m1) are written.
+ * t: the ternary values int8 [N x K] (unpacked once by the caller). */
+ORACLE_API int oracle_hbitlinear_forward_rows_t(const uint16_t* X, const float* gain, int M,
+                                                int K, int N, const int8_t* t, float alpha,
+                                                int act_bits, float norm_eps, float quant_eps,
+                                                int m0, int m1, uint16_t* Y) {
     if (m0 < 0 || m1 > M || m0 > m1) return -1;
     int rows = m1 - m0;
     if (rows == 0) return 0;
@@ -630,9 +640,27 @@ ORACLE_API int oracle_hbitlinear_forward_rows(const uint16_t* X, const float* ga
     int rc = oracle_norm_fwht_quant(X + (int64_t)m0 * K, gain, rows, K, norm_eps, quant_eps,
                                     act_bits, codes, scales, NULL);
     if (rc == 0)
-        rc = oracle_ternary_gemm(codes, scales, act_bits, rows, K, packed, alpha, N,
-                                 Y + (int64_t)m0 * N, NULL);
+        rc = oracle_ternary_gemm_rows_t(codes, scales, act_bits, rows, K, t, alpha, N, 0, rows,
+                                        Y + (int64_t)m0 * N, NULL);
     free(codes);
     free(scales);
+    return rc;
+}
+
+/* The same from the packed weights (unpacked here). */
+ORACLE_API int oracle_hbitlinear_forward_rows(const uint16_t* X, const float* gain, int M, int K,
+                                              int N, const uint32_t* packed, float alpha,
+                                              int act_bits, float norm_eps, float quant_eps,
+                                              int m0, int m1, uint16_t* Y) {
+    if (m0 < 0 || m1 > M || m0 > m1) return -1;
+    if (K <= 0 || K % 16 != 0 || N <= 0) return -1;
+    if (m1 == m0) return 0;
+    int8_t* t = (int8_t*)malloc((size_t)N * (size_t)K);
+    if (!t) return -2;
+    int rc = oracle_unpack_codes(packed, N, K, t);
+    if (rc == 0)
+        rc = oracle_hbitlinear_forward_rows_t(X, gain, M, K, N, t, alpha, act_bits, norm_eps,
+                                              quant_eps, m0, m1, Y);
+    free(t);
     return rc;
 }

@@ -171,6 +171,87 @@ def test_rmsnorm_matches_torch_fp64():
     assert np.max(np.abs(got - want) / np.abs(want).max(axis=1, keepdims=True)) < 1e-6
 
 
+def _f32_nearest(q):
+    """The binary32 value nearest to the positive rational q (ties to even) for a
+    q in the normal range, derived exactly (no floating-point arithmetic)."""
+    q = Fraction(q)
+    assert q > 0
+    e = 0
+    while q >= 2:
+        q /= 2
+        e += 1
+    while q < 1:
+        q *= 2
+        e -= 1
+    assert -126 <= e <= 127
+    m = q * 2 ** 23
+    n = m.numerator // m.denominator
+    rem = m - n
+    if rem > Fraction(1, 2) or (rem == Fraction(1, 2) and n % 2 == 1):
+        n += 1
+    return Fraction(n, 2 ** 23) * Fraction(2) ** e
+
+
+def _f32_sqrt_nearest(q):
+    """Nearest binary32 to sqrt(q) for a positive rational q with a normal root."""
+    q = Fraction(q)
+    e = 0
+    while q >= 4:
+        q /= 4
+        e += 1
+    while q < 1:
+        q *= 4
+        e -= 1
+    # sqrt(q) in [1, 2): candidates n / 2^23; pick by comparing squares exactly
+    target = q * 2 ** 46
+    n = int(target.numerator // target.denominator)
+    lo = int(np.floor(np.sqrt(float(n))))
+    while (lo + 1) ** 2 <= target:
+        lo += 1
+    while lo ** 2 > target:
+        lo -= 1
+    mid = Fraction(2 * lo + 1, 2)
+    if mid * mid < target or (mid * mid == target and lo % 2 == 1):
+        lo += 1
+    return Fraction(lo, 2 ** 23) * Fraction(2) ** e
+
+
+def test_sum_of_squares_rounds_every_square_hand_case():
+    # The RMS statistic is tree_sum(x*x): each square is one binary32 multiply
+    # (rounded), then the pairwise tree adds them.  Hand-derived row of K = 16
+    # pairs (a, b) = (2^-75, 1.5 * 2^-75), norm_eps = 2^-149:
+    #   a*a = 2^-150 rounds to 0 (a tie, to even); b*b = 1.125 * 2^-149 rounds to
+    #   2^-149; every pair adds to 2^-149 and the tree to 8 * 2^-149 = 2^-146;
+    #   mean 2^-146 / 16 = 2^-150 rounds to 0; + eps = 2^-149;
+    #   r = fl(1 / fl(sqrt(2^-149))) = 2^75 * fl(1 / fl(sqrt 2));
+    #   u = (fl(1/fl(sqrt 2)), fl(1.5 * fl(1/fl(sqrt 2)))) per pair.
+    # (Summing each pair with one rounding, a*a + fl(b*b) = 1.5 * 2^-149 -> 2^-148,
+    # would give r = 2^74 and u = (0.5, 0.75) instead.)
+    K = 16
+    a_bits, b_bits = 0x1A00, 0x1A40  # bf16 of 2^-75 and 1.5 * 2^-75
+    assert oracle.bf16_to_f32(np.array([a_bits], np.uint16))[0] == np.float32(2.0 ** -75)
+    assert oracle.bf16_to_f32(np.array([b_bits], np.uint16))[0] == np.float32(1.5 * 2.0 ** -75)
+    row = np.tile(np.array([a_bits, b_bits], np.uint16), K // 2)[None, :]
+    h = _f32_nearest(1 / _f32_sqrt_nearest(2))
+    want = np.tile(np.array([float(h), float(_f32_nearest(Fraction(3, 2) * h))],
+                            np.float32), K // 2)
+    eps = float(2.0 ** -149)
+    got = oracle.rmsnorm(row, norm_eps=eps)
+    assert np.array_equal(got[0].view(np.uint32), want.view(np.uint32))
+    # the same row through norm_transform without the transform
+    got_t = oracle.norm_transform(row, norm_eps=eps, hadamard=False)
+    assert np.array_equal(got_t[0].view(np.uint32), want.view(np.uint32))
+    # LayerNorm of the row with its second half negated: the tree sum of x is 0
+    # exactly (each half sums to +-10 * 2^-75), so d = x and the statistic is the
+    # same sum of rounded squares
+    neg = row.copy()
+    neg[0, K // 2:] |= 0x8000
+    want_ln = want.copy()
+    want_ln[K // 2:] = -want_ln[K // 2:]
+    got_ln = oracle.norm_transform(neg, norm_eps=eps, layernorm=True, hadamard=False)
+    assert np.array_equal(got_ln[0].view(np.uint32), want_ln.view(np.uint32))
+
+
 # ------------------------------------------------------- norm + transform
 
 @pytest.mark.parametrize("name,M,K", [("tiny", 16, 256), ("attn_wo", 8, 2048),
