@@ -453,11 +453,12 @@ __global__ void __launch_bounds__(Ext::template threads<L>(), Ext::template min_
             });
         }
         // ---- RMS of the row (of x - mean for LayerNorm): tree over the row in
-        // ascending index order; each leaf is d0*d0 + d1*d1 with one rounding
-        // (for RMSNorm of bf16 inputs the squares are exact in fp32)
+        // ascending index order of the squares, each square rounded to fp32
+        // (one packed multiply per pair), the first tree level adding the pair
         float ss = stream_tree<R / 2>([&](auto kk) {
             constexpr int k = decltype(kk)::value;
-            return __fmaf_rn(d[k].x, d[k].x, __fmul_rn(d[k].y, d[k].y));
+            const float2 sq = mul2(d[k], d[k]);
+            return __fadd_rn(sq.x, sq.y);
         });
         ss = row_sum(ss);
         [[maybe_unused]] const bool ss_ok = ss >= 0x1p-100f;

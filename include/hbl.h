@@ -75,22 +75,28 @@ HBL_API const char* hbl_status_string(int status);
 /* Library ABI version (major * 10000 + minor * 100 + patch). */
 HBL_API int hbl_version(void);
 
-/* Choice of ternary-GEMM back end (test and tuning aid; process-wide, not
- * synchronised with calls in flight on other threads):
- *   0 = automatic (and, in hbl_hbitlinear_forward, the one-kernel decode
- *       forward where it applies): CUDA-core GEMV for M <= 8 tokens (one weight row per warp
- *       for K >= 2048, split-K below); the tcgen05 kernel with activations in
- *       tensor memory (split over K for M <= 256) up to 256 tokens; above that
- *       the TMA-fed tcgen05 kernel when the codes are one byte each (it expands
- *       the packed weights to signed bytes in workspace first),
- *   1 = tcgen05 with both operands staged in shared memory by threads,
- *   2 = always the GEMV path (large M runs in chunks of 8 tokens),
- *   3 = always the tcgen05 kernel with activations in tensor memory,
- *   4 = the TMA-fed tcgen05 kernel whenever the codes are one byte each and
- *       K >= 128 (else as 3).
- * hbl_workspace_size() answers for the path in force.  Returns HBL_OK or
- * HBL_ERR_INVALID_ARG.  This call has no counterpart on the BitNet v2 pages. */
-HBL_API int hbl_set_gemm_path(int path);
+/* Ternary-GEMM back ends, chosen per call through the *_path variants below
+ * (a test and tuning aid; the library keeps no process-wide choice):
+ *   HBL_PATH_AUTO (0) = what hbl_ternary_gemm / hbl_hbitlinear_forward do: the
+ *       one-kernel decode forward where it applies; CUDA-core GEMV for M <= 8
+ *       tokens (one weight row per warp for K >= 2048, split-K below); the
+ *       tcgen05 kernel with activations in tensor memory (split over K for
+ *       M <= 256) up to 256 tokens; above that the TMA-fed tcgen05 kernel when
+ *       the codes are one byte each (it expands the packed weights to signed
+ *       bytes in workspace first),
+ *   HBL_PATH_TC_SS (1)  = tcgen05 with both operands staged in shared memory by threads,
+ *   HBL_PATH_GEMV (2)   = always the GEMV path (large M runs in chunks of 8 tokens),
+ *   HBL_PATH_TC_TS (3)  = always the tcgen05 kernel with activations in tensor memory,
+ *   HBL_PATH_TC_TMA (4) = the TMA-fed tcgen05 kernel whenever the codes are one
+ *       byte each and K >= 128 (else as 3).
+ * Every path computes the same values.  No counterpart on the BitNet v2 pages. */
+enum {
+    HBL_PATH_AUTO = 0,
+    HBL_PATH_TC_SS = 1,
+    HBL_PATH_GEMV = 2,
+    HBL_PATH_TC_TS = 3,
+    HBL_PATH_TC_TMA = 4
+};
 
 /* act_bits also accepts these two values: the same INT4 / INT8 codes stored
  * one byte per code (two's complement) in a 32-row interleaved layout.  Rows
@@ -100,7 +106,8 @@ HBL_API int hbl_set_gemm_path(int path);
  * owns 32 consecutive rows reads each chunk as 512 contiguous bytes; the
  * tensor-core GEMM takes this layout without widening, and
  * hbl_hbitlinear_forward uses it internally.  hbl_ternary_gemm always runs its
- * tcgen05 kernel for these layouts, whatever hbl_set_gemm_path says. */
+ * tcgen05 kernel with activations in tensor memory for these layouts, whatever
+ * path is asked for. */
 enum { HBL_ACT_INT4_I32 = 0x104, HBL_ACT_INT8_I32 = 0x108 };
 
 /* act_bits may also be HBL_ACT_INT4_BYTES: INT4 codes stored one byte each
@@ -122,6 +129,11 @@ enum {
  * HBL_ERR_INVALID_ARG on bad input. */
 HBL_API hbl_status hbl_workspace_size(int op, int M, int K, int N, int act_bits, size_t* bytes);
 
+/* hbl_workspace_size for the calls' *_path variants: the bytes `op` needs when
+ * run on back end `path` (HBL_PATH_*; HBL_ERR_INVALID_ARG for other values). */
+HBL_API hbl_status hbl_workspace_size_path(int op, int M, int K, int N, int act_bits, int path,
+                                           size_t* bytes);
+
 /* Ternary weight quantisation and packing (offline, once per weight).
  * Formula (per-tensor absmean; the page's formula is an image):
  *   alpha = S / (float)(N*K),  S = fp32 left-complete pairwise tree sum of |W|
@@ -136,6 +148,8 @@ HBL_API hbl_status hbl_pack_ternary(const float* W, int N, int K, float eps, uin
 
 /* RMSNorm followed by the normalised online Hadamard transform, fp32 out:
  *   r = 1 / sqrt(tree_sum(x*x) * (1/K) + norm_eps),   u = (x * r) * gain
+ *   (every square x*x rounded to fp32, then summed by the perfect pairwise
+ *   tree over index order)
  *   V = (u . H_K) * c_K,   c_K = fp32(1/sqrt(K)),
  * H_K the Sylvester Hadamard matrix in natural order, evaluated as butterfly
  * stages h = 1, 2, ..., K/2 in that order, (a, b) -> (a + b, a - b).
@@ -173,6 +187,15 @@ HBL_API hbl_status hbl_ternary_gemm(const void* codes, const float* scales, cons
                             const float* alpha, int N, uint16_t* Y, int32_t* acc_out,
                             void* ws, size_t ws_bytes, int32_t* dev_status, void* stream);
 
+/* hbl_ternary_gemm on the back end `path` (HBL_PATH_*; HBL_PATH_AUTO is
+ * hbl_ternary_gemm itself).  Same results on every path; ws sized by
+ * hbl_workspace_size_path(HBL_OP_TERNARY_GEMM, ..., path, ...). */
+HBL_API hbl_status hbl_ternary_gemm_path(const void* codes, const float* scales,
+                                         const int32_t* rowsum, int act_bits, int M, int K,
+                                         const uint32_t* W_packed, const float* alpha, int N,
+                                         uint16_t* Y, int32_t* acc_out, void* ws, size_t ws_bytes,
+                                         int32_t* dev_status, int path, void* stream);
+
 /* The whole layer: hbl_norm_fwht_quant into workspace, then hbl_ternary_gemm.
  * Decode batches (M <= 16384 / K tokens at K = 4096 / 8192 / 16384, while the
  * packed weight rows of one SM's share fit its shared memory, GEMM path 0) run
@@ -187,6 +210,17 @@ HBL_API hbl_status hbl_hbitlinear_forward(const uint16_t* X, const float* gain, 
                                   const uint32_t* W_packed, const float* alpha, int act_bits,
                                   float norm_eps, float quant_eps, uint16_t* Y, void* ws,
                                   size_t ws_bytes, int32_t* dev_status, void* stream);
+
+/* hbl_hbitlinear_forward with the GEMM on back end `path` (HBL_PATH_*); any
+ * path other than HBL_PATH_AUTO runs the two-kernel forward (quantiser, then
+ * that GEMM).  ws sized by hbl_workspace_size_path(HBL_OP_HBITLINEAR_FORWARD,
+ * ..., path, ...). */
+HBL_API hbl_status hbl_hbitlinear_forward_path(const uint16_t* X, const float* gain, int M, int K,
+                                               int N, const uint32_t* W_packed,
+                                               const float* alpha, int act_bits, float norm_eps,
+                                               float quant_eps, uint16_t* Y, void* ws,
+                                               size_t ws_bytes, int32_t* dev_status, int path,
+                                               void* stream);
 
 /* The whole layer with HOST activations in and HOST outputs out: copies X_host
  * to the device, runs hbl_hbitlinear_forward, copies Y back to Y_host
@@ -218,8 +252,8 @@ HBL_API hbl_status hbl_hbitlinear_forward_hostio(const uint16_t* X_host, const f
  *   HBL_NORM_LAYERNORM:   LayerNorm without bias instead of RMSNorm:
  *       mu = tree_sum(x) * (1/K);  d = x - mu;
  *       r = 1 / sqrt(tree_sum(d*d) * (1/K) + norm_eps);  u = (d * r) * gain
- *       (tree sums as for RMSNorm; the leaves of the d*d sum are
- *        d0*d0 + d1*d1 with one rounding).
+ *       (tree sums as for RMSNorm; every square d*d is rounded to fp32
+ *        before the tree adds it).
  *   HBL_NORM_NO_HADAMARD: no transform: the codes quantise u itself.
  * flags = 0 is exactly the H-BitLinear path of the calls above.  Other bits
  * return HBL_ERR_INVALID_ARG.  Shapes and layouts as above (K a power of two). */

@@ -99,6 +99,31 @@ def test_variant_edge_rows_and_zero_eps(flags, bits):
 
 
 @pytest.mark.parametrize("flags", FLAGS)
+@pytest.mark.parametrize("K", [16, 4096, 16384])
+def test_variant_values_with_underflowing_squares(flags, K):
+    # the squares of d = x (- mean) are rounded to fp32 before the tree sum:
+    # rows whose squares are subnormal decide that reading
+    rng = np.random.default_rng(K + flags)
+    X = np.empty((4, K), dtype=np.uint16)
+    X[0] = np.tile(np.array([0x1A00, 0x1A40], np.uint16), K // 2)
+    X[1] = X[0]
+    X[1, K // 2:] |= 0x8000
+    for r, sc in ((2, 1e-20), (3, 1e-22)):
+        v = torch.from_numpy((rng.standard_normal(K) * sc).astype(np.float32))
+        X[r] = v.to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    eps = float(2.0 ** -149)
+    V = hbl.norm_transform(to_dev_bf16(X), flags, norm_eps=eps).cpu().numpy()
+    want = oracle.norm_transform(X, norm_eps=eps, **okw(flags))
+    assert np.array_equal(V.view(np.uint32), want.view(np.uint32))
+    for bits in (4, 8):
+        codes, scales, rowsum = hbl.norm_quant(to_dev_bf16(X), bits, flags, norm_eps=eps)
+        wc, ws, wr = oracle.norm_quant(X, bits, norm_eps=eps, **okw(flags))
+        assert np.array_equal(codes.cpu().numpy(), wc)
+        assert np.array_equal(scales.cpu().numpy().view(np.uint32), ws.view(np.uint32))
+        assert np.array_equal(rowsum.cpu().numpy(), wr)
+
+
+@pytest.mark.parametrize("flags", FLAGS)
 @pytest.mark.parametrize("bits", [4, 8])
 @pytest.mark.parametrize("M,K,N", [(1, 4096, 4096), (8, 256, 128), (45, 2048, 272),
                                    (300, 4096, 256)])
