@@ -33,9 +33,11 @@ OP_PACK_TERNARY, OP_TERNARY_GEMM, OP_HBITLINEAR_FORWARD, OP_HBITLINEAR_FORWARD_H
 ACT_INT4_I32, ACT_INT8_I32 = 0x104, 0x108  # one byte per code, 32-row interleaved layout
 ACT_INT4_BYTES = 0x204                      # INT4 codes one byte each, row-major
 NORM_LAYERNORM, NORM_NO_HADAMARD = 1, 2     # variant flags of norm_transform / norm_quant / bitlinear_forward
-EXPORTS = ("hbl_status_string", "hbl_version", "hbl_set_gemm_path", "hbl_workspace_size",
+PATH_AUTO, PATH_TC_SS, PATH_GEMV, PATH_TC_TS, PATH_TC_TMA = 0, 1, 2, 3, 4  # GEMM back ends
+EXPORTS = ("hbl_status_string", "hbl_version", "hbl_workspace_size", "hbl_workspace_size_path",
            "hbl_pack_ternary", "hbl_norm_fwht", "hbl_norm_fwht_quant", "hbl_ternary_gemm",
-           "hbl_hbitlinear_forward", "hbl_hbitlinear_forward_hostio",
+           "hbl_ternary_gemm_path", "hbl_hbitlinear_forward", "hbl_hbitlinear_forward_path",
+           "hbl_hbitlinear_forward_hostio",
            "hbl_ternary_gemv_noalloc", "hbl_norm_transform", "hbl_norm_quant",
            "hbl_bitlinear_forward", "hbl_rotate_weights", "hbl_kv_quant",
            "hbl_expand_ternary", "hbl_ternary_gemm_s8w", "hbl_selftest_bounded_wait")
@@ -63,10 +65,10 @@ def lib():
         L.hbl_status_string.argtypes = [I]
         L.hbl_version.restype = I
         L.hbl_version.argtypes = []
-        L.hbl_set_gemm_path.restype = I
-        L.hbl_set_gemm_path.argtypes = [I]
         L.hbl_workspace_size.restype = I
         L.hbl_workspace_size.argtypes = [I, I, I, I, I, ctypes.POINTER(SZ)]
+        L.hbl_workspace_size_path.restype = I
+        L.hbl_workspace_size_path.argtypes = [I, I, I, I, I, I, ctypes.POINTER(SZ)]
         L.hbl_pack_ternary.restype = I
         L.hbl_pack_ternary.argtypes = [P, I, I, F, P, P, P, SZ, P]
         L.hbl_norm_fwht.restype = I
@@ -75,8 +77,12 @@ def lib():
         L.hbl_norm_fwht_quant.argtypes = [P, P, I, I, F, F, I, P, P, P, P, P]
         L.hbl_ternary_gemm.restype = I
         L.hbl_ternary_gemm.argtypes = [P, P, P, I, I, I, P, P, I, P, P, P, SZ, P, P]
+        L.hbl_ternary_gemm_path.restype = I
+        L.hbl_ternary_gemm_path.argtypes = [P, P, P, I, I, I, P, P, I, P, P, P, SZ, P, I, P]
         L.hbl_hbitlinear_forward.restype = I
         L.hbl_hbitlinear_forward.argtypes = [P, P, I, I, I, P, P, I, F, F, P, P, SZ, P, P]
+        L.hbl_hbitlinear_forward_path.restype = I
+        L.hbl_hbitlinear_forward_path.argtypes = [P, P, I, I, I, P, P, I, F, F, P, P, SZ, P, I, P]
         L.hbl_hbitlinear_forward_hostio.restype = I
         L.hbl_hbitlinear_forward_hostio.argtypes = [P, P, I, I, I, P, P, I, F, F, P, P, SZ, P, P]
         L.hbl_ternary_gemv_noalloc.restype = I
@@ -129,17 +135,12 @@ def _dev(t, dtype, name):
     return t
 
 
-def workspace_size(op, M, K, N, act_bits):
+def workspace_size(op, M, K, N, act_bits, path=PATH_AUTO):
+    """Workspace bytes of `op` on GEMM back end `path` (PATH_*)."""
     out = ctypes.c_size_t(0)
-    _check(lib().hbl_workspace_size(op, M, K, N, act_bits, ctypes.byref(out)), "workspace_size")
+    _check(lib().hbl_workspace_size_path(op, M, K, N, act_bits, int(path), ctypes.byref(out)),
+           "workspace_size")
     return out.value
-
-
-def set_gemm_path(path):
-    """0 = automatic, 1 = tensor cores (both operands staged by threads),
-    2 = CUDA-core GEMV, 3 = tensor cores with activations in TMEM, 4 = TMA-fed
-    tensor cores for one-byte codes (process-wide)."""
-    _check(lib().hbl_set_gemm_path(int(path)), "set_gemm_path")
 
 
 def _workspace(nbytes, device):
@@ -206,7 +207,11 @@ def norm_fwht_quant(X, act_bits, gain=None, norm_eps=1e-6, quant_eps=1e-5, out=N
 
 
 def ternary_gemm(codes, scales, rowsum, act_bits, K, W_packed, alpha, want_acc=False, ws=None,
-                 out=None, status=None):
+                 out=None, status=None, path=PATH_AUTO):
+    """hbl_ternary_gemm (hbl_ternary_gemm_path for a back end other than PATH_AUTO:
+    PATH_TC_SS tensor cores with both operands staged by threads, PATH_GEMV
+    CUDA-core GEMV, PATH_TC_TS tensor cores with activations in TMEM,
+    PATH_TC_TMA TMA-fed tensor cores for one-byte codes)."""
     import torch
 
     M = scales.shape[0]  # the interleaved layouts pad the codes buffer to 32 rows
@@ -214,12 +219,13 @@ def ternary_gemm(codes, scales, rowsum, act_bits, K, W_packed, alpha, want_acc=F
     Y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16,
                                                 device=codes.device)
     acc = torch.empty((M, N), dtype=torch.int32, device=codes.device) if want_acc else None
-    need = workspace_size(OP_TERNARY_GEMM, M, K, N, act_bits)
+    need = workspace_size(OP_TERNARY_GEMM, M, K, N, act_bits, path)
     if ws is None:
         ws = _workspace(need, codes.device)
-    _check(lib().hbl_ternary_gemm(_ptr(codes), _ptr(scales), _ptr(rowsum), int(act_bits), M, K,
-                                  _ptr(W_packed), _ptr(alpha), N, _ptr(Y), _ptr(acc), _ptr(ws),
-                                  ws.numel(), _ptr(status), _stream()), "hbl_ternary_gemm")
+    _check(lib().hbl_ternary_gemm_path(_ptr(codes), _ptr(scales), _ptr(rowsum), int(act_bits), M,
+                                       K, _ptr(W_packed), _ptr(alpha), N, _ptr(Y), _ptr(acc),
+                                       _ptr(ws), ws.numel(), _ptr(status), int(path), _stream()),
+           "hbl_ternary_gemm")
     return (Y, acc) if want_acc else Y
 
 
@@ -229,7 +235,7 @@ def ternary_gemv_noalloc(codes, scales, rowsum, act_bits, K, W_packed, alpha, wa
     array (no workspace argument; the library allocates nothing)."""
     import torch
 
-    M = codes.shape[0]
+    M = scales.shape[0]
     N = W_packed.shape[0]
     Y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16,
                                                 device=codes.device)
@@ -237,14 +243,13 @@ def ternary_gemv_noalloc(codes, scales, rowsum, act_bits, K, W_packed, alpha, wa
     _check(lib().hbl_ternary_gemv_noalloc(_ptr(codes), _ptr(scales), _ptr(rowsum),
                                           int(act_bits), M, K, _ptr(W_packed), _ptr(alpha), N,
                                           _ptr(Y), _ptr(acc), _ptr(status), _stream()),
-           "hbl_ternary_gemv_noalloc", "hbl_norm_transform", "hbl_norm_quant",
-           "hbl_bitlinear_forward", "hbl_rotate_weights", "hbl_kv_quant",
-           "hbl_expand_ternary", "hbl_ternary_gemm_s8w", "hbl_selftest_bounded_wait")
+           "hbl_ternary_gemv_noalloc")
     return (Y, acc) if want_acc else Y
 
 
 def hbitlinear_forward(X, W_packed, alpha, act_bits, gain=None, norm_eps=1e-6, quant_eps=1e-5,
-                       ws=None, out=None, status=None):
+                       ws=None, out=None, status=None, path=PATH_AUTO):
+    """hbl_hbitlinear_forward (hbl_hbitlinear_forward_path for another GEMM back end)."""
     import torch
 
     _dev(X, torch.bfloat16, "X")
@@ -252,11 +257,12 @@ def hbitlinear_forward(X, W_packed, alpha, act_bits, gain=None, norm_eps=1e-6, q
     N = W_packed.shape[0]
     Y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=X.device)
     if ws is None:
-        ws = _workspace(workspace_size(OP_HBITLINEAR_FORWARD, M, K, N, act_bits), X.device)
-    _check(lib().hbl_hbitlinear_forward(_ptr(X), _ptr(gain), M, K, N, _ptr(W_packed),
-                                        _ptr(alpha), int(act_bits), float(norm_eps),
-                                        float(quant_eps), _ptr(Y), _ptr(ws), ws.numel(),
-                                        _ptr(status), _stream()), "hbl_hbitlinear_forward")
+        ws = _workspace(workspace_size(OP_HBITLINEAR_FORWARD, M, K, N, act_bits, path), X.device)
+    _check(lib().hbl_hbitlinear_forward_path(_ptr(X), _ptr(gain), M, K, N, _ptr(W_packed),
+                                             _ptr(alpha), int(act_bits), float(norm_eps),
+                                             float(quant_eps), _ptr(Y), _ptr(ws), ws.numel(),
+                                             _ptr(status), int(path), _stream()),
+           "hbl_hbitlinear_forward")
     return Y
 
 

@@ -23,7 +23,6 @@ struct DevInfo {
     int sms = 0;
 };
 DevInfo g_dev[kMaxDevices];
-std::atomic<int> g_path{0};  // 0 auto, 1 SS tcgen05, 2 CUDA-core GEMV, 3 TS tcgen05, 4 TMA tcgen05
 
 bool is_pow2(int64_t v) { return v > 0 && (v & (v - 1)) == 0; }
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -79,9 +78,11 @@ bool rows_gemv(int64_t M, int K) { return gemv_rows_supported(K) && M <= gemv_ro
 // Batches above this many tokens take the TMA-fed kernel (automatic choice).
 constexpr int64_t kTmaMinM = 257;
 
-// The back end for M tokens; `bytes`: the codes are (or can be made) one byte each.
-Back pick(int64_t M, int K, bool bytes) {
-    const int path = g_path.load();
+bool path_valid(int path) { return path >= HBL_PATH_AUTO && path <= HBL_PATH_TC_TMA; }
+
+// The back end for M tokens under `path` (HBL_PATH_*); `bytes`: the codes are
+// (or can be made) one byte each.
+Back pick(int64_t M, int K, bool bytes, int path) {
     if (path == 1) return Back::SS;
     if (path == 2) return Back::GEMV;
     if (path == 3) return Back::TS;
@@ -155,9 +156,9 @@ struct FwdPlan {
     int gemm_act_bits;  // value width the GEMM reads (4 or 8)
     bool interleaved;
 };
-FwdPlan forward_plan(int64_t M, int K, int act_bits) {
+FwdPlan forward_plan(int64_t M, int K, int act_bits, int path) {
     FwdPlan f;
-    f.back = pick(M, K, true);
+    f.back = pick(M, K, true, path);
     f.interleaved = f.back == Back::TS;
     if (f.back == Back::TMA) {
         f.k1_mode = act_bits == 4 ? 6 : 8;
@@ -212,14 +213,13 @@ const char* hbl_status_string(int status) {
 
 int hbl_version(void) { return 100; }
 
-int hbl_set_gemm_path(int path) {
-    if (path < 0 || path > 4) return HBL_ERR_INVALID_ARG;
-    g_path.store(path);
-    return HBL_OK;
+hbl_status hbl_workspace_size(int op, int M, int K, int N, int act_bits, size_t* bytes) {
+    return hbl_workspace_size_path(op, M, K, N, act_bits, HBL_PATH_AUTO, bytes);
 }
 
-hbl_status hbl_workspace_size(int op, int M, int K, int N, int act_bits, size_t* bytes) {
-    if (bytes == nullptr) return HBL_ERR_INVALID_ARG;
+hbl_status hbl_workspace_size_path(int op, int M, int K, int N, int act_bits, int path,
+                                   size_t* bytes) {
+    if (bytes == nullptr || !path_valid(path)) return HBL_ERR_INVALID_ARG;
     *bytes = 0;
     switch (op) {
         case HBL_OP_PACK_TERNARY:
@@ -236,11 +236,11 @@ hbl_status hbl_workspace_size(int op, int M, int K, int N, int act_bits, size_t*
                 return HBL_ERR_INVALID_ARG;
             size_t b;
             if (op == HBL_OP_TERNARY_GEMM)
-                b = act_il(act_bits) ? up256(gemm_ts_workspace(M, K, N))
-                                     : up256(backend_ws(pick(M, K, act_width(act_bits) == 8), M,
-                                                        K, N));
+                b = act_il(act_bits)
+                        ? up256(gemm_ts_workspace(M, K, N))
+                        : up256(backend_ws(pick(M, K, act_width(act_bits) == 8, path), M, K, N));
             else
-                b = up256(backend_ws(forward_plan(M, K, act_bits).back, M, K, N));
+                b = up256(backend_ws(forward_plan(M, K, act_bits, path).back, M, K, N));
             if (op != HBL_OP_TERNARY_GEMM) {
                 b += up256((size_t)((M + 31) & ~31) * K);  // codes, one byte each, rows padded to 32
                 b += up256((size_t)M * 4) * 2;                         // scales, rowsum
@@ -327,7 +327,16 @@ hbl_status hbl_ternary_gemm(const void* codes, const float* scales, const int32_
                             int act_bits, int M, int K, const uint32_t* W_packed,
                             const float* alpha, int N, uint16_t* Y, int32_t* acc_out,
                             void* ws, size_t ws_bytes, int32_t* dev_status, void* stream) {
-    if (!act_valid(act_bits)) return HBL_ERR_INVALID_ARG;
+    return hbl_ternary_gemm_path(codes, scales, rowsum, act_bits, M, K, W_packed, alpha, N, Y,
+                                 acc_out, ws, ws_bytes, dev_status, HBL_PATH_AUTO, stream);
+}
+
+hbl_status hbl_ternary_gemm_path(const void* codes, const float* scales, const int32_t* rowsum,
+                                 int act_bits, int M, int K, const uint32_t* W_packed,
+                                 const float* alpha, int N, uint16_t* Y, int32_t* acc_out,
+                                 void* ws, size_t ws_bytes, int32_t* dev_status, int path,
+                                 void* stream) {
+    if (!act_valid(act_bits) || !path_valid(path)) return HBL_ERR_INVALID_ARG;
     if (M < 0 || check_k(K) != HBL_OK || check_n(N) != HBL_OK) return HBL_ERR_SHAPE;
     if (M == 0) return HBL_OK;
     if (!codes || !scales || !rowsum || !W_packed || !alpha || !Y) return HBL_ERR_INVALID_ARG;
@@ -335,7 +344,7 @@ hbl_status hbl_ternary_gemm(const void* codes, const float* scales, const int32_
         !aligned16(alpha) || !aligned16(Y) || (acc_out && !aligned16(acc_out)) ||
         (dev_status && !aligned16(dev_status)))
         return HBL_ERR_ALIGNMENT;
-    const Back bk = act_il(act_bits) ? Back::TS : pick(M, K, act_width(act_bits) == 8);
+    const Back bk = act_il(act_bits) ? Back::TS : pick(M, K, act_width(act_bits) == 8, path);
     const size_t need = backend_ws(bk, M, K, N);
     if (need > 0 && (ws == nullptr || ws_bytes < need)) return HBL_ERR_WORKSPACE;
     if (ws && !aligned16(ws)) return HBL_ERR_ALIGNMENT;
@@ -352,10 +361,10 @@ static hbl_status forward_impl(const uint16_t* X, const float* gain, int M, int 
                                const uint32_t* W_packed, const float* alpha, int act_bits,
                                float norm_eps, float quant_eps, uint16_t* Y, uint8_t* ws,
                                size_t ws_bytes, int32_t* dev_status, cudaStream_t s, int sms,
-                               unsigned variant = 0) {
+                               unsigned variant, int path) {
     // Decode batches: one kernel quantises and multiplies (no workspace used);
     // a forced GEMM path keeps the two-kernel forward.
-    if (g_path.load() == 0 && decode_fused_supported(M, K, N, act_bits, variant, sms)) {
+    if (path == HBL_PATH_AUTO && decode_fused_supported(M, K, N, act_bits, variant, sms)) {
         DecodeArgs d{X, gain, M, K, N, W_packed, alpha, act_bits, norm_eps, quant_eps, Y,
                      dev_status};
         return launch_decode_fused(d, s, sms);
@@ -374,7 +383,7 @@ static hbl_status forward_impl(const uint16_t* X, const float* gain, int M, int 
     // Other decode batches of up to 8 tokens at K = 16384: K1 (one byte per
     // code, row-major), then the one-kernel forward's GEMV half, its weight
     // rows streaming into shared memory under K1.
-    if (g_path.load() == 0 && decode_gemv_supported(M, K, N, sms)) {
+    if (path == HBL_PATH_AUTO && decode_gemv_supported(M, K, N, sms)) {
         hbl_status st = launch_norm_fwht_quant(X, gain, M, K, norm_eps, quant_eps,
                                                act_bits == 4 ? 6 : 8, codes, scales, rowsum,
                                                nullptr, s, sms, variant);
@@ -382,7 +391,7 @@ static hbl_status forward_impl(const uint16_t* X, const float* gain, int M, int 
         GemvArgs g{codes, scales, rowsum, M, K, N, W_packed, alpha, Y, dev_status};
         return launch_decode_gemv(g, s, sms);
     }
-    const FwdPlan f = forward_plan(M, K, act_bits);
+    const FwdPlan f = forward_plan(M, K, act_bits, path);
     hbl_status st = launch_norm_fwht_quant(X, gain, M, K, norm_eps, quant_eps, f.k1_mode, codes,
                                            scales, rowsum, nullptr, s, sms, variant);
     if (st != HBL_OK) return st;
@@ -396,8 +405,10 @@ static hbl_status forward_impl(const uint16_t* X, const float* gain, int M, int 
 static hbl_status check_forward(const uint16_t* X, const float* gain, int M, int K, int N,
                                 const uint32_t* W_packed, const float* alpha, int act_bits,
                                 float norm_eps, float quant_eps, const uint16_t* Y, void* ws,
-                                size_t ws_bytes, int32_t* dev_status, int op, bool host_xy) {
+                                size_t ws_bytes, int32_t* dev_status, int op, bool host_xy,
+                                int path) {
     if (act_bits != 4 && act_bits != 8) return HBL_ERR_INVALID_ARG;
+    if (!path_valid(path)) return HBL_ERR_INVALID_ARG;
     if (!finite_nonneg(norm_eps) || !finite_nonneg(quant_eps)) return HBL_ERR_INVALID_ARG;
     if (M < 0 || check_k(K) != HBL_OK || check_n(N) != HBL_OK) return HBL_ERR_SHAPE;
     if (M == 0) return HBL_OK;
@@ -406,7 +417,7 @@ static hbl_status check_forward(const uint16_t* X, const float* gain, int M, int
         !aligned16(W_packed) || !aligned16(alpha) || (dev_status && !aligned16(dev_status)))
         return HBL_ERR_ALIGNMENT;
     size_t need = 0;
-    hbl_workspace_size(op, M, K, N, act_bits, &need);
+    hbl_workspace_size_path(op, M, K, N, act_bits, path, &need);
     if (ws == nullptr || ws_bytes < need) return HBL_ERR_WORKSPACE;
     if (!aligned16(ws)) return HBL_ERR_ALIGNMENT;
     return HBL_OK;
@@ -416,16 +427,26 @@ hbl_status hbl_hbitlinear_forward(const uint16_t* X, const float* gain, int M, i
                                   const uint32_t* W_packed, const float* alpha, int act_bits,
                                   float norm_eps, float quant_eps, uint16_t* Y, void* ws,
                                   size_t ws_bytes, int32_t* dev_status, void* stream) {
+    return hbl_hbitlinear_forward_path(X, gain, M, K, N, W_packed, alpha, act_bits, norm_eps,
+                                       quant_eps, Y, ws, ws_bytes, dev_status, HBL_PATH_AUTO,
+                                       stream);
+}
+
+hbl_status hbl_hbitlinear_forward_path(const uint16_t* X, const float* gain, int M, int K, int N,
+                                       const uint32_t* W_packed, const float* alpha,
+                                       int act_bits, float norm_eps, float quant_eps,
+                                       uint16_t* Y, void* ws, size_t ws_bytes,
+                                       int32_t* dev_status, int path, void* stream) {
     hbl_status st = check_forward(X, gain, M, K, N, W_packed, alpha, act_bits, norm_eps,
                                   quant_eps, Y, ws, ws_bytes, dev_status,
-                                  HBL_OP_HBITLINEAR_FORWARD, false);
+                                  HBL_OP_HBITLINEAR_FORWARD, false, path);
     if (st != HBL_OK) return st;
     if (M == 0) return HBL_OK;
     int sms = 0;
     if ((st = device(&sms)) != HBL_OK) return st;
     return forward_impl(X, gain, M, K, N, W_packed, alpha, act_bits, norm_eps, quant_eps, Y,
                         static_cast<uint8_t*>(ws), ws_bytes, dev_status,
-                        static_cast<cudaStream_t>(stream), sms);
+                        static_cast<cudaStream_t>(stream), sms, 0, path);
 }
 
 namespace {
@@ -470,7 +491,7 @@ hbl_status hbl_hbitlinear_forward_hostio(const uint16_t* X_host, const float* ga
                                          size_t ws_bytes, int32_t* dev_status, void* stream) {
     hbl_status st = check_forward(X_host, gain, M, K, N, W_packed, alpha, act_bits, norm_eps,
                                   quant_eps, Y_host, ws, ws_bytes, dev_status,
-                                  HBL_OP_HBITLINEAR_FORWARD_HOSTIO, true);
+                                  HBL_OP_HBITLINEAR_FORWARD_HOSTIO, true, HBL_PATH_AUTO);
     if (st != HBL_OK) return st;
     if (M == 0) return HBL_OK;
     int sms = 0;
@@ -482,7 +503,7 @@ hbl_status hbl_hbitlinear_forward_hostio(const uint16_t* X_host, const float* ga
     uint16_t* Yd = reinterpret_cast<uint16_t*>(w8 + xb);
     uint8_t* fws = w8 + xb + yb;
     const size_t fws_bytes = ws_bytes - xb - yb;
-    const FwdPlan plan = forward_plan(M, K, act_bits);
+    const FwdPlan plan = forward_plan(M, K, act_bits, HBL_PATH_AUTO);
     // Batches on the TMA-fed GEMM run in row chunks of at least kTmaMinM rows
     // (so every chunk keeps that plan and fits its workspace): chunk c's input
     // copy, its layer and chunk c-1's output copy overlap on three streams.
@@ -495,7 +516,7 @@ hbl_status hbl_hbitlinear_forward_hostio(const uint16_t* X_host, const float* ga
             cudaSuccess)
             return HBL_ERR_CUDA;
         st = forward_impl(Xd, gain, M, K, N, W_packed, alpha, act_bits, norm_eps, quant_eps, Yd,
-                          fws, fws_bytes, dev_status, s, sms);
+                          fws, fws_bytes, dev_status, s, sms, 0, HBL_PATH_AUTO);
         if (st != HBL_OK) return st;
         if (cudaMemcpyAsync(Y_host, Yd, (size_t)M * N * 2, cudaMemcpyDeviceToHost, s) !=
             cudaSuccess)
@@ -592,14 +613,14 @@ hbl_status hbl_bitlinear_forward(const uint16_t* X, const float* gain, int M, in
     if (!flags_valid(flags)) return HBL_ERR_INVALID_ARG;
     hbl_status st = check_forward(X, gain, M, K, N, W_packed, alpha, act_bits, norm_eps,
                                   quant_eps, Y, ws, ws_bytes, dev_status,
-                                  HBL_OP_HBITLINEAR_FORWARD, false);
+                                  HBL_OP_HBITLINEAR_FORWARD, false, HBL_PATH_AUTO);
     if (st != HBL_OK) return st;
     if (M == 0) return HBL_OK;
     int sms = 0;
     if ((st = device(&sms)) != HBL_OK) return st;
     return forward_impl(X, gain, M, K, N, W_packed, alpha, act_bits, norm_eps, quant_eps, Y,
                         static_cast<uint8_t*>(ws), ws_bytes, dev_status,
-                        static_cast<cudaStream_t>(stream), sms, flags);
+                        static_cast<cudaStream_t>(stream), sms, flags, HBL_PATH_AUTO);
 }
 
 hbl_status hbl_rotate_weights(const float* W, const float* signs, int N, int K, float* W_rot,

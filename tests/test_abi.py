@@ -57,17 +57,14 @@ def test_workspace_sizes():
     assert hbl.workspace_size(hbl.OP_PACK_TERNARY, 0, 4096, 100, 0) == 512
     # forward: codes + scales + rowsum, each 256-aligned (tensor-core path: no GEMM scratch)
     M, K, N = 8192, 16384, 4096
-    hbl.set_gemm_path(1)
-    try:
-        got = hbl.workspace_size(hbl.OP_HBITLINEAR_FORWARD, M, K, N, 4)
-        assert got == M * K + 2 * M * 4  # codes one byte each inside the layer (M % 32 == 0)
-        got8 = hbl.workspace_size(hbl.OP_HBITLINEAR_FORWARD, M, K, N, 8)
-        assert got8 == M * K + 2 * M * 4
-        hio = hbl.workspace_size(hbl.OP_HBITLINEAR_FORWARD_HOSTIO, M, K, N, 4)
-        assert hio == got + M * K * 2 + M * N * 2
-        assert hbl.workspace_size(hbl.OP_TERNARY_GEMM, M, K, N, 4) == 0
-    finally:
-        hbl.set_gemm_path(0)
+    ss = hbl.PATH_TC_SS
+    got = hbl.workspace_size(hbl.OP_HBITLINEAR_FORWARD, M, K, N, 4, ss)
+    assert got == M * K + 2 * M * 4  # codes one byte each inside the layer (M % 32 == 0)
+    got8 = hbl.workspace_size(hbl.OP_HBITLINEAR_FORWARD, M, K, N, 8, ss)
+    assert got8 == M * K + 2 * M * 4
+    hio = hbl.workspace_size(hbl.OP_HBITLINEAR_FORWARD_HOSTIO, M, K, N, 4, ss)
+    assert hio == got + M * K * 2 + M * N * 2
+    assert hbl.workspace_size(hbl.OP_TERNARY_GEMM, M, K, N, 4, ss) == 0
     # automatic choice at this batch: the TMA-fed GEMM, plus N*K bytes of expanded weights
     auto = hbl.workspace_size(hbl.OP_HBITLINEAR_FORWARD, M, K, N, 4)
     assert auto == M * K + 2 * M * 4 + N * K
@@ -117,7 +114,15 @@ def test_validation_errors():
     assert pack(A, 16, 100, 1e-5, B, C, D, 1024, NUL) == 2
     assert pack(A, 16, 256, 1e-5, B, C, NUL, 0, NUL) == 5
     assert pack(A, 0, 256, 1e-5, B, C, D, 1024, NUL) == 2
-    assert lib.hbl_set_gemm_path(7) == 1
+    # per-call back-end choice: out-of-range paths are refused
+    sz = ctypes.c_size_t()
+    assert lib.hbl_workspace_size_path(hbl.OP_TERNARY_GEMM, 4, 256, 64, 4, 7, ctypes.byref(sz)) == 1
+    assert lib.hbl_workspace_size_path(hbl.OP_TERNARY_GEMM, 4, 256, 64, 4, -1,
+                                       ctypes.byref(sz)) == 1
+    assert lib.hbl_ternary_gemm_path(A, B, C, 4, 64, 256, D, E, 64, A, NUL, E, 1 << 20, NUL, 9,
+                                     NUL) == 1
+    assert lib.hbl_hbitlinear_forward_path(A, NUL, 64, 256, 64, B, C, 4, 1e-6, 1e-5, D, E,
+                                           1 << 20, NUL, 5, NUL) == 1
 
 
 def test_binding_rejects_non_cuda_tensors():
@@ -164,8 +169,6 @@ def test_expanded_weight_calls_validation():
     assert s8w(A, B, 8, 16, 64, C, D, 64, E, NUL, NUL, NUL) == 2     # K < 128
     assert s8w(A, B, 0x204, 16, 256, C, D, 40, E, NUL, NUL, NUL) == 2
     assert s8w(A, B, 8, 0, 256, C, D, 64, E, NUL, NUL, NUL) == 0
-    assert lib.hbl_set_gemm_path(4) == 0 and lib.hbl_set_gemm_path(0) == 0
-    assert lib.hbl_set_gemm_path(5) == 1
 
 
 def test_selftest_validation():
