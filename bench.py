@@ -213,7 +213,9 @@ def run_reference(args):
     W = inputs.weights("ffn_wdown")
     packed, alpha = oracle.pack_ternary(W)
     threads = os.cpu_count() or 1
-    rows_per_step = min(8192, max(1, threads))
+    # 4 token rows per thread per step (the oracle unpacks the weights once per
+    # call, shared by its threads), so a step times the oracle's arithmetic
+    rows_per_step = min(8192, 4 * max(1, threads))
     for i in range(args.warmup):
         oracle.hbitlinear_forward(X[i * rows_per_step:(i + 1) * rows_per_step], packed, alpha,
                                   BITS, threads=threads)
@@ -236,8 +238,9 @@ def run_reference(args):
                    "l2": "inputs larger than L2 (X 268 MB per step)"},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": used, "kind": "oracle",
                          "sample": "each step: %d token rows of the ffn_wdown workload (full K "
-                                   "and N), scalar C oracle over %d threads" % (rows_per_step,
-                                                                                used)},
+                                   "and N), scalar C oracle over %d threads (%d rows each)"
+                                   % (rows_per_step, used, -(-rows_per_step // used))},
+        "rows_per_step": rows_per_step,
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line))

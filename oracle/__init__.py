@@ -14,7 +14,9 @@ Pins (what fixes each function other than itself; see tests/test_oracle_pins.py)
   sylvester          closed form (-1)^popcount(i&j); H H^T = n I; scipy.linalg.hadamard
   fwht_f32/_f64      dense product with scipy's Hadamard matrix (bit-exact on
                      integer inputs); involution; Parseval; delta / all-ones cases
-  rmsnorm            constant-row closed form; torch.nn.functional.rms_norm in fp64
+  rmsnorm            constant-row closed form; torch.nn.functional.rms_norm in fp64;
+                     a hand-derived row whose squares underflow (each square rounded
+                     to binary32 before the tree: the plain reading of sum x^2)
   norm_fwht          within 1e-6 relative (fp32 vs fp64 composition of the pinned steps)
   quantize_rows      hand-made rows with exact .5 ties; absmax element -> +-127;
                      INT4 range [-8, 7] with -8 reachable; zero row; brute-force
@@ -79,7 +81,9 @@ def _load():
             "oracle_unpack_codes": (I, [P, I, I, P]),
             "oracle_pack_ternary": (I, [P, I, I, F, P, P]),
             "oracle_ternary_gemm_rows": (I, [P, P, I, I, I, P, F, I, I, I, P, P]),
+            "oracle_ternary_gemm_rows_t": (I, [P, P, I, I, I, P, F, I, I, I, P, P]),
             "oracle_hbitlinear_forward_rows": (I, [P, P, I, I, I, P, F, I, F, F, I, I, P]),
+            "oracle_hbitlinear_forward_rows_t": (I, [P, P, I, I, I, P, F, I, F, F, I, I, P]),
             "oracle_norm_transform": (I, [P, P, I, I, F, I, I, P]),
             "oracle_norm_quant": (I, [P, P, I, I, F, F, I, I, I, P, P, P]),
             "oracle_bitlinear_forward_rows": (I, [P, P, I, I, I, P, F, I, F, F, I, I, I, I, P]),
@@ -309,11 +313,12 @@ def ternary_gemm(codes, scales, act_bits, K, packed, alpha, rows=None, threads=N
         return ternary_gemm(sub_c, sub_s, act_bits, K, packed, alpha, None, threads, want_acc)
     Y = np.empty((M, N), dtype=np.uint16)
     acc = np.empty((M, N), dtype=np.int32) if want_acc else None
+    t = unpack_codes(packed, K) if M else None  # once, shared by the threads
 
     def run(r):
         a, b = r
-        _check(lib.oracle_ternary_gemm_rows(_p(codes), _p(scales), act_bits, M, K, _p(packed),
-                                            float(alpha), N, a, b, _p(Y), _p(acc)),
+        _check(lib.oracle_ternary_gemm_rows_t(_p(codes), _p(scales), act_bits, M, K, _p(t),
+                                              float(alpha), N, a, b, _p(Y), _p(acc)),
                "ternary_gemm")
 
     if M:
@@ -335,12 +340,13 @@ def hbitlinear_forward(X_bits, packed, alpha, act_bits, gain=None, norm_eps=1e-6
     g = None if gain is None else _c(gain, np.float32)
     Y = np.empty((M, N), dtype=np.uint16)
     lib = _load()
+    t = unpack_codes(packed, K) if M else None  # once, shared by the threads
 
     def run(r):
         a, b = r
-        _check(lib.oracle_hbitlinear_forward_rows(_p(X_bits), _p(g), M, K, N, _p(packed),
-                                                  float(alpha), act_bits, norm_eps, quant_eps,
-                                                  a, b, _p(Y)), "hbitlinear_forward")
+        _check(lib.oracle_hbitlinear_forward_rows_t(_p(X_bits), _p(g), M, K, N, _p(t),
+                                                    float(alpha), act_bits, norm_eps, quant_eps,
+                                                    a, b, _p(Y)), "hbitlinear_forward")
 
     if M:
         nt = _threads(M, threads)
