@@ -50,9 +50,11 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--kernel-iters", type=int, default=200,
                     help="iterations of the per-kernel timing loops")
-    ap.add_argument("--only", default=None, choices=["forward", "gemm", "quant4", "quant8", "nohad4", "ln4",
-                                                      "rotate", "kv3", "kv4", "kv8", "decode_wo",
-                                                      "decode_wdown"],
+    ap.add_argument("--only", default=None,
+                    choices=["forward", "gemm", "quant4", "quant8", "nohad4", "ln4", "rotate",
+                             "kv3", "kv4", "kv8", "decode_wo", "decode_wdown", "decode_wdown_t32",
+                             "decode_wo_t32", "gemv_rows", "gemv_splitk", "pack", "expand",
+                             "int8_probe"],
                     help="run only this case (a few launches, for profiler captures); prints a "
                          "short JSON line, not the benchmark line")
     return ap.parse_args()
@@ -334,6 +336,12 @@ def run_hbl(args):
     t_k2 = statistics.mean(e[2].elapsed_time(e[3]) for e in evs) * 1e-3
     del Ws
 
+    # ---- dense INT8 tensor-core rate of this GPU (the GEMM's roofline denominator)
+    probe_mmas = 1 << 15
+    probe_tops, probe_st = hbl.measure_int8_tensor_peak(n_sms, probe_mmas, reps=5)
+    int8_probe = {"tops": probe_tops, "mmas_per_cta": probe_mmas, "ctas": n_sms,
+                  "status": probe_st}
+
     # ---- quant workload: 8192 x 4096, a4 and a8, 4 rotating inputs (256 MB > L2)
     qX = [torch.from_numpy(inputs.activations("quant", seed=s).view(np.int16)).view(
         torch.bfloat16).to(dev) for s in range(4)]
@@ -493,15 +501,19 @@ def run_hbl(args):
     ops = 2.0 * M_TOK * N_OUT * K_IN
     if t_k2 >= t_k1:
         achieved = ops / t_k2 / 1e12
-        # the GEMM is timed in a sub-second loop at full clocks: the burst figure
-        peak = 2.0 * pk["bf16_tflops"]
+        # the GEMM is timed in a sub-second loop at full clocks: the burst rate
+        # of the same MMA instruction measured by the probe on this GPU
+        peak = int8_probe["tops"]
         roof = {"bound": "tensor",
                 "kernel": "gemm_tma (TMA-fed tcgen05 kind::i8, accumulators in TMEM)",
                 "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-                "peak_note": "int8 dense = %s burst bf16 %.1f TFLOP/s x 2 (nominal int8:bf16 "
-                             "ratio); against the sustained figure (%.1f x 2) frac would be %.2f"
-                             % (pk["source"], pk["bf16_tflops"], pk["bf16_tflops_sustained"],
-                                achieved / (2.0 * pk["bf16_tflops_sustained"])),
+                "peak_note": "dense INT8 (TOPS) measured on this GPU by hbl_probe_tc_int8: %d "
+                             "SMs x %d back-to-back tcgen05.mma kind::i8 128x256x32 from shared "
+                             "memory, best of 5, CUDA events; for context 2 x %s burst bf16 = "
+                             "%.1f (frac %.2f) and the 4500 TOPS datasheet figure (frac %.2f)"
+                             % (n_sms, int8_probe["mmas_per_cta"], pk["source"],
+                                2.0 * pk["bf16_tflops"], achieved / (2.0 * pk["bf16_tflops"]),
+                                achieved / 4500.0),
                 "traffic": recorded_traffic("gemm_tma_a4_ffn_wdown",
                                             source_hash("k2c_gemm_tma.cu")),
                 "us_per_launch": t_k2 * 1e6}
@@ -540,7 +552,8 @@ def run_hbl(args):
         "gpu_launches": 3 * args.steps,  # K1, weight expansion, GEMM per forward
         "clocks": clocks,
         "device_status": st,
-        "peaks": pk,
+        "peaks": dict(pk, int8_tops_probe=probe_tops),
+        "int8_probe": int8_probe,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import oracle
@@ -584,14 +597,38 @@ def run_only(args):
         QX = torch.from_numpy(inputs.qkv_states().view(np.int16)).view(torch.bfloat16).to(dev)
         kb = int(args.only[2:])
         fn = lambda: hbl.kv_quant(QX, kb)
-    elif args.only.startswith("decode"):  # one token through W_o or W_down
-        Kd = 4096 if args.only == "decode_wo" else 16384
-        Xt = torch.from_numpy(inputs.activations(args.only, M=1, K=Kd, seed=1).view(
+    elif args.only.startswith("decode"):  # 1 (or 32) tokens through W_o or W_down
+        Kd = 4096 if args.only.startswith("decode_wo") else 16384
+        T = 32 if args.only.endswith("_t32") else 1
+        name = "decode_wo" if Kd == 4096 else "decode_wdown"
+        Xt = torch.from_numpy(inputs.activations(name, M=T, K=Kd, seed=1).view(
             np.int16)).view(torch.bfloat16).to(dev)
         pd, ad = hbl.pack_ternary(torch.from_numpy(inputs.latent_weights(N_OUT, Kd, seed=7)).to(dev))
-        wsd = torch.empty(max(16, hbl.workspace_size(hbl.OP_HBITLINEAR_FORWARD, 1, Kd, N_OUT,
+        wsd = torch.empty(max(16, hbl.workspace_size(hbl.OP_HBITLINEAR_FORWARD, T, Kd, N_OUT,
                                                      BITS)), dtype=torch.uint8, device=dev)
         fn = lambda: hbl.hbitlinear_forward(Xt, pd, ad, BITS, ws=wsd)
+    elif args.only in ("gemv_rows", "gemv_splitk"):
+        # the CUDA-core GEMVs on 8 tokens: one weight row per warp (K = 16384),
+        # split-K with a reduction kernel (K = 1024); N = 4096
+        Kd = 16384 if args.only == "gemv_rows" else 1024
+        Xt = torch.from_numpy(inputs.activations("decode_wdown", M=8, K=Kd, seed=1).view(
+            np.int16)).view(torch.bfloat16).to(dev)
+        pd, ad = hbl.pack_ternary(torch.from_numpy(inputs.latent_weights(N_OUT, Kd, seed=7)).to(dev))
+        codes, scales, rowsum = hbl.norm_fwht_quant(Xt, BITS)
+        fn = lambda: hbl.ternary_gemm(codes, scales, rowsum, BITS, Kd, pd, ad, path=hbl.PATH_GEMV)
+    elif args.only in ("pack", "expand"):
+        Wd = torch.from_numpy(inputs.weights("ffn_wdown")).to(dev)
+        pd, ad = hbl.pack_ternary(Wd)
+        if args.only == "pack":
+            fn = lambda: hbl.pack_ternary(Wd)
+        else:
+            del Wd
+            Ws = torch.empty((N_OUT, K_IN), dtype=torch.int8, device=dev)
+            fn = lambda: hbl.expand_ternary(pd, K_IN, out=Ws)
+    elif args.only == "int8_probe":
+        st = hbl.new_status(dev)
+        n = torch.cuda.get_device_properties(dev).multi_processor_count
+        fn = lambda: hbl.probe_tc_int8(n, 1 << 12, st)
     else:
         X = torch.from_numpy(inputs.activations("ffn_wdown").view(np.int16)).view(
             torch.bfloat16).to(dev)

@@ -40,7 +40,8 @@ EXPORTS = ("hbl_status_string", "hbl_version", "hbl_workspace_size", "hbl_worksp
            "hbl_hbitlinear_forward_hostio",
            "hbl_ternary_gemv_noalloc", "hbl_norm_transform", "hbl_norm_quant",
            "hbl_bitlinear_forward", "hbl_rotate_weights", "hbl_kv_quant",
-           "hbl_expand_ternary", "hbl_ternary_gemm_s8w", "hbl_selftest_bounded_wait")
+           "hbl_expand_ternary", "hbl_ternary_gemm_s8w", "hbl_selftest_bounded_wait",
+           "hbl_probe_tc_int8")
 
 _lib = None
 
@@ -104,6 +105,8 @@ def lib():
         L.hbl_ternary_gemm_s8w.argtypes = [P, P, I, I, I, P, P, I, P, P, P, P]
         L.hbl_selftest_bounded_wait.restype = I
         L.hbl_selftest_bounded_wait.argtypes = [I, I, P, P]
+        L.hbl_probe_tc_int8.restype = I
+        L.hbl_probe_tc_int8.argtypes = [I, I, P, P]
         _lib = L
     return _lib
 
@@ -397,3 +400,34 @@ def selftest_bounded_wait(arrive, timeout_us, status):
     """hbl_selftest_bounded_wait: the bounded-wait failure path on one probe kernel."""
     _check(lib().hbl_selftest_bounded_wait(int(bool(arrive)), int(timeout_us), _ptr(status),
                                            _stream()), "hbl_selftest_bounded_wait")
+
+
+def probe_tc_int8(ctas, mmas_per_cta, status):
+    """hbl_probe_tc_int8: back-to-back 128 x 256 x 32 kind::i8 MMAs from shared
+    memory on `ctas` SMs (time it with events on the current stream)."""
+    _check(lib().hbl_probe_tc_int8(int(ctas), int(mmas_per_cta), _ptr(status), _stream()),
+           "hbl_probe_tc_int8")
+
+
+OPS_PER_PROBE_MMA = 2 * 128 * 256 * 32
+
+
+def measure_int8_tensor_peak(ctas, mmas_per_cta=1 << 15, reps=5):
+    """Best-of-reps dense INT8 rate (TOPS) from the probe, with its launch timed
+    by CUDA events on the current stream; returns (tops, status word)."""
+    import torch
+
+    status = new_status(torch.device("cuda", torch.cuda.current_device()))
+    probe_tc_int8(ctas, 64, status)  # warm-up (shared-memory attribute, clocks)
+    torch.cuda.synchronize()
+    best = None
+    for _ in range(reps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        probe_tc_int8(ctas, mmas_per_cta, status)
+        b.record()
+        torch.cuda.synchronize()
+        t = a.elapsed_time(b) * 1e-3
+        best = t if best is None else min(best, t)
+    tops = ctas * mmas_per_cta * OPS_PER_PROBE_MMA / best / 1e12
+    return tops, int(status[0].item())

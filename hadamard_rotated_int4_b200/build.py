@@ -7,6 +7,7 @@ one IEEE round-to-nearest operation.  Objects are linked into one shared
 library with the CUDA runtime linked statically.
 """
 import os
+import re
 import subprocess
 import sys
 from concurrent.futures import ThreadPoolExecutor
@@ -34,14 +35,41 @@ def _deps_mtime():
     return max(os.path.getmtime(f) for f in files)
 
 
+_INCLUDE = re.compile(r'^\s*#\s*include\s+"([^"]+)"', re.M)
+
+
+def _src_mtime(path, seen=None):
+    """Latest mtime of a source and the local headers it includes (recursively)."""
+    seen = set() if seen is None else seen
+    if path in seen or not os.path.exists(path):
+        return 0.0
+    seen.add(path)
+    t = os.path.getmtime(path)
+    with open(path, errors="replace") as f:
+        for name in _INCLUDE.findall(f.read()):
+            for d in (os.path.dirname(path), CSRC, INC):
+                cand = os.path.join(d, name)
+                if os.path.exists(cand):
+                    t = max(t, _src_mtime(cand, seen))
+                    break
+    return t
+
+
 def build(force=False, verbose=False, ptxas_info=False):
     if not force and os.path.exists(OUT) and os.path.getmtime(OUT) >= _deps_mtime():
         return OUT
     os.makedirs(BUILD, exist_ok=True)
     extra = ["-Xptxas", "-v"] if ptxas_info else []
+    flags_key = " ".join(FLAGS)
+    stamp = os.path.join(BUILD, "flags.txt")
+    same_flags = os.path.exists(stamp) and open(stamp).read() == flags_key
 
     def compile_one(src):
         obj = os.path.join(BUILD, os.path.basename(src) + ".o")
+        # objects newer than their source and its headers (same flags) are kept
+        if (not force and not ptxas_info and same_flags and os.path.exists(obj) and
+                os.path.getmtime(obj) >= _src_mtime(src)):
+            return obj
         cmd = [NVCC] + FLAGS + extra + ["-c", src, "-o", obj]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
@@ -52,6 +80,8 @@ def build(force=False, verbose=False, ptxas_info=False):
 
     with ThreadPoolExecutor(max(1, min(8, os.cpu_count() or 1))) as ex:
         objs = list(ex.map(compile_one, sources()))
+    with open(stamp, "w") as f:
+        f.write(flags_key)
     tmp = OUT + ".tmp%d" % os.getpid()
     cmd = [NVCC, "-shared", "-gencode", "arch=compute_100a,code=sm_100a", "-cudart", "static",
            "-o", tmp] + objs

@@ -696,6 +696,17 @@ hbl_status hbl_selftest_bounded_wait(int arrive, int timeout_us, int32_t* dev_st
                                      static_cast<cudaStream_t>(stream));
 }
 
+hbl_status hbl_probe_tc_int8(int ctas, int mmas_per_cta, int32_t* dev_status, void* stream) {
+    if (dev_status == nullptr) return HBL_ERR_INVALID_ARG;
+    if (ctas < 1 || ctas > 4096 || mmas_per_cta < 1 || mmas_per_cta > (1 << 22))
+        return HBL_ERR_INVALID_ARG;
+    if (!aligned16(dev_status)) return HBL_ERR_ALIGNMENT;
+    int sms = 0;
+    hbl_status st = device(&sms);
+    if (st != HBL_OK) return st;
+    return launch_tc_int8_probe(ctas, mmas_per_cta, dev_status, static_cast<cudaStream_t>(stream));
+}
+
 // Allocation-free ternary GEMV: the CUDA-core split-K path with its partial
 // sums in the library's fixed 2 MiB device array instead of caller workspace.
 hbl_status hbl_ternary_gemv_noalloc(const void* codes, const float* scales,

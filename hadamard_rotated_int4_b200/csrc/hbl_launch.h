@@ -90,6 +90,9 @@ hbl_status launch_kv_quant(const uint16_t* X, int64_t rows, int D, int bits, flo
 hbl_status launch_bounded_wait_probe(int arrive, int timeout_us, int32_t* status,
                                      cudaStream_t stream);
 
+// Dense INT8 tensor-core rate probe (see k9_tc_probe.cu).
+hbl_status launch_tc_int8_probe(int ctas, int mmas_per_cta, int32_t* status, cudaStream_t stream);
+
 // K0: absmean ternarisation + 2-bit packing (K a power of two).
 size_t pack_ternary_workspace(int N, int K);
 hbl_status launch_pack_ternary(const float* W, int N, int K, float eps, uint32_t* W_packed,

@@ -344,6 +344,20 @@ HBL_API hbl_status hbl_ternary_gemm_s8w(const void* codes, const float* scales, 
 HBL_API hbl_status hbl_selftest_bounded_wait(int arrive, int timeout_us, int32_t* dev_status,
                                              void* stream);
 
+/* Dense INT8 tensor-core rate probe (no counterpart on the pages; it measures
+ * the denominator of the ternary GEMM's roofline on the GPU at hand).  Launches
+ * `ctas` CTAs (at most one per SM); each zeroes a 128 x 128-byte and a
+ * 256 x 128-byte operand tile in its shared memory and one thread issues
+ * `mmas_per_cta` back-to-back tcgen05.mma.cta_group::1.kind::i8 instructions of
+ * shape M = 128, N = 256, K = 32 (2 * 128 * 256 * 32 integer operations each)
+ * into one TMEM accumulator, then waits (bounded) for them.  No global memory
+ * is touched except dev_status.  Time the launch with events on `stream`: the
+ * rate is ctas * mmas_per_cta * 2097152 operations over that time.
+ * ctas in [1, 4096]; mmas_per_cta in [1, 2^22]; dev_status: device int32
+ * (required; HBL_ERR_TIMEOUT if the MMAs did not finish within 2 s). */
+HBL_API hbl_status hbl_probe_tc_int8(int ctas, int mmas_per_cta, int32_t* dev_status,
+                                     void* stream);
+
 /* Allocation-free ternary GEMV (no counterpart on the BitNet v2 pages; it is a
  * deployment aid).  Same arguments, layouts and results as hbl_ternary_gemm
  * run on its CUDA-core split-K path, but without a workspace argument: the

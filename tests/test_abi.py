@@ -173,6 +173,11 @@ def test_expanded_weight_calls_validation():
 
 def test_selftest_validation():
     lib = hbl.lib()
+    assert lib.hbl_probe_tc_int8(148, 100, NUL, NUL) == 1
+    assert lib.hbl_probe_tc_int8(0, 100, A, NUL) == 1
+    assert lib.hbl_probe_tc_int8(148, 0, A, NUL) == 1
+    assert lib.hbl_probe_tc_int8(148, (1 << 22) + 1, A, NUL) == 1
+    assert lib.hbl_probe_tc_int8(148, 100, MIS, NUL) == 3
     assert lib.hbl_selftest_bounded_wait(0, 100, NUL, NUL) == 1
     assert lib.hbl_selftest_bounded_wait(0, 0, A, NUL) == 1
     assert lib.hbl_selftest_bounded_wait(0, 100, MIS, NUL) == 3

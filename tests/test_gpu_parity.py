@@ -557,6 +557,16 @@ def test_hostio_chunked_pipeline(M, bits):
     assert np.array_equal(Yh.view(torch.int16).numpy().view(np.uint16)[rows], want)
 
 
+def test_int8_tensor_probe_runs_and_is_plausible():
+    # the dense INT8 tensor-core probe (the GEMM roofline's denominator):
+    # finishes within its bounded wait and measures a rate between the GEMM's
+    # own measured rate (about 3 POPS) and well above the datasheet figure
+    n = torch.cuda.get_device_properties(0).multi_processor_count
+    tops, st = hbl.measure_int8_tensor_peak(n, mmas_per_cta=1 << 13, reps=3)
+    assert st == 0
+    assert 1000.0 < tops < 6000.0
+
+
 def test_status_word_stays_clear():
     st = hbl.new_status(DEV)
     X = to_dev_bf16(acts(200, 2048, seed=1))
