@@ -608,10 +608,11 @@ def run_only(args):
                                                      BITS)), dtype=torch.uint8, device=dev)
         fn = lambda: hbl.hbitlinear_forward(Xt, pd, ad, BITS, ws=wsd)
     elif args.only in ("gemv_rows", "gemv_splitk"):
-        # the CUDA-core GEMVs on 8 tokens: one weight row per warp (K = 16384),
-        # split-K with a reduction kernel (K = 1024); N = 4096
+        # the CUDA-core GEMVs: one weight row per warp (4 tokens, K = 16384),
+        # split-K with a reduction kernel (8 tokens, K = 1024); N = 4096
         Kd = 16384 if args.only == "gemv_rows" else 1024
-        Xt = torch.from_numpy(inputs.activations("decode_wdown", M=8, K=Kd, seed=1).view(
+        Mt = 4 if args.only == "gemv_rows" else 8
+        Xt = torch.from_numpy(inputs.activations("decode_wdown", M=Mt, K=Kd, seed=1).view(
             np.int16)).view(torch.bfloat16).to(dev)
         pd, ad = hbl.pack_ternary(torch.from_numpy(inputs.latent_weights(N_OUT, Kd, seed=7)).to(dev))
         codes, scales, rowsum = hbl.norm_fwht_quant(Xt, BITS)

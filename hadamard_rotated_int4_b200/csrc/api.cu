@@ -69,7 +69,7 @@ int act_width(int a) { return a == 4 ? 4 : 8; }
 int codes_row_bytes(int K, int act_bits) { return act_width(act_bits) == 4 ? K / 2 : K; }
 
 // Ternary-GEMM back ends.
-enum class Back { GEMV, SS, TS, TMA };
+enum class Back { GEMV, SS, TS, TMA, DEC };
 
 // The GEMV back end uses the row GEMV when K allows it and the tokens fit one
 // launch; otherwise the split-K GEMV (8-token chunks).
@@ -78,7 +78,14 @@ bool rows_gemv(int64_t M, int K) { return gemv_rows_supported(K) && M <= gemv_ro
 // Batches above this many tokens take the TMA-fed kernel (automatic choice).
 constexpr int64_t kTmaMinM = 257;
 
-bool path_valid(int path) { return path >= HBL_PATH_AUTO && path <= HBL_PATH_TC_TMA; }
+bool path_valid(int path) { return path >= HBL_PATH_AUTO && path <= HBL_PATH_TC_DECODE; }
+
+// Shapes the decode-batch tensor-core kernel takes (one-byte codes); whether a
+// launch plan fits the device is checked again at launch, which falls back to
+// the TMEM-activation kernel (its workspace is reserved for that).
+bool dec_shape(int64_t M, int K) { return M >= 1 && M <= decode_mma_max_m() && K >= 128; }
+// Automatic choice: batches of kDecMinM..kDecMaxM tokens take it.
+constexpr int64_t kDecMinM = 5, kDecMaxM = 128;
 
 // The back end for M tokens under `path` (HBL_PATH_*); `bytes`: the codes are
 // (or can be made) one byte each.
@@ -87,10 +94,12 @@ Back pick(int64_t M, int K, bool bytes, int path) {
     if (path == 2) return Back::GEMV;
     if (path == 3) return Back::TS;
     if (path == 4) return (bytes && K >= 128) ? Back::TMA : Back::TS;
+    if (path == 5) return (bytes && dec_shape(M, K)) ? Back::DEC : Back::TS;
     // CUDA cores for a few tokens: the row GEMV where it takes the batch in one
     // launch; past that at K >= 16384 the tensor-core kernel is faster than the
     // split-K GEMV
     if (M <= gemv_max_m() && (rows_gemv(M, K) || K < 16384)) return Back::GEMV;
+    if (bytes && dec_shape(M, K) && M >= kDecMinM && M <= kDecMaxM) return Back::DEC;
     if (bytes && K >= 128 && M >= kTmaMinM) return Back::TMA;
     return Back::TS;
 }
@@ -99,6 +108,7 @@ size_t backend_ws(Back b, int64_t M, int K, int N) {
     switch (b) {
         case Back::SS: return 0;
         case Back::TS: return gemm_ts_workspace(M, K, N);
+        case Back::DEC: return gemm_ts_workspace(M, K, N);  // its fallback's
         case Back::TMA: return gemm_tma_workspace(K, N);
         case Back::GEMV:
         default: {
@@ -118,6 +128,11 @@ hbl_status run_gemm(Back b, const GemmArgs& a, void* ws, size_t ws_bytes, cudaSt
     if (b == Back::SS) return launch_gemm_tc(a, s, sms);
     if (b == Back::TS) return launch_gemm_ts(a, ws, ws_bytes, s, sms);
     if (b == Back::TMA) return launch_gemm_tma(a, ws, ws_bytes, s, sms);
+    if (b == Back::DEC) {
+        if (!a.interleaved && a.act_bits == 8 && decode_mma_supported(a.M, a.K, a.N, sms))
+            return launch_decode_mma(a, s, sms);
+        return launch_gemm_ts(a, ws, ws_bytes, s, sms);
+    }
     if (rows_gemv(a.M, a.K)) {  // row GEMV in chunks of up to gemv_rows_max_m(K) tokens
         const int64_t step = gemv_rows_max_m(a.K);
         for (int64_t r0 = 0; r0 < a.M; r0 += step) {
@@ -160,7 +175,7 @@ FwdPlan forward_plan(int64_t M, int K, int act_bits, int path) {
     FwdPlan f;
     f.back = pick(M, K, true, path);
     f.interleaved = f.back == Back::TS;
-    if (f.back == Back::TMA) {
+    if (f.back == Back::TMA || f.back == Back::DEC) {
         f.k1_mode = act_bits == 4 ? 6 : 8;
         f.gemm_act_bits = 8;
     } else if (f.back == Back::TS) {

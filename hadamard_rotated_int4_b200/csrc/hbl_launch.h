@@ -157,6 +157,17 @@ size_t gemv_workspace(int64_t M, int K, int N, int num_sms);
 hbl_status launch_gemv(const GemmArgs& a, void* ws, size_t ws_bytes, cudaStream_t stream,
                        int num_sms);
 
+// K7: tensor-core GEMM for decode batches (1..decode_mma_max_m() tokens): the
+// weights as the MMA's A operand in TMEM (128 weight rows per CTA), the
+// tokens as B (TMA from one-byte row-major codes), K split over a thread-block
+// cluster and reduced through distributed shared memory.  Codes one byte per
+// code (a.act_bits 8), row-major; launched as a programmatic dependent (the
+// weight rows stream into shared memory before the dependency wait).  No
+// workspace.  decode_mma_supported: the shape has a plan that fits.
+int decode_mma_max_m();
+bool decode_mma_supported(int64_t M, int K, int N, int num_sms);
+hbl_status launch_decode_mma(const GemmArgs& a, cudaStream_t stream, int num_sms);
+
 // Fixed scratch of the allocation-free GEMV entry point (file-scope device array).
 size_t gemv_noalloc_scratch_bytes();
 void* gemv_noalloc_scratch(int dev);

@@ -1,0 +1,647 @@
+// k7_decode_mma.cu -- ternary-weight GEMM for decode batches (9 to 128
+// tokens) on the sm_100a tensor cores, bound by the stream of packed weights.
+//
+// Computes (BitNet v2 write-up, 0755model.com, section "H-BitLinear": the
+// ternary matmul of the per-token quantised activations, rescaled by the
+// weight and activation scales)
+//   acc[m][n] = sum_k q[m][k] * t[n][k]     (exact, int32)
+//   Y[m][n]   = bf16_rne((float)acc * (alpha * s[m]))
+// for codes q one byte each, row-major [M x K] (INT8, or INT4 values in
+// [-8, 7]), and the library's 2-bit packed weights.
+//
+// The roles of the operands are swapped against the large-batch GEMM: the
+// weights are the MMA's A operand (M = 128 weight rows per CTA, read from
+// tensor memory) and the tokens its B operand (N = NT = the batch rounded up to
+// 16, 32, 64 or 128, from shared memory), so a decode batch of 32 tokens wastes
+// no tensor-core rows.  Per CTA:
+//   - before the dependency wait (the weights are not the previous kernel's
+//     output), one warp starts 1-D bulk copies of the CTA's 128 weight rows,
+//     its K slice only, into shared memory (rows padded by 16 bytes, so the
+//     converters' 16-byte reads are free of bank conflicts), on G mbarriers
+//     of K groups: the whole weight stream runs under the quantiser kernel;
+//   - one thread TMA-loads the tokens' codes for each 128-byte K stage into a
+//     4-stage ring (SWIZZLE_128B: the K-major layout the MMA descriptor names;
+//     rows past M are zero-filled);
+//   - eight converter warps unpack each stage's 2-bit weights in registers
+//     ((w >> 2m) & 0x03030303 is the codes of weights 4m..4m+3 as bytes, in
+//     natural order) and store them with tcgen05.st into a 4-stage ring of A
+//     tiles in TMEM (32 columns = 128 bytes per row and stage);
+//   - one thread issues tcgen05.mma.cta_group::1.kind::i8 (A u8 from TMEM,
+//     B s8 from shared memory, D s32 in TMEM) and commits each stage back.
+// The weights enter as the unsigned code c = t + 1, so the result carries
+// sum_k q*c = acc + rowsum[m]; rowsum is subtracted once in the epilogue.
+//
+// K is split over the CS CTAs of a thread-block cluster (CS = 1, 2, 4 or 8,
+// chosen so that ceil(N/128) * CS CTAs fill the SMs in one wave).  Each CTA
+// leaves its int32 partials [NT x 128] in its own shared memory; after a
+// cluster barrier CTA c sums rows [c * 128/CS, (c + 1) * 128/CS) over the CS
+// CTAs through distributed shared memory (integer sums: exact in any order),
+// subtracts rowsum and writes bf16 Y.  No workspace, no second kernel.
+//
+// TMEM: 256 columns per CTA (D in [0, NT), the A ring in [128, 256)); the
+// dynamic shared memory is at least 80 KB, so no more than two CTAs share an
+// SM and their allocations always fit the SM's 512 columns.  Every mbarrier
+// wait is bounded by the global timer; on expiry the kernel records
+// HBL_ERR_TIMEOUT, stops issuing, lets its own copies and MMAs land (bounded
+// waits again), still takes part in both cluster barriers (every thread of
+// every CTA reaches them after bounded work) and frees its TMEM.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "hbl_internal.cuh"
+#include "hbl_launch.h"
+
+namespace hbl {
+namespace k7 {
+
+constexpr int kRows = 128;  // weight rows per CTA (MMA M, TMEM lanes)
+constexpr int BK = 128;     // K bytes per stage
+constexpr int S = 4;        // stages of the A (TMEM) and B (shared memory) rings
+constexpr int kConvWarps = 8;
+constexpr int kThreads = 32 * (2 + kConvWarps);
+constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kACol = 128;  // first TMEM column of the A ring
+constexpr int kMaxGroups = 8;
+constexpr int kMinSmem = 80 * 1024;  // caps residency at two CTAs per SM
+constexpr uint64_t kTimeoutNs = 2000000000ull;
+
+// kind::i8: D s32 (bits 4-5 = 2), A u8 (bits 7-9 = 0), B s8 (bits 10-12 = 1),
+// both K-major, N >> 3 at bit 17, M >> 4 at bit 24.
+template <int NT>
+__host__ __device__ constexpr uint32_t idesc() {
+    return (2u << 4) | (0u << 7) | (1u << 10) | ((uint32_t)(NT >> 3) << 17) |
+           ((uint32_t)(kRows >> 4) << 24);
+}
+
+struct Params {
+    int M, K, N;
+    int Kc;        // K per CTA (K / cluster size), a multiple of BK
+    int G;         // weight copy groups per row (Kc / 4 / G bytes each)
+    int rs;        // bytes per weight row in shared memory (Kc / 4 + 16)
+    uint32_t b_off;  // offset of the B ring from the 1024-aligned base
+    uint32_t bar_off;
+    const uint32_t* W;
+    const float* scales;
+    const int32_t* rowsum;
+    const float* alpha;
+    uint16_t* Y;
+    int32_t* acc_out;
+    int32_t* status;
+    int early_weights;  // launched after the kernel that writes the codes: the
+                        // weight copies start before the dependency wait
+};
+
+__device__ __forceinline__ bool mbar_wait(uint32_t a, uint32_t parity) {
+    return mbar_wait_bounded<false>(a, parity, kTimeoutNs);
+}
+__device__ __forceinline__ bool mbar_wait_sleep(uint32_t a, uint32_t parity) {
+    return mbar_wait_bounded<true>(a, parity, kTimeoutNs);
+}
+// Warp-uniform bounded wait: lane 0 waits, every lane gets its verdict.
+__device__ __forceinline__ bool warp_wait(uint32_t a, uint32_t parity) {
+    bool ok = true;
+    if ((threadIdx.x & 31) == 0) ok = mbar_wait_sleep(a, parity);
+    return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t a, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(a), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+// K-major, 128-byte-swizzled shared-memory matrix descriptor (8-row atoms of
+// 1024 bytes, SBO = 1024), version 1.
+__device__ __forceinline__ uint64_t sdesc(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)1 << 16;
+    d |= (uint64_t)(1024 >> 4) << 32;
+    d |= (uint64_t)1 << 46;
+    d |= (uint64_t)2 << 61;
+    return d;
+}
+template <int NT>
+__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
+                                       uint32_t accum) {
+    asm volatile(
+        "{\n.reg .pred p;\n"
+        "setp.ne.b32 p, %3, 0;\n"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %4, p;\n}\n" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(bdesc), "r"(accum), "r"(idesc<NT>())
+        : "memory");
+}
+__device__ __forceinline__ void mma_commit(uint32_t mbar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(mbar)
+        : "memory");
+}
+// 2-D tiled TMA load (no multicast) of box (x, y) into this CTA's shared memory.
+__device__ __forceinline__ void tma_load(uint32_t dst, const CUtensorMap* map, int x, int y,
+                                         uint32_t mbar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes "
+        "[%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(mbar)
+        : "memory");
+}
+// 1-D bulk copy (no multicast) global -> this CTA's shared memory.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
+                                          uint32_t mbar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            dst),
+        "l"(src), "r"(bytes), "r"(mbar)
+        : "memory");
+}
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ uint32_t cluster_size() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
+    return r;
+}
+// Every thread of every CTA of the cluster: prior shared-memory writes are
+// visible to the cluster after it.
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release;" ::: "memory");
+    asm volatile("barrier.cluster.wait.acquire;" ::: "memory");
+}
+__device__ __forceinline__ uint32_t mapa(uint32_t saddr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ uint4 ld_cluster_v4(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared::cluster.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(addr)
+                 : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+        "r"(r[15])
+        : "memory");
+}
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t* v) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+          "=r"(v[7])
+        : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t* v) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+        "%11, %12, %13, %14, %15}, [%16];"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+          "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]),
+          "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+        : "r"(taddr));
+}
+
+template <int NT>
+__global__ void __launch_bounds__(kThreads, 1)
+    decode_mma_kernel(const __grid_constant__ CUtensorMap tmB, Params p) {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_s = smem_addr(smem_raw);
+    const uint32_t base_s = (raw_s + 1023u) & ~1023u;
+    uint8_t* base = smem_raw + (base_s - raw_s);
+    const uint32_t w_s = base_s;              // weights, later the partial sums
+    const uint32_t b_s = base_s + p.b_off;    // B ring: S x NT x 128 bytes
+    const uint32_t bar_s = base_s + p.bar_off;
+    auto full_b = [&](int s) { return bar_s + 8u * s; };
+    auto full_a = [&](int s) { return bar_s + 8u * (S + s); };
+    auto empty = [&](int s) { return bar_s + 8u * (2 * S + s); };
+    auto wbar = [&](int g) { return bar_s + 8u * (3 * S + g); };
+    const uint32_t acc_bar = bar_s + 8u * (3 * S + kMaxGroups);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + p.bar_off + 8 * (3 * S + kMaxGroups + 1));
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t crank = cluster_rank(), csize = cluster_size();
+    const int n0 = (int)blockIdx.y * kRows;
+    const int k0 = (int)blockIdx.x * p.Kc;  // blockIdx.x == cluster rank (cluster along x)
+    const int nkb = p.Kc / BK;
+    const int rows = min(kRows, p.N - n0);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init_count(full_b(s), 1);
+            mbar_init_count(full_a(s), kConvWarps);
+            mbar_init_count(empty(s), 1);
+        }
+        for (int g = 0; g < kMaxGroups; ++g) mbar_init_count(wbar(g), 1);
+        mbar_init_count(acc_bar, 1);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmB)) : "memory");
+    }
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_addr(tmem_slot)),
+                     "r"(kTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    __syncthreads();  // barriers initialised
+
+    // ---- the CTA's weight rows (its K slice) into shared memory: the weights
+    // are not the previous kernel's output, so this runs before the dependency
+    // wait, under that kernel
+    const uint32_t cbytes = (uint32_t)(p.Kc / 4 / p.G);
+    auto load_weights = [&] {
+        if (lane == 0)
+            for (int g = 0; g < p.G; ++g) mbar_expect_tx(wbar(g), (uint32_t)rows * cbytes);
+        __syncwarp();
+        for (int r = lane; r < rows; r += 32) {
+            const uint8_t* src =
+                reinterpret_cast<const uint8_t*>(p.W + (int64_t)(n0 + r) * (p.K / 16)) + k0 / 4;
+            for (int g = 0; g < p.G; ++g)
+                bulk_load(w_s + (uint32_t)(r * p.rs) + g * cbytes, src + g * cbytes, cbytes,
+                          wbar(g));
+        }
+    };
+    if (warp == 1 && p.early_weights) load_weights();
+    pdl_wait();  // the codes, scales and row sums come from the previous kernel
+    if (warp == 1 && !p.early_weights) load_weights();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ---------------- MMA issuer (one thread)
+        if (lane == 0) {
+            bool ok = true;
+            for (int kb = 0; kb < nkb; ++kb) {
+                const int s = kb % S;
+                const uint32_t ph = (uint32_t)((kb / S) & 1);
+                if (!mbar_wait(full_a(s), ph) || !mbar_wait(full_b(s), ph) || *abort_flag) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t sb = b_s + (uint32_t)(s * NT * BK);
+#pragma unroll
+                for (int k = 0; k < BK / 32; ++k)
+                    mma_ts<NT>(tmem, tmem + kACol + 32u * s + 8u * k, sdesc(sb + 32 * k),
+                               (kb | k) != 0 ? 1u : 0u);
+                mma_commit(empty(s));
+            }
+            if (!ok) {
+                *abort_flag = 1;
+                report_status(p.status, HBL_ERR_TIMEOUT);
+            }
+            // arrives once every MMA issued above has completed; this thread
+            // also waits for it, so no MMA is in flight when TMEM is freed
+            mma_commit(acc_bar);
+            if (!mbar_wait_sleep(acc_bar, 0)) report_status(p.status, HBL_ERR_TIMEOUT);
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ---------------- TMA producer of the token stages (one thread)
+        if (lane == 0) {
+            bool ok = true;
+            int issued = 0;
+            for (int kb = 0; kb < nkb; ++kb) {
+                const int s = kb % S;
+                if (kb >= S && !mbar_wait_sleep(empty(s), (uint32_t)(((kb / S) - 1) & 1))) {
+                    ok = false;
+                    break;
+                }
+                if (*abort_flag) {
+                    ok = false;
+                    break;
+                }
+                mbar_expect_tx(full_b(s), (uint32_t)(NT * BK));
+                tma_load(b_s + (uint32_t)(s * NT * BK), &tmB, k0 + kb * BK, 0, full_b(s));
+                ++issued;
+            }
+            if (!ok) {
+                *abort_flag = 1;
+                report_status(p.status, HBL_ERR_TIMEOUT);
+            }
+            // every load issued lands before the CTA may move on
+            for (int j = issued > S ? issued - S : 0; j < issued; ++j)
+                if (!mbar_wait_sleep(full_b(j % S), (uint32_t)((j / S) & 1))) break;
+        }
+        __syncwarp();
+    } else {
+        // ---------------- converters: one weight row (TMEM lane) and one
+        // 64-weight half of each stage per thread
+        const int cw = warp - 2;
+        const int q = warp & 3;  // the TMEM lane quarter this warp may access
+        const int h = cw >> 2;
+        const int r = 32 * q + lane;
+        const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+        const uint32_t wrow = w_s + (uint32_t)(r * p.rs) + 16u * h;
+        const int kb_per_g = nkb / p.G;
+        bool ok = true;
+        for (int kb = 0; kb < nkb; ++kb) {
+            const int s = kb % S;
+            if (kb % kb_per_g == 0 && !warp_wait(wbar(kb / kb_per_g), 0)) {
+                ok = false;
+                break;
+            }
+            if (kb >= S && !warp_wait(empty(s), (uint32_t)(((kb / S) - 1) & 1))) {
+                ok = false;
+                break;
+            }
+            if (__shfl_sync(0xffffffffu, *abort_flag, 0) != 0) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const uint4 w = lds128(wrow + (uint32_t)(kb * 32));
+            const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+            uint32_t v[16];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                v[4 * j + 0] = wv[j] & 0x03030303u;
+                v[4 * j + 1] = (wv[j] >> 2) & 0x03030303u;
+                v[4 * j + 2] = (wv[j] >> 4) & 0x03030303u;
+                v[4 * j + 3] = (wv[j] >> 6) & 0x03030303u;
+            }
+            tmem_st16(tmem + lane_base + kACol + 32u * s + 16u * h, v);
+            asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_one(full_a(s));
+        }
+        if (!ok && lane == 0) {
+            *abort_flag = 1;
+            report_status(p.status, HBL_ERR_TIMEOUT);
+        }
+        // every weight copy has landed before its bytes are reused (bounded)
+        for (int g = 0; g < p.G; ++g)
+            if (!warp_wait(wbar(g), 0)) break;
+        const bool ready = warp_wait(acc_bar, 0);
+        if (!ready && lane == 0) report_status(p.status, HBL_ERR_TIMEOUT);
+        tc_fence_after();
+        const bool aborted = __shfl_sync(0xffffffffu, *abort_flag, 0) != 0;
+        if (ready && !aborted) {
+            // partials [NT][128] int32 over the (consumed) weight rows
+            int32_t* part = reinterpret_cast<int32_t*>(base);
+            constexpr int HC = NT / 2;  // columns (tokens) of this warp
+            const uint32_t taddr = tmem + lane_base + (uint32_t)(HC * h);
+#pragma unroll
+            for (int c0 = 0; c0 < HC; c0 += 8) {
+                uint32_t d[8];
+                tmem_ld8(taddr + (uint32_t)c0, d);
+                asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+                for (int e = 0; e < 8; ++e) part[(HC * h + c0 + e) * kRows + r] = (int32_t)d[e];
+            }
+        }
+    }
+    // ---- reduction over the cluster: CTA c sums rows [c RC, (c + 1) RC)
+    tc_fence_before();
+    __syncwarp();
+    cluster_sync_all();
+    {
+        const int RC = kRows / (int)csize;
+        const int quads = RC / 4;
+        const float alpha = *p.alpha;
+        const uint32_t part_s = w_s;
+        for (int it = threadIdx.x; it < p.M * quads; it += kThreads) {
+            const int j = it / quads;
+            const int r = (int)crank * RC + 4 * (it % quads);
+            const int n = n0 + r;
+            if (n >= p.N) continue;
+            const uint32_t off = part_s + (uint32_t)((j * kRows + r) * 4);
+            int a0 = 0, a1 = 0, a2 = 0, a3 = 0;
+            for (uint32_t c = 0; c < csize; ++c) {
+                const uint4 v = ld_cluster_v4(mapa(off, c));
+                a0 += (int)v.x;
+                a1 += (int)v.y;
+                a2 += (int)v.z;
+                a3 += (int)v.w;
+            }
+            const int rs = p.rowsum[j];
+            a0 -= rs;
+            a1 -= rs;
+            a2 -= rs;
+            a3 -= rs;
+            const float sc = __fmul_rn(alpha, p.scales[j]);
+            const uint32_t y01 =
+                (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn((float)a0, sc))) |
+                ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn((float)a1, sc)))
+                 << 16);
+            const uint32_t y23 =
+                (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn((float)a2, sc))) |
+                ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn((float)a3, sc)))
+                 << 16);
+            *reinterpret_cast<uint2*>(p.Y + (int64_t)j * p.N + n) = make_uint2(y01, y23);
+            if (p.acc_out != nullptr)
+                *reinterpret_cast<int4*>(p.acc_out + (int64_t)j * p.N + n) = make_int4(a0, a1, a2, a3);
+        }
+    }
+    // peers have finished reading this CTA's partials
+    __syncwarp();
+    cluster_sync_all();
+    if (warp == 0) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                     "r"(kTmemCols)
+                     : "memory");
+    }
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point.
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static std::once_flag once;
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    });
+    return fn;
+}
+
+// Codes [M x K] bytes, box (128 bytes x NT rows), 128-byte swizzle; rows past M
+// read as zeros.
+static bool make_codes_map(CUtensorMap* map, const void* codes, int M, int K, int NT) {
+    auto fn = encode_fn();
+    if (fn == nullptr) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M};
+    const cuuint64_t strides[1] = {(cuuint64_t)K};
+    const cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)NT};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(codes), dims, strides, box,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+struct Plan {
+    int NT, CS, Kc, G, rs, smem;
+    uint32_t b_off, bar_off;
+};
+
+static int nt_for(int M) { return M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : 128; }
+
+static int smem_for(int NT, int Kc, int G, int* rs, uint32_t* b_off, uint32_t* bar_off) {
+    (void)G;
+    *rs = Kc / 4 + 16;
+    const int wbytes = kRows * *rs;
+    const int pbytes = NT * kRows * 4;
+    const int region0 = ((wbytes > pbytes ? wbytes : pbytes) + 1023) & ~1023;
+    *b_off = (uint32_t)region0;
+    *bar_off = (uint32_t)(region0 + S * NT * BK);
+    const int total = region0 + S * NT * BK + 8 * (3 * S + kMaxGroups + 1) + 16 + 1024;
+    return total < kMinSmem ? kMinSmem : total;
+}
+
+template <int NT>
+static int max_active_clusters(int CS, int smem) {
+    // cached per (cluster size, shared memory) for this instantiation
+    static std::mutex mu;
+    static int cache[4][8] = {};  // [log2 CS][smem bucket] -> clusters + 1
+    int lcs = CS == 1 ? 0 : CS == 2 ? 1 : CS == 4 ? 2 : 3;
+    int bucket = smem / (32 * 1024);
+    if (bucket > 7) bucket = 7;
+    std::lock_guard<std::mutex> lock(mu);
+    if (cache[lcs][bucket] == 0) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(CS, 1, 1);
+        cfg.blockDim = dim3(kThreads);
+        cfg.dynamicSmemBytes = smem;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = CS;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, decode_mma_kernel<NT>, &cfg) != cudaSuccess) {
+            cudaGetLastError();
+            n = 0;
+        }
+        cache[lcs][bucket] = n + 1;
+    }
+    return cache[lcs][bucket] - 1;
+}
+
+template <int NT>
+static bool plan_for(int M, int K, int N, int sms, int optin, Plan* pl) {
+    const int RB = (N + kRows - 1) / kRows;
+    for (int CS = 8; CS >= 1; CS /= 2) {
+        if (CS > 1 && RB * CS > sms) continue;
+        const int Kc = K / CS;
+        if (Kc < BK || K % CS != 0) continue;
+        int G = Kc / 1024;
+        if (G < 1) G = 1;
+        if (G > kMaxGroups) G = kMaxGroups;
+        int rs;
+        uint32_t b_off, bar_off;
+        const int smem = smem_for(NT, Kc, G, &rs, &b_off, &bar_off);
+        if (smem > optin) continue;
+        if (!smem_attr_once(reinterpret_cast<const void*>(decode_mma_kernel<NT>), smem)) return false;
+        if (CS > 1 && max_active_clusters<NT>(CS, smem) < RB) continue;
+        *pl = Plan{NT, CS, Kc, G, rs, smem, b_off, bar_off};
+        return true;
+    }
+    return false;
+}
+
+template <int NT>
+static hbl_status launch_nt(const GemmArgs& a, cudaStream_t stream, int sms, int optin) {
+    Plan pl;
+    if (!plan_for<NT>((int)a.M, a.K, a.N, sms, optin, &pl)) return HBL_ERR_SHAPE;
+    CUtensorMap map;
+    if (!make_codes_map(&map, a.codes, (int)a.M, a.K, NT)) return HBL_ERR_CUDA;
+    Params p;
+    p.M = (int)a.M;
+    p.K = a.K;
+    p.N = a.N;
+    p.Kc = pl.Kc;
+    p.G = pl.G;
+    p.rs = pl.rs;
+    p.b_off = pl.b_off;
+    p.bar_off = pl.bar_off;
+    p.W = a.W_packed;
+    p.scales = a.scales;
+    p.rowsum = a.rowsum;
+    p.alpha = a.alpha;
+    p.Y = a.Y;
+    p.acc_out = a.acc_out;
+    p.status = a.dev_status;
+    p.early_weights = a.pdl ? 1 : 0;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(pl.CS, (a.N + kRows - 1) / kRows, 1);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = pl.smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = pl.CS;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    return cudaLaunchKernelEx(&cfg, decode_mma_kernel<NT>, map, p) == cudaSuccess ? HBL_OK
+                                                                                   : HBL_ERR_CUDA;
+}
+
+static int optin_smem() {
+    int dev = 0, optin = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+        return 0;
+    return optin;
+}
+
+}  // namespace k7
+
+int decode_mma_max_m() { return 128; }
+
+bool decode_mma_supported(int64_t M, int K, int N, int num_sms) {
+    if (M < 1 || M > decode_mma_max_m() || K < k7::BK || N < 16) return false;
+    const int optin = k7::optin_smem();
+    if (optin <= 0) return false;
+    k7::Plan pl;
+    switch (k7::nt_for((int)M)) {
+        case 16: return k7::plan_for<16>((int)M, K, N, num_sms, optin, &pl);
+        case 32: return k7::plan_for<32>((int)M, K, N, num_sms, optin, &pl);
+        case 64: return k7::plan_for<64>((int)M, K, N, num_sms, optin, &pl);
+        default: return k7::plan_for<128>((int)M, K, N, num_sms, optin, &pl);
+    }
+}
+
+hbl_status launch_decode_mma(const GemmArgs& a, cudaStream_t stream, int num_sms) {
+    if (a.M == 0) return HBL_OK;
+    if (a.M > decode_mma_max_m()) return HBL_ERR_SHAPE;
+    const int optin = k7::optin_smem();
+    switch (k7::nt_for((int)a.M)) {
+        case 16: return k7::launch_nt<16>(a, stream, num_sms, optin);
+        case 32: return k7::launch_nt<32>(a, stream, num_sms, optin);
+        case 64: return k7::launch_nt<64>(a, stream, num_sms, optin);
+        default: return k7::launch_nt<128>(a, stream, num_sms, optin);
+    }
+}
+
+}  // namespace hbl

@@ -346,6 +346,43 @@ def test_gemm_tma_one_byte_codes(bits, M, K, N):
     assert np.array_equal(bf16_bits(Y), wY)
 
 
+# decode-batch tensor-core kernel: weights as the MMA's A operand in TMEM,
+# tokens as B (NT = 16 / 32 / 64 / 128), K split over clusters of 1-8 CTAs and
+# reduced through distributed shared memory; ragged N (last 128-row block
+# partly filled) and shapes whose plan does not fit (largest K: the fallback)
+@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("M,K,N", [(1, 128, 16), (9, 256, 48), (16, 4096, 4096), (17, 4096, 1040),
+                                   (32, 16384, 4096), (33, 2048, 272), (64, 16384, 4096),
+                                   (65, 8192, 2048), (100, 4096, 11008), (128, 16384, 4096),
+                                   (5, 16384, 4096), (128, 32768, 4096)])
+def test_gemm_decode_mma(bits, M, K, N):
+    codes, scales, rowsum, packed, alpha = make_gemm_case(M, K, N, bits, seed=M + K + N)
+    q = oracle.decode_codes(codes, K, bits)
+    act = 8 if bits == 8 else hbl.ACT_INT4_BYTES
+    Y, acc = hbl.ternary_gemm(
+        torch.from_numpy(q.view(np.uint8).copy()).to(DEV), torch.from_numpy(scales).to(DEV),
+        torch.from_numpy(rowsum).to(DEV), act, K,
+        torch.from_numpy(packed.view(np.int32)).to(DEV),
+        torch.from_numpy(np.array([alpha, 0, 0, 0], dtype=np.float32)).to(DEV),
+        want_acc=True, path=hbl.PATH_TC_DECODE)
+    torch.cuda.synchronize()
+    wY, wacc = oracle.ternary_gemm(codes, scales, bits, K, packed, alpha)
+    assert np.array_equal(acc.cpu().numpy(), wacc)
+    assert np.array_equal(bf16_bits(Y), wY)
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("M,K,N", [(1, 4096, 4096), (3, 16384, 4096), (12, 4096, 4096),
+                                   (40, 16384, 4096), (128, 4096, 2048)])
+def test_forward_decode_mma_path(bits, M, K, N):
+    # the whole layer with its GEMM on the decode tensor-core kernel (K1 writes
+    # one-byte codes, the kernel follows it as a programmatic dependent)
+    X = acts(M, K, seed=M + 3 * K, kind="swiglu")
+    packed, alpha = oracle.pack_ternary(inputs.latent_weights(N, K, seed=M + N))
+    want = oracle.hbitlinear_forward(X, packed, alpha, bits)
+    assert np.array_equal(forward(X, packed, alpha, bits, path=hbl.PATH_TC_DECODE), want)
+
+
 @pytest.mark.parametrize("K", [16, 256, 4096, 16384])
 def test_quant_int4_one_byte_layout(K):
     X = acts(45, K, seed=K + 7, kind="t")
@@ -429,18 +466,18 @@ def test_ffn_wdown_workload_every_row(bits):
     assert bad.size == 0, "outputs differ at %d elements, first %s" % (len(bad), bad[:5].tolist())
 
 
-@pytest.mark.parametrize("T", list(inputs.DECODE_TOKENS))
+@pytest.mark.parametrize("T", sorted(set(inputs.DECODE_TOKENS) | {5, 9, 16, 64, 100}))
 @pytest.mark.parametrize("shape", ["wo", "wdown"])
 def test_decode_sweep(T, shape):
+    # every row of the decode batches the benchmark times, on the automatic path
     K = 4096 if shape == "wo" else 16384
     N = 4096
     X = inputs.activations("decode_" + shape, M=T, K=K, seed=T)
     W = inputs.latent_weights(N, K, seed=7)
     packed, alpha = oracle.pack_ternary(W)
     Y = forward(X, packed, alpha, 4)
-    rows = np.arange(T) if T <= 8 else np.concatenate([np.arange(4), [T - 1]])
-    want = oracle.hbitlinear_forward(X, packed, alpha, 4, rows=rows)
-    assert np.array_equal(Y[rows], want)
+    want = oracle.hbitlinear_forward(X, packed, alpha, 4)
+    assert np.array_equal(Y, want)
 
 
 # one-kernel decode forward (M <= 16384 / K tokens at K = 4096 / 8192 / 16384
