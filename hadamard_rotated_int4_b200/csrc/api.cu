@@ -69,7 +69,7 @@ int act_width(int a) { return a == 4 ? 4 : 8; }
 int codes_row_bytes(int K, int act_bits) { return act_width(act_bits) == 4 ? K / 2 : K; }
 
 // Ternary-GEMM back ends.
-enum class Back { GEMV, SS, TS, TMA, DEC };
+enum class Back { GEMV, SS, TS, TMA, DEC, WT };
 
 // The GEMV back end uses the row GEMV when K allows it and the tokens fit one
 // launch; otherwise the split-K GEMV (8-token chunks).
@@ -78,7 +78,7 @@ bool rows_gemv(int64_t M, int K) { return gemv_rows_supported(K) && M <= gemv_ro
 // Batches above this many tokens take the TMA-fed kernel (automatic choice).
 constexpr int64_t kTmaMinM = 257;
 
-bool path_valid(int path) { return path >= HBL_PATH_AUTO && path <= HBL_PATH_TC_DECODE; }
+bool path_valid(int path) { return path >= HBL_PATH_AUTO && path <= HBL_PATH_TC_PACKED; }
 
 // Shapes the decode-batch tensor-core kernel takes (one-byte codes); whether a
 // launch plan fits the device is checked again at launch, which falls back to
@@ -95,6 +95,7 @@ Back pick(int64_t M, int K, bool bytes, int path) {
     if (path == 3) return Back::TS;
     if (path == 4) return (bytes && K >= 128) ? Back::TMA : Back::TS;
     if (path == 5) return (bytes && dec_shape(M, K)) ? Back::DEC : Back::TS;
+    if (path == 6) return (bytes && K >= 128) ? Back::WT : Back::TS;
     // CUDA cores for a few tokens: the row GEMV where it takes the batch in one
     // launch; past that at K >= 16384 the tensor-core kernel is faster than the
     // split-K GEMV
@@ -109,6 +110,7 @@ size_t backend_ws(Back b, int64_t M, int K, int N) {
         case Back::SS: return 0;
         case Back::TS: return gemm_ts_workspace(M, K, N);
         case Back::DEC: return gemm_ts_workspace(M, K, N);  // its fallback's
+        case Back::WT: return 0;
         case Back::TMA: return gemm_tma_workspace(K, N);
         case Back::GEMV:
         default: {
@@ -128,6 +130,7 @@ hbl_status run_gemm(Back b, const GemmArgs& a, void* ws, size_t ws_bytes, cudaSt
     if (b == Back::SS) return launch_gemm_tc(a, s, sms);
     if (b == Back::TS) return launch_gemm_ts(a, ws, ws_bytes, s, sms);
     if (b == Back::TMA) return launch_gemm_tma(a, ws, ws_bytes, s, sms);
+    if (b == Back::WT) return launch_gemm_wt(a, s, sms);
     if (b == Back::DEC) {
         if (!a.interleaved && a.act_bits == 8 && decode_mma_supported(a.M, a.K, a.N, sms))
             return launch_decode_mma(a, s, sms);
@@ -175,7 +178,7 @@ FwdPlan forward_plan(int64_t M, int K, int act_bits, int path) {
     FwdPlan f;
     f.back = pick(M, K, true, path);
     f.interleaved = f.back == Back::TS;
-    if (f.back == Back::TMA || f.back == Back::DEC) {
+    if (f.back == Back::TMA || f.back == Back::DEC || f.back == Back::WT) {
         f.k1_mode = act_bits == 4 ? 6 : 8;
         f.gemm_act_bits = 8;
     } else if (f.back == Back::TS) {
@@ -522,9 +525,9 @@ hbl_status hbl_hbitlinear_forward_hostio(const uint16_t* X_host, const float* ga
     // Batches on the TMA-fed GEMM run in row chunks of at least kTmaMinM rows
     // (so every chunk keeps that plan and fits its workspace): chunk c's input
     // copy, its layer and chunk c-1's output copy overlap on three streams.
-    const int nch = plan.back == Back::TMA
-                        ? (int)((int64_t)M / kTmaMinM < kMaxChunks ? (int64_t)M / kTmaMinM
-                                                                    : kMaxChunks)
+    const bool big = plan.back == Back::TMA || plan.back == Back::WT;
+    const int nch = big ? (int)((int64_t)M / kTmaMinM < kMaxChunks ? (int64_t)M / kTmaMinM
+                                                                   : kMaxChunks)
                         : 1;
     if (nch <= 1) {
         if (cudaMemcpyAsync(Xd, X_host, (size_t)M * K * 2, cudaMemcpyHostToDevice, s) !=
@@ -549,13 +552,16 @@ hbl_status hbl_hbitlinear_forward_hostio(const uint16_t* X_host, const float* ga
     float* scales = reinterpret_cast<float*>(fws + cb);
     int32_t* rowsum = reinterpret_cast<int32_t*>(fws + cb + sb);
     int8_t* wexp = reinterpret_cast<int8_t*>(fws + cb + 2 * sb);
-    if (cb + 2 * sb + gemm_tma_workspace(K, N) > fws_bytes) return HBL_ERR_WORKSPACE;
+    const bool expand = plan.back == Back::TMA;
+    if (cb + 2 * sb + (expand ? gemm_tma_workspace(K, N) : 0) > fws_bytes)
+        return HBL_ERR_WORKSPACE;
 #define HBL_CK(x) \
     if ((x) != cudaSuccess) return HBL_ERR_CUDA
     HBL_CK(cudaEventRecord(c->start, s));
     HBL_CK(cudaStreamWaitEvent(c->in, c->start, 0));
     HBL_CK(cudaStreamWaitEvent(c->out, c->start, 0));
-    if ((st = launch_expand_ternary(W_packed, N, K, wexp, s, sms)) != HBL_OK) return st;
+    if (expand && (st = launch_expand_ternary(W_packed, N, K, wexp, s, sms)) != HBL_OK)
+        return st;
     for (int i = 0; i < nch; ++i) {
         const int64_t r0 = (int64_t)i * rows;
         const int64_t mc = ((int64_t)M - r0) < rows ? ((int64_t)M - r0) : rows;
@@ -570,7 +576,10 @@ hbl_status hbl_hbitlinear_forward_hostio(const uint16_t* X_host, const float* ga
             return st;
         GemmArgs a{codes, scales, rowsum, plan.gemm_act_bits, mc, K, W_packed, alpha, N,
                    Yd + r0 * N, nullptr, dev_status};
-        if ((st = launch_gemm_tma_s8w(a, wexp, s, sms)) != HBL_OK) return st;
+        a.pdl = true;  // right after K1 on the same stream
+        if ((st = expand ? launch_gemm_tma_s8w(a, wexp, s, sms) : launch_gemm_wt(a, s, sms)) !=
+            HBL_OK)
+            return st;
         HBL_CK(cudaEventRecord(c->fwd_ev[i], s));
         HBL_CK(cudaStreamWaitEvent(c->out, c->fwd_ev[i], 0));
         HBL_CK(cudaMemcpyAsync(Y_host + r0 * N, Yd + r0 * N, (size_t)mc * N * 2,

@@ -15,16 +15,19 @@
 // 16, 32, 64 or 128, from shared memory), so a decode batch of 32 tokens wastes
 // no tensor-core rows.  Per CTA:
 //   - before the dependency wait (the weights are not the previous kernel's
-//     output), one warp starts 1-D bulk copies of the CTA's 128 weight rows,
-//     its K slice only, into shared memory (rows padded by 16 bytes, so the
-//     converters' 16-byte reads are free of bank conflicts), on G mbarriers
-//     of K groups: the whole weight stream runs under the quantiser kernel;
+//     output), one thread starts TMA loads of the CTA's 128 weight rows, its
+//     K slice only, into shared memory: G boxes of 128 rows x 128 bytes with
+//     the 128-byte swizzle (so the converters' 16-byte reads are free of bank
+//     conflicts), each on its own mbarrier: the whole weight stream runs under
+//     the quantiser kernel, in a few large requests;
 //   - one thread TMA-loads the tokens' codes for each 128-byte K stage into a
-//     4-stage ring (SWIZZLE_128B: the K-major layout the MMA descriptor names;
+//     ring that takes the rest of shared memory (up to 32 stages, all of the
+//     CTA's codes when they fit: the loads are L2 round trips, so many must be
+//     in flight; SWIZZLE_128B, the K-major layout the MMA descriptor names;
 //     rows past M are zero-filled);
 //   - eight converter warps unpack each stage's 2-bit weights in registers
 //     ((w >> 2m) & 0x03030303 is the codes of weights 4m..4m+3 as bytes, in
-//     natural order) and store them with tcgen05.st into a 4-stage ring of A
+//     natural order) and store them with tcgen05.st into a 12-stage ring of A
 //     tiles in TMEM (32 columns = 128 bytes per row and stage);
 //   - one thread issues tcgen05.mma.cta_group::1.kind::i8 (A u8 from TMEM,
 //     B s8 from shared memory, D s32 in TMEM) and commits each stage back.
@@ -38,9 +41,10 @@
 // CTAs through distributed shared memory (integer sums: exact in any order),
 // subtracts rowsum and writes bf16 Y.  No workspace, no second kernel.
 //
-// TMEM: 256 columns per CTA (D in [0, NT), the A ring in [128, 256)); the
-// dynamic shared memory is at least 80 KB, so no more than two CTAs share an
-// SM and their allocations always fit the SM's 512 columns.  Every mbarrier
+// TMEM: all 512 columns (D in [0, NT), the A ring in [128, 512)); the dynamic
+// shared memory is at least 116 KB, so no two CTAs of this kernel share an SM.
+// The converters fill the A ring in batches of four stages with one wait for
+// their TMEM stores per batch.  Every mbarrier
 // wait is bounded by the global timer; on expiry the kernel records
 // HBL_ERR_TIMEOUT, stops issuing, lets its own copies and MMAs land (bounded
 // waits again), still takes part in both cluster barriers (every thread of
@@ -60,13 +64,15 @@ namespace k7 {
 
 constexpr int kRows = 128;  // weight rows per CTA (MMA M, TMEM lanes)
 constexpr int BK = 128;     // K bytes per stage
-constexpr int S = 4;        // stages of the A (TMEM) and B (shared memory) rings
+constexpr int kMaxSA = 12;  // stages of the A ring in TMEM (32 columns each)
+constexpr int kMaxSB = 32;  // stages of the B ring in shared memory
 constexpr int kConvWarps = 8;
 constexpr int kThreads = 32 * (2 + kConvWarps);
-constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kACol = 128;  // first TMEM column of the A ring
-constexpr int kMaxGroups = 8;
-constexpr int kMinSmem = 80 * 1024;  // caps residency at two CTAs per SM
+constexpr int kMaxGroups = 16;
+constexpr int kBoxBytes = 128 * 128;  // one swizzled weight box: 128 rows x 128 bytes
+constexpr int kMinSmem = 116 * 1024;  // one CTA per SM: it may take all 512 TMEM columns
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 
 // kind::i8: D s32 (bits 4-5 = 2), A u8 (bits 7-9 = 0), B s8 (bits 10-12 = 1),
@@ -80,10 +86,12 @@ __host__ __device__ constexpr uint32_t idesc() {
 struct Params {
     int M, K, N;
     int Kc;        // K per CTA (K / cluster size), a multiple of BK
-    int G;         // weight copy groups per row (Kc / 4 / G bytes each)
-    int rs;        // bytes per weight row in shared memory (Kc / 4 + 16)
+    int G;         // weight boxes: Kc / 512 swizzled 128-byte boxes, or one
+                   // unswizzled box of Kc / 4 bytes per row when Kc < 512
+    int sw;        // the weight boxes are 128-byte swizzled
     uint32_t b_off;  // offset of the B ring from the 1024-aligned base
     uint32_t bar_off;
+    int SA, SB;      // ring depths (A in TMEM, B in shared memory)
     const uint32_t* W;
     const float* scales;
     const int32_t* rowsum;
@@ -152,15 +160,6 @@ __device__ __forceinline__ void tma_load(uint32_t dst, const CUtensorMap* map, i
         "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(mbar)
         : "memory");
 }
-// 1-D bulk copy (no multicast) global -> this CTA's shared memory.
-__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
-                                          uint32_t mbar) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-            dst),
-        "l"(src), "r"(bytes), "r"(mbar)
-        : "memory");
-}
 __device__ __forceinline__ uint32_t cluster_rank() {
     uint32_t r;
     asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
@@ -219,20 +218,24 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t* v) {
 
 template <int NT>
 __global__ void __launch_bounds__(kThreads, 1)
-    decode_mma_kernel(const __grid_constant__ CUtensorMap tmB, Params p) {
+    decode_mma_kernel(const __grid_constant__ CUtensorMap tmB,
+                      const __grid_constant__ CUtensorMap tmW, Params p) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_s = smem_addr(smem_raw);
     const uint32_t base_s = (raw_s + 1023u) & ~1023u;
     uint8_t* base = smem_raw + (base_s - raw_s);
     const uint32_t w_s = base_s;              // weights, later the partial sums
-    const uint32_t b_s = base_s + p.b_off;    // B ring: S x NT x 128 bytes
+    const uint32_t b_s = base_s + p.b_off;    // B ring: SB x NT x 128 bytes
     const uint32_t bar_s = base_s + p.bar_off;
+    const int SA = p.SA, SB = p.SB;
     auto full_b = [&](int s) { return bar_s + 8u * s; };
-    auto full_a = [&](int s) { return bar_s + 8u * (S + s); };
-    auto empty = [&](int s) { return bar_s + 8u * (2 * S + s); };
-    auto wbar = [&](int g) { return bar_s + 8u * (3 * S + g); };
-    const uint32_t acc_bar = bar_s + 8u * (3 * S + kMaxGroups);
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + p.bar_off + 8 * (3 * S + kMaxGroups + 1));
+    auto empty_b = [&](int s) { return bar_s + 8u * (kMaxSB + s); };
+    auto full_a = [&](int s) { return bar_s + 8u * (2 * kMaxSB + s); };
+    auto empty_a = [&](int s) { return bar_s + 8u * (2 * kMaxSB + kMaxSA + s); };
+    auto wbar = [&](int g) { return bar_s + 8u * (2 * kMaxSB + 2 * kMaxSA + g); };
+    const uint32_t acc_bar = bar_s + 8u * (2 * kMaxSB + 2 * kMaxSA + kMaxGroups);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(
+        base + p.bar_off + 8 * (2 * kMaxSB + 2 * kMaxSA + kMaxGroups + 1));
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -243,16 +246,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int rows = min(kRows, p.N - n0);
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < S; ++s) {
+        for (int s = 0; s < SB; ++s) {
             mbar_init_count(full_b(s), 1);
+            mbar_init_count(empty_b(s), 1);
+        }
+        for (int s = 0; s < SA; ++s) {
             mbar_init_count(full_a(s), kConvWarps);
-            mbar_init_count(empty(s), 1);
+            mbar_init_count(empty_a(s), 1);
         }
         for (int g = 0; g < kMaxGroups; ++g) mbar_init_count(wbar(g), 1);
         mbar_init_count(acc_bar, 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmB)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmW)) : "memory");
     }
     if (warp == 0) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -266,18 +273,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---- the CTA's weight rows (its K slice) into shared memory: the weights
     // are not the previous kernel's output, so this runs before the dependency
     // wait, under that kernel
-    const uint32_t cbytes = (uint32_t)(p.Kc / 4 / p.G);
+    // box g: bytes [k0/4 + g * inner, + inner) of rows [n0, n0 + 128) (rows
+    // past N read as zeros; the full box counts toward the transaction bytes)
+    const int inner = p.sw ? 128 : p.Kc / 4;
     auto load_weights = [&] {
         if (lane == 0)
-            for (int g = 0; g < p.G; ++g) mbar_expect_tx(wbar(g), (uint32_t)rows * cbytes);
+            for (int g = 0; g < p.G; ++g) {
+                mbar_expect_tx(wbar(g), (uint32_t)(kRows * inner));
+                tma_load(w_s + (uint32_t)(g * kRows * inner), &tmW, k0 / 4 + g * inner, n0,
+                         wbar(g));
+            }
         __syncwarp();
-        for (int r = lane; r < rows; r += 32) {
-            const uint8_t* src =
-                reinterpret_cast<const uint8_t*>(p.W + (int64_t)(n0 + r) * (p.K / 16)) + k0 / 4;
-            for (int g = 0; g < p.G; ++g)
-                bulk_load(w_s + (uint32_t)(r * p.rs) + g * cbytes, src + g * cbytes, cbytes,
-                          wbar(g));
-        }
     };
     if (warp == 1 && p.early_weights) load_weights();
     pdl_wait();  // the codes, scales and row sums come from the previous kernel
@@ -291,20 +297,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ---------------- MMA issuer (one thread)
         if (lane == 0) {
             bool ok = true;
+            int sa = 0, sb = 0;
+            uint32_t pa = 0, pb = 0;  // phases of the current A and B slots
             for (int kb = 0; kb < nkb; ++kb) {
-                const int s = kb % S;
-                const uint32_t ph = (uint32_t)((kb / S) & 1);
-                if (!mbar_wait(full_a(s), ph) || !mbar_wait(full_b(s), ph) || *abort_flag) {
+                if (!mbar_wait(full_a(sa), pa) || !mbar_wait(full_b(sb), pb) || *abort_flag) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                const uint32_t sb = b_s + (uint32_t)(s * NT * BK);
+                const uint32_t bsm = b_s + (uint32_t)(sb * NT * BK);
 #pragma unroll
                 for (int k = 0; k < BK / 32; ++k)
-                    mma_ts<NT>(tmem, tmem + kACol + 32u * s + 8u * k, sdesc(sb + 32 * k),
+                    mma_ts<NT>(tmem, tmem + kACol + 32u * sa + 8u * k, sdesc(bsm + 32 * k),
                                (kb | k) != 0 ? 1u : 0u);
-                mma_commit(empty(s));
+                mma_commit(empty_a(sa));
+                mma_commit(empty_b(sb));
+                if (++sa == SA) { sa = 0; pa ^= 1u; }
+                if (++sb == SB) { sb = 0; pb ^= 1u; }
             }
             if (!ok) {
                 *abort_flag = 1;
@@ -322,8 +331,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             bool ok = true;
             int issued = 0;
             for (int kb = 0; kb < nkb; ++kb) {
-                const int s = kb % S;
-                if (kb >= S && !mbar_wait_sleep(empty(s), (uint32_t)(((kb / S) - 1) & 1))) {
+                const int s = kb % SB;
+                if (kb >= SB && !mbar_wait_sleep(empty_b(s), (uint32_t)(((kb / SB) - 1) & 1))) {
                     ok = false;
                     break;
                 }
@@ -340,8 +349,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 report_status(p.status, HBL_ERR_TIMEOUT);
             }
             // every load issued lands before the CTA may move on
-            for (int j = issued > S ? issued - S : 0; j < issued; ++j)
-                if (!mbar_wait_sleep(full_b(j % S), (uint32_t)((j / S) & 1))) break;
+            for (int j = issued > SB ? issued - SB : 0; j < issued; ++j)
+                if (!mbar_wait_sleep(full_b(j % SB), (uint32_t)((j / SB) & 1))) break;
         }
         __syncwarp();
     } else {
@@ -352,39 +361,61 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int h = cw >> 2;
         const int r = 32 * q + lane;
         const uint32_t lane_base = (uint32_t)(32 * q) << 16;
-        const uint32_t wrow = w_s + (uint32_t)(r * p.rs) + 16u * h;
         const int kb_per_g = nkb / p.G;
+        // stages go in batches of CB: the batch's stores are issued back to back
+        // and waited for once (a TMEM store round trip per batch, not per stage)
+        constexpr int CB = 4;
         bool ok = true;
-        for (int kb = 0; kb < nkb; ++kb) {
-            const int s = kb % S;
-            if (kb % kb_per_g == 0 && !warp_wait(wbar(kb / kb_per_g), 0)) {
-                ok = false;
-                break;
+        for (int kb0 = 0; kb0 < nkb && ok; kb0 += CB) {
+            const int nb = min(CB, nkb - kb0);
+            for (int i = 0; i < nb; ++i) {
+                const int kb = kb0 + i;
+                if (kb % kb_per_g == 0 && !warp_wait(wbar(kb / kb_per_g), 0)) {
+                    ok = false;
+                    break;
+                }
+                if (kb >= SA && !warp_wait(empty_a(kb % SA), (uint32_t)(((kb / SA) - 1) & 1))) {
+                    ok = false;
+                    break;
+                }
             }
-            if (kb >= S && !warp_wait(empty(s), (uint32_t)(((kb / S) - 1) & 1))) {
-                ok = false;
-                break;
-            }
-            if (__shfl_sync(0xffffffffu, *abort_flag, 0) != 0) {
+            if (!ok || __shfl_sync(0xffffffffu, *abort_flag, 0) != 0) {
                 ok = false;
                 break;
             }
             tc_fence_after();
-            const uint4 w = lds128(wrow + (uint32_t)(kb * 32));
-            const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
-            uint32_t v[16];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                v[4 * j + 0] = wv[j] & 0x03030303u;
-                v[4 * j + 1] = (wv[j] >> 2) & 0x03030303u;
-                v[4 * j + 2] = (wv[j] >> 4) & 0x03030303u;
-                v[4 * j + 3] = (wv[j] >> 6) & 0x03030303u;
+            for (int i = 0; i < CB; ++i) {
+                if (i < nb) {
+                    const int kb = kb0 + i;
+                    // this thread's 16 bytes (64 weights) of row r in stage kb:
+                    // chunk c of the row's 128-byte line in box kb / 4, swizzled by r % 8
+                    uint32_t waddr;
+                    if (p.sw) {
+                        const uint32_t c = (uint32_t)(((kb & 3) << 1) | h);
+                        waddr = w_s + (uint32_t)((kb >> 2) * kBoxBytes + r * 128) +
+                                ((c ^ (uint32_t)(r & 7)) << 4);
+                    } else {
+                        waddr = w_s + (uint32_t)(r * (p.Kc / 4) + kb * 32 + 16 * h);
+                    }
+                    const uint4 w = lds128(waddr);
+                    const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+                    uint32_t v[16];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        v[4 * j + 0] = wv[j] & 0x03030303u;
+                        v[4 * j + 1] = (wv[j] >> 2) & 0x03030303u;
+                        v[4 * j + 2] = (wv[j] >> 4) & 0x03030303u;
+                        v[4 * j + 3] = (wv[j] >> 6) & 0x03030303u;
+                    }
+                    tmem_st16(tmem + lane_base + kACol + 32u * (uint32_t)(kb % SA) + 16u * h, v);
+                }
             }
-            tmem_st16(tmem + lane_base + kACol + 32u * s + 16u * h, v);
             asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive_one(full_a(s));
+            if (lane == 0)
+                for (int i = 0; i < nb; ++i) mbar_arrive_one(full_a((kb0 + i) % SA));
         }
         if (!ok && lane == 0) {
             *abort_flag = 1;
@@ -494,22 +525,47 @@ static bool make_codes_map(CUtensorMap* map, const void* codes, int M, int K, in
               CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Packed weights as bytes [N x K/4], box (inner bytes x 128 rows): the
+// 128-byte swizzle when inner is 128, else no swizzle; rows past N read as zeros.
+static bool make_weight_map(CUtensorMap* map, const uint32_t* W, int N, int K, int inner, bool sw) {
+    auto fn = encode_fn();
+    if (fn == nullptr) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)(K / 4), (cuuint64_t)N};
+    const cuuint64_t strides[1] = {(cuuint64_t)(K / 4)};
+    const cuuint32_t box[2] = {(cuuint32_t)inner, (cuuint32_t)kRows};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint32_t*>(W), dims, strides, box,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              sw ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 struct Plan {
-    int NT, CS, Kc, G, rs, smem;
+    int NT, CS, Kc, G, sw, smem, SA, SB;
     uint32_t b_off, bar_off;
 };
 
 static int nt_for(int M) { return M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : 128; }
 
-static int smem_for(int NT, int Kc, int G, int* rs, uint32_t* b_off, uint32_t* bar_off) {
-    (void)G;
-    *rs = Kc / 4 + 16;
-    const int wbytes = kRows * *rs;
+constexpr int kBarBytes = 8 * (2 * kMaxSB + 2 * kMaxSA + kMaxGroups + 1) + 16;
+
+// Shared memory of a plan: the weights (or the partial sums, whichever is
+// larger), then as deep a B ring as fits `budget` bytes (all of the CTA's B
+// when it fits), then the barriers.  0 if not even two B stages fit.
+static int smem_for(int NT, int Kc, int budget, int* SB, uint32_t* b_off, uint32_t* bar_off) {
+    const int wbytes = kRows * Kc / 4;
     const int pbytes = NT * kRows * 4;
     const int region0 = ((wbytes > pbytes ? wbytes : pbytes) + 1023) & ~1023;
+    const int stage = NT * BK;
+    const int nkb = Kc / BK;
+    int sb = (budget - region0 - kBarBytes - 1024) / stage;
+    if (sb > nkb) sb = nkb;
+    if (sb > kMaxSB) sb = kMaxSB;
+    if (sb < 2 && sb < nkb) return 0;
+    *SB = sb;
     *b_off = (uint32_t)region0;
-    *bar_off = (uint32_t)(region0 + S * NT * BK);
-    const int total = region0 + S * NT * BK + 8 * (3 * S + kMaxGroups + 1) + 16 + 1024;
+    *bar_off = (uint32_t)(region0 + sb * stage);
+    const int total = region0 + sb * stage + kBarBytes + 1024;
     return total < kMinSmem ? kMinSmem : total;
 }
 
@@ -551,16 +607,17 @@ static bool plan_for(int M, int K, int N, int sms, int optin, Plan* pl) {
         if (CS > 1 && RB * CS > sms) continue;
         const int Kc = K / CS;
         if (Kc < BK || K % CS != 0) continue;
-        int G = Kc / 1024;
-        if (G < 1) G = 1;
-        if (G > kMaxGroups) G = kMaxGroups;
-        int rs;
+        const int sw = Kc >= 512 ? 1 : 0;
+        const int G = sw ? Kc / 512 : 1;
+        if (G > kMaxGroups) continue;
         uint32_t b_off, bar_off;
-        const int smem = smem_for(NT, Kc, G, &rs, &b_off, &bar_off);
-        if (smem > optin) continue;
+        int SB = 0;
+        const int smem = smem_for(NT, Kc, optin, &SB, &b_off, &bar_off);
+        if (smem == 0 || smem > optin) continue;
         if (!smem_attr_once(reinterpret_cast<const void*>(decode_mma_kernel<NT>), smem)) return false;
         if (CS > 1 && max_active_clusters<NT>(CS, smem) < RB) continue;
-        *pl = Plan{NT, CS, Kc, G, rs, smem, b_off, bar_off};
+        const int SA = kMaxSA < Kc / BK ? kMaxSA : Kc / BK;
+        *pl = Plan{NT, CS, Kc, G, sw, smem, SA, SB, b_off, bar_off};
         return true;
     }
     return false;
@@ -570,15 +627,19 @@ template <int NT>
 static hbl_status launch_nt(const GemmArgs& a, cudaStream_t stream, int sms, int optin) {
     Plan pl;
     if (!plan_for<NT>((int)a.M, a.K, a.N, sms, optin, &pl)) return HBL_ERR_SHAPE;
-    CUtensorMap map;
-    if (!make_codes_map(&map, a.codes, (int)a.M, a.K, NT)) return HBL_ERR_CUDA;
+    CUtensorMap map, wmap;
+    if (!make_codes_map(&map, a.codes, (int)a.M, a.K, NT) ||
+        !make_weight_map(&wmap, a.W_packed, a.N, a.K, pl.sw ? 128 : pl.Kc / 4, pl.sw != 0))
+        return HBL_ERR_CUDA;
     Params p;
     p.M = (int)a.M;
     p.K = a.K;
     p.N = a.N;
     p.Kc = pl.Kc;
     p.G = pl.G;
-    p.rs = pl.rs;
+    p.sw = pl.sw;
+    p.SA = pl.SA;
+    p.SB = pl.SB;
     p.b_off = pl.b_off;
     p.bar_off = pl.bar_off;
     p.W = a.W_packed;
@@ -603,8 +664,9 @@ static hbl_status launch_nt(const GemmArgs& a, cudaStream_t stream, int sms, int
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    return cudaLaunchKernelEx(&cfg, decode_mma_kernel<NT>, map, p) == cudaSuccess ? HBL_OK
-                                                                                   : HBL_ERR_CUDA;
+    return cudaLaunchKernelEx(&cfg, decode_mma_kernel<NT>, map, wmap, p) == cudaSuccess
+               ? HBL_OK
+               : HBL_ERR_CUDA;
 }
 
 static int optin_smem() {

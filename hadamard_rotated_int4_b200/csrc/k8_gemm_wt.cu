@@ -1,0 +1,470 @@
+// k8_gemm_wt.cu -- ternary-weight GEMM for large token batches on the sm_100a
+// tensor cores, reading the 2-bit packed weights directly (no expanded copy).
+//
+// Computes (BitNet v2 write-up, 0755model.com, section "H-BitLinear": the
+// ternary matmul of the per-token quantised activations, rescaled by the
+// weight and activation scales)
+//   acc[m][n] = sum_k q[m][k] * t[n][k]     (exact, int32)
+//   Y[m][n]   = bf16_rne((float)acc * (alpha * s[m]))
+// for codes q one byte each, row-major [M x K] (INT8, or INT4 values in
+// [-8, 7]) and the library's packed weights (16 per uint32, code t + 1).
+//
+// The weights are the MMA's A operand, in tensor memory: 128 weight rows per
+// tile (TMEM lanes), and the tokens its B operand from shared memory: 256
+// tokens per tile (MMA N).  Shared memory then carries only the tokens' codes
+// (TMA, 128-byte swizzle) and the packed weights (TMA, 32 bytes per row and
+// stage, 32-byte swizzle): per 128 x 256 x 32 MMA it reads 8 KB and is written
+// 9 KB, against 12 + 12 KB when both byte operands sit in shared memory; the
+// weights are widened to bytes in registers by eight converter warps
+// ((w >> 2m) & 0x03030303 is the codes of weights 4m..4m+3 in natural order)
+// and stored with tcgen05.st.  The weights enter as c = t + 1 (unsigned), so
+// the accumulator holds acc + rowsum[m]; the epilogue subtracts rowsum.
+//
+// Persistent CTAs, one per SM, walk the tiles token block by token block (the
+// weight block varies fastest): the packed weights (16.8 MB for 4096 x 16384)
+// and the token blocks in flight stay in L2, so HBM sees each code once.
+// Warp 0 allocates TMEM (512 columns: the 128 x 256 int32 accumulator in
+// [0, 256), an 8-stage ring of A tiles in [256, 512)) and one lane issues the
+// MMAs; warp 1 issues the TMA loads (5-stage ring of 36 KB: 32 KB of codes and
+// 4 KB of packed weights); warps 2-9 convert, four stages per wait for their
+// TMEM stores; warps 10-17 drain the
+// accumulator (tcgen05.ld), subtract rowsum, scale and store bf16 Y.  Every
+// mbarrier wait is bounded by the global timer; on expiry the kernel records
+// HBL_ERR_TIMEOUT, stops issuing, lets its copies and MMAs land (bounded) and
+// frees its TMEM.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "hbl_internal.cuh"
+#include "hbl_launch.h"
+
+namespace hbl {
+namespace k8 {
+
+constexpr int kRows = 128;  // weight rows per tile (MMA M, TMEM lanes)
+constexpr int NT = 256;     // tokens per tile (MMA N)
+constexpr int BK = 128;     // K bytes per stage
+constexpr int S = 5;        // stages of the shared-memory ring (codes + packed weights)
+constexpr int SA = 8;       // stages of the TMEM A ring (32 columns each)
+constexpr int CB = 4;       // converter batch: stages stored per wait for the TMEM stores
+constexpr int kConvWarps = 8;
+constexpr int kEpiWarps = 8;
+constexpr int kThreads = 32 * (2 + kConvWarps + kEpiWarps);
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kACol = 256;
+constexpr int kBBytes = NT * BK;         // 32 KB of codes per stage
+constexpr int kWBytes = kRows * BK / 4;  // 4 KB of packed weights per stage
+constexpr int kStage = kBBytes + kWBytes;
+constexpr int kBarOff = S * kStage;
+constexpr int kSmemBytes = kBarOff + 256 + 1024;
+constexpr uint64_t kTimeoutNs = 2000000000ull;
+
+// kind::i8: D s32, A u8 (weights from TMEM), B s8 (codes), K-major, N = 256, M = 128.
+constexpr uint32_t kIdesc = (2u << 4) | (0u << 7) | (1u << 10) | ((uint32_t)(NT >> 3) << 17) |
+                            ((uint32_t)(kRows >> 4) << 24);
+
+struct Params {
+    int64_t M;
+    int N, K;
+    int tiles_n;  // weight blocks
+    int64_t tiles;
+    const float* scales;
+    const int32_t* rowsum;
+    const float* alpha;
+    uint16_t* Y;
+    int32_t* acc_out;
+    int32_t* status;
+};
+
+__device__ __forceinline__ bool mbar_wait(uint32_t a, uint32_t parity) {
+    return mbar_wait_bounded<false>(a, parity, kTimeoutNs);
+}
+__device__ __forceinline__ bool mbar_wait_sleep(uint32_t a, uint32_t parity) {
+    return mbar_wait_bounded<true>(a, parity, kTimeoutNs);
+}
+__device__ __forceinline__ bool warp_wait(uint32_t a, uint32_t parity) {
+    bool ok = true;
+    if ((threadIdx.x & 31) == 0) ok = mbar_wait_sleep(a, parity);
+    return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t a, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(a), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+// K-major, 128-byte-swizzled shared-memory matrix descriptor (8-row atoms of
+// 1024 bytes, SBO = 1024), version 1.
+__device__ __forceinline__ uint64_t sdesc(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)1 << 16;
+    d |= (uint64_t)(1024 >> 4) << 32;
+    d |= (uint64_t)1 << 46;
+    d |= (uint64_t)2 << 61;
+    return d;
+}
+__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
+                                       uint32_t accum) {
+    asm volatile(
+        "{\n.reg .pred p;\n"
+        "setp.ne.b32 p, %3, 0;\n"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %4, p;\n}\n" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(bdesc), "r"(accum), "r"(kIdesc)
+        : "memory");
+}
+__device__ __forceinline__ void mma_commit(uint32_t mbar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(mbar)
+        : "memory");
+}
+// 2-D tiled TMA load (no multicast) of box (x, y) into this CTA's shared memory.
+__device__ __forceinline__ void tma_load(uint32_t dst, const CUtensorMap* map, int x, int y,
+                                         uint32_t mbar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes "
+        "[%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(mbar)
+        : "memory");
+}
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+        "r"(r[15])
+        : "memory");
+}
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, "
+        "%31}, [%32];"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+          "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]),
+          "=r"(v[13]), "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]),
+          "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]),
+          "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]),
+          "=r"(v[31])
+        : "r"(taddr));
+}
+
+// tile t -> token block mb, weight block nb (weight blocks fastest)
+__device__ __forceinline__ void tile_coords(const Params& p, int64_t t, int64_t& mb, int& nb) {
+    mb = t / p.tiles_n;
+    nb = (int)(t - mb * p.tiles_n);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_wt_kernel(const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmW,
+                   Params p) {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_s = smem_addr(smem_raw);
+    const uint32_t base_s = (raw_s + 1023u) & ~1023u;
+    uint8_t* base = smem_raw + (base_s - raw_s);
+    const uint32_t bar_s = base_s + kBarOff;
+    auto full = [&](int s) { return bar_s + 8u * s; };
+    auto empty = [&](int s) { return bar_s + 8u * (S + s); };
+    auto full_a = [&](int s) { return bar_s + 8u * (2 * S + s); };
+    auto empty_a = [&](int s) { return bar_s + 8u * (2 * S + SA + s); };
+    const uint32_t acc_full = bar_s + 8u * (2 * S + 2 * SA);
+    const uint32_t acc_empty = bar_s + 8u * (2 * S + 2 * SA + 1);
+    const uint32_t drain = bar_s + 8u * (2 * S + 2 * SA + 2);
+    uint32_t* tmem_slot =
+        reinterpret_cast<uint32_t*>(base + kBarOff + 8 * (2 * S + 2 * SA + 3));
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nkb = p.K / BK;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init_count(full(s), 1);
+            mbar_init_count(empty(s), 1);
+        }
+        for (int s = 0; s < SA; ++s) {
+            mbar_init_count(full_a(s), kConvWarps);
+            mbar_init_count(empty_a(s), 1);
+        }
+        mbar_init_count(acc_full, 1);
+        mbar_init_count(acc_empty, kEpiWarps);
+        mbar_init_count(drain, 1);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmB)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmW)) : "memory");
+    }
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_addr(tmem_slot)),
+                     "r"(kTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    pdl_wait();  // the codes come from the previous kernel
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ---------------- MMA issuer (one thread)
+        if (lane == 0) {
+            uint32_t it = 0, tc = 0;
+            bool ok = true;
+            for (int64_t t = blockIdx.x; t < p.tiles && ok; t += gridDim.x, ++tc) {
+                if (tc >= 1 && !mbar_wait_sleep(acc_empty, (tc - 1) & 1)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                for (int kb = 0; kb < nkb; ++kb, ++it) {
+                    const int s = (int)(it % S), a = (int)(it % SA);
+                    if (!mbar_wait(full_a(a), (it / SA) & 1) || !mbar_wait(full(s), (it / S) & 1) ||
+                        *abort_flag) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t sb = base_s + (uint32_t)(s * kStage);
+#pragma unroll
+                    for (int k = 0; k < BK / 32; ++k)
+                        mma_ts(tmem, tmem + kACol + 32u * a + 8u * k, sdesc(sb + 32 * k),
+                               (kb | k) != 0 ? 1u : 0u);
+                    mma_commit(empty(s));
+                    mma_commit(empty_a(a));
+                }
+                if (ok) mma_commit(acc_full);
+            }
+            if (!ok) {
+                *abort_flag = 1;
+                report_status(p.status, HBL_ERR_TIMEOUT);
+            }
+            // every MMA issued has completed once this commit arrives
+            mma_commit(drain);
+            if (!mbar_wait_sleep(drain, 0)) report_status(p.status, HBL_ERR_TIMEOUT);
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ---------------- TMA producer (one thread): codes and packed weights
+        if (lane == 0) {
+            uint32_t it = 0;
+            bool ok = true;
+            for (int64_t t = blockIdx.x; t < p.tiles && ok; t += gridDim.x) {
+                int64_t mb;
+                int nb;
+                tile_coords(p, t, mb, nb);
+                for (int kb = 0; kb < nkb; ++kb, ++it) {
+                    const int s = (int)(it % S);
+                    if (it >= (uint32_t)S && !mbar_wait_sleep(empty(s), ((it / S) - 1) & 1)) {
+                        ok = false;
+                        break;
+                    }
+                    if (*abort_flag) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t sb = base_s + (uint32_t)(s * kStage);
+                    mbar_expect_tx(full(s), (uint32_t)kStage);
+                    tma_load(sb, &tmB, kb * BK, (int)(mb * NT), full(s));
+                    tma_load(sb + kBBytes, &tmW, kb * (BK / 4), nb * kRows, full(s));
+                }
+            }
+            if (!ok) {
+                *abort_flag = 1;
+                report_status(p.status, HBL_ERR_TIMEOUT);
+            }
+            // let every load issued land before the CTA may exit
+            const uint32_t first = it > (uint32_t)S ? it - S : 0;
+            for (uint32_t j = first; j < it; ++j)
+                if (!mbar_wait_sleep(full((int)(j % S)), (j / S) & 1)) break;
+        }
+        __syncwarp();
+    } else if (warp < 2 + kConvWarps) {
+        // ---------------- converters: weight row r (TMEM lane), 64-weight half h
+        const int cw = warp - 2;
+        const int q = warp & 3;
+        const int h = cw >> 2;
+        const int r = 32 * q + lane;
+        const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+        // the 32-byte swizzle of the weight box: 16-byte chunk h of row r sits
+        // at chunk h ^ ((r >> 2) & 1)
+        const uint32_t woff = (uint32_t)kBBytes + (uint32_t)(r * 32) +
+                              ((uint32_t)(h ^ ((r >> 2) & 1)) << 4);
+        // stages in batches of CB (within a tile): the batch's TMEM stores are
+        // issued back to back and waited for once
+        uint32_t it = 0;
+        bool ok = true;
+        for (int64_t t = blockIdx.x; t < p.tiles && ok; t += gridDim.x) {
+            for (int kb0 = 0; kb0 < nkb && ok; kb0 += CB) {
+                const int nb = min(CB, nkb - kb0);
+                for (int i = 0; i < nb; ++i) {
+                    const uint32_t j = it + (uint32_t)i;
+                    if (!warp_wait(full((int)(j % S)), (j / S) & 1) ||
+                        (j >= (uint32_t)SA && !warp_wait(empty_a((int)(j % SA)), ((j / SA) - 1) & 1))) {
+                        ok = false;
+                        break;
+                    }
+                }
+                if (!ok || __shfl_sync(0xffffffffu, *abort_flag, 0) != 0) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+#pragma unroll
+                for (int i = 0; i < CB; ++i) {
+                    if (i < nb) {
+                        const uint32_t j = it + (uint32_t)i;
+                        const uint4 w = lds128(base_s + (uint32_t)((j % S) * kStage) + woff);
+                        const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+                        uint32_t v[16];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            v[4 * e + 0] = wv[e] & 0x03030303u;
+                            v[4 * e + 1] = (wv[e] >> 2) & 0x03030303u;
+                            v[4 * e + 2] = (wv[e] >> 4) & 0x03030303u;
+                            v[4 * e + 3] = (wv[e] >> 6) & 0x03030303u;
+                        }
+                        tmem_st16(tmem + lane_base + kACol + 32u * (j % SA) + 16u * h, v);
+                    }
+                }
+                asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0)
+                    for (int i = 0; i < nb; ++i) mbar_arrive_one(full_a((int)((it + i) % SA)));
+                it += (uint32_t)nb;
+            }
+        }
+        if (!ok && lane == 0) {
+            *abort_flag = 1;
+            report_status(p.status, HBL_ERR_TIMEOUT);
+        }
+    } else {
+        // ---------------- epilogue: weight row r (TMEM lane), 128 of the 256 token columns
+        const int ew = warp - 2 - kConvWarps;
+        const int q = warp & 3;
+        const int half = ew >> 2;
+        const int r = 32 * q + lane;
+        const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+        const float alpha = *p.alpha;
+        uint32_t tc = 0;
+        for (int64_t t = blockIdx.x; t < p.tiles; t += gridDim.x, ++tc) {
+            int64_t mb;
+            int nb;
+            tile_coords(p, t, mb, nb);
+            const bool ready = warp_wait(acc_full, tc & 1);
+            if (!ready || __shfl_sync(0xffffffffu, *abort_flag, 0) != 0) {
+                if (lane == 0) {
+                    *abort_flag = 1;
+                    report_status(p.status, HBL_ERR_TIMEOUT);
+                }
+                break;
+            }
+            tc_fence_after();
+            const int n = nb * kRows + r;
+            const bool nok = n < p.N;
+#pragma unroll 1
+            for (int cc = 0; cc < NT / 2 / 32; ++cc) {
+                const int c0 = 128 * half + 32 * cc;
+                uint32_t v[32];
+                tmem_ld32(tmem + lane_base + (uint32_t)c0, v);
+                asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+                if (cc == NT / 2 / 32 - 1) {  // the accumulator is free for the next tile
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive_one(acc_empty);
+                }
+                const int64_t m0 = mb * NT + c0;
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    const int64_t m = m0 + e;
+                    if (nok && m < p.M) {
+                        const int a = (int)v[e] - p.rowsum[m];
+                        const float sc = __fmul_rn(alpha, p.scales[m]);
+                        p.Y[m * p.N + n] =
+                            __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn((float)a, sc)));
+                        if (p.acc_out != nullptr) p.acc_out[m * p.N + n] = a;
+                    }
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                     "r"(kTmemCols)
+                     : "memory");
+    }
+}
+
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static std::once_flag once;
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    });
+    return fn;
+}
+
+// 2-D uint8 map [rows x cols] (row stride = cols bytes) with the given box and swizzle.
+static bool make_map(CUtensorMap* map, const void* ptr, int64_t rows, int64_t cols, int box_x,
+                     int box_y, CUtensorMapSwizzle sw) {
+    auto fn = encode_fn();
+    if (fn == nullptr) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)cols};
+    const cuuint32_t box[2] = {(cuuint32_t)box_x, (cuuint32_t)box_y};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace k8
+
+hbl_status launch_gemm_wt(const GemmArgs& a, cudaStream_t stream, int num_sms) {
+    if (a.M == 0) return HBL_OK;
+    if (a.K < k8::BK || a.K % k8::BK != 0) return HBL_ERR_SHAPE;
+    CUtensorMap mB, mW;
+    if (!k8::make_map(&mB, a.codes, a.M, a.K, k8::BK, k8::NT, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !k8::make_map(&mW, a.W_packed, a.N, a.K / 4, k8::BK / 4, k8::kRows,
+                      CU_TENSOR_MAP_SWIZZLE_32B))
+        return HBL_ERR_CUDA;
+    k8::Params prm;
+    prm.M = a.M;
+    prm.N = a.N;
+    prm.K = a.K;
+    prm.tiles_n = (a.N + k8::kRows - 1) / k8::kRows;
+    prm.tiles = (int64_t)prm.tiles_n * ((a.M + k8::NT - 1) / k8::NT);
+    prm.scales = a.scales;
+    prm.rowsum = a.rowsum;
+    prm.alpha = a.alpha;
+    prm.Y = a.Y;
+    prm.acc_out = a.acc_out;
+    prm.status = a.dev_status;
+    if (!smem_attr_once(reinterpret_cast<const void*>(k8::gemm_wt_kernel), k8::kSmemBytes))
+        return HBL_ERR_CUDA;
+    const int64_t grid = prm.tiles < num_sms ? prm.tiles : num_sms;
+    return launch_pdl(k8::gemm_wt_kernel, dim3((unsigned)grid), dim3(k8::kThreads),
+                      (size_t)k8::kSmemBytes, stream, mB, mW, prm);
+}
+
+}  // namespace hbl

@@ -122,7 +122,7 @@ def test_validation_errors():
     assert lib.hbl_ternary_gemm_path(A, B, C, 4, 64, 256, D, E, 64, A, NUL, E, 1 << 20, NUL, 9,
                                      NUL) == 1
     assert lib.hbl_hbitlinear_forward_path(A, NUL, 64, 256, 64, B, C, 4, 1e-6, 1e-5, D, E,
-                                           1 << 20, NUL, 6, NUL) == 1
+                                           1 << 20, NUL, 7, NUL) == 1
 
 
 def test_binding_rejects_non_cuda_tensors():

@@ -371,6 +371,38 @@ def test_gemm_decode_mma(bits, M, K, N):
     assert np.array_equal(bf16_bits(Y), wY)
 
 
+# large-batch tensor-core kernel on the packed weights (weights widened into
+# TMEM as A, codes as B by TMA): ragged token blocks (M % 256), ragged weight
+# blocks (N % 128), several tiles per CTA (more than 148 tiles)
+@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("M,K,N", [(1, 128, 16), (45, 256, 272), (256, 512, 128),
+                                   (300, 4096, 400), (1000, 2048, 512), (257, 16384, 4096),
+                                   (600, 4096, 11008), (1300, 1024, 4096)])
+def test_gemm_packed_weights(bits, M, K, N):
+    codes, scales, rowsum, packed, alpha = make_gemm_case(M, K, N, bits, seed=M + K + 2 * N)
+    q = oracle.decode_codes(codes, K, bits)
+    act = 8 if bits == 8 else hbl.ACT_INT4_BYTES
+    Y, acc = hbl.ternary_gemm(
+        torch.from_numpy(q.view(np.uint8).copy()).to(DEV), torch.from_numpy(scales).to(DEV),
+        torch.from_numpy(rowsum).to(DEV), act, K,
+        torch.from_numpy(packed.view(np.int32)).to(DEV),
+        torch.from_numpy(np.array([alpha, 0, 0, 0], dtype=np.float32)).to(DEV),
+        want_acc=True, path=hbl.PATH_TC_PACKED)
+    torch.cuda.synchronize()
+    wY, wacc = oracle.ternary_gemm(codes, scales, bits, K, packed, alpha)
+    assert np.array_equal(acc.cpu().numpy(), wacc)
+    assert np.array_equal(bf16_bits(Y), wY)
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("M,K,N", [(520, 4096, 256), (1000, 2048, 528), (300, 16384, 1024)])
+def test_forward_packed_weights_path(bits, M, K, N):
+    X = acts(M, K, seed=M + 5 * K, kind="swiglu")
+    packed, alpha = oracle.pack_ternary(inputs.latent_weights(N, K, seed=M + N))
+    want = oracle.hbitlinear_forward(X, packed, alpha, bits)
+    assert np.array_equal(forward(X, packed, alpha, bits, path=hbl.PATH_TC_PACKED), want)
+
+
 @pytest.mark.parametrize("bits", [4, 8])
 @pytest.mark.parametrize("M,K,N", [(1, 4096, 4096), (3, 16384, 4096), (12, 4096, 4096),
                                    (40, 16384, 4096), (128, 4096, 2048)])
