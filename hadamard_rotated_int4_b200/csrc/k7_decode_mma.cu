@@ -25,10 +25,13 @@
 //     CTA's codes when they fit: the loads are L2 round trips, so many must be
 //     in flight; SWIZZLE_128B, the K-major layout the MMA descriptor names;
 //     rows past M are zero-filled);
-//   - eight converter warps unpack each stage's 2-bit weights in registers
-//     ((w >> 2m) & 0x03030303 is the codes of weights 4m..4m+3 as bytes, in
-//     natural order) and store them with tcgen05.st into a 12-stage ring of A
-//     tiles in TMEM (32 columns = 128 bytes per row and stage);
+//   - four groups of four converter warps take the stages round-robin (a
+//     stage's conversion is a chain of waits, loads and a TMEM store round
+//     trip; four in flight keep up with the MMAs); a thread unpacks its
+//     weight row's 128 weights of the stage in registers ((w >> 2m) &
+//     0x03030303 is the codes of weights 4m..4m+3 as bytes, in natural order)
+//     and stores them with one tcgen05.st into a 12-stage ring of A tiles in
+//     TMEM (32 columns = 128 bytes per row and stage);
 //   - one thread issues tcgen05.mma.cta_group::1.kind::i8 (A u8 from TMEM,
 //     B s8 from shared memory, D s32 in TMEM) and commits each stage back.
 // The weights enter as the unsigned code c = t + 1, so the result carries
@@ -43,8 +46,7 @@
 //
 // TMEM: all 512 columns (D in [0, NT), the A ring in [128, 512)); the dynamic
 // shared memory is at least 116 KB, so no two CTAs of this kernel share an SM.
-// The converters fill the A ring in batches of four stages with one wait for
-// their TMEM stores per batch.  Every mbarrier
+// Every mbarrier
 // wait is bounded by the global timer; on expiry the kernel records
 // HBL_ERR_TIMEOUT, stops issuing, lets its own copies and MMAs land (bounded
 // waits again), still takes part in both cluster barriers (every thread of
@@ -66,7 +68,8 @@ constexpr int kRows = 128;  // weight rows per CTA (MMA M, TMEM lanes)
 constexpr int BK = 128;     // K bytes per stage
 constexpr int kMaxSA = 12;  // stages of the A ring in TMEM (32 columns each)
 constexpr int kMaxSB = 32;  // stages of the B ring in shared memory
-constexpr int kConvWarps = 8;
+constexpr int kConvGroups = 4;  // converter warp groups (stages round-robin)
+constexpr int kConvWarps = 4 * kConvGroups;
 constexpr int kThreads = 32 * (2 + kConvWarps);
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kACol = 128;  // first TMEM column of the A ring
@@ -199,6 +202,19 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
         "r"(r[15])
         : "memory");
 }
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+        "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
+        "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(
+            taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+        "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
+        "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
+        "r"(r[29]), "r"(r[30]), "r"(r[31])
+        : "memory");
+}
 __device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t* v) {
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
@@ -251,7 +267,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init_count(empty_b(s), 1);
         }
         for (int s = 0; s < SA; ++s) {
-            mbar_init_count(full_a(s), kConvWarps);
+            mbar_init_count(full_a(s), 4);  // the four warps of one converter group
             mbar_init_count(empty_a(s), 1);
         }
         for (int g = 0; g < kMaxGroups; ++g) mbar_init_count(wbar(g), 1);
@@ -354,68 +370,58 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         __syncwarp();
     } else {
-        // ---------------- converters: one weight row (TMEM lane) and one
-        // 64-weight half of each stage per thread
+        // ---------------- converters: kConvGroups groups of four warps; group g
+        // takes the stages kb = g (mod kConvGroups), each thread one weight row
+        // (its TMEM lane) of the stage: two 16-byte reads, 32 words, one store
         const int cw = warp - 2;
         const int q = warp & 3;  // the TMEM lane quarter this warp may access
-        const int h = cw >> 2;
+        const int grp = cw >> 2;
         const int r = 32 * q + lane;
         const uint32_t lane_base = (uint32_t)(32 * q) << 16;
         const int kb_per_g = nkb / p.G;
-        // stages go in batches of CB: the batch's stores are issued back to back
-        // and waited for once (a TMEM store round trip per batch, not per stage)
-        constexpr int CB = 4;
         bool ok = true;
-        for (int kb0 = 0; kb0 < nkb && ok; kb0 += CB) {
-            const int nb = min(CB, nkb - kb0);
-            for (int i = 0; i < nb; ++i) {
-                const int kb = kb0 + i;
-                if (kb % kb_per_g == 0 && !warp_wait(wbar(kb / kb_per_g), 0)) {
+        int landed = 0;  // weight boxes this warp has seen land
+        for (int kb = grp; kb < nkb; kb += kConvGroups) {
+            if (kb / kb_per_g >= landed) {
+                if (!warp_wait(wbar(kb / kb_per_g), 0)) {
                     ok = false;
                     break;
                 }
-                if (kb >= SA && !warp_wait(empty_a(kb % SA), (uint32_t)(((kb / SA) - 1) & 1))) {
-                    ok = false;
-                    break;
-                }
+                landed = kb / kb_per_g + 1;
             }
-            if (!ok || __shfl_sync(0xffffffffu, *abort_flag, 0) != 0) {
+            if ((kb >= SA && !warp_wait(empty_a(kb % SA), (uint32_t)(((kb / SA) - 1) & 1))) ||
+                __shfl_sync(0xffffffffu, *abort_flag, 0) != 0) {
                 ok = false;
                 break;
             }
             tc_fence_after();
-#pragma unroll
-            for (int i = 0; i < CB; ++i) {
-                if (i < nb) {
-                    const int kb = kb0 + i;
-                    // this thread's 16 bytes (64 weights) of row r in stage kb:
-                    // chunk c of the row's 128-byte line in box kb / 4, swizzled by r % 8
-                    uint32_t waddr;
-                    if (p.sw) {
-                        const uint32_t c = (uint32_t)(((kb & 3) << 1) | h);
-                        waddr = w_s + (uint32_t)((kb >> 2) * kBoxBytes + r * 128) +
-                                ((c ^ (uint32_t)(r & 7)) << 4);
-                    } else {
-                        waddr = w_s + (uint32_t)(r * (p.Kc / 4) + kb * 32 + 16 * h);
-                    }
-                    const uint4 w = lds128(waddr);
-                    const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
-                    uint32_t v[16];
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        v[4 * j + 0] = wv[j] & 0x03030303u;
-                        v[4 * j + 1] = (wv[j] >> 2) & 0x03030303u;
-                        v[4 * j + 2] = (wv[j] >> 4) & 0x03030303u;
-                        v[4 * j + 3] = (wv[j] >> 6) & 0x03030303u;
-                    }
-                    tmem_st16(tmem + lane_base + kACol + 32u * (uint32_t)(kb % SA) + 16u * h, v);
-                }
+            // row r's 32 bytes (128 weights) of stage kb: chunks 2(kb%4), +1 of
+            // the row's 128-byte line in box kb / 4, swizzled by r % 8
+            uint32_t a0, a1;
+            if (p.sw) {
+                const uint32_t line = w_s + (uint32_t)((kb >> 2) * kBoxBytes + r * 128);
+                const uint32_t c0 = (uint32_t)((kb & 3) << 1);
+                a0 = line + ((c0 ^ (uint32_t)(r & 7)) << 4);
+                a1 = line + (((c0 + 1u) ^ (uint32_t)(r & 7)) << 4);
+            } else {
+                a0 = w_s + (uint32_t)(r * (p.Kc / 4) + kb * 32);
+                a1 = a0 + 16u;
             }
+            const uint4 w0 = lds128(a0), w1 = lds128(a1);
+            const uint32_t wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+            uint32_t v[32];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                v[4 * j + 0] = wv[j] & 0x03030303u;
+                v[4 * j + 1] = (wv[j] >> 2) & 0x03030303u;
+                v[4 * j + 2] = (wv[j] >> 4) & 0x03030303u;
+                v[4 * j + 3] = (wv[j] >> 6) & 0x03030303u;
+            }
+            tmem_st32(tmem + lane_base + kACol + 32u * (uint32_t)(kb % SA), v);
             asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
             tc_fence_before();
             __syncwarp();
-            if (lane == 0)
-                for (int i = 0; i < nb; ++i) mbar_arrive_one(full_a((kb0 + i) % SA));
+            if (lane == 0) mbar_arrive_one(full_a(kb % SA));
         }
         if (!ok && lane == 0) {
             *abort_flag = 1;
@@ -428,7 +434,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ready && lane == 0) report_status(p.status, HBL_ERR_TIMEOUT);
         tc_fence_after();
         const bool aborted = __shfl_sync(0xffffffffu, *abort_flag, 0) != 0;
-        if (ready && !aborted) {
+        if (ready && !aborted && cw < 8) {  // the first two groups drain D
+            const int h = cw >> 2;
             // partials [NT][128] int32 over the (consumed) weight rows
             int32_t* part = reinterpret_cast<int32_t*>(base);
             constexpr int HC = NT / 2;  // columns (tokens) of this warp

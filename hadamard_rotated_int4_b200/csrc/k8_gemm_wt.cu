@@ -24,10 +24,12 @@
 // weight block varies fastest): the packed weights (16.8 MB for 4096 x 16384)
 // and the token blocks in flight stay in L2, so HBM sees each code once.
 // Warp 0 allocates TMEM (512 columns: the 128 x 256 int32 accumulator in
-// [0, 256), an 8-stage ring of A tiles in [256, 512)) and one lane issues the
+// [0, 256), a 5-stage ring of A tiles in [256, 416)) and one lane issues the
 // MMAs; warp 1 issues the TMA loads (5-stage ring of 36 KB: 32 KB of codes and
-// 4 KB of packed weights); warps 2-9 convert, four stages per wait for their
-// TMEM stores; warps 10-17 drain the
+// 4 KB of packed weights); warps 2-13 convert, in three groups of four warps
+// that take the stages round-robin (one stage's conversion is a chain of
+// waits, loads and a TMEM store round trip; three in flight keep up with the
+// MMAs); warps 14-21 drain the
 // accumulator (tcgen05.ld), subtract rowsum, scale and store bf16 Y.  Every
 // mbarrier wait is bounded by the global timer; on expiry the kernel records
 // HBL_ERR_TIMEOUT, stops issuing, lets its copies and MMAs land (bounded) and
@@ -49,9 +51,13 @@ constexpr int kRows = 128;  // weight rows per tile (MMA M, TMEM lanes)
 constexpr int NT = 256;     // tokens per tile (MMA N)
 constexpr int BK = 128;     // K bytes per stage
 constexpr int S = 5;        // stages of the shared-memory ring (codes + packed weights)
-constexpr int SA = 8;       // stages of the TMEM A ring (32 columns each)
-constexpr int CB = 4;       // converter batch: stages stored per wait for the TMEM stores
-constexpr int kConvWarps = 8;
+// stages of the TMEM A ring (32 columns each).  SA <= S keeps every mbarrier
+// wait within one phase of the barrier's state: a converter group waits for
+// stage j's codes and weights only after the MMAs of stage j - SA (hence the
+// loads of stage j - S) are done, and groups run at most one A round apart.
+constexpr int SA = S;
+constexpr int kConvGroups = 3;  // converter groups of four warps, stages round-robin
+constexpr int kConvWarps = 4 * kConvGroups;
 constexpr int kEpiWarps = 8;
 constexpr int kThreads = 32 * (2 + kConvWarps + kEpiWarps);
 constexpr uint32_t kTmemCols = 512;
@@ -60,7 +66,8 @@ constexpr int kBBytes = NT * BK;         // 32 KB of codes per stage
 constexpr int kWBytes = kRows * BK / 4;  // 4 KB of packed weights per stage
 constexpr int kStage = kBBytes + kWBytes;
 constexpr int kBarOff = S * kStage;
-constexpr int kSmemBytes = kBarOff + 256 + 1024;
+constexpr int kEpiOff = kBarOff + 256;  // per-tile token scales and row sums, double-buffered
+constexpr int kSmemBytes = kEpiOff + 2 * NT * 8 + 1024;
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 
 // kind::i8: D s32, A u8 (weights from TMEM), B s8 (codes), K-major, N = 256, M = 128.
@@ -144,6 +151,19 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
         "r"(r[15])
         : "memory");
 }
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+        "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
+        "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(
+            taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+        "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
+        "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
+        "r"(r[29]), "r"(r[30]), "r"(r[31])
+        : "memory");
+}
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
@@ -193,7 +213,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init_count(empty(s), 1);
         }
         for (int s = 0; s < SA; ++s) {
-            mbar_init_count(full_a(s), kConvWarps);
+            mbar_init_count(full_a(s), 4);  // the four warps of one converter group
             mbar_init_count(empty_a(s), 1);
         }
         mbar_init_count(acc_full, 1);
@@ -291,60 +311,45 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         __syncwarp();
     } else if (warp < 2 + kConvWarps) {
-        // ---------------- converters: weight row r (TMEM lane), 64-weight half h
+        // ---------------- converters: group g takes the stages it = g (mod
+        // kConvGroups) of the CTA's stage sequence; a thread converts its weight
+        // row (TMEM lane) of the stage: 32 bytes read (the 32-byte swizzle puts
+        // 16-byte chunk c of row r at chunk c ^ ((r >> 2) & 1)), 32 words, one store
         const int cw = warp - 2;
         const int q = warp & 3;
-        const int h = cw >> 2;
+        const int grp = cw >> 2;
         const int r = 32 * q + lane;
         const uint32_t lane_base = (uint32_t)(32 * q) << 16;
-        // the 32-byte swizzle of the weight box: 16-byte chunk h of row r sits
-        // at chunk h ^ ((r >> 2) & 1)
-        const uint32_t woff = (uint32_t)kBBytes + (uint32_t)(r * 32) +
-                              ((uint32_t)(h ^ ((r >> 2) & 1)) << 4);
-        // stages in batches of CB (within a tile): the batch's TMEM stores are
-        // issued back to back and waited for once
-        uint32_t it = 0;
+        const uint32_t sw = (uint32_t)((r >> 2) & 1);
+        const uint32_t w0off = (uint32_t)kBBytes + (uint32_t)(r * 32) + (sw << 4);
+        const uint32_t w1off = (uint32_t)kBBytes + (uint32_t)(r * 32) + ((sw ^ 1u) << 4);
+        const uint32_t total = (uint32_t)(((p.tiles - blockIdx.x + gridDim.x - 1) / gridDim.x) * nkb);
         bool ok = true;
-        for (int64_t t = blockIdx.x; t < p.tiles && ok; t += gridDim.x) {
-            for (int kb0 = 0; kb0 < nkb && ok; kb0 += CB) {
-                const int nb = min(CB, nkb - kb0);
-                for (int i = 0; i < nb; ++i) {
-                    const uint32_t j = it + (uint32_t)i;
-                    if (!warp_wait(full((int)(j % S)), (j / S) & 1) ||
-                        (j >= (uint32_t)SA && !warp_wait(empty_a((int)(j % SA)), ((j / SA) - 1) & 1))) {
-                        ok = false;
-                        break;
-                    }
-                }
-                if (!ok || __shfl_sync(0xffffffffu, *abort_flag, 0) != 0) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-#pragma unroll
-                for (int i = 0; i < CB; ++i) {
-                    if (i < nb) {
-                        const uint32_t j = it + (uint32_t)i;
-                        const uint4 w = lds128(base_s + (uint32_t)((j % S) * kStage) + woff);
-                        const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
-                        uint32_t v[16];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            v[4 * e + 0] = wv[e] & 0x03030303u;
-                            v[4 * e + 1] = (wv[e] >> 2) & 0x03030303u;
-                            v[4 * e + 2] = (wv[e] >> 4) & 0x03030303u;
-                            v[4 * e + 3] = (wv[e] >> 6) & 0x03030303u;
-                        }
-                        tmem_st16(tmem + lane_base + kACol + 32u * (j % SA) + 16u * h, v);
-                    }
-                }
-                asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0)
-                    for (int i = 0; i < nb; ++i) mbar_arrive_one(full_a((int)((it + i) % SA)));
-                it += (uint32_t)nb;
+        for (uint32_t it = (uint32_t)grp; it < total; it += kConvGroups) {
+            const int s = (int)(it % S), a = (int)(it % SA);
+            if (!warp_wait(full(s), (it / S) & 1) ||
+                (it >= (uint32_t)SA && !warp_wait(empty_a(a), ((it / SA) - 1) & 1)) ||
+                __shfl_sync(0xffffffffu, *abort_flag, 0) != 0) {
+                ok = false;
+                break;
             }
+            tc_fence_after();
+            const uint32_t st_s = base_s + (uint32_t)(s * kStage);
+            const uint4 w0 = lds128(st_s + w0off), w1 = lds128(st_s + w1off);
+            const uint32_t wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+            uint32_t v[32];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                v[4 * e + 0] = wv[e] & 0x03030303u;
+                v[4 * e + 1] = (wv[e] >> 2) & 0x03030303u;
+                v[4 * e + 2] = (wv[e] >> 4) & 0x03030303u;
+                v[4 * e + 3] = (wv[e] >> 6) & 0x03030303u;
+            }
+            tmem_st32(tmem + lane_base + kACol + 32u * (uint32_t)a, v);
+            asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_one(full_a(a));
         }
         if (!ok && lane == 0) {
             *abort_flag = 1;
@@ -372,6 +377,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                 break;
             }
             tc_fence_after();
+            // the tile's 256 token scales (alpha * s) and row sums, one per thread
+            float* tsc = reinterpret_cast<float*>(base + kEpiOff) + (tc & 1) * 2 * NT;
+            int* trs = reinterpret_cast<int*>(tsc + NT);
+            {
+                const int j = 32 * ew + lane;
+                const int64_t m = mb * NT + j;
+                tsc[j] = m < p.M ? __fmul_rn(alpha, p.scales[m]) : 0.f;
+                trs[j] = m < p.M ? p.rowsum[m] : 0;
+            }
+            named_barrier(1, 32 * kEpiWarps);
             const int n = nb * kRows + r;
             const bool nok = n < p.N;
 #pragma unroll 1
@@ -390,8 +405,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int e = 0; e < 32; ++e) {
                     const int64_t m = m0 + e;
                     if (nok && m < p.M) {
-                        const int a = (int)v[e] - p.rowsum[m];
-                        const float sc = __fmul_rn(alpha, p.scales[m]);
+                        const int a = (int)v[e] - trs[c0 + e];
+                        const float sc = tsc[c0 + e];
                         p.Y[m * p.N + n] =
                             __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn((float)a, sc)));
                         if (p.acc_out != nullptr) p.acc_out[m * p.N + n] = a;
