@@ -417,9 +417,12 @@ def run_hbl(args):
                                     if T <= 16384 // Kd
                                     else "K1 + GEMV half of the one-kernel forward (weights "
                                          "bulk-copied under K1)"
-                                    if Kd == 16384 and T <= 8
+                                    if Kd == 16384 and T <= 4
                                     else "row GEMV (weight rows per warp, PDL after K1)"
-                                    if T <= (4 if Kd >= 16384 else 8)
+                                    if T <= 4
+                                    else "K1 + decode tensor-core kernel (weights in TMEM as "
+                                         "A, tokens as B, cluster K-split, DSMEM reduction)"
+                                    if T <= 64 or (T <= 128 and Kd <= 8192)
                                     else "gemm_ts (TMEM activations, one-wave split-K)"),
                            "timing": "CUDA graph replay, one forward per weight copy"})
         del pcs

@@ -83,8 +83,9 @@ bool path_valid(int path) { return path >= HBL_PATH_AUTO && path <= HBL_PATH_TC_
 // Shapes the decode-batch tensor-core kernel takes (one-byte codes); whether a
 // launch plan fits the device is checked again at launch, which falls back to
 // the TMEM-activation kernel (its workspace is reserved for that).
-bool dec_shape(int64_t M, int K) { return M >= 1 && M <= decode_mma_max_m() && K >= 128; }
-// Automatic choice: batches of kDecMinM..kDecMaxM tokens take it.
+bool dec_shape(int64_t M, int K) { return M >= 1 && M <= decode_mma_max_m() && K >= 512; }
+// Automatic choice: batches of kDecMinM..kDecMaxM tokens take it (when its
+// launch plan fits the device; otherwise the TMEM-activation kernel).
 constexpr int64_t kDecMinM = 5, kDecMaxM = 128;
 
 // The back end for M tokens under `path` (HBL_PATH_*); `bytes`: the codes are
@@ -95,12 +96,12 @@ Back pick(int64_t M, int K, bool bytes, int path) {
     if (path == 3) return Back::TS;
     if (path == 4) return (bytes && K >= 128) ? Back::TMA : Back::TS;
     if (path == 5) return (bytes && dec_shape(M, K)) ? Back::DEC : Back::TS;
-    if (path == 6) return (bytes && K >= 128) ? Back::WT : Back::TS;
+    if (path == 6) return (bytes && K >= 256) ? Back::WT : Back::TS;
     // CUDA cores for a few tokens: the row GEMV where it takes the batch in one
     // launch; past that at K >= 16384 the tensor-core kernel is faster than the
     // split-K GEMV
-    if (M <= gemv_max_m() && (rows_gemv(M, K) || K < 16384)) return Back::GEMV;
     if (bytes && dec_shape(M, K) && M >= kDecMinM && M <= kDecMaxM) return Back::DEC;
+    if (M <= gemv_max_m() && (rows_gemv(M, K) || K < 16384)) return Back::GEMV;
     if (bytes && K >= 128 && M >= kTmaMinM) return Back::TMA;
     return Back::TS;
 }
@@ -401,7 +402,7 @@ static hbl_status forward_impl(const uint16_t* X, const float* gain, int M, int 
     // Other decode batches of up to 8 tokens at K = 16384: K1 (one byte per
     // code, row-major), then the one-kernel forward's GEMV half, its weight
     // rows streaming into shared memory under K1.
-    if (path == HBL_PATH_AUTO && decode_gemv_supported(M, K, N, sms)) {
+    if (path == HBL_PATH_AUTO && M < kDecMinM && decode_gemv_supported(M, K, N, sms)) {
         hbl_status st = launch_norm_fwht_quant(X, gain, M, K, norm_eps, quant_eps,
                                                act_bits == 4 ? 6 : 8, codes, scales, rowsum,
                                                nullptr, s, sms, variant);
@@ -409,7 +410,14 @@ static hbl_status forward_impl(const uint16_t* X, const float* gain, int M, int 
         GemvArgs g{codes, scales, rowsum, M, K, N, W_packed, alpha, Y, dev_status};
         return launch_decode_gemv(g, s, sms);
     }
-    const FwdPlan f = forward_plan(M, K, act_bits, path);
+    FwdPlan f = forward_plan(M, K, act_bits, path);
+    if (f.back == Back::DEC && path == HBL_PATH_AUTO && !decode_mma_supported(M, K, N, sms)) {
+        // no decode plan fits (e.g. too many tokens for the shared memory left
+        // next to the weights): the TMEM-activation kernel with its codes layout
+        f.back = Back::TS;
+        f.k1_mode = act_bits == 4 ? 5 : 9;
+        f.interleaved = true;
+    }
     hbl_status st = launch_norm_fwht_quant(X, gain, M, K, norm_eps, quant_eps, f.k1_mode, codes,
                                            scales, rowsum, nullptr, s, sms, variant);
     if (st != HBL_OK) return st;

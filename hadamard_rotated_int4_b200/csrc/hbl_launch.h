@@ -171,7 +171,7 @@ hbl_status launch_decode_mma(const GemmArgs& a, cudaStream_t stream, int num_sms
 // K8: tensor-core GEMM for large batches on the packed weights: weights widened
 // in registers into TMEM as the MMA's A operand (128 rows per tile), codes one
 // byte each (a.act_bits 8, row-major) as B by TMA (256 tokens per tile).  No
-// workspace.  K a multiple of 128.
+// workspace.  K a multiple of 256.
 hbl_status launch_gemm_wt(const GemmArgs& a, cudaStream_t stream, int num_sms);
 
 // Fixed scratch of the allocation-free GEMV entry point (file-scope device array).

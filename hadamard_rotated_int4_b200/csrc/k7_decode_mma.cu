@@ -20,20 +20,22 @@
 //     the 128-byte swizzle (so the converters' 16-byte reads are free of bank
 //     conflicts), each on its own mbarrier: the whole weight stream runs under
 //     the quantiser kernel, in a few large requests;
-//   - one thread TMA-loads the tokens' codes for each 128-byte K stage into a
-//     ring that takes the rest of shared memory (up to 32 stages, all of the
-//     CTA's codes when they fit: the loads are L2 round trips, so many must be
-//     in flight; SWIZZLE_128B, the K-major layout the MMA descriptor names;
-//     rows past M are zero-filled);
-//   - four groups of four converter warps take the stages round-robin (a
-//     stage's conversion is a chain of waits, loads and a TMEM store round
-//     trip; four in flight keep up with the MMAs); a thread unpacks its
-//     weight row's 128 weights of the stage in registers ((w >> 2m) &
+//   - one thread TMA-loads the tokens' codes for each 512-byte K stage (four
+//     128-byte-wide boxes) into a ring that takes the rest of shared memory
+//     (all of the CTA's codes when they fit: the loads are L2 round trips, so
+//     many must be in flight; SWIZZLE_128B, the K-major layout the MMA
+//     descriptor names; rows past M are zero-filled);
+//   - three groups of four converter warps take the stages round-robin (a
+//     stage's conversion is a chain of waits, loads and TMEM store round
+//     trips; three in flight keep up with the MMAs); a thread unpacks its
+//     weight row's 512 weights of the stage in registers ((w >> 2m) &
 //     0x03030303 is the codes of weights 4m..4m+3 as bytes, in natural order)
-//     and stores them with one tcgen05.st into a 12-stage ring of A tiles in
-//     TMEM (32 columns = 128 bytes per row and stage);
+//     and stores them with four tcgen05.st into a 3-stage ring of A tiles in
+//     TMEM (128 columns = 512 bytes per row and stage);
 //   - one thread issues tcgen05.mma.cta_group::1.kind::i8 (A u8 from TMEM,
-//     B s8 from shared memory, D s32 in TMEM) and commits each stage back.
+//     B s8 from shared memory, D s32 in TMEM), sixteen per stage (a stage's
+//     barrier waits and commits cost about as much issue time as four MMAs),
+//     and commits each stage back.
 // The weights enter as the unsigned code c = t + 1, so the result carries
 // sum_k q*c = acc + rowsum[m]; rowsum is subtracted once in the epilogue.
 //
@@ -65,10 +67,15 @@ namespace hbl {
 namespace k7 {
 
 constexpr int kRows = 128;  // weight rows per CTA (MMA M, TMEM lanes)
-constexpr int BK = 128;     // K bytes per stage
-constexpr int kMaxSA = 12;  // stages of the A ring in TMEM (32 columns each)
+constexpr int BK = 512;     // K bytes per stage: 16 MMAs of K = 32 (a stage's barrier
+                            // waits and commits cost about as much issue time as
+                            // four MMAs, so stages are long)
+constexpr int kSub = BK / 128;  // 128-byte K sub-tiles per stage (one TMA box of codes each)
+constexpr int kMaxSA = 3;   // stages of the A ring in TMEM (128 columns each)
 constexpr int kMaxSB = 32;  // stages of the B ring in shared memory
-constexpr int kConvGroups = 4;  // converter warp groups (stages round-robin)
+// converter warp groups (stages round-robin); no more groups than A stages, so
+// every empty-slot wait is within one phase of the barrier's state
+constexpr int kConvGroups = kMaxSA;
 constexpr int kConvWarps = 4 * kConvGroups;
 constexpr int kThreads = 32 * (2 + kConvWarps);
 constexpr uint32_t kTmemCols = 512;
@@ -89,9 +96,8 @@ __host__ __device__ constexpr uint32_t idesc() {
 struct Params {
     int M, K, N;
     int Kc;        // K per CTA (K / cluster size), a multiple of BK
-    int G;         // weight boxes: Kc / 512 swizzled 128-byte boxes, or one
-                   // unswizzled box of Kc / 4 bytes per row when Kc < 512
-    int sw;        // the weight boxes are 128-byte swizzled
+    int G;         // weight boxes: Kc / 512 swizzled 128-byte boxes, one per stage
+    int sw;        // the weight boxes are 128-byte swizzled (always, Kc >= 512)
     uint32_t b_off;  // offset of the B ring from the 1024-aligned base
     uint32_t bar_off;
     int SA, SB;      // ring depths (A in TMEM, B in shared memory)
@@ -289,9 +295,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---- the CTA's weight rows (its K slice) into shared memory: the weights
     // are not the previous kernel's output, so this runs before the dependency
     // wait, under that kernel
-    // box g: bytes [k0/4 + g * inner, + inner) of rows [n0, n0 + 128) (rows
-    // past N read as zeros; the full box counts toward the transaction bytes)
-    const int inner = p.sw ? 128 : p.Kc / 4;
+    // box g (= stage g): bytes [k0/4 + 128 g, + 128) of rows [n0, n0 + 128)
+    // (rows past N read as zeros; the full box counts toward the transaction
+    // bytes)
+    constexpr int inner = 128;
     auto load_weights = [&] {
         if (lane == 0)
             for (int g = 0; g < p.G; ++g) {
@@ -324,7 +331,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t bsm = b_s + (uint32_t)(sb * NT * BK);
 #pragma unroll
                 for (int k = 0; k < BK / 32; ++k)
-                    mma_ts<NT>(tmem, tmem + kACol + 32u * sa + 8u * k, sdesc(bsm + 32 * k),
+                    mma_ts<NT>(tmem, tmem + kACol + (uint32_t)(BK / 4) * sa + 8u * k,
+                               sdesc(bsm + (k >> 2) * NT * 128 + 32 * (k & 3)),
                                (kb | k) != 0 ? 1u : 0u);
                 mma_commit(empty_a(sa));
                 mma_commit(empty_b(sb));
@@ -357,7 +365,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     break;
                 }
                 mbar_expect_tx(full_b(s), (uint32_t)(NT * BK));
-                tma_load(b_s + (uint32_t)(s * NT * BK), &tmB, k0 + kb * BK, 0, full_b(s));
+#pragma unroll
+                for (int j = 0; j < kSub; ++j)
+                    tma_load(b_s + (uint32_t)(s * NT * BK + j * NT * 128), &tmB,
+                             k0 + kb * BK + 128 * j, 0, full_b(s));
                 ++issued;
             }
             if (!ok) {
@@ -378,46 +389,35 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int grp = cw >> 2;
         const int r = 32 * q + lane;
         const uint32_t lane_base = (uint32_t)(32 * q) << 16;
-        const int kb_per_g = nkb / p.G;
         bool ok = true;
-        int landed = 0;  // weight boxes this warp has seen land
         for (int kb = grp; kb < nkb; kb += kConvGroups) {
-            if (kb / kb_per_g >= landed) {
-                if (!warp_wait(wbar(kb / kb_per_g), 0)) {
-                    ok = false;
-                    break;
-                }
-                landed = kb / kb_per_g + 1;
-            }
-            if ((kb >= SA && !warp_wait(empty_a(kb % SA), (uint32_t)(((kb / SA) - 1) & 1))) ||
+            if (!warp_wait(wbar(kb), 0) ||
+                (kb >= SA && !warp_wait(empty_a(kb % SA), (uint32_t)(((kb / SA) - 1) & 1))) ||
                 __shfl_sync(0xffffffffu, *abort_flag, 0) != 0) {
                 ok = false;
                 break;
             }
             tc_fence_after();
-            // row r's 32 bytes (128 weights) of stage kb: chunks 2(kb%4), +1 of
-            // the row's 128-byte line in box kb / 4, swizzled by r % 8
-            uint32_t a0, a1;
-            if (p.sw) {
-                const uint32_t line = w_s + (uint32_t)((kb >> 2) * kBoxBytes + r * 128);
-                const uint32_t c0 = (uint32_t)((kb & 3) << 1);
-                a0 = line + ((c0 ^ (uint32_t)(r & 7)) << 4);
-                a1 = line + (((c0 + 1u) ^ (uint32_t)(r & 7)) << 4);
-            } else {
-                a0 = w_s + (uint32_t)(r * (p.Kc / 4) + kb * 32);
-                a1 = a0 + 16u;
-            }
-            const uint4 w0 = lds128(a0), w1 = lds128(a1);
-            const uint32_t wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-            uint32_t v[32];
+            // row r's 128 bytes (512 weights) of stage kb: the row's line in box
+            // kb, 16-byte chunk c at c ^ (r % 8); sub-tile j = chunks 2j, 2j + 1
+            const uint32_t line = w_s + (uint32_t)(kb * kBoxBytes + r * 128);
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                v[4 * j + 0] = wv[j] & 0x03030303u;
-                v[4 * j + 1] = (wv[j] >> 2) & 0x03030303u;
-                v[4 * j + 2] = (wv[j] >> 4) & 0x03030303u;
-                v[4 * j + 3] = (wv[j] >> 6) & 0x03030303u;
+            for (int j = 0; j < kSub; ++j) {
+                const uint4 w0 = lds128(line + (((uint32_t)(2 * j) ^ (uint32_t)(r & 7)) << 4));
+                const uint4 w1 = lds128(line + (((uint32_t)(2 * j + 1) ^ (uint32_t)(r & 7)) << 4));
+                const uint32_t wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+                uint32_t v[32];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    v[4 * e + 0] = wv[e] & 0x03030303u;
+                    v[4 * e + 1] = (wv[e] >> 2) & 0x03030303u;
+                    v[4 * e + 2] = (wv[e] >> 4) & 0x03030303u;
+                    v[4 * e + 3] = (wv[e] >> 6) & 0x03030303u;
+                }
+                tmem_st32(tmem + lane_base + kACol + (uint32_t)(BK / 4) * (uint32_t)(kb % SA) +
+                              32u * j,
+                          v);
             }
-            tmem_st32(tmem + lane_base + kACol + 32u * (uint32_t)(kb % SA), v);
             asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
             tc_fence_before();
             __syncwarp();
@@ -525,7 +525,7 @@ static bool make_codes_map(CUtensorMap* map, const void* codes, int M, int K, in
     if (fn == nullptr) return false;
     const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M};
     const cuuint64_t strides[1] = {(cuuint64_t)K};
-    const cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)NT};
+    const cuuint32_t box[2] = {128u, (cuuint32_t)NT};
     const cuuint32_t estr[2] = {1, 1};
     return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(codes), dims, strides, box,
               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,

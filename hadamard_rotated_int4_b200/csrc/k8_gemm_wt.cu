@@ -24,9 +24,11 @@
 // weight block varies fastest): the packed weights (16.8 MB for 4096 x 16384)
 // and the token blocks in flight stay in L2, so HBM sees each code once.
 // Warp 0 allocates TMEM (512 columns: the 128 x 256 int32 accumulator in
-// [0, 256), a 5-stage ring of A tiles in [256, 416)) and one lane issues the
-// MMAs; warp 1 issues the TMA loads (5-stage ring of 36 KB: 32 KB of codes and
-// 4 KB of packed weights); warps 2-13 convert, in three groups of four warps
+// [0, 256), a 3-stage ring of A tiles in [256, 448)) and one lane issues the
+// MMAs, eight per 256-byte K stage (a stage's barrier waits and commits cost
+// about as much issue time as four MMAs, so stages are long); warp 1 issues
+// the TMA loads (3-stage ring of 72 KB: 64 KB of codes in two 128-byte-wide
+// boxes and 8 KB of packed weights in two 32-byte-wide boxes); warps 2-13 convert, in three groups of four warps
 // that take the stages round-robin (one stage's conversion is a chain of
 // waits, loads and a TMEM store round trip; three in flight keep up with the
 // MMAs); warps 14-21 drain the
@@ -49,8 +51,9 @@ namespace k8 {
 
 constexpr int kRows = 128;  // weight rows per tile (MMA M, TMEM lanes)
 constexpr int NT = 256;     // tokens per tile (MMA N)
-constexpr int BK = 128;     // K bytes per stage
-constexpr int S = 5;        // stages of the shared-memory ring (codes + packed weights)
+constexpr int BK = 256;     // K bytes per stage: 8 MMAs of K = 32
+constexpr int kSub = BK / 128;  // 128-byte K sub-tiles per stage (one TMA box of codes each)
+constexpr int S = 3;        // stages of the shared-memory ring (codes + packed weights)
 // stages of the TMEM A ring (32 columns each).  SA <= S keeps every mbarrier
 // wait within one phase of the barrier's state: a converter group waits for
 // stage j's codes and weights only after the MMAs of stage j - SA (hence the
@@ -62,8 +65,8 @@ constexpr int kEpiWarps = 8;
 constexpr int kThreads = 32 * (2 + kConvWarps + kEpiWarps);
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kACol = 256;
-constexpr int kBBytes = NT * BK;         // 32 KB of codes per stage
-constexpr int kWBytes = kRows * BK / 4;  // 4 KB of packed weights per stage
+constexpr int kBBytes = NT * BK;         // 64 KB of codes per stage (two 32 KB boxes)
+constexpr int kWBytes = kRows * BK / 4;  // 8 KB of packed weights per stage (two 4 KB boxes)
 constexpr int kStage = kBBytes + kWBytes;
 constexpr int kBarOff = S * kStage;
 constexpr int kEpiOff = kBarOff + 256;  // per-tile token scales and row sums, double-buffered
@@ -259,7 +262,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint32_t sb = base_s + (uint32_t)(s * kStage);
 #pragma unroll
                     for (int k = 0; k < BK / 32; ++k)
-                        mma_ts(tmem, tmem + kACol + 32u * a + 8u * k, sdesc(sb + 32 * k),
+                        mma_ts(tmem, tmem + kACol + (uint32_t)(BK / 4) * a + 8u * k,
+                               sdesc(sb + (k >> 2) * NT * 128 + 32 * (k & 3)),
                                (kb | k) != 0 ? 1u : 0u);
                     mma_commit(empty(s));
                     mma_commit(empty_a(a));
@@ -296,8 +300,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     const uint32_t sb = base_s + (uint32_t)(s * kStage);
                     mbar_expect_tx(full(s), (uint32_t)kStage);
-                    tma_load(sb, &tmB, kb * BK, (int)(mb * NT), full(s));
-                    tma_load(sb + kBBytes, &tmW, kb * (BK / 4), nb * kRows, full(s));
+#pragma unroll
+                    for (int j = 0; j < kSub; ++j) {
+                        tma_load(sb + j * NT * 128, &tmB, kb * BK + 128 * j, (int)(mb * NT), full(s));
+                        tma_load(sb + kBBytes + j * kRows * 32, &tmW, kb * (BK / 4) + 32 * j,
+                                 nb * kRows, full(s));
+                    }
                 }
             }
             if (!ok) {
@@ -323,6 +331,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t sw = (uint32_t)((r >> 2) & 1);
         const uint32_t w0off = (uint32_t)kBBytes + (uint32_t)(r * 32) + (sw << 4);
         const uint32_t w1off = (uint32_t)kBBytes + (uint32_t)(r * 32) + ((sw ^ 1u) << 4);
+        static_assert(kSub * kRows * 32 == kWBytes, "weight boxes fill the stage's weight part");
         const uint32_t total = (uint32_t)(((p.tiles - blockIdx.x + gridDim.x - 1) / gridDim.x) * nkb);
         bool ok = true;
         for (uint32_t it = (uint32_t)grp; it < total; it += kConvGroups) {
@@ -335,17 +344,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             tc_fence_after();
             const uint32_t st_s = base_s + (uint32_t)(s * kStage);
-            const uint4 w0 = lds128(st_s + w0off), w1 = lds128(st_s + w1off);
-            const uint32_t wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-            uint32_t v[32];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                v[4 * e + 0] = wv[e] & 0x03030303u;
-                v[4 * e + 1] = (wv[e] >> 2) & 0x03030303u;
-                v[4 * e + 2] = (wv[e] >> 4) & 0x03030303u;
-                v[4 * e + 3] = (wv[e] >> 6) & 0x03030303u;
+            for (int j = 0; j < kSub; ++j) {  // each 4 KB weight box: 128 weights of row r
+                const uint32_t bx = st_s + (uint32_t)(j * kRows * 32);
+                const uint4 w0 = lds128(bx + w0off), w1 = lds128(bx + w1off);
+                const uint32_t wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+                uint32_t v[32];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    v[4 * e + 0] = wv[e] & 0x03030303u;
+                    v[4 * e + 1] = (wv[e] >> 2) & 0x03030303u;
+                    v[4 * e + 2] = (wv[e] >> 4) & 0x03030303u;
+                    v[4 * e + 3] = (wv[e] >> 6) & 0x03030303u;
+                }
+                tmem_st32(tmem + lane_base + kACol + (uint32_t)(BK / 4) * a + 32u * j, v);
             }
-            tmem_st32(tmem + lane_base + kACol + 32u * (uint32_t)a, v);
             asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
             tc_fence_before();
             __syncwarp();
@@ -459,8 +472,8 @@ hbl_status launch_gemm_wt(const GemmArgs& a, cudaStream_t stream, int num_sms) {
     if (a.M == 0) return HBL_OK;
     if (a.K < k8::BK || a.K % k8::BK != 0) return HBL_ERR_SHAPE;
     CUtensorMap mB, mW;
-    if (!k8::make_map(&mB, a.codes, a.M, a.K, k8::BK, k8::NT, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !k8::make_map(&mW, a.W_packed, a.N, a.K / 4, k8::BK / 4, k8::kRows,
+    if (!k8::make_map(&mB, a.codes, a.M, a.K, 128, k8::NT, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !k8::make_map(&mW, a.W_packed, a.N, a.K / 4, 32, k8::kRows,
                       CU_TENSOR_MAP_SWIZZLE_32B))
         return HBL_ERR_CUDA;
     k8::Params prm;

@@ -92,11 +92,11 @@ HBL_API int hbl_version(void);
  *   HBL_PATH_TC_DECODE (5) = the decode-batch tcgen05 kernel (weights as the
  *       MMA's A operand in tensor memory, tokens as B, K split over a cluster
  *       of CTAs and reduced in distributed shared memory) whenever the codes
- *       are one byte each, M <= 128 and K >= 128 (else as 3),
+ *       are one byte each, M <= 128 and K >= 512 (else as 3),
  *   HBL_PATH_TC_PACKED (6) = the large-batch tcgen05 kernel on the packed
  *       weights (widened in registers into tensor memory as the MMA's A
  *       operand, codes as B by TMA; no expanded copy) whenever the codes are
- *       one byte each and K >= 128 (else as 3).
+ *       one byte each and K >= 256 (else as 3).
  * Every path computes the same values.  No counterpart on the BitNet v2 pages. */
 enum {
     HBL_PATH_AUTO = 0,
