@@ -54,7 +54,7 @@ def parse():
                     choices=["forward", "gemm", "quant4", "quant8", "nohad4", "ln4", "rotate",
                              "kv3", "kv4", "kv8", "decode_wo", "decode_wdown", "decode_wdown_t32",
                              "decode_wo_t32", "gemv_rows", "gemv_splitk", "pack", "expand",
-                             "int8_probe"],
+                             "int8_probe", "gemm_packed"],
                     help="run only this case (a few launches, for profiler captures); prints a "
                          "short JSON line, not the benchmark line")
     return ap.parse_args()
@@ -641,6 +641,12 @@ def run_only(args):
             ws = torch.empty(hbl.workspace_size(hbl.OP_HBITLINEAR_FORWARD, M_TOK, K_IN, N_OUT,
                                                 BITS), dtype=torch.uint8, device=dev)
             fn = lambda: hbl.hbitlinear_forward(X, packed, alpha, BITS, ws=ws)
+        elif args.only == "gemm_packed":  # the tensor-core GEMM on the packed weights
+            B8 = hbl.ACT_INT4_BYTES
+            codes, scales, rowsum = hbl.norm_fwht_quant(X, B8)
+            Yp = torch.empty((M_TOK, N_OUT), dtype=torch.bfloat16, device=dev)
+            fn = lambda: hbl.ternary_gemm(codes, scales, rowsum, B8, K_IN, packed, alpha, out=Yp,
+                                          path=hbl.PATH_TC_PACKED)
         else:  # the forward's GEMM: one-byte INT4 codes, expanded weights
             B8 = hbl.ACT_INT4_BYTES
             codes, scales, rowsum = hbl.norm_fwht_quant(X, B8)
