@@ -20,73 +20,124 @@
 namespace hbl {
 namespace k0 {
 
+// Pushes x, the perfect-tree sum of the 2^lvl elements that follow the cnt
+// elements already pushed (cnt a multiple of 2^lvl), onto a binary-counter
+// stack of partial sums: level l holds the sum of a 2^l-element block.
+__device__ __forceinline__ void push_block(float (&stk)[40], int64_t& cnt, float x, int lvl) {
+    int64_t c = cnt >> lvl;
+    int l = lvl;
+    while (c & 1) {
+        x = __fadd_rn(stk[l], x);
+        c >>= 1;
+        ++l;
+    }
+    stk[l] = x;
+    cnt += (int64_t)1 << lvl;
+}
+
+// Perfect pairwise tree of |W| over the 128 consecutive floats that lane l
+// holds four of (l*4 .. l*4+3): in-lane pairs, then xor shuffles (lane bit b =
+// block bit b).  Every lane ends with the sum.
+__device__ __forceinline__ float warp_tree128(float4 q) {
+    float s = __fadd_rn(__fadd_rn(fabsf(q.x), fabsf(q.y)), __fadd_rn(fabsf(q.z), fabsf(q.w)));
+#pragma unroll
+    for (int b = 1; b < 32; b <<= 1) s = __fadd_rn(s, __shfl_xor_sync(0xffffffffu, s, b));
+    return s;
+}
+
 // One warp per row: perfect pairwise tree of |W| over the row (K = 2^L).
-// Lane l owns the contiguous chunk [l*E, (l+1)*E) (E = K/32, or 1 element per
-// lane for K < 32); chunks are reduced in index order with a binary-counter
-// stack, then lanes combine by xor shuffles (lane bit b = chunk bit b).
+// K >= 1024: the warp reads the row in coalesced 1024-float blocks (eight
+// 16-byte loads per lane in flight), reduces each 128-float sub-block as a
+// perfect tree across the warp, the eight sub-blocks as a perfect tree, and
+// pushes the block on a (warp-uniform) binary-counter stack.  K < 1024: lane
+// l reduces [l*E, (l+1)*E) (E = K/32, or one element per lane for K < 32) in
+// index order and lanes combine by xor shuffles.
 __global__ void row_abs_sum_kernel(const float* __restrict__ W, int N, int K,
                                    float* __restrict__ rowsums) {
     const int lane = threadIdx.x & 31;
     const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int nwarps = (gridDim.x * blockDim.x) >> 5;
-    const int lanes = K < 32 ? K : 32;
-    const int E = K / lanes;
     for (int n = warp; n < N; n += nwarps) {
+        const float* row = W + (int64_t)n * K;
         float total = 0.f;
-        if (lane < lanes) {
-            const float* src = W + (int64_t)n * K + (int64_t)lane * E;
-            float stk[16];
-            int cnt = 0;  // elements consumed; stack level l holds a 2^l partial
-            for (int e = 0; e < E; ++e) {
-                float x = fabsf(src[e]);
-                int c = cnt;
-                int l = 0;
-                while (c & 1) {
-                    x = __fadd_rn(stk[l], x);
-                    c >>= 1;
-                    ++l;
-                }
-                stk[l] = x;
-                ++cnt;
+        if (K >= 1024) {
+            float stk[40];
+            int64_t cnt = 0;
+            for (int e0 = 0; e0 < K; e0 += 1024) {
+                const float4* s4 = reinterpret_cast<const float4*>(row + e0) + lane;
+                float4 q[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) q[i] = __ldg(s4 + 32 * i);
+                float t[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) t[i] = warp_tree128(q[i]);
+#pragma unroll
+                for (int w = 1; w < 8; w <<= 1)
+#pragma unroll
+                    for (int i = 0; i < 8; i += 2 * w) t[i] = __fadd_rn(t[i], t[i + w]);
+                push_block(stk, cnt, t[0], 10);
             }
-            total = stk[ilog2((unsigned)E)];
-        }
-        for (int b = 1; b < lanes; b <<= 1) {
-            float o = __shfl_xor_sync(0xffffffffu, total, b);
-            total = __fadd_rn(total, o);
+            total = stk[ilog2((unsigned)K)];
+        } else {
+            const int lanes = K < 32 ? K : 32;
+            const int E = K / lanes;
+            if (lane < lanes) {
+                const float* src = row + (int64_t)lane * E;
+                float stk[40];
+                int64_t cnt = 0;
+                for (int e = 0; e < E; ++e) push_block(stk, cnt, fabsf(src[e]), 0);
+                total = stk[ilog2((unsigned)E)];
+            }
+            for (int b = 1; b < lanes; b <<= 1)
+                total = __fadd_rn(total, __shfl_xor_sync(0xffffffffu, total, b));
         }
         if (lane == 0) rowsums[n] = total;
     }
 }
 
-// Single thread: left-complete tree over the N row sums, then alpha.
-// The left-complete tree equals perfect trees over the blocks given by the
-// binary digits of N (largest first), combined right to left.
-__global__ void alpha_kernel(const float* __restrict__ rowsums, int N, int64_t nk,
-                             float* __restrict__ alpha) {
-    if (threadIdx.x != 0 || blockIdx.x != 0) return;
-    float stk[32];
-    int64_t cnt = 0;
-    for (int n = 0; n < N; ++n) {
-        float x = rowsums[n];
-        int64_t c = cnt;
-        int l = 0;
-        while (c & 1) {
-            x = __fadd_rn(stk[l], x);
-            c >>= 1;
-            ++l;
+// One block of kAlphaThreads: left-complete tree over the N row sums, then
+// alpha.  The left-complete tree equals perfect trees over the blocks given by
+// the binary digits of N (largest first), combined right to left.  Each block
+// of 2^b sums is reduced by min(2^b, kAlphaThreads) threads, each summing a
+// contiguous power-of-two run in index order, then by adjacent pairs in
+// shared memory.
+constexpr int kAlphaThreads = 1024;
+
+__global__ void __launch_bounds__(kAlphaThreads) alpha_kernel(const float* __restrict__ rowsums,
+                                                              int N, int64_t nk,
+                                                              float* __restrict__ alpha) {
+    __shared__ float part[kAlphaThreads];
+    __shared__ float blk[32];
+    const int t = threadIdx.x;
+    int64_t off = 0;
+    int nb = 0;
+    for (int b = 30; b >= 0; --b) {
+        if (!((N >> b) & 1)) continue;
+        const int P = 1 << b;
+        const int T = P < kAlphaThreads ? P : kAlphaThreads;
+        const int E = P / T;
+        if (t < T) {
+            const float* src = rowsums + off + (int64_t)t * E;
+            float stk[40];
+            int64_t cnt = 0;
+            for (int e = 0; e < E; ++e) push_block(stk, cnt, src[e], 0);
+            part[t] = stk[ilog2((unsigned)E)];
         }
-        stk[l] = x;
-        ++cnt;
+        __syncthreads();
+        for (int w = 1; w < T; w <<= 1) {
+            if (t < T && (t & (2 * w - 1)) == 0) part[t] = __fadd_rn(part[t], part[t + w]);
+            __syncthreads();
+        }
+        if (t == 0) blk[nb] = part[0];
+        ++nb;
+        off += P;
+        __syncthreads();
     }
-    float acc = 0.f;
-    bool have = false;
-    for (int l = 0; l < 32; ++l)
-        if ((cnt >> l) & 1) {
-            acc = have ? __fadd_rn(stk[l], acc) : stk[l];
-            have = true;
-        }
-    *alpha = __fdiv_rn(acc, __ll2float_rn((long long)nk));
+    if (t == 0) {
+        float acc = nb > 0 ? blk[nb - 1] : 0.f;
+        for (int i = nb - 2; i >= 0; --i) acc = __fadd_rn(blk[i], acc);
+        *alpha = __fdiv_rn(acc, __ll2float_rn((long long)nk));
+    }
 }
 
 // One thread per packed word (16 weights).
@@ -130,7 +181,7 @@ hbl_status launch_pack_ternary(const float* W, int N, int K, float eps, uint32_t
     int blocks = (warps_needed + 7) / 8;
     if (blocks > num_sms * 8) blocks = num_sms * 8;
     k0::row_abs_sum_kernel<<<blocks, 256, 0, stream>>>(W, N, K, rowsums);
-    k0::alpha_kernel<<<1, 32, 0, stream>>>(rowsums, N, (int64_t)N * K, alpha);
+    k0::alpha_kernel<<<1, k0::kAlphaThreads, 0, stream>>>(rowsums, N, (int64_t)N * K, alpha);
     const int64_t nwords = (int64_t)N * (K / 16);
     int64_t pb = (nwords + 255) / 256;
     if (pb > (int64_t)num_sms * 16) pb = (int64_t)num_sms * 16;

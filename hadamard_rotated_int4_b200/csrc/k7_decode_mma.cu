@@ -328,11 +328,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                     break;
                 }
                 tc_fence_after();
-                const uint32_t bsm = b_s + (uint32_t)(sb * NT * BK);
+                // descriptors of the stage: the 16 MMAs step through them by
+                // constant offsets of the start-address field
+                const uint64_t bd0 = sdesc(b_s + (uint32_t)(sb * NT * BK));
+                const uint32_t ad0 = tmem + kACol + (uint32_t)(BK / 4) * sa;
 #pragma unroll
                 for (int k = 0; k < BK / 32; ++k)
-                    mma_ts<NT>(tmem, tmem + kACol + (uint32_t)(BK / 4) * sa + 8u * k,
-                               sdesc(bsm + (k >> 2) * NT * 128 + 32 * (k & 3)),
+                    mma_ts<NT>(tmem, ad0 + 8u * k,
+                               bd0 + (uint64_t)(((k >> 2) * NT * 128 + 32 * (k & 3)) >> 4),
                                (kb | k) != 0 ? 1u : 0u);
                 mma_commit(empty_a(sa));
                 mma_commit(empty_b(sb));

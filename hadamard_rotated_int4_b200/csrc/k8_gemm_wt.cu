@@ -259,11 +259,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t sb = base_s + (uint32_t)(s * kStage);
+                    // descriptors of the stage: the MMAs step through them by
+                    // constant offsets of the start-address field
+                    const uint64_t bd0 = sdesc(base_s + (uint32_t)(s * kStage));
+                    const uint32_t ad0 = tmem + kACol + (uint32_t)(BK / 4) * a;
 #pragma unroll
                     for (int k = 0; k < BK / 32; ++k)
-                        mma_ts(tmem, tmem + kACol + (uint32_t)(BK / 4) * a + 8u * k,
-                               sdesc(sb + (k >> 2) * NT * 128 + 32 * (k & 3)),
+                        mma_ts(tmem, ad0 + 8u * k,
+                               bd0 + (uint64_t)(((k >> 2) * NT * 128 + 32 * (k & 3)) >> 4),
                                (kb | k) != 0 ? 1u : 0u);
                     mma_commit(empty(s));
                     mma_commit(empty_a(a));

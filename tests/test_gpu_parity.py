@@ -278,9 +278,12 @@ def test_gemm_interleaved_layout(bits, M, K, N):
 
 # ------------------------------------------------------------ ternary pack
 
-@pytest.mark.parametrize("N,K", [(16, 16), (48, 256), (128, 256), (100, 2048), (4096, 4096),
-                                 (4096, 16384)])
+@pytest.mark.parametrize("N,K", [(16, 16), (1, 16), (7, 32), (48, 256), (128, 256), (100, 2048),
+                                 (1500, 512), (3001, 1024), (4096, 4096), (4096, 16384)])
 def test_pack_ternary(N, K):
+    # N = 3001 = 2048 + 512 + 256 + 128 + 32 + 16 + 8 + 1 exercises every
+    # block size of the left-complete tree over the row sums (two row sums
+    # per thread in the 2048 block); K < 1024 takes the lane-chunk row sums
     W = inputs.latent_weights(N, K, seed=N + K)
     packed, alpha = hbl.pack_ternary(torch.from_numpy(W).to(DEV))
     wp, wa = oracle.pack_ternary(W)
