@@ -54,7 +54,7 @@ def parse():
                     choices=["forward", "gemm", "quant4", "quant8", "nohad4", "ln4", "rotate",
                              "kv3", "kv4", "kv8", "decode_wo", "decode_wdown", "decode_wdown_t32",
                              "decode_wo_t32", "gemv_rows", "gemv_splitk", "pack", "expand",
-                             "int8_probe", "gemm_packed"],
+                             "int8_probe", "gemm_packed", "gemm_pair"],
                     help="run only this case (a few launches, for profiler captures); prints a "
                          "short JSON line, not the benchmark line")
     return ap.parse_args()
@@ -508,7 +508,8 @@ def run_hbl(args):
         # of the same MMA instruction measured by the probe on this GPU
         peak = int8_probe["tops"]
         roof = {"bound": "tensor",
-                "kernel": "gemm_tma (TMA-fed tcgen05 kind::i8, accumulators in TMEM)",
+                "kernel": "gemm_pair (TMA-fed tcgen05.mma.cta_group::2 kind::i8 on pairs of SMs, "
+                          "256 x 256 tiles, accumulators in TMEM)",
                 "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                 "peak_note": "dense INT8 (TOPS) measured on this GPU by hbl_probe_tc_int8: %d "
                              "SMs x %d back-to-back tcgen05.mma kind::i8 128x256x32 from shared "
@@ -517,8 +518,8 @@ def run_hbl(args):
                              % (n_sms, int8_probe["mmas_per_cta"], pk["source"],
                                 2.0 * pk["bf16_tflops"], achieved / (2.0 * pk["bf16_tflops"]),
                                 achieved / 4500.0),
-                "traffic": recorded_traffic("gemm_tma_a4_ffn_wdown",
-                                            source_hash("k2c_gemm_tma.cu")),
+                "traffic": recorded_traffic("gemm_pair_a4_ffn_wdown",
+                                            source_hash("k10_gemm_pair.cu")),
                 "us_per_launch": t_k2 * 1e6}
     else:
         nbytes = M_TOK * K_IN * 2 + M_TOK * K_IN + 8 * M_TOK  # one-byte codes in the forward
@@ -540,7 +541,7 @@ def run_hbl(args):
                    "l2": "inputs larger than L2 (X 268 MB per step)"},
         "roofline": roof,
         "kernels_us": {"norm_fwht_quant": t_k1 * 1e6, "expand_ternary": t_kx * 1e6,
-                       "gemm_tma": t_k2 * 1e6},
+                       "gemm_pair": t_k2 * 1e6},
         "norm_fwht_quant_views": {
             "hbm": {"bytes": M_TOK * K_IN * 3 + 8 * M_TOK,
                     "achieved_gbs": (M_TOK * K_IN * 3 + 8 * M_TOK) / t_k1 / 1e9,
@@ -647,6 +648,12 @@ def run_only(args):
             Yp = torch.empty((M_TOK, N_OUT), dtype=torch.bfloat16, device=dev)
             fn = lambda: hbl.ternary_gemm(codes, scales, rowsum, B8, K_IN, packed, alpha, out=Yp,
                                           path=hbl.PATH_TC_PACKED)
+        elif args.only == "gemm_pair":  # the paired-SM GEMM (weights expanded by the call)
+            B8 = hbl.ACT_INT4_BYTES
+            codes, scales, rowsum = hbl.norm_fwht_quant(X, B8)
+            Yp = torch.empty((M_TOK, N_OUT), dtype=torch.bfloat16, device=dev)
+            fn = lambda: hbl.ternary_gemm(codes, scales, rowsum, B8, K_IN, packed, alpha, out=Yp,
+                                          path=hbl.PATH_TC_PAIR)
         else:  # the forward's GEMM: one-byte INT4 codes, expanded weights
             B8 = hbl.ACT_INT4_BYTES
             codes, scales, rowsum = hbl.norm_fwht_quant(X, B8)

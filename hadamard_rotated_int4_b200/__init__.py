@@ -34,7 +34,7 @@ ACT_INT4_I32, ACT_INT8_I32 = 0x104, 0x108  # one byte per code, 32-row interleav
 ACT_INT4_BYTES = 0x204                      # INT4 codes one byte each, row-major
 NORM_LAYERNORM, NORM_NO_HADAMARD = 1, 2     # variant flags of norm_transform / norm_quant / bitlinear_forward
 PATH_AUTO, PATH_TC_SS, PATH_GEMV, PATH_TC_TS, PATH_TC_TMA, PATH_TC_DECODE = 0, 1, 2, 3, 4, 5
-PATH_TC_PACKED = 6
+PATH_TC_PACKED, PATH_TC_PAIR = 6, 7
 EXPORTS = ("hbl_status_string", "hbl_version", "hbl_workspace_size", "hbl_workspace_size_path",
            "hbl_pack_ternary", "hbl_norm_fwht", "hbl_norm_fwht_quant", "hbl_ternary_gemm",
            "hbl_ternary_gemm_path", "hbl_hbitlinear_forward", "hbl_hbitlinear_forward_path",
@@ -217,7 +217,8 @@ def ternary_gemm(codes, scales, rowsum, act_bits, K, W_packed, alpha, want_acc=F
     CUDA-core GEMV, PATH_TC_TS tensor cores with activations in TMEM,
     PATH_TC_TMA TMA-fed tensor cores for one-byte codes, PATH_TC_DECODE the
     decode-batch tensor-core kernel for one-byte codes and M <= 128,
-    PATH_TC_PACKED the large-batch tensor-core kernel on the packed weights)."""
+    PATH_TC_PACKED the large-batch tensor-core kernel on the packed weights,
+    PATH_TC_PAIR the TMA-fed large-batch kernel on pairs of SMs)."""
     import torch
 
     M = scales.shape[0]  # the interleaved layouts pad the codes buffer to 32 rows

@@ -69,7 +69,10 @@ int act_width(int a) { return a == 4 ? 4 : 8; }
 int codes_row_bytes(int K, int act_bits) { return act_width(act_bits) == 4 ? K / 2 : K; }
 
 // Ternary-GEMM back ends.
-enum class Back { GEMV, SS, TS, TMA, DEC, WT };
+// TMA: the one-SM TMA-fed kernel; PAIR: the paired-SM kernel; BIG (automatic
+// choice for large batches): whichever of the two fills the device in fewer
+// waves of tiles, the pair on a tie.
+enum class Back { GEMV, SS, TS, TMA, DEC, WT, PAIR, BIG };
 
 // The GEMV back end uses the row GEMV when K allows it and the tokens fit one
 // launch; otherwise the split-K GEMV (8-token chunks).
@@ -78,7 +81,7 @@ bool rows_gemv(int64_t M, int K) { return gemv_rows_supported(K) && M <= gemv_ro
 // Batches above this many tokens take the TMA-fed kernel (automatic choice).
 constexpr int64_t kTmaMinM = 257;
 
-bool path_valid(int path) { return path >= HBL_PATH_AUTO && path <= HBL_PATH_TC_PACKED; }
+bool path_valid(int path) { return path >= HBL_PATH_AUTO && path <= HBL_PATH_TC_PAIR; }
 
 // Shapes the decode-batch tensor-core kernel takes (one-byte codes); whether a
 // launch plan fits the device is checked again at launch, which falls back to
@@ -97,14 +100,23 @@ Back pick(int64_t M, int K, bool bytes, int path) {
     if (path == 4) return (bytes && K >= 128) ? Back::TMA : Back::TS;
     if (path == 5) return (bytes && dec_shape(M, K)) ? Back::DEC : Back::TS;
     if (path == 6) return (bytes && K >= 256) ? Back::WT : Back::TS;
+    if (path == 7) return (bytes && K >= 128) ? Back::PAIR : Back::TS;
     // CUDA cores for a few tokens: the row GEMV where it takes the batch in one
     // launch; past that at K >= 16384 the tensor-core kernel is faster than the
     // split-K GEMV
     if (bytes && dec_shape(M, K) && M >= kDecMinM && M <= kDecMaxM) return Back::DEC;
     if (M <= gemv_max_m() && (rows_gemv(M, K) || K < 16384)) return Back::GEMV;
-    if (bytes && K >= 128 && M >= kTmaMinM) return Back::TMA;
+    if (bytes && K >= 128 && M >= kTmaMinM) return Back::BIG;
     return Back::TS;
 }
+
+// Large-batch back ends on expanded weights: whether the paired-SM kernel runs.
+bool use_pair(Back b, int64_t M, int K, int N, int sms) {
+    if (b == Back::PAIR) return gemm_pair_supported(K);
+    if (b == Back::BIG) return gemm_pair_supported(K) && gemm_pair_preferred(M, N, sms);
+    return false;
+}
+bool big_back(Back b) { return b == Back::TMA || b == Back::PAIR || b == Back::BIG; }
 
 size_t backend_ws(Back b, int64_t M, int K, int N) {
     switch (b) {
@@ -112,7 +124,9 @@ size_t backend_ws(Back b, int64_t M, int K, int N) {
         case Back::TS: return gemm_ts_workspace(M, K, N);
         case Back::DEC: return gemm_ts_workspace(M, K, N);  // its fallback's
         case Back::WT: return 0;
-        case Back::TMA: return gemm_tma_workspace(K, N);
+        case Back::TMA:
+        case Back::PAIR:
+        case Back::BIG: return gemm_tma_workspace(K, N);
         case Back::GEMV:
         default: {
             if (rows_gemv(M, K)) return 0;  // the row GEMV needs no scratch
@@ -131,6 +145,9 @@ hbl_status run_gemm(Back b, const GemmArgs& a, void* ws, size_t ws_bytes, cudaSt
     if (b == Back::SS) return launch_gemm_tc(a, s, sms);
     if (b == Back::TS) return launch_gemm_ts(a, ws, ws_bytes, s, sms);
     if (b == Back::TMA) return launch_gemm_tma(a, ws, ws_bytes, s, sms);
+    if (b == Back::PAIR || b == Back::BIG)
+        return use_pair(b, a.M, a.K, a.N, sms) ? launch_gemm_pair(a, ws, ws_bytes, s, sms)
+                                               : launch_gemm_tma(a, ws, ws_bytes, s, sms);
     if (b == Back::WT) return launch_gemm_wt(a, s, sms);
     if (b == Back::DEC) {
         if (!a.interleaved && a.act_bits == 8 && decode_mma_supported(a.M, a.K, a.N, sms))
@@ -179,7 +196,7 @@ FwdPlan forward_plan(int64_t M, int K, int act_bits, int path) {
     FwdPlan f;
     f.back = pick(M, K, true, path);
     f.interleaved = f.back == Back::TS;
-    if (f.back == Back::TMA || f.back == Back::DEC || f.back == Back::WT) {
+    if (big_back(f.back) || f.back == Back::DEC || f.back == Back::WT) {
         f.k1_mode = act_bits == 4 ? 6 : 8;
         f.gemm_act_bits = 8;
     } else if (f.back == Back::TS) {
@@ -533,7 +550,7 @@ hbl_status hbl_hbitlinear_forward_hostio(const uint16_t* X_host, const float* ga
     // Batches on the TMA-fed GEMM run in row chunks of at least kTmaMinM rows
     // (so every chunk keeps that plan and fits its workspace): chunk c's input
     // copy, its layer and chunk c-1's output copy overlap on three streams.
-    const bool big = plan.back == Back::TMA || plan.back == Back::WT;
+    const bool big = big_back(plan.back) || plan.back == Back::WT;
     const int nch = big ? (int)((int64_t)M / kTmaMinM < kMaxChunks ? (int64_t)M / kTmaMinM
                                                                    : kMaxChunks)
                         : 1;
@@ -560,7 +577,7 @@ hbl_status hbl_hbitlinear_forward_hostio(const uint16_t* X_host, const float* ga
     float* scales = reinterpret_cast<float*>(fws + cb);
     int32_t* rowsum = reinterpret_cast<int32_t*>(fws + cb + sb);
     int8_t* wexp = reinterpret_cast<int8_t*>(fws + cb + 2 * sb);
-    const bool expand = plan.back == Back::TMA;
+    const bool expand = big_back(plan.back);
     if (cb + 2 * sb + (expand ? gemm_tma_workspace(K, N) : 0) > fws_bytes)
         return HBL_ERR_WORKSPACE;
 #define HBL_CK(x) \
@@ -585,8 +602,9 @@ hbl_status hbl_hbitlinear_forward_hostio(const uint16_t* X_host, const float* ga
         GemmArgs a{codes, scales, rowsum, plan.gemm_act_bits, mc, K, W_packed, alpha, N,
                    Yd + r0 * N, nullptr, dev_status};
         a.pdl = true;  // right after K1 on the same stream
-        if ((st = expand ? launch_gemm_tma_s8w(a, wexp, s, sms) : launch_gemm_wt(a, s, sms)) !=
-            HBL_OK)
+        if ((st = use_pair(plan.back, mc, K, N, sms) ? launch_gemm_pair_s8w(a, wexp, s)
+                   : expand ? launch_gemm_tma_s8w(a, wexp, s, sms)
+                            : launch_gemm_wt(a, s, sms)) != HBL_OK)
             return st;
         HBL_CK(cudaEventRecord(c->fwd_ev[i], s));
         HBL_CK(cudaStreamWaitEvent(c->out, c->fwd_ev[i], 0));
@@ -713,6 +731,8 @@ hbl_status hbl_ternary_gemm_s8w(const void* codes, const float* scales, int act_
     hbl_status st = device(&sms);
     if (st != HBL_OK) return st;
     GemmArgs a{codes, scales, nullptr, 8, M, K, nullptr, alpha, N, Y, acc_out, dev_status};
+    if (use_pair(Back::BIG, M, K, N, sms))
+        return launch_gemm_pair_s8w(a, W_s8, static_cast<cudaStream_t>(stream));
     return launch_gemm_tma_s8w(a, W_s8, static_cast<cudaStream_t>(stream), sms);
 }
 

@@ -112,10 +112,10 @@ struct GemmArgs {
     uint16_t* Y;
     int32_t* acc_out;
     int32_t* dev_status;
-    bool interleaved = false;
+    bool interleaved = false;  // codes one per byte in the 32-row interleaved layout
     // launched right after the activation kernel of the fused forward: the
     // weights (not produced by that kernel) may be read before the dependency wait
-    bool pdl = false;  // codes one per byte in the 32-row interleaved layout
+    bool pdl = false;
 };
 
 // K2: tcgen05 tensor-core GEMM, both operands in shared memory, any M.
@@ -143,6 +143,17 @@ hbl_status launch_expand_ternary(const uint32_t* W_packed, int N, int K, int8_t*
                                  cudaStream_t stream, int num_sms);
 hbl_status launch_gemm_tma_s8w(const GemmArgs& a, const int8_t* W_s8, cudaStream_t stream,
                                int num_sms);
+// K10: the large-batch GEMM on pairs of SMs (tcgen05 cta_group::2, a
+// 256-token x 256-weight-row tile per cluster of two CTAs, both operands
+// TMA-fed; same expanded weights and workspace as K2c).  Supported when K is a
+// multiple of 128 and the device can hold a pair of its CTAs.
+bool gemm_pair_supported(int K);
+// Whether M x N fills the device in no more waves of paired tiles (256 x 256
+// per pair) than of one-SM tiles (128 x 256 per SM of `num_sms`).
+bool gemm_pair_preferred(int64_t M, int N, int num_sms);
+hbl_status launch_gemm_pair(const GemmArgs& a, void* ws, size_t ws_bytes, cudaStream_t stream,
+                            int num_sms);
+hbl_status launch_gemm_pair_s8w(const GemmArgs& a, const int8_t* W_s8, cudaStream_t stream);
 
 // Row GEMV (one weight row per warp over the whole K, epilogue fused, no
 // workspace) for M <= gemv_rows_max_m(K) tokens and 2048 <= K <= 32768.

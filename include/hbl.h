@@ -96,7 +96,12 @@ HBL_API int hbl_version(void);
  *   HBL_PATH_TC_PACKED (6) = the large-batch tcgen05 kernel on the packed
  *       weights (widened in registers into tensor memory as the MMA's A
  *       operand, codes as B by TMA; no expanded copy) whenever the codes are
- *       one byte each and K >= 256 (else as 3).
+ *       one byte each and K >= 256 (else as 3),
+ *   HBL_PATH_TC_PAIR (7) = the TMA-fed large-batch kernel on pairs of SMs
+ *       (tcgen05.mma.cta_group::2: a 256-token x 256-weight-row tile per
+ *       cluster of two CTAs, each holding half of each operand) whenever the
+ *       codes are one byte each and K >= 128 (else as 3; as 4 on a device
+ *       that cannot hold a pair of its CTAs).
  * Every path computes the same values.  No counterpart on the BitNet v2 pages. */
 enum {
     HBL_PATH_AUTO = 0,
@@ -105,7 +110,8 @@ enum {
     HBL_PATH_TC_TS = 3,
     HBL_PATH_TC_TMA = 4,
     HBL_PATH_TC_DECODE = 5,
-    HBL_PATH_TC_PACKED = 6
+    HBL_PATH_TC_PACKED = 6,
+    HBL_PATH_TC_PAIR = 7
 };
 
 /* act_bits also accepts these two values: the same INT4 / INT8 codes stored

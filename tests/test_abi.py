@@ -116,13 +116,13 @@ def test_validation_errors():
     assert pack(A, 0, 256, 1e-5, B, C, D, 1024, NUL) == 2
     # per-call back-end choice: out-of-range paths are refused
     sz = ctypes.c_size_t()
-    assert lib.hbl_workspace_size_path(hbl.OP_TERNARY_GEMM, 4, 256, 64, 4, 7, ctypes.byref(sz)) == 1
+    assert lib.hbl_workspace_size_path(hbl.OP_TERNARY_GEMM, 4, 256, 64, 4, 8, ctypes.byref(sz)) == 1
     assert lib.hbl_workspace_size_path(hbl.OP_TERNARY_GEMM, 4, 256, 64, 4, -1,
                                        ctypes.byref(sz)) == 1
     assert lib.hbl_ternary_gemm_path(A, B, C, 4, 64, 256, D, E, 64, A, NUL, E, 1 << 20, NUL, 9,
                                      NUL) == 1
     assert lib.hbl_hbitlinear_forward_path(A, NUL, 64, 256, 64, B, C, 4, 1e-6, 1e-5, D, E,
-                                           1 << 20, NUL, 7, NUL) == 1
+                                           1 << 20, NUL, 8, NUL) == 1
 
 
 def test_binding_rejects_non_cuda_tensors():

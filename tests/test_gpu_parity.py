@@ -377,11 +377,16 @@ def test_gemm_decode_mma(bits, M, K, N):
 # large-batch tensor-core kernel on the packed weights (weights widened into
 # TMEM as A, codes as B by TMA): ragged token blocks (M % 256), ragged weight
 # blocks (N % 128), several tiles per CTA (more than 148 tiles)
+# PATH_TC_PAIR: a 256 x 256 tile per pair of CTAs; M = 300 and N = 272 leave the
+# odd CTA's half of the last tile wholly past the end of A / B
+@pytest.mark.parametrize("path", ["packed", "pair"])
 @pytest.mark.parametrize("bits", [4, 8])
 @pytest.mark.parametrize("M,K,N", [(1, 128, 16), (45, 256, 272), (256, 512, 128),
                                    (300, 4096, 400), (1000, 2048, 512), (257, 16384, 4096),
-                                   (600, 4096, 11008), (1300, 1024, 4096)])
-def test_gemm_packed_weights(bits, M, K, N):
+                                   (600, 4096, 11008), (1300, 1024, 4096), (300, 128, 272)])
+def test_gemm_packed_weights(path, bits, M, K, N):
+    if path == "packed" and K < 256:
+        pytest.skip("the packed-weight kernel takes K >= 256 (smaller K runs as path 3)")
     codes, scales, rowsum, packed, alpha = make_gemm_case(M, K, N, bits, seed=M + K + 2 * N)
     q = oracle.decode_codes(codes, K, bits)
     act = 8 if bits == 8 else hbl.ACT_INT4_BYTES
@@ -390,20 +395,22 @@ def test_gemm_packed_weights(bits, M, K, N):
         torch.from_numpy(rowsum).to(DEV), act, K,
         torch.from_numpy(packed.view(np.int32)).to(DEV),
         torch.from_numpy(np.array([alpha, 0, 0, 0], dtype=np.float32)).to(DEV),
-        want_acc=True, path=hbl.PATH_TC_PACKED)
+        want_acc=True, path=hbl.PATH_TC_PACKED if path == "packed" else hbl.PATH_TC_PAIR)
     torch.cuda.synchronize()
     wY, wacc = oracle.ternary_gemm(codes, scales, bits, K, packed, alpha)
     assert np.array_equal(acc.cpu().numpy(), wacc)
     assert np.array_equal(bf16_bits(Y), wY)
 
 
+@pytest.mark.parametrize("path", [6, 7])
 @pytest.mark.parametrize("bits", [4, 8])
 @pytest.mark.parametrize("M,K,N", [(520, 4096, 256), (1000, 2048, 528), (300, 16384, 1024)])
-def test_forward_packed_weights_path(bits, M, K, N):
+def test_forward_packed_weights_path(path, bits, M, K, N):
+    # path 6: packed-weight kernel; path 7: the paired-SM kernel
     X = acts(M, K, seed=M + 5 * K, kind="swiglu")
     packed, alpha = oracle.pack_ternary(inputs.latent_weights(N, K, seed=M + N))
     want = oracle.hbitlinear_forward(X, packed, alpha, bits)
-    assert np.array_equal(forward(X, packed, alpha, bits, path=hbl.PATH_TC_PACKED), want)
+    assert np.array_equal(forward(X, packed, alpha, bits, path=path), want)
 
 
 @pytest.mark.parametrize("bits", [4, 8])
@@ -493,12 +500,16 @@ def test_ffn_wdown_workload_every_row(bits):
     assert np.array_equal(scales.cpu().numpy().view(np.uint32), ws.view(np.uint32))
     assert np.array_equal(rowsum.cpu().numpy(), wr)
     del codes, scales, rowsum
-    Y = bf16_bits(hbl.hbitlinear_forward(
-        Xd, torch.from_numpy(packed.view(np.int32)).to(DEV),
-        torch.from_numpy(np.array([alpha, 0, 0, 0], dtype=np.float32)).to(DEV), bits))
     wY, _ = oracle.ternary_gemm(wc, ws, bits, 16384, packed, alpha, want_acc=False)
-    bad = np.argwhere(Y != wY)
-    assert bad.size == 0, "outputs differ at %d elements, first %s" % (len(bad), bad[:5].tolist())
+    Wd = torch.from_numpy(packed.view(np.int32)).to(DEV)
+    ad = torch.from_numpy(np.array([alpha, 0, 0, 0], dtype=np.float32)).to(DEV)
+    # the automatic path, and both large-batch tensor-core kernels forced (one
+    # SM per tile; pairs of SMs per 256 x 256 tile)
+    for path in (hbl.PATH_AUTO, hbl.PATH_TC_TMA, hbl.PATH_TC_PAIR):
+        Y = bf16_bits(hbl.hbitlinear_forward(Xd, Wd, ad, bits, path=path))
+        bad = np.argwhere(Y != wY)
+        assert bad.size == 0, "path %d: outputs differ at %d elements, first %s" % (
+            path, len(bad), bad[:5].tolist())
 
 
 @pytest.mark.parametrize("T", sorted(set(inputs.DECODE_TOKENS) | {5, 9, 16, 64, 100}))
