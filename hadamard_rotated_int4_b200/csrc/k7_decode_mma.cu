@@ -309,8 +309,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
     };
     if (warp == 1 && p.early_weights) load_weights();
-    pdl_wait();  // the codes, scales and row sums come from the previous kernel
-    if (warp == 1 && !p.early_weights) load_weights();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -353,7 +351,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         __syncwarp();
     } else if (warp == 1) {
-        // ---------------- TMA producer of the token stages (one thread)
+        // ---------------- TMA producer of the token stages (one thread).  Only
+        // this warp waits for the previous kernel, whose output the codes are:
+        // the converters unpack the first stages' weights meanwhile, and all
+        // that reads the codes, scales or row sums is ordered after these
+        // loads (MMAs after "full", the epilogue after the accumulator).
+        pdl_wait();
+        if (!p.early_weights) load_weights();
         if (lane == 0) {
             bool ok = true;
             int issued = 0;
