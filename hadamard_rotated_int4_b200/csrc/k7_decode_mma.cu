@@ -267,34 +267,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int nkb = p.Kc / BK;
     const int rows = min(kRows, p.N - n0);
 
-    if (threadIdx.x == 0) {
-        for (int s = 0; s < SB; ++s) {
-            mbar_init_count(full_b(s), 1);
-            mbar_init_count(empty_b(s), 1);
-        }
-        for (int s = 0; s < SA; ++s) {
-            mbar_init_count(full_a(s), 4);  // the four warps of one converter group
-            mbar_init_count(empty_a(s), 1);
-        }
-        for (int g = 0; g < kMaxGroups; ++g) mbar_init_count(wbar(g), 1);
-        mbar_init_count(acc_bar, 1);
-        *abort_flag = 0;
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmB)) : "memory");
-        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmW)) : "memory");
-    }
-    if (warp == 0) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                         smem_addr(tmem_slot)),
-                     "r"(kTmemCols)
-                     : "memory");
-        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-    }
-    __syncthreads();  // barriers initialised
-
     // ---- the CTA's weight rows (its K slice) into shared memory: the weights
     // are not the previous kernel's output, so this runs before the dependency
-    // wait, under that kernel
+    // wait, under that kernel, and first of all: warp 1 initialises the weight
+    // barriers itself and starts the copies while the other barriers are set up
     // box g (= stage g): bytes [k0/4 + 128 g, + 128) of rows [n0, n0 + 128)
     // (rows past N read as zeros; the full box counts toward the transaction
     // bytes)
@@ -308,9 +284,46 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         __syncwarp();
     };
-    if (warp == 1 && p.early_weights) load_weights();
+    if (warp == 1) {
+        if (lane == 0) {
+            for (int g = 0; g < kMaxGroups; ++g) mbar_init_count(wbar(g), 1);
+            asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmW))
+                         : "memory");
+        }
+        __syncwarp();
+        if (p.early_weights) load_weights();
+    }
+    // the other barriers, one per thread of warps 2 and up
+    {
+        const int i = (int)threadIdx.x - 64;
+        const int nb = 2 * SB + 2 * SA + 1;
+        if (i >= 0 && i < nb) {
+            uint32_t a;
+            uint32_t count = 1;
+            if (i < SB) a = full_b(i);
+            else if (i < 2 * SB) a = empty_b(i - SB);
+            else if (i < 2 * SB + SA) { a = full_a(i - 2 * SB); count = 4; }  // a converter group
+            else if (i < 2 * SB + 2 * SA) a = empty_a(i - 2 * SB - SA);
+            else a = acc_bar;
+            mbar_init_count(a, count);
+            asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        }
+        if (threadIdx.x == 64) {
+            *abort_flag = 0;
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmB))
+                         : "memory");
+        }
+    }
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_addr(tmem_slot)),
+                     "r"(kTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
     tc_fence_before();
-    __syncthreads();
+    __syncthreads();  // every barrier initialised, TMEM allocated
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
