@@ -339,7 +339,8 @@ HBL_API hbl_status hbl_kv_quant(const uint16_t* X, int64_t rows, int D, int bits
 HBL_API hbl_status hbl_expand_ternary(const uint32_t* W_packed, int N, int K, int8_t* W_s8,
                                       int32_t* dev_status, void* stream);
 
-/* The TMA-fed tensor-core GEMM on expanded weights:
+/* The TMA-fed tensor-core GEMM on expanded weights (the paired-SM kernel, or
+ * the one-SM kernel where that fills the device in fewer waves of tiles):
  *   Y[m][n] = bf16_rne((float)(sum_k q[m][k] * W_s8[n][k]) * (alpha * scales[m]))
  * codes: one byte per code, row-major [M x K]: act_bits 8 (INT8) or
  * HBL_ACT_INT4_BYTES.  K >= 128 (a power of two as above).  acc_out: int32
