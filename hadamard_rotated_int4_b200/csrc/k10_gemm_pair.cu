@@ -189,8 +189,9 @@ struct Params {
 // within a group, so a group's weights stay in L2 (loaded with evict_last)
 // while the activations stream past (evict_first).  A wave of 74 pairs covers
 // about 9 token blocks x 8 weight blocks, all reading the same K slice at about
-// the same time.  (W_down, 8192 tokens: DRAM reads 533 MB without the
-// eviction hints, 414 MB with them; groups of 4 or 16 read more.)
+// the same time.  (W_down, 8192 tokens, a stand-alone copy of the kernel:
+// DRAM reads 533 MB without the eviction hints, 414 MB with them; groups of 4
+// or 16 read more.)
 constexpr int kGroup = 8;
 __device__ __forceinline__ void tile_coords(const Params& p, int64_t t, int& mb, int& nb) {
     const int64_t per_group = (int64_t)p.tiles_m * kGroup;
