@@ -15,11 +15,12 @@
 // and code j of a group sits at bits [b*j, b*j + b) of the group read as a
 // little-endian integer.
 //
-// Mapping: D/8 lanes per row, 8 values (one 16-byte load) per lane, so a warp
-// covers 32*8/D rows per step and a lane's 8 codes are 8*b contiguous bits;
-// lanes combine them with one shuffle where a 32-bit word spans two lanes.
-// Memory-bound: 2*D bytes in, D*b/8 + 4 out per row; each warp keeps U steps of
-// loads in flight.
+// Mapping: D/16 lanes per row, 16 values (two 16-byte loads) per lane, so a
+// warp covers 32*16/D rows per step and a lane's 16 codes are 16*b contiguous
+// bits; the per-step costs (the max over the row's lanes, the division, the
+// scale) are shared by 16 values per lane.  For b = 3 lane pairs make one
+// 12-byte group (one shuffle).  Memory-bound: 2*D bytes in, D*b/8 + 4 out per
+// row; each warp keeps U steps of loads in flight.
 #include <cuda_runtime.h>
 
 #include <type_traits>
@@ -31,14 +32,15 @@ namespace hbl {
 namespace k5 {
 
 constexpr int kThreads = 256;
-constexpr int U = 4;  // row steps per warp with their loads in flight together
+constexpr int U = 2;     // row steps per warp with their loads in flight together
+constexpr int VPL = 16;  // values per lane
 
 template <int D, int B>
 __global__ void __launch_bounds__(kThreads) kv_quant_kernel(const uint16_t* __restrict__ X,
                                                             int64_t rows, float eps,
                                                             uint8_t* __restrict__ codes,
                                                             float* __restrict__ scales) {
-    constexpr int LPR = D / 8;       // lanes per row
+    constexpr int LPR = D / VPL;     // lanes per row
     constexpr int RPW = 32 / LPR;    // rows per warp step
     constexpr int ROW_BYTES = D * B / 8;
     constexpr int QP = (1 << (B - 1)) - 1;
@@ -50,21 +52,23 @@ __global__ void __launch_bounds__(kThreads) kv_quant_kernel(const uint16_t* __re
     const float qp = (float)QP;
 
     for (int64_t base = warp0 * (RPW * U); base < rows; base += nwarps * (RPW * U)) {
-        uint4 raw[U];
+        uint4 raw[U][2];
 #pragma unroll
         for (int u = 0; u < U; ++u) {
             const int64_t row = base + u * RPW + sub;
-            raw[u] = row < rows ? *reinterpret_cast<const uint4*>(X + row * D + li * 8)
-                                : make_uint4(0, 0, 0, 0);
+            const uint4* src = reinterpret_cast<const uint4*>(X + row * D + li * VPL);
+            raw[u][0] = row < rows ? src[0] : make_uint4(0, 0, 0, 0);
+            raw[u][1] = row < rows ? src[1] : make_uint4(0, 0, 0, 0);
         }
 #pragma unroll
         for (int u = 0; u < U; ++u) {
             const int64_t row = base + u * RPW + sub;
-            float x[8];
+            float x[VPL];
             {
-                const uint32_t w[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};
+                const uint32_t w[8] = {raw[u][0].x, raw[u][0].y, raw[u][0].z, raw[u][0].w,
+                                       raw[u][1].x, raw[u][1].y, raw[u][1].z, raw[u][1].w};
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
+                for (int i = 0; i < 8; ++i) {
                     const float2 f = bf16x2_to_f2(w[i]);
                     x[2 * i] = f.x;
                     x[2 * i + 1] = f.y;
@@ -72,45 +76,44 @@ __global__ void __launch_bounds__(kThreads) kv_quant_kernel(const uint16_t* __re
             }
             float g = 0.f;
 #pragma unroll
-            for (int i = 0; i < 8; ++i) g = fmaxf(g, fabsf(x[i]));
+            for (int i = 0; i < VPL; ++i) g = fmaxf(g, fabsf(x[i]));
 #pragma unroll
             for (int o = 1; o < LPR; o <<= 1) g = fmaxf(g, __shfl_xor_sync(0xffffffffu, g, o));
             const float den = __fadd_rn(g, eps);
             const float inv = den > 0.f ? __fdiv_rn(qp, den) : 0.f;
-            // 8 codes of this lane, code i at bits [B*i, B*i + B).  No clamp is
-            // needed: |x| <= gamma, so |x * inv| <= Qp * gamma / (gamma + eps)
-            // up to the rounding of inv (well under half a unit), and rounding
-            // to the nearest integer stays within [-Qp, Qp].
-            using Word = typename std::conditional<(8 * B <= 32), uint32_t, uint64_t>::type;
-            Word bits = 0;
+            // 16 codes of this lane, code i at bits [B*i, B*i + B) of a 16*B-bit
+            // field (two 32-bit halves of 8 codes each).  No clamp is needed:
+            // |x| <= gamma, so |x * inv| <= Qp * gamma / (gamma + eps) up to the
+            // rounding of inv (well under half a unit), and rounding to the
+            // nearest integer stays within [-Qp, Qp].
+            using Half = typename std::conditional<(8 * B <= 32), uint32_t, uint64_t>::type;
+            Half h[2] = {0, 0};
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
+            for (int i = 0; i < VPL; ++i) {
                 const int32_t b = __float_as_int(__fmaf_rn(x[i], inv, 12582912.0f));
                 const uint32_t code = (uint32_t)(b - kMagicBits + (QP + 1));
-                bits |= (Word)code << (B * i);
+                h[i / 8] |= (Half)code << (B * (i % 8));
             }
             const bool ok = row < rows;
             uint8_t* dst = codes + row * ROW_BYTES;
-            if constexpr (B == 8) {
+            if constexpr (B == 8) {  // 16 bytes per lane
                 if (ok)
-                    *reinterpret_cast<uint2*>(dst + li * 8) =
-                        make_uint2((uint32_t)bits, (uint32_t)((uint64_t)bits >> 32));
-            } else if constexpr (B == 4) {
-                if (ok) *reinterpret_cast<uint32_t*>(dst + li * 4) = (uint32_t)bits;
-            } else if constexpr (B == 2) {  // 16 bits per lane: even lanes write pairs
-                const uint32_t mine = (uint32_t)bits;
-                const uint32_t next = __shfl_down_sync(0xffffffffu, mine, 1);
-                if (ok && (li & 1) == 0)
-                    *reinterpret_cast<uint32_t*>(dst + (li >> 1) * 4) = mine | (next << 16);
-            } else {  // B == 3: 24 bits per lane; four lanes make one 12-byte group
-                const uint32_t mine = (uint32_t)bits;
-                const uint32_t next = __shfl_down_sync(0xffffffffu, mine, 1);
-                const int k = li & 3;
-                const uint32_t word = k == 0 ? (mine | (next << 24))
-                                    : k == 1 ? ((mine >> 8) | (next << 16))
-                                             : ((mine >> 16) | (next << 8));
-                if (ok && k < 3)
-                    *reinterpret_cast<uint32_t*>(dst + (li >> 2) * 12 + 4 * k) = word;
+                    *reinterpret_cast<uint4*>(dst + li * 16) =
+                        make_uint4((uint32_t)h[0], (uint32_t)((uint64_t)h[0] >> 32), (uint32_t)h[1],
+                                   (uint32_t)((uint64_t)h[1] >> 32));
+            } else if constexpr (B == 4) {  // 8 bytes per lane
+                if (ok) *reinterpret_cast<uint2*>(dst + li * 8) = make_uint2(h[0], h[1]);
+            } else if constexpr (B == 2) {  // 4 bytes per lane
+                if (ok) *reinterpret_cast<uint32_t*>(dst + li * 4) = h[0] | (h[1] << 16);
+            } else {  // B == 3: 48 bits per lane; a lane pair makes one 12-byte group
+                const uint64_t mine = (uint64_t)h[0] | ((uint64_t)h[1] << 24);
+                const uint64_t next = __shfl_down_sync(0xffffffffu, mine, 1);
+                if (ok && (li & 1) == 0) {
+                    uint32_t* d32 = reinterpret_cast<uint32_t*>(dst + (li >> 1) * 12);
+                    d32[0] = (uint32_t)mine;
+                    d32[1] = (uint32_t)(mine >> 32) | ((uint32_t)next << 16);
+                    d32[2] = (uint32_t)(next >> 16);
+                }
             }
             if (ok && li == 0) scales[row] = __fdiv_rn(g, qp);
         }
@@ -120,7 +123,7 @@ __global__ void __launch_bounds__(kThreads) kv_quant_kernel(const uint16_t* __re
 template <int D, int B>
 static hbl_status launch_one(const uint16_t* X, int64_t rows, float eps, uint8_t* codes,
                              float* scales, cudaStream_t stream, int sms) {
-    constexpr int RPW = 32 / (D / 8);
+    constexpr int RPW = 32 / (D / VPL);
     const int64_t per_cta = (int64_t)(kThreads / 32) * RPW * U;
     int64_t grid = (rows + per_cta - 1) / per_cta;
     const int64_t cap = (int64_t)sms * 8;
