@@ -342,6 +342,32 @@ def run_hbl(args):
     int8_probe = {"tops": probe_tops, "mmas_per_cta": probe_mmas, "ctas": n_sms,
                   "status": probe_st}
 
+    # Device time per call of a short kernel: `iters` calls (cycling over n
+    # inputs) captured in one CUDA graph and replayed, CUDA events around the
+    # replays on this stream, so the host's per-call cost stays out of it.
+    def graph_time(fn, n, iters, reps=5):
+        for i in range(3):
+            fn(i % n)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream()
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            with torch.cuda.graph(g, stream=side):
+                for i in range(iters):
+                    fn(i % n)
+        stream.wait_stream(side)
+        g.replay()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(reps):
+            g.replay()
+        b.record(stream)
+        torch.cuda.synchronize()
+        del g
+        return a.elapsed_time(b) * 1e-3 / (reps * iters)
+
     # ---- quant workload: 8192 x 4096, a4 and a8, 4 rotating inputs (256 MB > L2)
     qX = [torch.from_numpy(inputs.activations("quant", seed=s).view(np.int16)).view(
         torch.bfloat16).to(dev) for s in range(4)]
@@ -350,17 +376,8 @@ def run_hbl(args):
         qc = torch.empty((QM, QK if bits == 8 else QK // 2), dtype=torch.uint8, device=dev)
         qs = torch.empty(QM, dtype=torch.float32, device=dev)
         qr = torch.empty(QM, dtype=torch.int32, device=dev)
-        for i in range(4):
-            hbl.norm_fwht_quant(qX[i], bits, out=(qc, qs, qr))
-        torch.cuda.synchronize()
-        qi = max(args.kernel_iters, 40)
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        for i in range(qi):
-            hbl.norm_fwht_quant(qX[i % 4], bits, out=(qc, qs, qr))
-        b.record(stream)
-        torch.cuda.synchronize()
-        t = a.elapsed_time(b) * 1e-3 / qi
+        t = graph_time(lambda i: hbl.norm_fwht_quant(qX[i], bits, out=(qc, qs, qr)), 4,
+                       max(args.kernel_iters, 40))
         nbytes = QM * QK * 2 + QM * QK * bits // 8 + QM * 4 + QM * 4
         gbs = nbytes / t / 1e9
         quant["a%d" % bits] = {"workload": "quant 8192 x 4096 Student-t nu=3, 1% channels x20",
@@ -428,17 +445,7 @@ def run_hbl(args):
         del pcs
 
     # ---- the other rows of the hot path, each against the HBM roofline
-    def ev_time(fn, n, iters):
-        for i in range(3):
-            fn(i % n)
-        torch.cuda.synchronize()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        for i in range(iters):
-            fn(i % n)
-        b.record(stream)
-        torch.cuda.synchronize()
-        return a.elapsed_time(b) * 1e-3 / iters
+    ev_time = graph_time
 
     others = {}
     # BitLinear variants (no Hadamard / LayerNorm) on the quant workload, a4 packed
