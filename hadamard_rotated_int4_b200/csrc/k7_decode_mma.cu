@@ -485,14 +485,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int n = n0 + r;
             if (n >= p.N) continue;
             const uint32_t off = part_s + (uint32_t)((j * kRows + r) * 4);
+            // the cluster's partials: all remote loads in flight, then the sums
+            constexpr int kMaxCS = 8;
+            uint4 v[kMaxCS];
+#pragma unroll
+            for (int c = 0; c < kMaxCS; ++c)
+                if (c < (int)csize) v[c] = ld_cluster_v4(mapa(off, (uint32_t)c));
             int a0 = 0, a1 = 0, a2 = 0, a3 = 0;
-            for (uint32_t c = 0; c < csize; ++c) {
-                const uint4 v = ld_cluster_v4(mapa(off, c));
-                a0 += (int)v.x;
-                a1 += (int)v.y;
-                a2 += (int)v.z;
-                a3 += (int)v.w;
-            }
+#pragma unroll
+            for (int c = 0; c < kMaxCS; ++c)
+                if (c < (int)csize) {
+                    a0 += (int)v[c].x;
+                    a1 += (int)v[c].y;
+                    a2 += (int)v[c].z;
+                    a3 += (int)v[c].w;
+                }
             const int rs = p.rowsum[j];
             a0 -= rs;
             a1 -= rs;
