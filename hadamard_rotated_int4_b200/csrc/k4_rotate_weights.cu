@@ -44,21 +44,47 @@ __global__ void __launch_bounds__(kThreads) rotate_kernel(const float* W, const 
     for (int64_t n = blockIdx.x; n < N; n += gridDim.x) {
         const float* src = W + n * K;
         float* dst = out + n * K;
-        // coalesced load (times the signs) into the padded row
-        for (int c = tid; c < K / 4; c += kThreads) {
-            float4 v = *reinterpret_cast<const float4*>(src + 4 * c);
-            if (signs != nullptr) {
-                const float4 sg = *reinterpret_cast<const float4*>(signs + 4 * c);
-                v.x = __fmul_rn(v.x, sg.x);
-                v.y = __fmul_rn(v.y, sg.y);
-                v.z = __fmul_rn(v.z, sg.z);
-                v.w = __fmul_rn(v.w, sg.w);
+        // coalesced load (times the signs) into the padded row; with signs,
+        // kLoadBatch 16-byte loads per thread are issued before any is used
+        // (the signs' loads otherwise serialise the row's; without signs the
+        // one-at-a-time loop measured faster: 126 against 131 us on W_down)
+        constexpr int kChunks = K / 4;
+        constexpr int kLoadBatch = 8;
+        if (signs == nullptr) {
+            for (int c = tid; c < kChunks; c += kThreads) {
+                const float4 v = *reinterpret_cast<const float4*>(src + 4 * c);
+                const int i = 4 * c;  // four consecutive words never straddle a pad
+                row[pad(i)] = v.x;
+                row[pad(i) + 1] = v.y;
+                row[pad(i) + 2] = v.z;
+                row[pad(i) + 3] = v.w;
             }
-            const int i = 4 * c;  // four consecutive words never straddle a pad
-            row[pad(i)] = v.x;
-            row[pad(i) + 1] = v.y;
-            row[pad(i) + 2] = v.z;
-            row[pad(i) + 3] = v.w;
+        } else {
+            for (int c0 = 0; c0 < kChunks; c0 += kThreads * kLoadBatch) {
+                float4 v[kLoadBatch];
+#pragma unroll
+                for (int b = 0; b < kLoadBatch; ++b) {
+                    const int c = c0 + b * kThreads + tid;
+                    if (c < kChunks) v[b] = *reinterpret_cast<const float4*>(src + 4 * c);
+                }
+#pragma unroll
+                for (int b = 0; b < kLoadBatch; ++b) {
+                    const int c = c0 + b * kThreads + tid;
+                    if (c < kChunks) {
+                        float4 x = v[b];
+                        const float4 sg = *reinterpret_cast<const float4*>(signs + 4 * c);
+                        x.x = __fmul_rn(x.x, sg.x);
+                        x.y = __fmul_rn(x.y, sg.y);
+                        x.z = __fmul_rn(x.z, sg.z);
+                        x.w = __fmul_rn(x.w, sg.w);
+                        const int i = 4 * c;  // four consecutive words never straddle a pad
+                        row[pad(i)] = x.x;
+                        row[pad(i) + 1] = x.y;
+                        row[pad(i) + 2] = x.z;
+                        row[pad(i) + 3] = x.w;
+                    }
+                }
+            }
         }
         __syncthreads();
         static_for<0, (L + 4) / 5>([&](auto pp) {
