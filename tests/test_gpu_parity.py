@@ -571,6 +571,26 @@ def test_decode_one_kernel_edge_rows():
                               oracle.hbitlinear_forward(X, packed, alpha, bits))
 
 
+@pytest.mark.parametrize("K,N", [(4096, 4096), (8192, 1008), (16384, 4096)])
+def test_decode_one_token_edge_rows(K, N):
+    # one token through the one-kernel forward: zero, constant, single-spike
+    # and a Hadamard-row input (whose transform is a spike), and a normal row,
+    # each as its own one-token forward
+    W = inputs.latent_weights(N, K, seed=K + 1)
+    packed, alpha = oracle.pack_ternary(W)
+    rows = np.zeros((5, K), dtype=np.uint16)
+    rows[1] = np.float32(0.75).view(np.uint32) >> 16
+    rows[2, K // 3] = np.float32(-3.0).view(np.uint32) >> 16
+    h = np.array([1.0 - 2.0 * (bin(5 & j).count("1") & 1) for j in range(K)], np.float32)  # row 5 of H_K
+    rows[3] = h.view(np.uint32) >> 16
+    rows[4] = acts(1, K, seed=K)[0]
+    for r in range(5):
+        X = rows[r:r + 1].copy()
+        for bits in (4, 8):
+            assert np.array_equal(forward(X, packed, alpha, bits),
+                                  oracle.hbitlinear_forward(X, packed, alpha, bits)), (r, bits)
+
+
 @pytest.mark.parametrize("T,K", [(1, 4096), (32, 16384), (300, 2048)])
 def test_forward_replays_from_cuda_graph(T, K):
     # the forward launches only on the caller's stream, so it can be captured
