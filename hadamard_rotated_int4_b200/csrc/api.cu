@@ -435,13 +435,28 @@ static hbl_status forward_impl(const uint16_t* X, const float* gain, int M, int 
         f.k1_mode = act_bits == 4 ? 5 : 9;
         f.interleaved = true;
     }
+    // The GEMMs on expanded weights get them from K1, which widens the packed
+    // words beside its rows (its FP32 work leaves HBM bandwidth to spare), so
+    // the GEMM follows K1 directly -- where the rows are enough to carry the
+    // expansion; other shapes and the norm variants keep the separate
+    // expansion kernel.
+    const bool expand = big_back(f.back) &&
+                        (variant & (HBL_NORM_NO_HADAMARD | HBL_NORM_LAYERNORM)) == 0 &&
+                        norm_quant_expand_rides_along(M, K, N, sms);
+    if (expand && gws_bytes < gemm_tma_workspace(K, N)) return HBL_ERR_WORKSPACE;
+    int8_t* wexp = reinterpret_cast<int8_t*>(gws);
     hbl_status st = launch_norm_fwht_quant(X, gain, M, K, norm_eps, quant_eps, f.k1_mode, codes,
-                                           scales, rowsum, nullptr, s, sms, variant);
+                                           scales, rowsum, nullptr, s, sms, variant,
+                                           expand ? W_packed : nullptr, expand ? N : 0,
+                                           expand ? wexp : nullptr);
     if (st != HBL_OK) return st;
     GemmArgs a{codes, scales, rowsum, f.gemm_act_bits, M, K, W_packed, alpha, N, Y, nullptr,
                dev_status};
     a.interleaved = f.interleaved;
     a.pdl = true;  // right after K1 on the same stream
+    if (expand)
+        return use_pair(f.back, M, K, N, sms) ? launch_gemm_pair_s8w(a, wexp, s)
+                                              : launch_gemm_tma_s8w(a, wexp, s, sms);
     return run_gemm(f.back, a, gws, gws_bytes, s, sms);
 }
 

@@ -121,6 +121,11 @@ __device__ __forceinline__ uint4 lds128(uint32_t addr) {
                  : "memory");
     return v;
 }
+__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1];\n" : "=r"(v) : "r"(addr) : "memory");
+    return v;
+}
 __device__ __forceinline__ void sts128(uint32_t addr, uint4 v) {
     asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};\n" ::"r"(addr), "r"(v.x), "r"(v.y),
                  "r"(v.z), "r"(v.w)
@@ -149,6 +154,20 @@ __device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a
 // bit-identical to an IEEE subtraction.
 __device__ __forceinline__ float2 sub2(float2 a, float2 b) {
     return __ffma2_rn(b, make_float2(-1.0f, -1.0f), a);
+}
+
+// One packed ternary word (16 two-bit codes t + 1; weight j at bits 8(j%4) +
+// 2(j/4)) -> its 16 weights t as signed bytes in index order: bytes 4i..4i+3
+// are ((w >> 2i) & 0x03030303) - 1 per byte.  The per-byte subtraction sets
+// each byte's top bit first, so no borrow crosses a byte, and clears it after:
+// a byte b <= 3 becomes (0x80 + b - 1) ^ 0x80 = b - 1 (mod 256).
+__device__ __forceinline__ uint32_t ternary_bytes(uint32_t m) {
+    return ((m | 0x80808080u) - 0x01010101u) ^ 0x80808080u;
+}
+__device__ __forceinline__ uint4 expand_ternary_word(uint32_t w) {
+    return make_uint4(ternary_bytes(w & 0x03030303u), ternary_bytes((w >> 2) & 0x03030303u),
+                      ternary_bytes((w >> 4) & 0x03030303u),
+                      ternary_bytes((w >> 6) & 0x03030303u));
 }
 
 // bf16 pair (low half = first element) -> two fp32 (exact widening).

@@ -35,11 +35,19 @@ hbl_status launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem
 // scales (+ rowsum); mode 6 writes INT4 codes one per byte, row-major;
 // modes 5 / 9 write INT4 / INT8 codes one per byte in the
 // 32-row interleaved layout of the fused forward.  variant: HBL_NORM_* bits
-// (LayerNorm instead of RMSNorm, no Hadamard transform).
+// (LayerNorm instead of RMSNorm, no Hadamard transform).  Modes 6 and 8 with
+// W_packed set also widen the N x K packed ternary weights to one signed byte
+// each into W_s8 (N*K bytes, 16-byte aligned; K a multiple of 128, N of 16), beside the
+// rows -- the large-batch forward's operand, without a kernel of its own.
 hbl_status launch_norm_fwht_quant(const uint16_t* X, const float* gain, int64_t M, int K,
                                   float norm_eps, float quant_eps, int mode, void* codes,
                                   float* scales, int32_t* rowsum, float* V, cudaStream_t stream,
-                                  int num_sms, unsigned variant = 0);
+                                  int num_sms, unsigned variant = 0,
+                                  const uint32_t* W_packed = nullptr, int N = 0,
+                                  int8_t* W_s8 = nullptr);
+// Whether that expansion rides along K1's rows for this shape (nearly all of it
+// inside the row loop); otherwise the separate expansion kernel is faster.
+bool norm_quant_expand_rides_along(int64_t M, int K, int N, int num_sms);
 
 // K6: the whole forward of a decode batch in one kernel (quantiser and ternary
 // GEMV fused; see k6_decode_fused.cuh).  Supported for M <= 16384 / K tokens

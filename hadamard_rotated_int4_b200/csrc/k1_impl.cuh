@@ -46,6 +46,7 @@ constexpr int kRedFloats = 128;  // per-group cross-warp reduction scratch
 constexpr int kFlGain = 1;
 constexpr int kFlNoHadamard = 2;
 constexpr int kFlLayerNorm = 4;
+constexpr int kFlExpand = 8;  // modes 6 and 8: also widen the packed weights (Params::W)
 
 // log2 of the fp32 values each thread holds: 128 in general (K = 16384: four
 // warps per row, three rows per SM, 149 us on 8192 rows against 169 us with
@@ -168,10 +169,19 @@ struct Params {
     // INT4 at K >= 16384: rows with norm_eps-free energy (sum x^2 >= 2^-100)
     // and den > thr16 have every |q| < 2^15 (see the quantisation below)
     float thr16;
-    // used only by an extension (Ext below) that consumes the codes in-kernel
+    // used only by an extension (Ext below) that consumes the codes in-kernel,
+    // and (W, N, wdst) by the weight expansion run beside the rows (FL &
+    // kFlExpand, modes 6 and 8 of the plain kernel, for the large-batch
+    // forward): the N x K packed ternary weights W widened to one signed byte
+    // per weight in wdst (16 bytes per packed word).  The struct keeps its
+    // size: a larger parameter block changed the plain kernels' register
+    // allocation.
     const uint32_t* W;
     const float* alpha;
-    uint16_t* Y;
+    union {
+        uint16_t* Y;
+        uint4* wdst;
+    };
     int32_t* status;
     int N, rows;
 };
@@ -289,7 +299,8 @@ __device__ __forceinline__ float stream_tree(F&& f) {
 // FL: kFlGain = multiply by the per-channel gain (else a gain of one, exact
 // skip); kFlNoHadamard = no transform (the plain BitLinear of the layers
 // without H: the codes are those of the normalised row itself); kFlLayerNorm =
-// subtract the row mean first (LayerNorm without bias) instead of RMSNorm.
+// subtract the row mean first (LayerNorm without bias) instead of RMSNorm;
+// kFlExpand = widen the packed ternary weights beside the rows (below).
 template <int L, int MODE, int FL, class Ext = NoExt>
 __global__ void __launch_bounds__(Ext::template threads<L>(), Ext::template min_blocks<L>())
     norm_fwht_quant_kernel(Params p) {
@@ -409,11 +420,49 @@ __global__ void __launch_bounds__(Ext::template threads<L>(), Ext::template min_
         }
     };
 
+    // Weight expansion beside the rows (the large-batch forward): the packed
+    // words go in chunks of W x 4 words, and a group widens the chunks whose
+    // index is one of its row groups' (rg_first, rg_first + stride_groups, ...,
+    // continuing past the rows).  At a row's start (after the wait and group
+    // barrier that the staged row needs anyway, before the row's values are
+    // live) each thread copies 16 bytes of the next chunk with cp.async into
+    // one of the group's two slots (it lands while the row is worked on), and
+    // the group widens the chunk in the other, thread w taking words w, w + W,
+    // w + 2W, w + 3W, so every warp store is 512 contiguous bytes.
+    // Chunks left when the rows run out are widened after the loop straight
+    // from global memory.  Chunks are whole: the launcher takes N % 16 == 0
+    // and K % 128 == 0, so the W x 4 = max(K / 32, 128) words of a chunk
+    // divide the N K / 16 words.
+    constexpr bool kExpand = !Ext::kOn && (FL & kFlExpand) != 0;
+    static_assert(!kExpand || MODE == 6 || MODE == 8, "expansion beside modes 6 and 8 only");
+    constexpr int kWChunkLog = ilog2(W) + 2;  // W x 4 words per chunk
+    auto w_chunks = [&]() -> int64_t { return ((int64_t)p.N << (L - 4)) >> kWChunkLog; };
+    // two slots per group, taken in turn
+    [[maybe_unused]] uint32_t w_buf = 0;  // byte offset of the slot the next chunk lands in
+    auto w_slot = [&]() -> uint32_t {
+        return smem_addr(smem + C::kSmemBytes) + (uint32_t)grp * (uint32_t)(W * 32);
+    };
+    auto w_issue = [&](int64_t c) {
+        if (c >= w_chunks()) return;  // uniform over the group
+        cp_async16(w_slot() + w_buf + (uint32_t)w * 16u, p.W + (c << kWChunkLog) + w * 4, 16);
+        cp_async_commit();
+    };
+    auto w_widen = [&](int64_t c, uint32_t buf) {  // the group's copies of chunk c have landed
+        if (c >= w_chunks()) return;
+        uint4* dst = p.wdst + (c << kWChunkLog) + w;
+        static_for<0, 4>([&](auto jj) {
+            constexpr int jw = decltype(jj)::value;
+            dst[jw * W] = expand_ternary_word(lds32(w_slot() + buf + (uint32_t)(jw * W + w) * 4u));
+        });
+    };
+
     // One row group per thread (small M, e.g. decode): let the next kernel
     // start its prologue (weight prefetch) while this one works.
     if (!Ext::kOn && stride_groups * C::kRowsPerGroup >= p.M) pdl_launch_dependents();
     issue_load(rg_first);
-    for (int64_t rg = rg_first;; rg += stride_groups) {
+    if constexpr (kExpand) w_issue(rg_first);
+    int64_t rg = rg_first;
+    for (;; rg += stride_groups) {
         const int64_t row0 = rg * C::kRowsPerGroup;
         if (row0 >= p.M) break;
         const int64_t row = row0 + rig;
@@ -421,6 +470,13 @@ __global__ void __launch_bounds__(Ext::template threads<L>(), Ext::template min_
         group_sync<T>(grp);
         if constexpr (Ext::kOn) {
             if (rg == rg_first && tid == 0) Ext::staged(p);
+        }
+        if constexpr (kExpand) {
+            // the other slot was last read a row ago, before this row's barrier
+            const uint32_t cur = w_buf;
+            w_buf ^= (uint32_t)(W * 16);
+            w_issue(rg + stride_groups);
+            w_widen(rg, cur);
         }
 
         float2 d[R / 2];
@@ -779,6 +835,33 @@ __global__ void __launch_bounds__(Ext::template threads<L>(), Ext::template min_
             }
         }
     }
+    if constexpr (kExpand) {
+        // chunk rg is in flight (or past the end): finish it, then the rest
+        // from global memory with four chunks' loads in flight per thread
+        cp_async_wait_all();
+        group_sync<T>(grp);
+        w_widen(rg, w_buf);  // the last copy went to slot w_buf
+        for (int64_t c0 = rg + stride_groups; c0 < w_chunks(); c0 += 4 * stride_groups) {
+            uint32_t v[4][4];
+            static_for<0, 4>([&](auto ee) {
+                constexpr int e = decltype(ee)::value;
+                const int64_t c = c0 + e * stride_groups;
+                static_for<0, 4>([&](auto jj) {
+                    constexpr int jw = decltype(jj)::value;
+                    v[e][jw] = c < w_chunks() ? __ldg(p.W + (c << kWChunkLog) + jw * W + w) : 0u;
+                });
+            });
+            static_for<0, 4>([&](auto ee) {
+                constexpr int e = decltype(ee)::value;
+                const int64_t c = c0 + e * stride_groups;
+                static_for<0, 4>([&](auto jj) {
+                    constexpr int jw = decltype(jj)::value;
+                    if (c < w_chunks())
+                        p.wdst[(c << kWChunkLog) + jw * W + w] = expand_ternary_word(v[e][jw]);
+                });
+            });
+        }
+    }
     if constexpr (Ext::kOn) Ext::finish(p);
 }
 
@@ -786,14 +869,39 @@ template <int L, int MODE, int FL, class Ext>
 static hbl_status launch_cfg(const Params& prm, cudaStream_t stream, int num_sms) {
     using C = Cfg<L, Ext::template rlog<L>()>;
     auto kern = norm_fwht_quant_kernel<L, MODE, FL, Ext>;
-    if (!smem_attr_once(reinterpret_cast<const void*>(kern), C::kSmemBytes)) return HBL_ERR_CUDA;
+    // the weight expansion's two slots: 32 bytes per thread after the rows' buffers
+    constexpr bool expand = !Ext::kOn && (FL & kFlExpand) != 0;
+    const int smem = C::kSmemBytes + (expand ? C::kCtaThreads * 32 : 0);
+    if (!smem_attr_once(reinterpret_cast<const void*>(kern), smem)) return HBL_ERR_CUDA;
     const int64_t groups = (prm.M + C::kRowsPerGroup - 1) / C::kRowsPerGroup;
     const int64_t ctas_needed = (groups + C::kGroupsPerCta - 1) / C::kGroupsPerCta;
     int64_t grid = (int64_t)num_sms * C::kMinBlocks;
     if (ctas_needed < grid) grid = ctas_needed;
     if (grid < 1) grid = 1;
-    kern<<<(unsigned)grid, C::kCtaThreads, C::kSmemBytes, stream>>>(prm);
+    kern<<<(unsigned)grid, C::kCtaThreads, smem, stream>>>(prm);
     return cudaGetLastError() == cudaSuccess ? HBL_OK : HBL_ERR_CUDA;
+}
+
+// Whether K1's rows carry the weight expansion well: every group widens at
+// most one chunk more than it has row groups, so hardly any of it is left for
+// after the rows (measured: 8192 tokens at K = 16384 gained 6 us over the
+// separate expansion kernel; 2048 tokens, most chunks after the rows, lost 12).
+template <int L, int RL>
+static bool expand_rides_along_cfg(int64_t M, int N, int num_sms) {
+    using C = Cfg<L, RL>;
+    const int64_t groups = (M + C::kRowsPerGroup - 1) / C::kRowsPerGroup;
+    int64_t ctas = (groups + C::kGroupsPerCta - 1) / C::kGroupsPerCta;
+    if (ctas > (int64_t)num_sms * C::kMinBlocks) ctas = (int64_t)num_sms * C::kMinBlocks;
+    const int64_t ng = (ctas < 1 ? 1 : ctas) * C::kGroupsPerCta;
+    const int64_t chunks = ((int64_t)N << (L - 4)) >> (ilog2(C::W) + 2);
+    return (chunks + ng - 1) / ng <= (groups + ng - 1) / ng + 1;
+}
+template <int L>
+static bool expand_rides_along_l(int64_t M, int N, int num_sms) {
+    if constexpr (L == 14)  // the launch choice of launch_one below
+        if (M <= (int64_t)num_sms * Cfg<L>::kMinBlocks)
+            return expand_rides_along_cfg<L, 6>(M, N, num_sms);
+    return expand_rides_along_cfg<L, reg_log(L)>(M, N, num_sms);
 }
 
 template <int L, int MODE, int FL>

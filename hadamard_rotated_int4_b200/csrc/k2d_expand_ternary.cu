@@ -12,17 +12,11 @@
 namespace hbl {
 namespace k2d {
 
-// Packed 2-bit codes (16 per word; weight j of a word at bits 8(j%4) + 2(j/4),
-// code t + 1) -> one signed byte t per weight, row-major [N x K].  Bytes 4i..4i+3
-// of a word's 16 are ((w >> 2i) & 0x03030303) - 1 per byte.  Consecutive threads
-// take consecutive words, so every warp load is 128 contiguous bytes and every
-// warp store 512; each thread has four words in flight per step.
-__device__ __forceinline__ uint4 expand_word(uint32_t w) {
-    return make_uint4(__vsub4(w & 0x03030303u, 0x01010101u),
-                      __vsub4((w >> 2) & 0x03030303u, 0x01010101u),
-                      __vsub4((w >> 4) & 0x03030303u, 0x01010101u),
-                      __vsub4((w >> 6) & 0x03030303u, 0x01010101u));
-}
+// Packed 2-bit codes (16 per word, expand_ternary_word) -> one signed byte t
+// per weight, row-major [N x K].  Consecutive threads take consecutive words,
+// so every warp load is 128 contiguous bytes and every warp store 512; each
+// thread has four words in flight per step.  (The large-batch forward runs the
+// same expansion inside K1 instead, beside the token rows.)
 __global__ void expand_kernel(const uint32_t* __restrict__ Wp, int64_t words,
                               uint4* __restrict__ out) {
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
@@ -37,7 +31,7 @@ __global__ void expand_kernel(const uint32_t* __restrict__ Wp, int64_t words,
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             const int64_t i = base + j * stride;
-            if (i < words) out[i] = expand_word(w[j]);
+            if (i < words) out[i] = expand_ternary_word(w[j]);
         }
     }
 }

@@ -414,6 +414,28 @@ def test_forward_packed_weights_path(path, bits, M, K, N):
 
 
 @pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("M,K,N,with_gain", [(257, 128, 16, False), (1777, 4096, 2048, True),
+                                             (445, 16384, 656, True), (600, 8192, 1200, False)])
+def test_forward_widens_weights_beside_the_rows(bits, M, K, N, with_gain):
+    # Where the token rows are enough to carry it, the large-batch forward's
+    # quantiser (K1) also widens the packed weights for the GEMM: one chunk
+    # per row group while the rows are worked on, the rest after them.  These
+    # shapes give some groups one row and up to three chunks (so the loop
+    # after the rows runs), groups without a row (257 tokens: 9 row groups
+    # over 12), a single chunk (N = 16), and the gain variant; every column
+    # of Y checks one widened weight row.
+    X = acts(M, K, seed=M + K)
+    g = (np.random.default_rng(N).uniform(0.25, 2.0, K).astype(np.float32)
+         if with_gain else None)
+    W = inputs.latent_weights(N, K, seed=N)
+    packed, alpha = oracle.pack_ternary(W)
+    Y = forward(X, packed, alpha, bits, gain=g)
+    rows = np.array([0, 1, M // 2, M - 2, M - 1])
+    want = oracle.hbitlinear_forward(X, packed, alpha, bits, gain=g, rows=rows)
+    assert np.array_equal(Y[rows], want)
+
+
+@pytest.mark.parametrize("bits", [4, 8])
 @pytest.mark.parametrize("M,K,N", [(1, 4096, 4096), (3, 16384, 4096), (12, 4096, 4096),
                                    (40, 16384, 4096), (128, 4096, 2048)])
 def test_forward_decode_mma_path(bits, M, K, N):
