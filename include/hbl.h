@@ -82,8 +82,10 @@ HBL_API int hbl_version(void);
  *       tokens (one weight row per warp for K >= 2048, split-K below); the
  *       tcgen05 kernel with activations in tensor memory (split over K for
  *       M <= 256) up to 256 tokens; above that the TMA-fed tcgen05 kernel when
- *       the codes are one byte each (it expands the packed weights to signed
- *       bytes in workspace first),
+ *       the codes are one byte each (the packed weights are widened to
+ *       signed bytes in workspace first: by hbl_hbitlinear_forward's quantiser
+ *       beside its token rows where the batch is large enough to carry it,
+ *       else by a separate kernel),
  *   HBL_PATH_TC_SS (1)  = tcgen05 with both operands staged in shared memory by threads,
  *   HBL_PATH_GEMV (2)   = always the GEMV path (large M runs in chunks of 8 tokens),
  *   HBL_PATH_TC_TS (3)  = always the tcgen05 kernel with activations in tensor memory,
@@ -330,7 +332,8 @@ HBL_API hbl_status hbl_kv_quant(const uint16_t* X, int64_t rows, int D, int bits
  * For large token batches the tensor-core GEMM reads the ternary weights as
  * one signed byte each (tcgen05 has no integer MMA narrower than 8 bits);
  * hbl_ternary_gemm and hbl_hbitlinear_forward expand the packed weights into
- * workspace on every call.  A caller that keeps the expanded copy (N*K bytes,
+ * workspace on every call (the forward inside its quantiser kernel where the
+ * token rows carry it).  A caller that keeps the expanded copy (N*K bytes,
  * 4x the packed size) can skip that step with these two calls.  No
  * counterpart on the BitNet v2 pages: a deployment aid.
  *
