@@ -15,8 +15,8 @@ namespace k2d {
 // Packed 2-bit codes (16 per word, expand_ternary_word) -> one signed byte t
 // per weight, row-major [N x K].  Consecutive threads take consecutive words,
 // so every warp load is 128 contiguous bytes and every warp store 512; each
-// thread has four words in flight per step.  (The large-batch forward runs the
-// same expansion inside K1 instead, beside the token rows.)
+// thread has four words in flight per step.  (Where its token rows carry it,
+// the large-batch forward widens the weights inside K1 instead.)
 __global__ void expand_kernel(const uint32_t* __restrict__ Wp, int64_t words,
                               uint4* __restrict__ out) {
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
