@@ -3,7 +3,10 @@ compiled with nvcc against the kernel header and run on the CPU.  It uses the
 header's own constexpr layout functions to check, for every (K, values per
 thread) the kernels instantiate, that each register/thread layout covers the
 row one-to-one and that every 16-byte shared-memory exchange access is free of
-bank conflicts, with writer and reader addressing each element identically."""
+bank conflicts, with writer and reader addressing each element identically.
+tests/host/k1_expand_plan_check.cu checks, the same way, how the large-batch
+forward's K1 shares out the widening of the packed weights over its groups
+(every chunk exactly once) and which shapes its routing rule gives it."""
 import os
 import shutil
 import subprocess
