@@ -161,10 +161,10 @@ __device__ __forceinline__ float2 sub2(float2 a, float2 b) {
 // are ((w >> 2i) & 0x03030303) - 1 per byte.  The per-byte subtraction sets
 // each byte's top bit first, so no borrow crosses a byte, and clears it after:
 // a byte b <= 3 becomes (0x80 + b - 1) ^ 0x80 = b - 1 (mod 256).
-__device__ __forceinline__ uint32_t ternary_bytes(uint32_t m) {
+__host__ __device__ __forceinline__ uint32_t ternary_bytes(uint32_t m) {
     return ((m | 0x80808080u) - 0x01010101u) ^ 0x80808080u;
 }
-__device__ __forceinline__ uint4 expand_ternary_word(uint32_t w) {
+__host__ __device__ __forceinline__ uint4 expand_ternary_word(uint32_t w) {
     return make_uint4(ternary_bytes(w & 0x03030303u), ternary_bytes((w >> 2) & 0x03030303u),
                       ternary_bytes((w >> 4) & 0x03030303u),
                       ternary_bytes((w >> 6) & 0x03030303u));

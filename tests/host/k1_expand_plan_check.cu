@@ -9,7 +9,10 @@
 //   2. every chunk is widened exactly once,
 //   3. the routing rule takes the expansion into K1 exactly for the shapes
 //      expected (the ones the GPU tests and the benchmark run through it),
-// and prints one line per shape; exits non-zero on any failure.
+// and prints one line per shape; and that the word widening both expansion
+// paths share (expand_ternary_word) gives byte 4i + b = the two-bit field at
+// bits 8b + 2i minus one (mod 256) for every low and high half-word, so no
+// borrow crosses a byte.  Exits non-zero on any failure.
 #include <cstdio>
 #include <vector>
 
@@ -58,8 +61,32 @@ static int check(long long M, int N, int expect_fused) {
     return ok ? 0 : 1;
 }
 
-int main() {
+// expand_ternary_word against the packing's definition (weight j of a word at
+// bits 8(j%4) + 2(j/4), code t + 1), for words w = lo | hi << 16.
+static int check_widening() {
     int bad = 0;
+    auto one = [&](uint32_t w) {
+        const uint4 v = hbl::expand_ternary_word(w);
+        const uint32_t part[4] = {v.x, v.y, v.z, v.w};
+        for (int i = 0; i < 4; ++i)
+            for (int b = 0; b < 4; ++b) {
+                const uint32_t code = (w >> (8 * b + 2 * i)) & 3u;
+                const uint32_t want = (code + 255u) & 255u;  // code - 1 mod 256
+                if (((part[i] >> (8 * b)) & 255u) != want) ++bad;
+            }
+    };
+    const uint32_t others[] = {0x0000u, 0xffffu, 0x5555u, 0xaaaau, 0x1234u};
+    for (uint32_t h = 0; h < 65536u; ++h)
+        for (uint32_t o : others) {
+            one(h | (o << 16));
+            one(o | (h << 16));
+        }
+    printf("word widening, %d half-word patterns x %d: %s\n", 65536, 2 * 5, bad ? "FAIL" : "ok");
+    return bad ? 1 : 0;
+}
+
+int main() {
+    int bad = check_widening();
     // taken into K1: the benchmark's W_down and the GPU test shapes
     bad += check<14>(8192, 4096, 1);
     bad += check<12>(8192, 4096, 1);

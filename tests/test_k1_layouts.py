@@ -37,9 +37,10 @@ def test_k1_layouts_bijective_and_conflict_free():
 
 @pytest.mark.skipif(not (os.path.exists(NVCC) or shutil.which("nvcc")), reason="nvcc not found")
 def test_k1_weight_expansion_plan():
-    # tests/host/k1_expand_plan_check.cu: every chunk of the packed weights
-    # widened exactly once by K1's groups, and the rule that takes the
-    # expansion into K1 picking the expected shapes
+    # tests/host/k1_expand_plan_check.cu: the word widening against the
+    # packing's definition, every chunk of the packed weights widened exactly
+    # once by K1's groups, and the rule that takes the expansion into K1
+    # picking the expected shapes
     out_dir = os.path.join(ROOT, "_build")
     os.makedirs(out_dir, exist_ok=True)
     exe = os.path.join(out_dir, "k1_expand_plan_check")
@@ -52,5 +53,5 @@ def test_k1_weight_expansion_plan():
     assert r.returncode == 0, r.stderr[-2000:]
     run = subprocess.run([exe], capture_output=True, text=True, timeout=120)
     lines = run.stdout.strip().splitlines()
-    assert len(lines) == 10 + 7 * 4 * 4, run.stdout
+    assert len(lines) == 1 + 10 + 7 * 4 * 4, run.stdout
     assert run.returncode == 0 and all(l.endswith(": ok") for l in lines), run.stdout
