@@ -1,6 +1,9 @@
 """The C ABI: the library loads, exports every call include/hbl.h declares, and
 rejects bad arguments on the host before touching the GPU.  CPU only: every
-call here fails validation before any CUDA call, so no device is needed."""
+call here fails validation before any CUDA call, so no device is needed --
+except one, which runs in a child process with no device visible and checks
+that a well-formed call then fails with HBL_ERR_CUDA instead of running on the
+host."""
 import ctypes
 import os
 import re
@@ -181,3 +184,41 @@ def test_selftest_validation():
     assert lib.hbl_selftest_bounded_wait(0, 100, NUL, NUL) == 1
     assert lib.hbl_selftest_bounded_wait(0, 0, A, NUL) == 1
     assert lib.hbl_selftest_bounded_wait(0, 100, MIS, NUL) == 3
+
+
+def test_no_device_is_an_error_not_a_fallback():
+    # With no GPU visible, a well-formed call reaches the device query and
+    # returns HBL_ERR_CUDA (nothing runs on the host instead), and the binding
+    # raises when the library is missing.  Run in a child process with no
+    # device visible, so the fake pointers can never reach a GPU.
+    import subprocess
+    import sys
+
+    code = r'''
+import ctypes, sys
+sys.path.insert(0, %r)
+import hadamard_rotated_int4_b200 as hbl
+lib = hbl.lib()
+A, B, C, D, E = (ctypes.c_void_p(a) for a in (0x10000, 0x20000, 0x30000, 0x40000, 0x50000))
+need = ctypes.c_size_t(0)
+assert lib.hbl_workspace_size(hbl.OP_HBITLINEAR_FORWARD, 512, 4096, 256, 4, ctypes.byref(need)) == 0
+st = lib.hbl_hbitlinear_forward(A, None, 512, 4096, 256, B, C, 4, ctypes.c_float(1e-6),
+                                ctypes.c_float(1e-5), D, E, ctypes.c_size_t(need.value), None, None)
+print("forward", st)
+st = lib.hbl_norm_fwht_quant(A, None, 512, 4096, ctypes.c_float(1e-6), ctypes.c_float(1e-5), 4,
+                             B, C, D, None, None)
+print("quant", st)
+hbl.LIB_PATH = "/nonexistent/libhbl.so"
+hbl._lib = None
+try:
+    hbl.lib()
+    print("missing none")
+except RuntimeError:
+    print("missing raises")
+''' % ROOT
+    env = dict(os.environ, CUDA_VISIBLE_DEVICES="")
+    r = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True,
+                       timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    out = r.stdout.split()
+    assert out == ["forward", "6", "quant", "6", "missing", "raises"], r.stdout
